@@ -1,0 +1,198 @@
+"""Seeded synthetic workloads for the W4A4 linear layer.
+
+This module only draws numbers: it holds none of the layer's arithmetic
+(no transform, no scale, no rounding to codes, no GEMM).  Both the CPU oracle
+and the CUDA path receive the arrays built here.
+
+Shapes follow the LLaMA-family layers the pages quantize (FlatQuant notes,
+"Transformer 集成"; MergeQuant, "实验亮点": Llama-2-7B/70B; FRM-PTQ, "实验设置"):
+the pages measure on WikiText-2 / C4 activations of trained models, which are
+not available here, so these seeded Gaussian / Student-t tensors with planted
+outlier channels and a pivot token stand in for them.
+
+Every tensor is drawn in float64 from ``numpy.random.Generator(PCG64(seed))``
+in the order stated in each builder's docstring, then cast to float16
+(round-to-nearest-even) or float32.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+GROUP = 128
+_CHUNK = 1 << 22  # elements drawn per call; the stream is consumed in order
+
+
+def generator(seed: int) -> np.random.Generator:
+    return np.random.Generator(np.random.PCG64(seed))
+
+
+def _draw(g: np.random.Generator, shape, kind: str, scale: float, df: float = 5.0,
+          col_scale: np.ndarray | None = None, row_scale: np.ndarray | None = None,
+          dtype=np.float16) -> np.ndarray:
+    """Draw ``shape`` values row-chunk by row-chunk (same stream order as one call)."""
+    rows, cols = shape
+    out = np.empty((rows, cols), dtype=dtype)
+    step = max(1, _CHUNK // cols)
+    for r0 in range(0, rows, step):
+        r1 = min(rows, r0 + step)
+        if kind == "normal":
+            v = g.standard_normal((r1 - r0, cols))
+        elif kind == "t":
+            v = g.standard_t(df, (r1 - r0, cols))
+        else:
+            raise ValueError(kind)
+        v *= scale
+        if col_scale is not None:
+            v *= col_scale[None, :]
+        if row_scale is not None:
+            v *= row_scale[r0:r1, None]
+        out[r0:r1] = v.astype(dtype)
+    return out
+
+
+def kron_factors(k: int) -> tuple[int, int]:
+    """(n1, n2) with n1*n2 = k and the smallest n1 + n2 (FlatQuant notes,
+    "Kronecker 分解": the pair with the least n1 + n2, e.g. 8192 -> (64, 128)).
+
+    Reading: n2 is kept at most 128 so that one row of the n1 x n2 tile never
+    straddles a 128-wide quantization group; ties go to the larger n2.
+    """
+    best = None
+    for n2 in range(1, 129):
+        if k % n2:
+            continue
+        n1 = k // n2
+        key = (n1 + n2, -n2)
+        if best is None or key < best[0]:
+            best = (key, (n1, n2))
+    if best is None:
+        raise ValueError(f"no factorization for {k}")
+    return best[1]
+
+
+def orthogonal_scaled(g: np.random.Generator, n: int):
+    """P = Q @ diag(u): Q from the QR factorization of a Gaussian matrix with
+    the signs fixed so that R has a positive diagonal, u ~ U[0.8, 1.2].
+
+    Returns (P, P_inv) as float32, both computed in float64 first
+    (P_inv = diag(1/u) @ Q^T).  Draw order: n*n normals, then n uniforms.
+    """
+    a = g.standard_normal((n, n))
+    q, r = np.linalg.qr(a)
+    q = q * np.sign(np.diag(r))[None, :]
+    u = g.uniform(0.8, 1.2, n)
+    p = q * u[None, :]
+    p_inv = (q / u[None, :]).T
+    return p.astype(np.float32), p_inv.astype(np.float32)
+
+
+def outlier_channels(g: np.random.Generator, k: int, frac: float = 0.01) -> np.ndarray:
+    """A seeded choice of round(frac * k) channel indices (a permutation prefix)."""
+    n = int(round(frac * k))
+    return np.sort(g.permutation(k)[:n])
+
+
+# ---------------------------------------------------------------- workloads
+
+
+def tiny_linear(seed: int = 0) -> dict:
+    """Tiny W4A4 linear, no transform.
+
+    X fp16 [16, 256] ~ N(0, 1) with channels 3 and 77 scaled x50;
+    W fp16 [256, 256] ~ N(0, 0.02).  Draw order: X, W.
+    """
+    g = generator(seed)
+    m, k, n = 16, 256, 256
+    cs = np.ones(k)
+    cs[[3, 77]] = 50.0
+    x = _draw(g, (m, k), "normal", 1.0, col_scale=cs)
+    w = _draw(g, (n, k), "normal", 0.02)
+    return dict(name="tiny_linear_16x256x256", x=x, w=w, m=m, k=k, n=n,
+                alpha_a=1.0, alpha_w=1.0)
+
+
+def transform_quant(seed: int = 0, m: int = 2048, k: int = 4096) -> dict:
+    """Transform + quantize, LLaMA-3-8B-like hidden size.
+
+    X fp16 [m, k] ~ N(0, 1); 1% of the channels (seeded permutation) x30; token 0
+    x100 (the pivot token); P1, P2 = random orthogonal x diag(U[0.8, 1.2]) with
+    (n1, n2) = kron_factors(k); c ~ U[0.5, 2]; alpha_a = 0.9.
+    Draw order: X, P1, P2, c; the outlier channels come from a second stream
+    (seed + 1_000_003) because they must be known before X is cast.
+    """
+    g = generator(seed)
+    h = generator(seed + 1_000_003)
+    cols = outlier_channels(h, k)
+    cs = np.ones(k)
+    cs[cols] = 30.0
+    rs = np.ones(m)
+    rs[0] = 100.0
+    x = _draw(g, (m, k), "normal", 1.0, col_scale=cs, row_scale=rs)
+    n1, n2 = kron_factors(k)
+    p1, p1i = orthogonal_scaled(g, n1)
+    p2, p2i = orthogonal_scaled(g, n2)
+    c = g.uniform(0.5, 2.0, k).astype(np.float32)
+    return dict(name=f"transform_quant_{m}x{k}", x=x, m=m, k=k, n1=n1, n2=n2,
+                p1=p1, p2=p2, p1_inv=p1i, p2_inv=p2i, c=c, alpha_a=0.9,
+                outlier_cols=cols)
+
+
+def prefill_linear(k: int, n: int, m: int = 2048, seed: int = 0,
+                   w_kind: str = "normal", transform: bool = True) -> dict:
+    """Prefill W4A4 linear at LLaMA-like shapes.
+
+    X fp16 [m, k] ~ N(0, 1) with channels 3 and 77 x50 (the tiny recipe);
+    W fp16 [n, k] ~ N(0, 0.02) (w_kind="normal") or Student-t(5) * 0.02
+    (w_kind="t"); Kronecker factors P1, P2 (random orthogonal x diag(U[0.8,1.2]),
+    (n1, n2) = kron_factors(k)); c = 1; alpha_a = alpha_w = 1.
+    Draw order: X, W, P1, P2.
+    """
+    g = generator(seed)
+    cs = np.ones(k)
+    cs[[3, 77]] = 50.0
+    x = _draw(g, (m, k), "normal", 1.0, col_scale=cs)
+    w = _draw(g, (n, k), w_kind, 0.02)
+    d = dict(name=f"prefill_{m}x{k}x{n}_{w_kind}", x=x, w=w, m=m, k=k, n=n,
+             alpha_a=1.0, alpha_w=1.0)
+    if transform:
+        n1, n2 = kron_factors(k)
+        p1, p1i = orthogonal_scaled(g, n1)
+        p2, p2i = orthogonal_scaled(g, n2)
+        d.update(n1=n1, n2=n2, p1=p1, p2=p2, p1_inv=p1i, p2_inv=p2i)
+    return d
+
+
+def decode_static(m: int, k: int, n: int, seed: int = 0, calib_seed: int = 1,
+                  calib_tokens: int = 512) -> dict:
+    """Decode, static per-channel activation scales (MergeQuant-style).
+
+    X fp16 [m, k] ~ N(0, 1) with 1% outlier channels x30; W fp16 [n, k] ~ N(0, 0.02).
+    The calibration draw is X_cal fp16 [calib_tokens, k] from the same recipe
+    with ``calib_seed``; the outlier channels are shared (drawn from a stream
+    of ``seed`` + 1_000_003).  The stand-in static scale is
+    s_k = float32(max_t |X_cal[t, k]|) / 7 (the pages leave MergeQuant's
+    calibration unspecified).  Draw order: X, W; calibration stream: X_cal.
+    """
+    h = generator(seed + 1_000_003)
+    cols = outlier_channels(h, k)
+    cs = np.ones(k)
+    cs[cols] = 30.0
+    g = generator(seed)
+    x = _draw(g, (m, k), "normal", 1.0, col_scale=cs)
+    w = _draw(g, (n, k), "normal", 0.02)
+    gc = generator(calib_seed)
+    xc = _draw(gc, (calib_tokens, k), "normal", 1.0, col_scale=cs)
+    amax = np.abs(xc.astype(np.float32)).max(axis=0)
+    s_k = (amax / np.float32(7.0)).astype(np.float32)
+    return dict(name=f"decode_static_{m}x{k}x{n}", x=x, w=w, m=m, k=k, n=n,
+                static_scale=s_k, alpha_a=1.0, alpha_w=1.0, outlier_cols=cols)
+
+
+# The LLaMA-3-8B-like decoder-layer linears at prefill, M = 2048 tokens:
+# (K, N) for qkv, o, gate+up, down.
+PREFILL_8B_SHAPES = [(4096, 6144), (4096, 4096), (4096, 28672), (14336, 4096)]
+# The LLaMA-3-70B-like group-128 shapes at M = 4096.
+GROUP_70B_SHAPES = [(8192, 10240), (8192, 57344), (28672, 8192)]
+# Decode shapes.
+DECODE_70B_SHAPES = [(8192, 57344), (28672, 8192)]
+DECODE_TOKENS = [1, 8, 32, 64]

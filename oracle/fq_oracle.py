@@ -1,0 +1,288 @@
+"""CPU oracle for the W4A4 quantized linear layer.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the library imports this module: the
+tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py``
+are its only callers.  It shares no code with the CUDA path.
+
+It restates, step by step and in plain numpy, what the pages define:
+
+* the uniform quantizer Q(W) = clamp(round(W/s) + z, 0, 2^b - 1)
+  (FRM-PTQ page, section 初步介绍), used symmetric with b = 4 and z = 2^(b-1);
+* the per-channel scaling diag(c) placed before the affine transform and the
+  clip ratios alpha_w, alpha_a (FlatQuant notes, "额外可学习组件");
+* the Kronecker-factored affine transform P = P1 (x) P2 applied to the
+  n1 x n2 reshape of a row: activations go through P1^T x1 X x2 P2, weights
+  through P1^-1 x1 W x2 (P2^-1)^T (FlatQuant notes, "Kronecker 分解");
+* static per-channel activation scales and quantization-step migration into
+  the weights (MergeQuant page, 核心思路 / 关键设计);
+* group-wise quantization in groups of 128 along K (FRM-PTQ abstract,
+  multi-granularity group quantization);
+* the INT4 x INT4 product with integer accumulation and the dequantization
+  y = acc * s_x * s_w (FlatQuant notes, 核心思想: Y ~ Q(XP) Q(P^-1 W^T)).
+
+Precision: the transform is evaluated in float64 and rounded once to float32
+(the "transformed value"); scales, the division and round-half-to-even are
+float32 exactly as written; integer products are exact.
+
+Every function carries "parity pinned by" notes naming the CPU tests that
+check it against something other than itself.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+BITS = 4                      # b in Q(W)
+ZERO_POINT = 1 << (BITS - 1)  # z = 2^(b-1) = 8: the symmetric case
+QMAX_U = (1 << BITS) - 1      # 2^b - 1 = 15
+QMAX = QMAX_U - ZERO_POINT    # 7: largest signed code, the scale denominator
+QMIN = -ZERO_POINT            # -8
+GROUP = 128
+
+ROW, GROUPED, STATIC = 0, 1, 2   # per-token/per-channel, group-128, static per-channel
+
+
+# ------------------------------------------------------------------ quantizer
+
+def quantize(v32: np.ndarray, s32: np.ndarray) -> np.ndarray:
+    """Signed INT4 codes of Q(W) = clamp(round(W/s) + z, 0, 2^b - 1) - z.
+
+    FRM-PTQ page, 初步介绍 (the garbled brackets read as round-to-nearest,
+    ties to even; the garbled "2^b?1" read as 2^b - 1).  The division is an
+    IEEE float32 division; s = 0 gives code 0.
+    Parity pinned by: tests/golden/rtn_worked.txt, the |v - s*q| <= s/2 bound.
+    """
+    v32 = np.asarray(v32, dtype=np.float32)
+    s32 = np.asarray(s32, dtype=np.float32)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        ratio = v32 / s32                       # float32 / float32 -> float32
+    u = np.clip(np.rint(ratio) + ZERO_POINT, 0, QMAX_U)   # unsigned form of Q(W)
+    q = u - ZERO_POINT
+    q = np.where(s32 == 0, 0, q)
+    return q.astype(np.int8)
+
+
+def scale_row(v32: np.ndarray, alpha: float) -> np.ndarray:
+    """One float32 scale per row: s = (max|v| * alpha) / 7.
+
+    Symmetric absmax scale with the clip ratio alpha (FlatQuant notes,
+    "可学习裁剪阈值"); 7 = 2^(b-1) - 1 maps the clipped absmax to the largest code.
+    Parity pinned by: tests/golden/rtn_worked.txt.
+    """
+    amax = np.abs(v32).max(axis=-1).astype(np.float32)
+    return (amax * np.float32(alpha)) / np.float32(QMAX)
+
+
+def scale_group(v32: np.ndarray, alpha: float, group: int = GROUP) -> np.ndarray:
+    """One scale per row and group of ``group`` columns, stored in float16.
+
+    Same rule as scale_row on each group (FRM-PTQ multi-granularity group
+    quantization); the scale is rounded to float16 before it is used, so
+    quantization and dequantization use the same value.
+    Returns float32 [rows, K/group] holding float16 values.
+    Parity pinned by: the group == row special case, tests/golden/rtn_worked.txt.
+    """
+    r, k = v32.shape
+    amax = np.abs(v32.reshape(r, k // group, group)).max(axis=-1).astype(np.float32)
+    s = (amax * np.float32(alpha)) / np.float32(QMAX)
+    return s.astype(np.float16).astype(np.float32)
+
+
+def pack_int4(q: np.ndarray) -> np.ndarray:
+    """Two's-complement nibbles, element 2j in bits 0-3 and 2j+1 in bits 4-7 of byte j.
+
+    Parity pinned by: tests/golden/pack_int4.txt and the round trip over all codes.
+    """
+    q = np.asarray(q, dtype=np.int16)
+    lo = q[..., 0::2] & 0xF
+    hi = q[..., 1::2] & 0xF
+    return (lo | (hi << 4)).astype(np.uint8)
+
+
+def unpack_int4(p: np.ndarray) -> np.ndarray:
+    p = np.asarray(p, dtype=np.int16)
+    lo = p & 0xF
+    hi = (p >> 4) & 0xF
+    lo = np.where(lo >= 8, lo - 16, lo)
+    hi = np.where(hi >= 8, hi - 16, hi)
+    out = np.empty(p.shape[:-1] + (p.shape[-1] * 2,), dtype=np.int8)
+    out[..., 0::2] = lo
+    out[..., 1::2] = hi
+    return out
+
+
+# ------------------------------------------------------------------ transform
+
+def kron_apply(v64: np.ndarray, left: np.ndarray, right: np.ndarray) -> np.ndarray:
+    """Row-wise left @ Xbar @ right, where Xbar is the row-major n1 x n2 reshape.
+
+    Evaluated in float64: first T = left @ Xbar, then T @ right.
+    """
+    n1, n2 = left.shape[0], right.shape[0]
+    r = v64.shape[0]
+    xbar = v64.reshape(r, n1, n2)
+    t = np.matmul(left.astype(np.float64)[None], xbar)
+    out = np.matmul(t, right.astype(np.float64)[None])
+    return out.reshape(r, n1 * n2)
+
+
+def act_transform(x: np.ndarray, p1=None, p2=None, c=None) -> np.ndarray:
+    """float64 value of (x * c) (P1 (x) P2) for each token row x.
+
+    The channel scale c multiplies before the transform (FlatQuant notes,
+    "逐通道缩放 diag(c)...在仿射变换之前引入"); the transform is
+    P1^T x1 Xbar x2 P2 on the n1 x n2 reshape (FlatQuant notes, "Kronecker 分解").
+    Parity pinned by: explicit np.kron(P1, P2) product, the worked example in
+    tests/golden/kron_worked.txt, function preservation with weight_transform.
+    """
+    v = np.asarray(x, dtype=np.float64)
+    if c is not None:
+        v = v * np.asarray(c, dtype=np.float64)[None, :]
+    if p1 is not None:
+        v = kron_apply(v, np.asarray(p1).T, np.asarray(p2))
+    return v
+
+
+def weight_transform(w: np.ndarray, p1_inv=None, p2_inv=None, c=None) -> np.ndarray:
+    """float64 value of P^-1 applied to each weight row (as a column of W^T).
+
+    The weight side divides by c and applies P1^-1 x1 Wbar x2 (P2^-1)^T
+    (FlatQuant notes, "Kronecker 分解"); the inverses are the caller's.
+    Parity pinned by: explicit np.kron(P1^-1, P2^-1) product and function
+    preservation X P P^-1 W^T = X W^T.
+    """
+    v = np.asarray(w, dtype=np.float64)
+    if c is not None:
+        v = v / np.asarray(c, dtype=np.float64)[None, :]
+    if p1_inv is not None:
+        v = kron_apply(v, np.asarray(p1_inv), np.asarray(p2_inv).T)
+    return v
+
+
+# ------------------------------------------------------------------ quant steps
+
+def quant_act(x, gran=ROW, alpha=1.0, p1=None, p2=None, c=None, static_scale=None):
+    """Online activation quantization of fp16 rows.
+
+    Returns (codes int8 [M, K], scales, transformed float32 [M, K]) where the
+    scales are float32 [M] (ROW), float32-held float16 [M, K/128] (GROUPED) or
+    the given static scale float32 [K] (STATIC, MergeQuant page).
+    """
+    v32 = act_transform(x, p1, p2, c).astype(np.float32)
+    if gran == ROW:
+        s = scale_row(v32, alpha)
+        q = quantize(v32, s[:, None])
+    elif gran == GROUPED:
+        s = scale_group(v32, alpha)
+        q = quantize(v32, np.repeat(s, GROUP, axis=1))
+    elif gran == STATIC:
+        s = np.asarray(static_scale, dtype=np.float32)
+        q = quantize(v32, s[None, :])
+    else:
+        raise ValueError(gran)
+    return q, s, v32
+
+
+def quant_weight(w, gran=ROW, alpha=1.0, p1_inv=None, p2_inv=None, c=None,
+                 qsm_scale=None):
+    """Offline weight quantization of fp16 rows W [N, K].
+
+    Steps: divide by c, apply the inverse Kronecker transform (float64), round
+    once to float32, fold the static activation scales s_k into the weights
+    with one float32 multiply (quantization step migration, MergeQuant page,
+    关键设计), then per-output-channel (ROW) or group-128 (GROUPED) scales and
+    codes.  Returns (codes int8 [N, K], scales, float32 values quantized).
+    """
+    v32 = weight_transform(w, p1_inv, p2_inv, c).astype(np.float32)
+    if qsm_scale is not None:
+        v32 = v32 * np.asarray(qsm_scale, dtype=np.float32)[None, :]
+    if gran == ROW:
+        s = scale_row(v32, alpha)
+        q = quantize(v32, s[:, None])
+    elif gran == GROUPED:
+        s = scale_group(v32, alpha)
+        q = quantize(v32, np.repeat(s, GROUP, axis=1))
+    else:
+        raise ValueError(gran)
+    return q, s, v32
+
+
+# ------------------------------------------------------------------ GEMM + dequant
+
+def gemm_int(qx: np.ndarray, qw: np.ndarray) -> np.ndarray:
+    """acc[m, n] = sum_k qx[m, k] * qw[n, k], exact, as int64.
+
+    The matmul runs on float64 holding integers: every product is at most 64
+    in magnitude and every partial sum at most 64*K < 2^53, so each float64
+    operation is exact whatever the summation order.
+    Parity pinned by: the pure-Python triple loop on tiny shapes.
+    """
+    k = qx.shape[1]
+    assert 64 * k < (1 << 53)
+    acc = np.asarray(qx, np.float64) @ np.asarray(qw, np.float64).T
+    return acc.astype(np.int64)
+
+
+def dequant_row(acc: np.ndarray, s_x: np.ndarray, s_w: np.ndarray) -> np.ndarray:
+    """y = fp16_rne((float32(acc) * s_x[m]) * s_w[n]), two float32 multiplies."""
+    assert np.abs(acc).max(initial=0) < (1 << 24)
+    a = acc.astype(np.float32)
+    y = (a * np.asarray(s_x, np.float32)[:, None]) * np.asarray(s_w, np.float32)[None, :]
+    return y.astype(np.float16)
+
+
+def dequant_static(acc: np.ndarray, s_w: np.ndarray) -> np.ndarray:
+    """y = fp16_rne(float32(acc) * s_w'[n]) where s_w' already carries the migrated
+    activation scales (MergeQuant quantization step migration)."""
+    assert np.abs(acc).max(initial=0) < (1 << 24)
+    y = acc.astype(np.float32) * np.asarray(s_w, np.float32)[None, :]
+    return y.astype(np.float16)
+
+
+def dequant_group(qx, qw, s_x, s_w) -> np.ndarray:
+    """y = fp16_rne(sum_g acc_g * s_x[m, g] * s_w[n, g]) in float64, g ascending,
+    where acc_g is the exact integer product over k in [128 g, 128 g + 128).
+
+    s_x [M, K/128] and s_w [N, K/128] hold float16 values.
+    Parity pinned by: the single-group case against dequant_row and the
+    float64 dequantize-then-multiply bound.
+    """
+    m, k = qx.shape
+    n = qw.shape[0]
+    y = np.zeros((m, n), dtype=np.float64)
+    for g in range(k // GROUP):
+        sl = slice(g * GROUP, (g + 1) * GROUP)
+        acc_g = gemm_int(qx[:, sl], qw[:, sl]).astype(np.float64)
+        y += acc_g * np.asarray(s_x, np.float64)[:, g:g + 1] * np.asarray(s_w, np.float64)[None, :, g]
+    return y.astype(np.float16)
+
+
+def linear(x, wq, s_w, gran=ROW, alpha=1.0, p1=None, p2=None, c=None,
+           static_scale=None):
+    """Y = dequant(Q(X P) Q(P^-1 W^T)) for fp16 X [M, K] and weight codes wq [N, K]."""
+    qx, s_x, _ = quant_act(x, gran, alpha, p1, p2, c, static_scale)
+    if gran == ROW:
+        return dequant_row(gemm_int(qx, wq), s_x, s_w)
+    if gran == STATIC:
+        return dequant_static(gemm_int(qx, wq), s_w)
+    return dequant_group(qx, wq, s_x, s_w)
+
+
+# ------------------------------------------------------------------ sampled rows
+
+def linear_rows(rows, x, wq, s_w, **kw):
+    """The rows ``rows`` of linear(...): every step above is row-independent."""
+    rows = np.asarray(rows)
+    return linear(np.asarray(x)[rows], wq, s_w, **kw)
+
+
+# ------------------------------------------------------------------ counts
+
+def kron_flops(n1: int, n2: int) -> int:
+    """Multiply-adds x2 per row for P1^T Xbar P2: 2 n (n1 + n2), n = n1 n2
+    (FlatQuant notes: computation saving sqrt(n)/2 against a dense n x n P)."""
+    n = n1 * n2
+    return 2 * n * (n1 + n2)
+
+
+def dense_transform_flops(n: int) -> int:
+    return 2 * n * n

@@ -1,0 +1,320 @@
+"""Checks that pin the CPU oracle to what the pages and the mathematics fix.
+
+Each check takes the oracle module (or a copy with one planted mistake) and
+raises AssertionError when it disagrees.  ``test_oracle_pins`` runs every check
+on the oracle as it stands and, through ``test_oracle_mutants``, shows that a
+plausible mistake in any step (a transposed factor, a dropped term, a wrong
+sign, rounding or nibble order) fails at least one of them.
+"""
+from __future__ import annotations
+
+import os
+import types
+
+import numpy as np
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _lines(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        for ln in f:
+            ln = ln.strip()
+            if ln and not ln.startswith("#"):
+                yield ln
+
+
+# ------------------------------------------------------------------ quantizer
+
+def check_rtn_golden(o):
+    """Hand-worked rows in tests/golden/rtn_worked.txt (Q(W), FRM-PTQ page 初步介绍)."""
+    for ln in _lines("rtn_worked.txt"):
+        head, xs, ss, qs = [p.strip() for p in ln.split("|")]
+        mode, alpha = head.split()
+        x = np.array([float(v) for v in xs.split()], dtype=np.float16)
+        s_exp = np.float32(float(ss))
+        q_exp = np.array([int(v) for v in qs.split()], dtype=np.int8)
+        if mode == "row":
+            q, s, _ = o.quant_act(x[None, :], o.ROW, float(alpha))
+            assert np.float32(s[0]) == s_exp, (ln, s[0])
+            assert np.array_equal(q[0], q_exp), (ln, q[0])
+        elif mode == "group1":
+            xx = np.zeros((1, o.GROUP), dtype=np.float16)
+            xx[0, :x.size] = x
+            q, s, _ = o.quant_act(xx, o.GROUPED, float(alpha))
+            assert np.float32(s[0, 0]) == s_exp, (ln, s[0, 0])
+            assert np.array_equal(q[0, :x.size], q_exp), (ln, q[0, :x.size])
+        else:
+            raise ValueError(mode)
+
+
+def check_rtn_bounds(o):
+    """Every unclipped element satisfies |v - s q| <= s/2; codes lie in [-8, 7];
+    alpha = 1 never produces -8 and maps each row's absmax to +-7."""
+    g = np.random.Generator(np.random.PCG64(11))
+    x = (g.standard_normal((64, 256)) * g.uniform(0.01, 30, (64, 1))).astype(np.float16)
+    for alpha in (1.0, 0.8):
+        q, s, v = o.quant_act(x, o.ROW, alpha)
+        assert q.min() >= -8 and q.max() <= 7
+        deq = q.astype(np.float64) * s[:, None].astype(np.float64)
+        unclipped = (q > -8) & (q < 7)
+        err = np.abs(v.astype(np.float64) - deq)
+        bound = s[:, None].astype(np.float64) / 2 * (1 + 1e-6)
+        assert np.all(err[unclipped] <= np.broadcast_to(bound, err.shape)[unclipped])
+        if alpha == 1.0:
+            assert q.min() > -8
+            idx = np.abs(v).argmax(axis=1)
+            assert np.all(np.abs(q[np.arange(64), idx]) == 7)
+    qg, sg, vg = o.quant_act(x, o.GROUPED, 1.0)
+    deq = qg.astype(np.float64) * np.repeat(sg, o.GROUP, axis=1)
+    unclipped = (qg > -8) & (qg < 7)
+    err = np.abs(vg.astype(np.float64) - deq)
+    bound = np.repeat(sg, o.GROUP, axis=1) / 2 * (1 + 1e-6)
+    assert np.all(err[unclipped] <= bound[unclipped])
+
+
+def check_pack(o):
+    """tests/golden/pack_int4.txt and the round trip over all 16 x 16 code pairs."""
+    for ln in _lines("pack_int4.txt"):
+        codes, byte = [p.strip() for p in ln.split("|")]
+        q = np.array([[int(v) for v in codes.split()]], dtype=np.int8)
+        assert o.pack_int4(q)[0, 0] == int(byte, 16), ln
+    a, b = np.meshgrid(np.arange(-8, 8), np.arange(-8, 8))
+    q = np.stack([a.ravel(), b.ravel()], axis=1).reshape(1, -1).astype(np.int8)
+    assert np.array_equal(o.unpack_int4(o.pack_int4(q)), q)
+
+
+# ------------------------------------------------------------------ transform
+
+def check_kron_golden(o):
+    """tests/golden/kron_worked.txt (FlatQuant notes, Kronecker 分解)."""
+    d = {}
+    for ln in _lines("kron_worked.txt"):
+        key, *vals = ln.split()
+        d[key] = np.array([float(v) for v in vals])
+    n1, n2 = int(d["n1"][0]), int(d["n2"][0])
+    p1 = d["P1"].reshape(n1, n1)
+    p2 = d["P2"].reshape(n2, n2)
+    p1i = d["P1inv"].reshape(n1, n1)
+    p2i = d["P2inv"].reshape(n2, n2)
+    xh = o.act_transform(d["x"][None, :], p1, p2)
+    assert np.array_equal(xh[0], d["xhat"]), xh
+    wh = o.weight_transform(d["w"][None, :], p1i, p2i)
+    assert np.array_equal(wh[0], d["what"]), wh
+
+
+def check_kron_explicit(o):
+    """x (P1 (x) P2) against the explicit n x n Kronecker matrix, and the weight
+    side against (P1^-1 (x) P2^-1) w, on tiny n, float64, <= 1e-12 relative."""
+    g = np.random.Generator(np.random.PCG64(5))
+    for n1, n2 in [(2, 4), (3, 5), (8, 8), (4, 2)]:
+        n = n1 * n2
+        x = g.standard_normal((3, n))
+        p1 = g.standard_normal((n1, n1))
+        p2 = g.standard_normal((n2, n2))
+        c = g.uniform(0.5, 2, n)
+        ref = (x * c) @ np.kron(p1, p2)
+        got = o.act_transform(x, p1, p2, c)
+        assert np.abs(got - ref).max() <= 1e-12 * np.abs(ref).max(), (n1, n2)
+        p1i, p2i = np.linalg.inv(p1), np.linalg.inv(p2)
+        w = g.standard_normal((2, n))
+        refw = (w / c) @ np.kron(p1i, p2i).T
+        gotw = o.weight_transform(w, p1i, p2i, c)
+        assert np.abs(gotw - refw).max() <= 1e-12 * np.abs(refw).max(), (n1, n2)
+
+
+def check_function_preservation(o):
+    """X P (P^-1 W^T) = X W^T in float64 (FlatQuant notes, 核心思想), with the
+    channel scale c on both sides; and a permutation P (PT2-LLM page, SSR:
+    X' W'^T = X W^T) is exact."""
+    g = np.random.Generator(np.random.PCG64(6))
+    n1, n2 = 8, 16
+    n = n1 * n2
+    x = g.standard_normal((5, n))
+    w = g.standard_normal((7, n))
+    p1 = g.standard_normal((n1, n1)) + 4 * np.eye(n1)
+    p2 = g.standard_normal((n2, n2)) + 4 * np.eye(n2)
+    c = g.uniform(0.5, 2, n)
+    y = o.act_transform(x, p1, p2, c) @ o.weight_transform(w, np.linalg.inv(p1), np.linalg.inv(p2), c).T
+    ref = x @ w.T
+    assert np.abs(y - ref).max() <= 1e-10 * np.abs(ref).max()
+    # permutation factors (PT2-LLM page, SSR: W' = W P, X' = X P): the transform
+    # only moves values, and on integer data the product is exactly unchanged
+    e1 = np.eye(n1)[g.permutation(n1)]
+    e2 = np.eye(n2)[g.permutation(n2)]
+    xi = g.integers(-50, 50, (5, n)).astype(np.float64)
+    wi = g.integers(-50, 50, (7, n)).astype(np.float64)
+    xp = o.act_transform(xi, e1, e2)
+    wp = o.weight_transform(wi, e1.T, e2.T)
+    assert np.array_equal(np.sort(xp, axis=1), np.sort(xi, axis=1))
+    assert np.array_equal(xp @ wp.T, xi @ wi.T)
+
+
+def check_identity_transform(o):
+    """P1 = P2 = I and c = 1 reduce the transformed path to the plain one, bit for bit."""
+    g = np.random.Generator(np.random.PCG64(7))
+    x = g.standard_normal((4, 256)).astype(np.float16)
+    a = o.quant_act(x, o.ROW, 0.9, np.eye(16, dtype=np.float32), np.eye(16, dtype=np.float32),
+                    np.ones(256, np.float32))
+    b = o.quant_act(x, o.ROW, 0.9)
+    assert all(np.array_equal(u, v) for u, v in zip(a, b))
+
+
+def check_flop_count(o):
+    """Per row, a dense n x n transform costs 2 n^2 flops and the Kronecker form
+    2 n (n1 + n2); with n1 = n2 = sqrt(n) the saving is sqrt(n)/2, and the
+    parameters shrink from n^2 to n1^2 + n2^2, a saving of n/2 (FlatQuant notes,
+    Kronecker 分解)."""
+    for r in (8, 16, 64, 128):
+        n = r * r
+        assert o.kron_flops(r, r) == 2 * n * 2 * r
+        assert o.dense_transform_flops(n) / o.kron_flops(r, r) == np.sqrt(n) / 2
+        assert (n * n) / (r * r + r * r) == n / 2
+    assert o.kron_flops(64, 128) == 2 * 8192 * 192
+
+
+# ------------------------------------------------------------------ GEMM + dequant
+
+def _brute(qx, qw):
+    m, k = qx.shape
+    n = qw.shape[0]
+    out = [[0] * n for _ in range(m)]
+    for i in range(m):
+        for j in range(n):
+            t = 0
+            for kk in range(k):
+                t += int(qx[i, kk]) * int(qw[j, kk])
+            out[i][j] = t
+    return np.array(out, dtype=np.int64)
+
+
+def check_gemm_bruteforce(o):
+    """Integer accumulation against a pure-Python triple loop on tiny shapes, and
+    the extreme -8 * -8 over K = 28672 (the largest K in use)."""
+    g = np.random.Generator(np.random.PCG64(8))
+    for m, n, k in [(1, 1, 1), (3, 5, 7), (4, 6, 128), (2, 3, 256)]:
+        qx = g.integers(-8, 8, (m, k), dtype=np.int8)
+        qw = g.integers(-8, 8, (n, k), dtype=np.int8)
+        assert np.array_equal(o.gemm_int(qx, qw), _brute(qx, qw)), (m, n, k)
+    k = 28672
+    qx = np.full((1, k), -8, np.int8)
+    assert o.gemm_int(qx, qx)[0, 0] == 64 * k
+    qw = np.full((1, k), 7, np.int8)
+    assert o.gemm_int(qx, qw)[0, 0] == -56 * k
+
+
+def check_linear_golden(o):
+    """tests/golden/linear_worked.txt: the whole layer on a hand-worked 1 x 4 x 2 case."""
+    d = {}
+    for ln in _lines("linear_worked.txt"):
+        key, *vals = ln.split()
+        d[key] = np.array([float(v) for v in vals])
+    x = d["x"].astype(np.float16)[None, :]
+    w = np.stack([d["w0"], d["w1"]]).astype(np.float16)
+    qw, sw, _ = o.quant_weight(w, o.ROW, 1.0)
+    assert np.array_equal(qw[0], d["qw0"]) and np.array_equal(qw[1], d["qw1"]), qw
+    qx, sx, _ = o.quant_act(x, o.ROW, 1.0)
+    assert np.array_equal(qx[0], d["qx"]), qx
+    acc = o.gemm_int(qx, qw)
+    assert np.array_equal(acc[0], d["acc"]), acc
+    y = o.linear(x, qw, sw, o.ROW, 1.0)
+    assert np.array_equal(y[0].astype(np.float64), d["y"]), y
+
+
+def check_dequant_bound(o):
+    """The per-row epilogue equals the float64 product of the dequantized
+    operands up to the float32 and float16 roundings: |y - ref| <= 1 fp16 ulp
+    of ref + 2^-22 |ref|; the group epilogue likewise with per-group scales."""
+    g = np.random.Generator(np.random.PCG64(9))
+    m, n, k = 8, 16, 512
+    x = (g.standard_normal((m, k)) * 3).astype(np.float16)
+    w = (g.standard_normal((n, k)) * 0.02).astype(np.float16)
+    for gran in (o.ROW, o.GROUPED):
+        qx, sx, _ = o.quant_act(x, gran, 1.0)
+        qw, sw, _ = o.quant_weight(w, gran, 1.0)
+        y = o.linear(x, qw, sw, gran, 1.0).astype(np.float64)
+        if gran == o.ROW:
+            xd = qx * sx[:, None].astype(np.float64)
+            wd = qw * sw[:, None].astype(np.float64)
+        else:
+            xd = qx * np.repeat(sx, o.GROUP, axis=1)
+            wd = qw * np.repeat(sw, o.GROUP, axis=1)
+        ref = xd @ wd.T
+        ulp = np.spacing(np.abs(ref).astype(np.float16)).astype(np.float64)
+        assert np.all(np.abs(y - ref) <= ulp + 2.0 ** -22 * np.abs(ref)), gran
+
+
+def check_group_equals_row(o):
+    """With K = 128 (one group) and float16-exact scales the group path equals the
+    per-row path (FRM-PTQ: the granularities differ only in the scale's extent)."""
+    g = np.random.Generator(np.random.PCG64(10))
+    m, n, k = 4, 8, 128
+    x = g.standard_normal((m, k))
+    x = x / np.abs(x).max(axis=1, keepdims=True) * (7 * 2.0 ** g.integers(-3, 3, (m, 1)))
+    w = g.standard_normal((n, k))
+    w = w / np.abs(w).max(axis=1, keepdims=True) * (7 * 2.0 ** g.integers(-9, -5, (n, 1)))
+    x, w = x.astype(np.float16), w.astype(np.float16)
+    qxr, sxr, _ = o.quant_act(x, o.ROW, 1.0)
+    qxg, sxg, _ = o.quant_act(x, o.GROUPED, 1.0)
+    assert np.array_equal(qxr, qxg) and np.array_equal(sxr, sxg[:, 0])
+    qwr, swr, _ = o.quant_weight(w, o.ROW, 1.0)
+    qwg, swg, _ = o.quant_weight(w, o.GROUPED, 1.0)
+    assert np.array_equal(qwr, qwg)
+    yr = o.linear(x, qwr, swr, o.ROW, 1.0)
+    yg = o.linear(x, qwg, swg, o.GROUPED, 1.0)
+    assert np.array_equal(yr, yg)
+
+
+def check_static_equals_row(o):
+    """Static per-channel scales all equal to a row's dynamic scale give that row's
+    dynamic codes (MergeQuant static vs per-token dynamic calibration)."""
+    g = np.random.Generator(np.random.PCG64(12))
+    x = g.standard_normal((3, 256)).astype(np.float16)
+    q, s, _ = o.quant_act(x, o.ROW, 1.0)
+    for r in range(3):
+        qs, _, _ = o.quant_act(x[r:r + 1], o.STATIC, static_scale=np.full(256, s[r], np.float32))
+        assert np.array_equal(qs[0], q[r])
+
+
+def check_qsm_fold(o):
+    """Quantization step migration: folding s_k into the weights and dequantizing
+    with s_w' alone approximates sum_k q_x s_k w (MergeQuant 核心思路), and the fold
+    multiplies the weight columns, not the rows."""
+    g = np.random.Generator(np.random.PCG64(13))
+    m, n, k = 4, 6, 256
+    x = g.standard_normal((m, k)).astype(np.float16)
+    w = (g.standard_normal((n, k)) * 0.02).astype(np.float16)
+    s_k = g.uniform(0.2, 0.6, k).astype(np.float32)
+    qx, _, _ = o.quant_act(x, o.STATIC, static_scale=s_k)
+    qw, sw, v = o.quant_weight(w, o.ROW, 1.0, qsm_scale=s_k)
+    assert np.array_equal(v, w.astype(np.float32) * s_k[None, :])
+    y = o.linear(x, qw, sw, o.STATIC, static_scale=s_k).astype(np.float64)
+    ref = (qx * s_k.astype(np.float64)) @ w.astype(np.float64).T
+    # error of W4 weights: |sum_k qx_k dq_k| <= sum |qx| s_w / 2 per output
+    bound = np.abs(qx).sum(axis=1, keepdims=True) * sw[None, :] / 2 + 1e-2 * np.abs(ref)
+    assert np.all(np.abs(y - ref) <= bound)
+
+
+ALL_CHECKS = [
+    check_rtn_golden, check_rtn_bounds, check_pack, check_kron_golden,
+    check_kron_explicit, check_function_preservation, check_identity_transform,
+    check_flop_count, check_gemm_bruteforce, check_linear_golden,
+    check_dequant_bound, check_group_equals_row, check_static_equals_row,
+    check_qsm_fold,
+]
+
+
+def mutant(o, **overrides):
+    """A copy of the oracle module with some functions replaced."""
+    m = types.ModuleType(o.__name__ + "_mutant")
+    m.__dict__.update(o.__dict__)
+    m.__dict__.update(overrides)
+    # functions resolve globals in their own module: rebind them to the copy
+    for name, f in list(m.__dict__.items()):
+        if isinstance(f, types.FunctionType) and f.__module__ == o.__name__ and name not in overrides:
+            m.__dict__[name] = types.FunctionType(f.__code__, m.__dict__, f.__name__, f.__defaults__, f.__closure__)
+    for name in overrides:
+        f = m.__dict__[name]
+        if isinstance(f, types.FunctionType):
+            m.__dict__[name] = types.FunctionType(f.__code__, m.__dict__, f.__name__, f.__defaults__, f.__closure__)
+    return m
