@@ -1,0 +1,182 @@
+/*
+ * fq.h - C ABI of libfq.so, a B200 (sm_100a) W4A4 quantized linear layer.
+ *
+ * The layer computes Y ~ Q(X P) Q(P^-1 W^T): activations X are optionally
+ * scaled per channel and passed through a Kronecker-factored affine transform
+ * P = P1 (x) P2, quantized online to signed INT4 codes, multiplied with
+ * offline-quantized INT4 weights with exact integer accumulation, and
+ * dequantized to fp16 (FlatQuant notes, sections 核心思想 and Kronecker 分解;
+ * the quantizer Q(W) = clamp(round(W/s) + z, 0, 2^b - 1) of the FRM-PTQ page,
+ * section 初步介绍; static per-channel activation scales and quantization-step
+ * migration from the MergeQuant page, 核心思路; group-128 scales from FRM-PTQ's
+ * multi-granularity group quantization).
+ *
+ * Conventions shared by every entry point
+ * ----------------------------------------
+ * - Memory. Every tensor pointer is DEVICE memory owned by the caller; the
+ *   library never allocates, frees or keeps a pointer after a call returns.
+ *   fp16 tensors are passed as uint16_t* holding IEEE binary16 bits.
+ *   Matrices are row-major and densely packed.  Pointers read by the tensor
+ *   memory accelerator (Xq, Wq, and group scales) must be 16-byte aligned;
+ *   all others 4-byte aligned (16-byte for X and Y is recommended).
+ * - Streams. `stream` is a cudaStream_t (NULL = the legacy default stream).
+ *   Every call is asynchronous: it validates its arguments on the host,
+ *   enqueues its kernels on `stream` and returns.  No call synchronizes,
+ *   except fq_check_device_error.
+ * - Errors. On any non-FQ_OK status nothing has been enqueued, except
+ *   FQ_ERR_CUDA from a failed launch.  fq_last_error() returns a message
+ *   for the calling thread's last failure.  Kernels never trap: a bounded
+ *   wait that gives up records FQ_ERR_TIMEOUT in a device word that
+ *   fq_check_device_error reads and clears.
+ * - INT4 codes. Symmetric, b = 4, zero point z = 2^(b-1) = 8, so the signed
+ *   code is q = clamp(round(x/s), -8, 7), round half to even, IEEE float32
+ *   division, s = 0 giving q = 0.  Codes are stored two per byte as
+ *   two's-complement nibbles: element 2j in bits 0-3 and element 2j+1 in
+ *   bits 4-7 of byte j.  A packed [R, K] matrix is uint8 [R, K/2].
+ * - Scales. Per row (token or output channel): float32 [R],
+ *   s = (max|v| * alpha) / 7 in float32.  Per group of 128 along K: fp16,
+ *   the same rule on each group, rounded to fp16 before it is used, stored
+ *   GROUP-MAJOR as [K/128][R] (row r of group g at g*R + r).  Static
+ *   per-input-channel activation scales: float32 [K], given by the caller.
+ * - Sizes. K % 128 == 0 and 128 <= K <= 65536 (quantization kernels: K <=
+ *   32768); N % 8 == 0; M >= 1; a transform needs n1 * n2 == K with
+ *   1 <= n1, n2 <= 256.
+ */
+#ifndef FQ_H_
+#define FQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FQ_OK = 0,
+  FQ_ERR_INVALID = 1,      /* a NULL/misaligned pointer or a size outside the ranges above */
+  FQ_ERR_UNSUPPORTED = 2,  /* b != 4, z != 2^(b-1), group size != 128, or a mode/argument combination not provided */
+  FQ_ERR_CUDA = 3,         /* the CUDA runtime or driver reported an error (launch, tensor-map encode) */
+  FQ_ERR_TIMEOUT = 4       /* a kernel's bounded wait gave up (reported by fq_check_device_error) */
+} fq_status;
+
+/* Extent of one scale (FRM-PTQ multi-granularity; MergeQuant static calibration). */
+typedef enum {
+  FQ_DYNAMIC_ROW = 0,    /* one scale per token (activations) / per output channel (weights) */
+  FQ_DYNAMIC_GROUP = 1,  /* one scale per row and group of 128 along K */
+  FQ_STATIC_CHANNEL = 2  /* activations only: caller-given float32 scale per input channel */
+} fq_gran;
+
+/* Parameters of Q(W) = clamp(round(W/s) + z, 0, 2^b - 1) (FRM-PTQ page, 初步介绍)
+ * and the clip ratio alpha of s = max|v| * alpha / 7 (FlatQuant notes,
+ * 可学习裁剪阈值).  Host memory, read during the call only. */
+typedef struct {
+  int bits;         /* b: only 4 */
+  int zero_point;   /* z: only 2^(b-1) = 8 (the symmetric quantizer) */
+  fq_gran gran;     /* scale extent */
+  int group_size;   /* 128 when gran == FQ_DYNAMIC_GROUP, ignored otherwise */
+  float alpha;      /* clip ratio in (0, 1]; unused for FQ_STATIC_CHANNEL */
+} fq_qparams;
+
+/* Kronecker-factored transform P = P1 (x) P2 and channel scale c (FlatQuant
+ * notes, Kronecker 分解 and 逐通道缩放).  Host struct; the matrix pointers are
+ * device float32, row-major.  For activations P1 [n1,n1], P2 [n2,n2] are the
+ * factors and each row is mapped to c * x followed by P1^T Xbar P2 on its
+ * row-major n1 x n2 reshape Xbar.  For weights the caller passes the
+ * INVERSES P1^-1, P2^-1 and each weight row w (a column of W^T) is mapped to
+ * w / c followed by P1^-1 Wbar (P2^-1)^T.  P1 == NULL means no transform
+ * (then P2, n1, n2 are ignored); c == NULL means c = 1. */
+typedef struct {
+  int n1, n2;
+  const float* P1;
+  const float* P2;
+  const float* c;   /* [K] */
+} fq_transform;
+
+/* Offline weight quantization (FlatQuant notes, Kronecker 分解: Q(P1^-1 W P2^-T);
+ * MergeQuant 核心思路: quantization step migration).
+ * W      fp16 [N, K]: weights, one row per output channel.
+ * qp     gran FQ_DYNAMIC_ROW (s_w float32 [N]) or FQ_DYNAMIC_GROUP (s_w fp16 [K/128][N]);
+ *        alpha = alpha_w.
+ * inv    NULL or the inverse transform (P1^-1, P2^-1, c): see fq_transform.
+ * qsm_scale NULL or float32 [K]: static activation scales s_k folded into the
+ *        weights, w'[n,k] = v[n,k] * s_k in float32 after the transform, so
+ *        that the GEMM epilogue needs s_w' only.
+ * Wq     uint8 [N, K/2] packed codes (out).  s_w: scales (out).
+ * Order per row: /c, inverse transform, x s_k, scale, round, pack. */
+fq_status fq_quant_weight(const uint16_t* W, int N, int K, const fq_qparams* qp,
+                          const fq_transform* inv, const float* qsm_scale,
+                          uint8_t* Wq, void* s_w, void* stream);
+
+/* Online activation quantization (FlatQuant notes, 高效 Kernel 设计: the
+ * transform and the quantization fused, intermediates kept on chip).
+ * X      fp16 [M, K] token rows.
+ * qp     FQ_DYNAMIC_ROW: s_x float32 [M];  FQ_DYNAMIC_GROUP: s_x fp16 [K/128][M];
+ *        FQ_STATIC_CHANNEL: static_scale float32 [K] is used and s_x is not written
+ *        (may be NULL); alpha = alpha_a.
+ * t      NULL or the transform (P1, P2, c).
+ * Xq     uint8 [M, K/2] packed codes (out). */
+fq_status fq_quant_act(const uint16_t* X, int M, int K, const fq_qparams* qp,
+                       const fq_transform* t, const float* static_scale,
+                       uint8_t* Xq, void* s_x, void* stream);
+
+/* fq_quant_act that also writes xhat float32 [M, K], the transformed values
+ * that were quantized (for checking the transform on its own). */
+fq_status fq_quant_act_debug(const uint16_t* X, int M, int K, const fq_qparams* qp,
+                             const fq_transform* t, const float* static_scale,
+                             uint8_t* Xq, void* s_x, float* xhat, void* stream);
+
+/* INT4 x INT4 GEMM with exact integer accumulation and fp16 dequantization
+ * (FlatQuant notes, 核心思想: Y ~ Q(XP) Q(P^-1 W^T)).
+ * Xq uint8 [M, K/2], Wq uint8 [N, K/2] packed codes; Y fp16 [M, N] (out):
+ *   FQ_DYNAMIC_ROW:    y = fp16((float(acc) * s_x[m]) * s_w[n]), s_x float32 [M], s_w float32 [N]
+ *   FQ_STATIC_CHANNEL: y = fp16(float(acc) * s_w[n]), s_x unused (may be NULL)
+ *   FQ_DYNAMIC_GROUP:  y = fp16(sum_g float(acc_g) * s_x[g][m] * s_w[g][n]), the sum in
+ *                      float32, acc_g the exact product over k in [128g, 128g+128);
+ *                      s_x fp16 [K/128][M], s_w fp16 [K/128][N].
+ * workspace / ws_bytes: device scratch of at least fq_gemm_workspace_size()
+ *   bytes (may be NULL when that size is 0); contents on entry are ignored. */
+fq_status fq_w4a4_gemm(const uint8_t* Xq, const void* s_x, const uint8_t* Wq, const void* s_w,
+                       int M, int N, int K, fq_gran gran, uint16_t* Y,
+                       void* workspace, size_t ws_bytes, void* stream);
+
+/* The exact integer accumulators acc[m][n] = sum_k qx[m,k] qw[n,k] as int32
+ * [M, N] (out), for checking the GEMM's integer part on its own. */
+fq_status fq_w4a4_gemm_s32(const uint8_t* Xq, const uint8_t* Wq, int M, int N, int K,
+                           int32_t* acc, void* stream);
+
+/* The linear layer: fq_quant_act into the workspace, then fq_w4a4_gemm, on
+ * one stream.  Arguments as in those two calls; Wq/s_w come from
+ * fq_quant_weight with the matching inverse transform (and, for
+ * FQ_STATIC_CHANNEL, the same static scales folded in).  workspace must hold
+ * fq_linear_workspace_size() bytes (packed activations, their scales and the
+ * GEMM's scratch). */
+fq_status fq_linear(const uint16_t* X, int M, int K, const fq_qparams* act_qp,
+                    const fq_transform* t, const float* static_scale,
+                    const uint8_t* Wq, const void* s_w, int N, uint16_t* Y,
+                    void* workspace, size_t ws_bytes, void* stream);
+
+/* Scratch sizes in bytes (0 when none is needed).  gran as in the calls. */
+size_t fq_gemm_workspace_size(int M, int N, int K, fq_gran gran);
+size_t fq_linear_workspace_size(int M, int N, int K, fq_gran gran);
+
+/* Static text for a status. */
+const char* fq_status_string(fq_status s);
+
+/* Message describing the calling thread's last non-FQ_OK status ("" if none). */
+const char* fq_last_error(void);
+
+/* Synchronizes `stream`, then reads and clears the current device's timeout
+ * word: FQ_ERR_TIMEOUT if a kernel's bounded wait gave up since the last
+ * check, FQ_ERR_CUDA if the synchronization failed, FQ_OK otherwise. */
+fq_status fq_check_device_error(void* stream);
+
+/* Test hook for the timeout path: one CTA waits on a barrier that nothing
+ * arrives at, gives up after `limit_us` microseconds (1..100000) and records
+ * FQ_ERR_TIMEOUT as every kernel of the library does; the context stays usable. */
+fq_status fq_debug_wait_timeout(unsigned limit_us, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FQ_H_ */

@@ -1,0 +1,47 @@
+// Host-side helpers shared by the library's translation units: error
+// reporting, argument checks, the device error word and TMA tensor maps.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/fq.h"
+
+namespace fq {
+
+// Record a message for fq_last_error() and return `s`.
+fq_status fail(fq_status s, const char* fmt, ...);
+// Clear the calling thread's message.
+void clear_error();
+
+// Device address of the current device's timeout word (nullptr on failure).
+unsigned* device_error_word();
+
+// Number of SMs of the current device (cached).
+int sm_count();
+
+// cudaGetLastError() -> FQ_ERR_CUDA with the launch name, else FQ_OK.
+fq_status check_launch(const char* what);
+
+inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// 2-D row-major tensor map over uint8/fp16 data (no swizzle, zero fill for
+// out-of-range boxes).  inner = elements per row, rows = rows,
+// row_bytes = stride, box = {box_inner, box_rows}.
+fq_status make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, uint64_t inner,
+                       uint64_t rows, uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows);
+
+constexpr int kGroup = 128;
+constexpr int kMaxK = 65536;
+constexpr int kMaxQuantK = 32768;
+
+}  // namespace fq
+
+#define FQ_CHECK_ARG(cond, ...)                                   \
+  do {                                                            \
+    if (!(cond)) return ::fq::fail(FQ_ERR_INVALID, __VA_ARGS__); \
+  } while (0)

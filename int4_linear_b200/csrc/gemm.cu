@@ -1,0 +1,588 @@
+// INT4 x INT4 GEMM on the 5th-generation tensor cores (tcgen05, kind::i8).
+//
+// Blackwell has no 4-bit integer MMA, so each 128-deep K slice of both
+// operands is unpacked from nibbles to bytes in shared memory and multiplied
+// with s8 x s8 -> s32 MMAs accumulating in tensor memory (FlatQuant notes,
+// 核心思想: Y ~ Q(XP) Q(P^-1 W^T) with integer accumulation).
+//
+// Warp roles inside one CTA (one 128 x BN output tile, a K range):
+//   warp 0      TMA producer: packed A/B slices into a ring of SP stages
+//   warp 1      tensor-memory allocation and the single MMA-issuing thread
+//   warps 2-5   epilogue: tcgen05.ld of the accumulator, dequantization, stores
+//   warps 6-13  unpackers: packed stage -> int8 stage in the 128-byte
+//               swizzled K-major layout the MMA descriptors describe
+// Stages are handed over with mbarriers; every wait is bounded and a wait
+// that gives up records a timeout code in the device error word.
+//
+// The nibble is unpacked into the high half of its byte (16 q, see
+// unpack8_hi), so the tensor core accumulates 256 * sum(qx qw); the epilogue
+// removes the factor with an exact arithmetic shift.
+//
+// Epilogues: per-token x per-output-channel scales, static (migrated) scales,
+// per-group scales summed in float32 (FRM-PTQ group quantization, one group
+// per K slice, double-buffered accumulators), raw int32, or atomic int32
+// partial sums for split-K.  For few tokens (decode) the operands swap roles:
+// the weights fill the 128-row MMA side and the tokens the N side.
+#include <cuda_fp16.h>
+
+#include <algorithm>
+#include <cmath>
+
+#include "fq_device.cuh"
+#include "fq_host.h"
+
+namespace fq {
+
+namespace {
+
+enum Epi { kEpiRow = 0, kEpiStatic = 1, kEpiGroup = 2, kEpiS32 = 3, kEpiAtomic = 4 };
+
+constexpr int kBM = 128;        // rows of the A operand per tile (MMA M)
+constexpr int kBK = 128;        // int8 K per stage; equals the quantization group
+constexpr int kPK = kBK / 2;    // packed bytes per row per stage
+constexpr int kEpiWarps = 4;
+constexpr int kUnpackWarps = 8;
+constexpr int kThreads = 32 * (2 + kEpiWarps + kUnpackWarps);
+
+template <int BN, int EPI>
+struct Cfg {
+  static constexpr int SP = BN >= 128 ? 4 : (BN >= 64 ? 6 : 8);
+  static constexpr int SU = EPI == kEpiGroup ? 3 : 2;
+  static constexpr int A_PACK = kBM * kPK;
+  static constexpr int B_PACK = BN * kPK;
+  static constexpr int A_UNP = kBM * kBK;
+  static constexpr int B_UNP = BN * kBK;
+  static constexpr int TMEM_COLS = EPI == kEpiGroup ? 512 : (BN < 32 ? 32 : BN);
+  static constexpr int UNP_STAGE = A_UNP + B_UNP;
+  static constexpr int PACK_STAGE = A_PACK + B_PACK;
+  static constexpr int OFF_UNP = 0;
+  static constexpr int OFF_PACK = OFF_UNP + SU * UNP_STAGE;
+  static constexpr int OFF_SCALE = OFF_PACK + SP * PACK_STAGE;
+  static constexpr int SCALE_BYTES = EPI == kEpiGroup ? kEpiWarps * BN * 4 : 0;
+  static constexpr int OFF_BAR = OFF_SCALE + SCALE_BYTES;
+  static constexpr int NBAR = 2 * SP + 2 * SU + 5;
+  static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM = OFF_TMEM + 16 + 1024;  // + slack to align the base to 1024
+  static_assert(UNP_STAGE % 1024 == 0, "unpacked stages must keep 1024-byte alignment");
+  static_assert(PACK_STAGE % 128 == 0, "packed stages must keep 128-byte alignment");
+  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
+  static_assert(EPI != kEpiGroup || 3 * BN <= 512, "group epilogue needs 3 x BN tensor-memory columns");
+};
+
+struct GemmParams {
+  int M, N, K;        // Y is [M][N]
+  int rowsA, rowsB;   // rows of the A (128-row tiles) and B (BN-row tiles) operands
+  int num_kb;         // K / 128
+  int kb_per_split;   // K slices per CTA along gridDim.z
+  const float* sx;    // [M]           per-token scales
+  const float* sw;    // [N]           per-channel (or migrated static) scales
+  const __half* gsx;  // [K/128][M]    group scales of the activations
+  const __half* gsw;  // [K/128][N]    group scales of the weights
+  __half* Y;          // [M][N]
+  int32_t* acc;       // [M][N]        int32 output / split-K partial sums
+  unsigned* err;
+};
+
+__device__ __forceinline__ void store_half8(__half* dst, const float* v) {
+  uint4 o;
+  __half2* h = reinterpret_cast<__half2*>(&o);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) h[j] = __floats2half2_rn(v[2 * j], v[2 * j + 1]);
+  *reinterpret_cast<uint4*>(dst) = o;
+}
+
+template <int BN, int EPI, bool SWAP>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_w4a4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const GemmParams p) {
+  using C = Cfg<BN, EPI>;
+  constexpr int SP = C::SP, SU = C::SU;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* full_p = bars;
+  uint64_t* empty_p = full_p + SP;
+  uint64_t* full_u = empty_p + SP;
+  uint64_t* empty_u = full_u + SU;
+  uint64_t* acc_full = empty_u + SU;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* done_bar = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tileA = blockIdx.x, tileB = blockIdx.y;
+  const int kb0 = blockIdx.z * p.kb_per_split;
+  const int nkb = max(0, min(p.num_kb, kb0 + p.kb_per_split) - kb0);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < SP; ++s) {
+      mbar_init(&full_p[s], 1);
+      mbar_init(&empty_p[s], kUnpackWarps);
+    }
+    for (int s = 0; s < SU; ++s) {
+      mbar_init(&full_u[s], kUnpackWarps);
+      mbar_init(&empty_u[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], kEpiWarps);
+    }
+    mbar_init(done_bar, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int issued = 0;
+      for (int i = 0; i < nkb; ++i) {
+        const int s = i % SP;
+        if (!mbar_wait(&empty_p[s], ((i / SP) & 1) ^ 1)) {
+          record_error(p.err, kErrTimeoutProducer);
+          break;
+        }
+        uint8_t* pa = smem + C::OFF_PACK + s * C::PACK_STAGE;
+        mbar_arrive_expect_tx(&full_p[s], C::PACK_STAGE);
+        const int kx = (kb0 + i) * kPK;
+        tma_load_2d(pa, &tmA, &full_p[s], kx, tileA * kBM);
+        tma_load_2d(pa + C::A_PACK, &tmB, &full_p[s], kx, tileB * BN);
+        ++issued;
+      }
+      // Every load this thread issued has landed before the CTA can exit.
+      for (int i = max(0, issued - SP); i < issued; ++i)
+        if (!mbar_wait(&full_p[i % SP], (i / SP) & 1)) record_error(p.err, kErrTimeoutDrain);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_i8_m128(BN);
+      for (int i = 0; i < nkb; ++i) {
+        const int su = i % SU;
+        uint32_t d = tmem;
+        if (EPI == kEpiGroup) {
+          const int b = i & 1;
+          if (!mbar_wait(&acc_empty[b], ((i >> 1) & 1) ^ 1)) {
+            record_error(p.err, kErrTimeoutMma);
+            break;
+          }
+          tc_fence_after();
+          d = tmem + uint32_t(b * BN);
+        }
+        if (!mbar_wait(&full_u[su], (i / SU) & 1)) {
+          record_error(p.err, kErrTimeoutMma);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a0 = smem_u32(smem + C::OFF_UNP + su * C::UNP_STAGE);
+        const uint32_t b0 = a0 + C::A_UNP;
+#pragma unroll
+        for (int k = 0; k < kBK / 32; ++k) {
+          const uint32_t accum = EPI == kEpiGroup ? uint32_t(k > 0) : uint32_t(i > 0 || k > 0);
+          mma_i8(d, sdesc_k128_sw128(a0 + 32 * k), sdesc_k128_sw128(b0 + 32 * k), idesc, accum);
+        }
+        mma_commit(&empty_u[su]);
+        if (EPI == kEpiGroup) mma_commit(&acc_full[i & 1]);
+      }
+      if (EPI != kEpiGroup) mma_commit(&acc_full[0]);
+      mma_commit(done_bar);
+      if (!mbar_wait(done_bar, 0)) record_error(p.err, kErrTimeoutDrain);
+    }
+  } else if (warp < 2 + kEpiWarps) {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // tensor-memory lane quadrant this warp may access
+    const int rloc = q * 32 + lane;
+    const uint32_t tl = tmem + (uint32_t(q * 32) << 16);
+    const int arow = tileA * kBM + rloc;
+    const int bbase = tileB * BN;
+    if (EPI != kEpiGroup) {
+      if (!warp_wait(&acc_full[0], 0) && lane == 0) record_error(p.err, kErrTimeoutEpilogue);
+      tc_fence_after();
+      constexpr int CW = BN >= 32 ? 32 : 16;
+      for (int c0 = 0; c0 < BN; c0 += CW) {
+        uint32_t v[32];
+        if (CW == 32)
+          tmem_ld_32x32(tl + c0, v);
+        else
+          tmem_ld_32x16(tl + c0, v);
+        tmem_wait_ld();
+        if (!SWAP) {
+          // thread owns token row m = arow, columns n = bbase + c0 + j
+          const int m = arow;
+          if (m < p.M) {
+            const int n0 = bbase + c0;
+            float y[32];
+            if (EPI == kEpiRow || EPI == kEpiStatic) {
+              const float sxm = EPI == kEpiRow ? p.sx[m] : 1.0f;
+#pragma unroll
+              for (int j = 0; j < CW; ++j) {
+                const int n = min(n0 + j, p.N - 1);
+                const float a = float(int(v[j]) >> 8);
+                y[j] = EPI == kEpiRow ? __fmul_rn(__fmul_rn(a, sxm), __ldg(p.sw + n)) : __fmul_rn(a, __ldg(p.sw + n));
+              }
+              __half* dst = p.Y + size_t(m) * p.N + n0;
+              if (n0 + CW <= p.N) {
+#pragma unroll
+                for (int j = 0; j < CW; j += 8) store_half8(dst + j, y + j);
+              } else {
+                for (int j = 0; j < CW && n0 + j < p.N; ++j) dst[j] = __float2half_rn(y[j]);
+              }
+            } else {
+              int32_t* dst = p.acc + size_t(m) * p.N + n0;
+              for (int j = 0; j < CW; ++j) {
+                if (n0 + j >= p.N) break;
+                const int32_t a = int32_t(v[j]) >> 8;
+                if (EPI == kEpiS32)
+                  dst[j] = a;
+                else
+                  atomicAdd(dst + j, a);
+              }
+            }
+          }
+        } else {
+          // swapped: thread owns output channel n = arow, columns are tokens m
+          const int n = arow;
+          if (n < p.N) {
+            const float swn = (EPI == kEpiRow || EPI == kEpiStatic) ? __ldg(p.sw + n) : 0.f;
+            for (int j = 0; j < CW; ++j) {
+              const int m = bbase + c0 + j;
+              if (m >= p.M) break;
+              const int32_t ai = int32_t(v[j]) >> 8;
+              if (EPI == kEpiRow) {
+                p.Y[size_t(m) * p.N + n] = __float2half_rn(__fmul_rn(__fmul_rn(float(ai), __ldg(p.sx + m)), swn));
+              } else if (EPI == kEpiStatic) {
+                p.Y[size_t(m) * p.N + n] = __float2half_rn(__fmul_rn(float(ai), swn));
+              } else if (EPI == kEpiS32) {
+                p.acc[size_t(m) * p.N + n] = ai;
+              } else {
+                atomicAdd(p.acc + size_t(m) * p.N + n, ai);
+              }
+            }
+          }
+        }
+      }
+    } else {
+      // group-128: one accumulator per K slice, double-buffered in tensor
+      // memory; the running float32 sum lives in columns [2 BN, 3 BN).
+      float* sbuf = reinterpret_cast<float*>(smem + C::OFF_SCALE) + (warp - 2) * BN;
+      const uint32_t tsum = tl + uint32_t(2 * BN);
+      const int m = arow;
+      const bool mok = m < p.M;
+      for (int i = 0; i < nkb; ++i) {
+        const int g = kb0 + i, b = i & 1;
+        for (int c = lane; c < BN; c += 32) {
+          const int n = bbase + c;
+          sbuf[c] = n < p.N ? __half2float(p.gsw[size_t(g) * p.N + n]) : 0.f;
+        }
+        const float sxg = mok ? __half2float(p.gsx[size_t(g) * p.M + m]) : 0.f;
+        __syncwarp();
+        if (!warp_wait(&acc_full[b], (i >> 1) & 1)) {
+          if (lane == 0) record_error(p.err, kErrTimeoutEpilogue);
+          break;
+        }
+        tc_fence_after();
+        for (int c0 = 0; c0 < BN; c0 += 32) {
+          uint32_t v[32], s[32];
+          tmem_ld_32x32(tl + uint32_t(b * BN + c0), v);
+          if (i > 0) tmem_ld_32x32(tsum + c0, s);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float prev = i > 0 ? __uint_as_float(s[j]) : 0.f;
+            const float t = __fmul_rn(sxg, sbuf[c0 + j]);
+            s[j] = __float_as_uint(fmaf(float(int32_t(v[j]) >> 8), t, prev));
+          }
+          tmem_st_32x32(tsum + c0, s);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[b]);
+      }
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        uint32_t s[32];
+        tmem_ld_32x32(tsum + c0, s);
+        tmem_wait_ld();
+        if (mok) {
+          const int n0 = bbase + c0;
+          float y[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) y[j] = nkb > 0 ? __uint_as_float(s[j]) : 0.f;
+          __half* dst = p.Y + size_t(m) * p.N + n0;
+          if (n0 + 32 <= p.N) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 8) store_half8(dst + j, y + j);
+          } else {
+            for (int j = 0; j < 32 && n0 + j < p.N; ++j) dst[j] = __float2half_rn(y[j]);
+          }
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ unpackers
+    const int uw = warp - (2 + kEpiWarps);
+    constexpr int kJobs = (kBM + BN) * 4;  // 16-byte packed chunks per stage (A rows, then B rows)
+    for (int i = 0; i < nkb; ++i) {
+      const int sp = i % SP, su = i % SU;
+      if (!warp_wait(&full_p[sp], (i / SP) & 1) || !warp_wait(&empty_u[su], ((i / SU) & 1) ^ 1)) {
+        if (lane == 0) record_error(p.err, kErrTimeoutUnpack);
+        break;
+      }
+      const uint8_t* pk = smem + C::OFF_PACK + sp * C::PACK_STAGE;
+      uint8_t* uk = smem + C::OFF_UNP + su * C::UNP_STAGE;
+      for (int j = uw * 32 + lane; j < kJobs; j += kUnpackWarps * 32) {
+        const int row = j >> 2, c = j & 3;
+        const uint4 w = *reinterpret_cast<const uint4*>(pk + row * kPK + c * 16);
+        uint4 o0, o1;
+        unpack8_hi(w.x, o0.x, o0.y);
+        unpack8_hi(w.y, o0.z, o0.w);
+        unpack8_hi(w.z, o1.x, o1.y);
+        unpack8_hi(w.w, o1.z, o1.w);
+        uint8_t* rb = uk + (row >> 3) * 1024 + (row & 7) * 128;
+        const int r7 = row & 7;
+        *reinterpret_cast<uint4*>(rb + (((2 * c) ^ r7) << 4)) = o0;
+        *reinterpret_cast<uint4*>(rb + (((2 * c + 1) ^ r7) << 4)) = o1;
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&full_u[su]);
+        mbar_arrive(&empty_p[sp]);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// y = dequant(split-K int32 sums): per-token x per-channel or static scales.
+__global__ void splitk_finalize_kernel(const int32_t* __restrict__ acc, const float* __restrict__ sx,
+                                       const float* __restrict__ sw, __half* __restrict__ Y, int M, int N,
+                                       int row_mode) {
+  const size_t total = size_t(M) * N;
+  for (size_t e = blockIdx.x * size_t(blockDim.x) + threadIdx.x; e < total; e += size_t(gridDim.x) * blockDim.x) {
+    const int m = int(e / N), n = int(e % N);
+    const float a = float(acc[e]);
+    const float y = row_mode ? __fmul_rn(__fmul_rn(a, sx[m]), sw[n]) : __fmul_rn(a, sw[n]);
+    Y[e] = __float2half_rn(y);
+  }
+}
+
+struct Plan {
+  bool swap;
+  int bn;
+  int epi;
+  int splits;
+  int kb_per_split;
+};
+
+int pick_bn_swap(int M) { return M <= 16 ? 16 : (M <= 32 ? 32 : 64); }
+
+Plan make_plan(int M, int N, int K, int epi_final, int sms) {
+  Plan pl{};
+  const int nkb = K / kBK;
+  pl.splits = 1;
+  pl.kb_per_split = nkb;
+  if (epi_final == kEpiGroup) {
+    pl.swap = false;
+    pl.bn = 128;
+    pl.epi = kEpiGroup;
+    return pl;
+  }
+  if (epi_final == kEpiS32 || M > 64) {
+    pl.swap = false;
+    pl.bn = 256;
+    pl.epi = epi_final;
+    return pl;
+  }
+  // decode: weights on the 128-row side, tokens on the N side
+  pl.swap = true;
+  pl.bn = pick_bn_swap(M);
+  pl.epi = epi_final;
+  const int tiles = (N + kBM - 1) / kBM;
+  const int per_sm = pl.bn <= 16 ? 2 : 1;
+  const int slots = sms * per_sm;
+  double best = -1.0;
+  int best_s = 1;
+  for (int s = 1; s <= 16; ++s) {
+    if (nkb / s < 4) break;
+    const int ctas = tiles * s;
+    const int waves = (ctas + slots - 1) / slots;
+    const double eff = double(ctas) / double(waves * slots);
+    // extra traffic of split-K partial sums relative to the weight stream
+    const double extra = s > 1 ? double(M) * N * 4.0 * (s + 1) / (double(N) * K / 2.0) : 0.0;
+    const double score = eff / (1.0 + extra);
+    if (score > best + 1e-3) {
+      best = score;
+      best_s = s;
+    }
+  }
+  pl.splits = best_s;
+  pl.kb_per_split = (nkb + best_s - 1) / best_s;
+  pl.splits = (nkb + pl.kb_per_split - 1) / pl.kb_per_split;
+  if (pl.splits > 1) pl.epi = kEpiAtomic;
+  return pl;
+}
+
+template <int BN, int EPI, bool SWAP>
+fq_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& gp, dim3 grid,
+                      cudaStream_t stream) {
+  using C = Cfg<BN, EPI>;
+  auto kern = gemm_w4a4_kernel<BN, EPI, SWAP>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
+    return fail(FQ_ERR_CUDA, "cannot reserve %d bytes of shared memory for the GEMM", C::SMEM);
+  kern<<<grid, kThreads, C::SMEM, stream>>>(ta, tb, gp);
+  return check_launch("gemm_w4a4_kernel");
+}
+
+fq_status dispatch(const Plan& pl, const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& gp, dim3 grid,
+                   cudaStream_t s) {
+  if (!pl.swap) {
+    switch (pl.epi) {
+      case kEpiRow: return launch_gemm<256, kEpiRow, false>(ta, tb, gp, grid, s);
+      case kEpiStatic: return launch_gemm<256, kEpiStatic, false>(ta, tb, gp, grid, s);
+      case kEpiS32: return launch_gemm<256, kEpiS32, false>(ta, tb, gp, grid, s);
+      case kEpiGroup: return launch_gemm<128, kEpiGroup, false>(ta, tb, gp, grid, s);
+      default: break;
+    }
+  } else {
+#define FQ_SWAP_CASES(BNV)                                                           \
+  if (pl.bn == BNV) {                                                                \
+    switch (pl.epi) {                                                                \
+      case kEpiRow: return launch_gemm<BNV, kEpiRow, true>(ta, tb, gp, grid, s);       \
+      case kEpiStatic: return launch_gemm<BNV, kEpiStatic, true>(ta, tb, gp, grid, s); \
+      case kEpiAtomic: return launch_gemm<BNV, kEpiAtomic, true>(ta, tb, gp, grid, s); \
+      default: break;                                                                \
+    }                                                                                \
+  }
+    FQ_SWAP_CASES(16)
+    FQ_SWAP_CASES(32)
+    FQ_SWAP_CASES(64)
+#undef FQ_SWAP_CASES
+  }
+  return fail(FQ_ERR_UNSUPPORTED, "no GEMM variant for this plan");
+}
+
+fq_status check_sizes(int M, int N, int K) {
+  FQ_CHECK_ARG(M >= 1, "M = %d must be >= 1", M);
+  FQ_CHECK_ARG(N >= 8 && N % 8 == 0, "N = %d must be a positive multiple of 8", N);
+  FQ_CHECK_ARG(K >= kBK && K <= kMaxK && K % kBK == 0, "K = %d must be a multiple of 128 in [128, %d]", K, kMaxK);
+  return FQ_OK;
+}
+
+fq_status gemm_impl(const uint8_t* Xq, const void* s_x, const uint8_t* Wq, const void* s_w, int M, int N, int K,
+                    int epi_final, uint16_t* Y, int32_t* acc_out, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  fq_status st = check_sizes(M, N, K);
+  if (st != FQ_OK) return st;
+  FQ_CHECK_ARG(Xq && Wq, "Xq and Wq must be non-NULL");
+  FQ_CHECK_ARG(aligned(Xq, 16) && aligned(Wq, 16), "Xq and Wq must be 16-byte aligned");
+  if (epi_final == kEpiS32) {
+    FQ_CHECK_ARG(acc_out && aligned(acc_out, 4), "the int32 output must be non-NULL and aligned");
+  } else {
+    FQ_CHECK_ARG(Y && aligned(Y, 16), "Y must be non-NULL and 16-byte aligned");
+    FQ_CHECK_ARG(s_w && aligned(s_w, 4), "s_w must be non-NULL and aligned");
+    if (epi_final != kEpiStatic) FQ_CHECK_ARG(s_x && aligned(s_x, 2), "s_x must be non-NULL and aligned");
+  }
+  unsigned* err = device_error_word();
+  if (!err) return fail(FQ_ERR_CUDA, "device error word unavailable");
+  const int sms = sm_count();
+  Plan pl = make_plan(M, N, K, epi_final, sms);
+  const size_t need = pl.splits > 1 ? size_t(M) * N * sizeof(int32_t) : 0;
+  if (need > 0) FQ_CHECK_ARG(ws && ws_bytes >= need && aligned(ws, 16), "workspace of %zu bytes required", need);
+
+  GemmParams gp{};
+  gp.M = M;
+  gp.N = N;
+  gp.K = K;
+  gp.num_kb = K / kBK;
+  gp.kb_per_split = pl.kb_per_split;
+  gp.err = err;
+  gp.Y = reinterpret_cast<__half*>(Y);
+  if (epi_final == kEpiRow) gp.sx = static_cast<const float*>(s_x);
+  if (epi_final == kEpiRow || epi_final == kEpiStatic) gp.sw = static_cast<const float*>(s_w);
+  if (epi_final == kEpiGroup) {
+    gp.gsx = static_cast<const __half*>(s_x);
+    gp.gsw = static_cast<const __half*>(s_w);
+  }
+  gp.acc = epi_final == kEpiS32 ? acc_out : (pl.splits > 1 ? static_cast<int32_t*>(ws) : nullptr);
+
+  const uint8_t* A = pl.swap ? Wq : Xq;
+  const uint8_t* B = pl.swap ? Xq : Wq;
+  gp.rowsA = pl.swap ? N : M;
+  gp.rowsB = pl.swap ? M : N;
+  CUtensorMap ta, tb;
+  st = make_tmap_2d(&ta, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, uint64_t(K / 2), uint64_t(gp.rowsA), uint64_t(K / 2),
+                    kPK, kBM);
+  if (st != FQ_OK) return st;
+  st = make_tmap_2d(&tb, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, uint64_t(K / 2), uint64_t(gp.rowsB), uint64_t(K / 2),
+                    kPK, uint32_t(pl.bn));
+  if (st != FQ_OK) return st;
+
+  const dim3 grid((gp.rowsA + kBM - 1) / kBM, (gp.rowsB + pl.bn - 1) / pl.bn, pl.splits);
+  if (pl.splits > 1) {
+    if (cudaMemsetAsync(ws, 0, need, stream) != cudaSuccess) return fail(FQ_ERR_CUDA, "workspace clear failed");
+  }
+  st = dispatch(pl, ta, tb, gp, grid, stream);
+  if (st != FQ_OK) return st;
+  if (pl.splits > 1) {
+    const int threads = 256;
+    const int blocks = int(std::min<size_t>((size_t(M) * N + threads - 1) / threads, size_t(sms) * 8));
+    splitk_finalize_kernel<<<blocks, threads, 0, stream>>>(gp.acc, gp.sx, gp.sw, gp.Y, M, N,
+                                                           epi_final == kEpiRow ? 1 : 0);
+    st = check_launch("splitk_finalize_kernel");
+  }
+  return st;
+}
+
+}  // namespace
+
+size_t gemm_workspace_bytes(int M, int N, int K, fq_gran gran) {
+  if (M < 1 || N < 8 || K < kBK || K % kBK) return 0;
+  const int epi = gran == FQ_DYNAMIC_GROUP ? kEpiGroup : (gran == FQ_STATIC_CHANNEL ? kEpiStatic : kEpiRow);
+  const Plan pl = make_plan(M, N, K, epi, sm_count());
+  return pl.splits > 1 ? size_t(M) * N * sizeof(int32_t) : 0;
+}
+
+}  // namespace fq
+
+extern "C" {
+
+fq_status fq_w4a4_gemm(const uint8_t* Xq, const void* s_x, const uint8_t* Wq, const void* s_w, int M, int N, int K,
+                       fq_gran gran, uint16_t* Y, void* workspace, size_t ws_bytes, void* stream) {
+  fq::clear_error();
+  int epi;
+  switch (gran) {
+    case FQ_DYNAMIC_ROW: epi = fq::kEpiRow; break;
+    case FQ_STATIC_CHANNEL: epi = fq::kEpiStatic; break;
+    case FQ_DYNAMIC_GROUP: epi = fq::kEpiGroup; break;
+    default: return fq::fail(FQ_ERR_UNSUPPORTED, "granularity %d is not provided", int(gran));
+  }
+  return fq::gemm_impl(Xq, s_x, Wq, s_w, M, N, K, epi, Y, nullptr, workspace, ws_bytes,
+                       static_cast<cudaStream_t>(stream));
+}
+
+fq_status fq_w4a4_gemm_s32(const uint8_t* Xq, const uint8_t* Wq, int M, int N, int K, int32_t* acc, void* stream) {
+  fq::clear_error();
+  return fq::gemm_impl(Xq, nullptr, Wq, nullptr, M, N, K, fq::kEpiS32, nullptr, acc, nullptr, 0,
+                       static_cast<cudaStream_t>(stream));
+}
+
+size_t fq_gemm_workspace_size(int M, int N, int K, fq_gran gran) { return fq::gemm_workspace_bytes(M, N, K, gran); }
+
+}  // extern "C"

@@ -1,0 +1,55 @@
+// The W4A4 linear layer: online activation quantization into the caller's
+// workspace, then the INT4 x INT4 GEMM, on one stream (FlatQuant notes,
+// 核心思想: Y ~ Q(XP) Q(P^-1 W^T)).
+#include "fq_host.h"
+
+namespace fq {
+size_t gemm_workspace_bytes(int M, int N, int K, fq_gran gran);
+
+namespace {
+constexpr size_t kAlign = 256;
+size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+size_t act_scale_bytes(int M, int K, fq_gran gran) {
+  if (gran == FQ_DYNAMIC_ROW) return size_t(M) * sizeof(float);
+  if (gran == FQ_DYNAMIC_GROUP) return size_t(K / kGroup) * M * 2;
+  return 0;
+}
+}  // namespace
+
+size_t linear_workspace_bytes(int M, int N, int K, fq_gran gran) {
+  if (M < 1 || K < kGroup || K % kGroup) return 0;
+  return up(size_t(M) * (K / 2)) + up(act_scale_bytes(M, K, gran)) + up(gemm_workspace_bytes(M, N, K, gran));
+}
+
+}  // namespace fq
+
+extern "C" {
+
+size_t fq_linear_workspace_size(int M, int N, int K, fq_gran gran) {
+  return fq::linear_workspace_bytes(M, N, K, gran);
+}
+
+fq_status fq_linear(const uint16_t* X, int M, int K, const fq_qparams* act_qp, const fq_transform* t,
+                    const float* static_scale, const uint8_t* Wq, const void* s_w, int N, uint16_t* Y,
+                    void* workspace, size_t ws_bytes, void* stream) {
+  fq::clear_error();
+  if (!act_qp) return fq::fail(FQ_ERR_INVALID, "act_qp is NULL");
+  if (M < 1 || K < fq::kGroup || K % fq::kGroup || N < 8 || N % 8)
+    return fq::fail(FQ_ERR_INVALID, "sizes M = %d, N = %d, K = %d out of range", M, N, K);
+  const size_t need = fq::linear_workspace_bytes(M, N, K, act_qp->gran);
+  if (!workspace || ws_bytes < need || !fq::aligned(workspace, 256))
+    return fq::fail(FQ_ERR_INVALID, "workspace of %zu bytes (256-byte aligned) required, got %zu", need, ws_bytes);
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  uint8_t* xq = base;
+  size_t off = fq::up(size_t(M) * (K / 2));
+  void* sx = act_qp->gran == FQ_STATIC_CHANNEL ? nullptr : static_cast<void*>(base + off);
+  off += fq::up(fq::act_scale_bytes(M, K, act_qp->gran));
+  void* gws = base + off;
+  const size_t gws_bytes = ws_bytes - off;
+  fq_status st = fq_quant_act(X, M, K, act_qp, t, static_scale, xq, sx, stream);
+  if (st != FQ_OK) return st;
+  return fq_w4a4_gemm(xq, sx, Wq, s_w, M, N, K, act_qp->gran, Y, gws, gws_bytes, stream);
+}
+
+}  // extern "C"

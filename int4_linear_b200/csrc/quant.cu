@@ -1,0 +1,357 @@
+// Row quantization kernels: online activation quantization (fq_quant_act)
+// and offline weight quantization (fq_quant_weight).
+//
+// One CTA owns one row at a time (grid-stride over rows), keeps the whole
+// row in shared memory as float32, and in order:
+//   1. loads the fp16 row with 128-bit loads and applies the channel scale
+//      (activations: x * c; weights: w / c)  (FlatQuant notes, 逐通道缩放);
+//   2. applies the Kronecker-factored transform on the n1 x n2 reshape,
+//      activations P1^T Xbar P2, weights P1^-1 Wbar P2^-T (FlatQuant notes,
+//      Kronecker 分解), as two in-place passes: first every tile row times the
+//      right factor, then every tile column times the left factor;
+//   3. weights only: folds the static activation scales s_k into the columns
+//      (MergeQuant, quantization step migration);
+//   4. reduces the absmax per row or per 128-group with warp shuffles, forms
+//      s = (amax * alpha) / 7 (group scales rounded to fp16), or reads the
+//      static scales (FRM-PTQ page, 初步介绍; FlatQuant notes, 可学习裁剪阈值);
+//   5. rounds half-to-even after an IEEE division, clamps to [-8, 7], packs
+//      two codes per byte and stores 32 bits per thread, coalesced.
+// The transform factors live in shared memory (read once per CTA) when they
+// fit, otherwise they are read through L1.
+#include <cuda_fp16.h>
+
+#include <algorithm>
+
+#include "fq_device.cuh"
+#include "fq_host.h"
+
+namespace fq {
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kSmemBudget = 220 * 1024;
+
+enum Side { kAct = 0, kWeight = 1 };
+
+struct QuantParams {
+  const __half* X;
+  int R, K;
+  int gran;
+  float alpha;
+  int n1, n2;            // transform tile (0 = none)
+  const float* L;        // P1 (act) or P1^-1 (weight), [n1][n1]
+  const float* Rt;       // P2 (act) or P2^-1 (weight), [n2][n2]
+  const float* c;        // [K] or null
+  const float* qsm;      // weights: [K] or null
+  const float* sstatic;  // act static: [K]
+  uint8_t* Q;            // [R][K/2]
+  float* s_row;          // [R]
+  __half* s_grp;         // [K/128][R]
+  float* xhat;           // [R][K] or null
+};
+
+// Left factor as used by the column pass: Lc(k, i) multiplies U[i][l] into
+// Xhat[k][l].  Activations: P1^T, so Lc(k, i) = P1[i][k]; weights: P1^-1.
+template <int SIDE>
+__device__ __forceinline__ float left_at(const float* L, int n1, int k, int i) {
+  return SIDE == kAct ? L[i * n1 + k] : L[k * n1 + i];
+}
+// Right factor as used by the row pass: Rr(j, l) multiplies Xbar[i][j] into
+// U[i][l].  Activations: P2, so Rr(j, l) = P2[j][l]; weights: P2^-T.
+template <int SIDE>
+__device__ __forceinline__ float right_at(const float* Rt, int n2, int j, int l) {
+  return SIDE == kAct ? Rt[j * n2 + l] : Rt[l * n2 + j];
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+__device__ __forceinline__ int rtn_code(float v, float s) {
+  if (s == 0.0f) return 0;
+  const float r = rintf(__fdiv_rn(v, s));
+  return static_cast<int>(fminf(fmaxf(r, -8.0f), 7.0f));
+}
+
+// Index of flat element e in the row buffer: padded by one float per tile row
+// when a transform is applied, so that the column pass is free of bank conflicts.
+__device__ __forceinline__ int slot(int e, int n2, int pad) { return pad ? (e / n2) * (n2 + 1) + (e % n2) : e; }
+
+template <int SIDE, bool PSMEM>
+__global__ void __launch_bounds__(kThreads) quant_rows_kernel(QuantParams p) {
+  extern __shared__ __align__(16) float smem[];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int K = p.K, n1 = p.n1, n2 = p.n2;
+  const bool xf = n1 > 0;
+  const int pad = xf ? 1 : 0;
+  const int row_floats = xf ? n1 * (n2 + 1) : K;
+  float* xs = smem;                       // row buffer
+  float* sL = xs + row_floats;            // [i][k] = Lc(k, i)   (PSMEM)
+  float* sR = sL + (PSMEM ? n1 * n1 : 0); // [j][l] = Rr(j, l)   (PSMEM)
+  float* red = sR + (PSMEM ? n2 * n2 : 0);  // [kWarps]
+  float* gsc = red + kWarps;                // [K/128] group scales
+
+  if (PSMEM && xf) {
+    for (int e = tid; e < n1 * n1; e += kThreads) {
+      const int i = e / n1, k = e % n1;
+      sL[e] = left_at<SIDE>(p.L, n1, k, i);
+    }
+    for (int e = tid; e < n2 * n2; e += kThreads) {
+      const int j = e / n2, l = e % n2;
+      sR[e] = right_at<SIDE>(p.Rt, n2, j, l);
+    }
+  }
+  __syncthreads();
+
+  const int ngroups = K / kGroup;
+  for (int r = blockIdx.x; r < p.R; r += gridDim.x) {
+    // 1. load + channel scale
+    const __half* xrow = p.X + size_t(r) * K;
+    for (int e0 = tid * 8; e0 < K; e0 += kThreads * 8) {
+      const uint4 raw = *reinterpret_cast<const uint4*>(xrow + e0);
+      const __half2* h2 = reinterpret_cast<const __half2*>(&raw);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = __half22float2(h2[j]);
+        float v0 = f.x, v1 = f.y;
+        if (p.c) {
+          if (SIDE == kAct) {
+            v0 = __fmul_rn(v0, p.c[e0 + 2 * j]);
+            v1 = __fmul_rn(v1, p.c[e0 + 2 * j + 1]);
+          } else {
+            v0 = __fdiv_rn(v0, p.c[e0 + 2 * j]);
+            v1 = __fdiv_rn(v1, p.c[e0 + 2 * j + 1]);
+          }
+        }
+        xs[slot(e0 + 2 * j, n2, pad)] = v0;
+        xs[slot(e0 + 2 * j + 1, n2, pad)] = v1;
+      }
+    }
+    __syncthreads();
+
+    // 2. transform
+    if (xf) {
+      // row pass: U[i][l] = sum_j Xbar[i][j] Rr(j, l), rows split over warps
+      for (int i = warp; i < n1; i += kWarps) {
+        float acc[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) acc[t] = 0.f;
+        const float* xr = xs + i * (n2 + 1);
+        for (int j = 0; j < n2; ++j) {
+          const float x = xr[j];
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            const int l = lane + 32 * t;
+            if (l < n2) {
+              const float rv = PSMEM ? sR[j * n2 + l] : right_at<SIDE>(p.Rt, n2, j, l);
+              acc[t] = fmaf(x, rv, acc[t]);
+            }
+          }
+        }
+        __syncwarp();
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          const int l = lane + 32 * t;
+          if (l < n2) xs[i * (n2 + 1) + l] = acc[t];
+        }
+      }
+      __syncthreads();
+      // column pass: Xhat[k][l] = sum_i Lc(k, i) U[i][l], columns split over warps
+      for (int l = warp; l < n2; l += kWarps) {
+        float acc[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) acc[t] = 0.f;
+        for (int i = 0; i < n1; ++i) {
+          const float u = xs[i * (n2 + 1) + l];
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            const int k = lane + 32 * t;
+            if (k < n1) {
+              const float lv = PSMEM ? sL[i * n1 + k] : left_at<SIDE>(p.L, n1, k, i);
+              acc[t] = fmaf(lv, u, acc[t]);
+            }
+          }
+        }
+        __syncwarp();
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          const int k = lane + 32 * t;
+          if (k < n1) xs[k * (n2 + 1) + l] = acc[t];
+        }
+      }
+      __syncthreads();
+    }
+
+    // 3. weights: quantization step migration
+    if (SIDE == kWeight && p.qsm) {
+      for (int e = tid; e < K; e += kThreads) xs[slot(e, n2, pad)] = __fmul_rn(xs[slot(e, n2, pad)], p.qsm[e]);
+      __syncthreads();
+    }
+
+    if (p.xhat) {
+      float* xo = p.xhat + size_t(r) * K;
+      for (int e = tid; e < K; e += kThreads) xo[e] = xs[slot(e, n2, pad)];
+    }
+
+    // 4. scales
+    float s_row = 0.f;
+    if (p.gran == FQ_DYNAMIC_ROW) {
+      float m = 0.f;
+      for (int e = tid; e < K; e += kThreads) m = fmaxf(m, fabsf(xs[slot(e, n2, pad)]));
+      m = warp_max(m);
+      if (lane == 0) red[warp] = m;
+      __syncthreads();
+      float amax = red[0];
+#pragma unroll
+      for (int w = 1; w < kWarps; ++w) amax = fmaxf(amax, red[w]);
+      s_row = __fdiv_rn(__fmul_rn(amax, p.alpha), 7.0f);
+      if (tid == 0) p.s_row[r] = s_row;
+    } else if (p.gran == FQ_DYNAMIC_GROUP) {
+      for (int g = warp; g < ngroups; g += kWarps) {
+        float m = 0.f;
+#pragma unroll
+        for (int t = 0; t < 4; ++t) m = fmaxf(m, fabsf(xs[slot(g * kGroup + lane + 32 * t, n2, pad)]));
+        m = warp_max(m);
+        const __half sh = __float2half_rn(__fdiv_rn(__fmul_rn(m, p.alpha), 7.0f));
+        if (lane == 0) {
+          gsc[g] = __half2float(sh);
+          p.s_grp[size_t(g) * p.R + r] = sh;
+        }
+      }
+      __syncthreads();
+    }
+
+    // 5. codes, packed 8 per thread-iteration (one 32-bit store)
+    uint32_t* qrow = reinterpret_cast<uint32_t*>(p.Q + size_t(r) * (K / 2));
+    for (int e0 = tid * 8; e0 < K; e0 += kThreads * 8) {
+      uint32_t word = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int e = e0 + j;
+        const float v = xs[slot(e, n2, pad)];
+        float s;
+        if (p.gran == FQ_DYNAMIC_ROW)
+          s = s_row;
+        else if (p.gran == FQ_DYNAMIC_GROUP)
+          s = gsc[e / kGroup];
+        else
+          s = p.sstatic[e];
+        word |= (uint32_t(rtn_code(v, s)) & 0xFu) << (4 * j);
+      }
+      qrow[e0 / 8] = word;
+    }
+    __syncthreads();
+  }
+}
+
+size_t smem_bytes(int K, int n1, int n2, bool psmem) {
+  const size_t row = n1 > 0 ? size_t(n1) * (n2 + 1) : size_t(K);
+  const size_t pm = (psmem && n1 > 0) ? size_t(n1) * n1 + size_t(n2) * n2 : 0;
+  return (row + pm + kWarps + K / kGroup) * sizeof(float);
+}
+
+template <int SIDE, bool PSMEM>
+fq_status launch_quant(const QuantParams& qp, cudaStream_t stream) {
+  const size_t smem = smem_bytes(qp.K, qp.n1, qp.n2, PSMEM);
+  auto kern = quant_rows_kernel<SIDE, PSMEM>;
+  if (smem > 48 * 1024) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
+      return fail(FQ_ERR_CUDA, "cannot reserve %zu bytes of shared memory", smem);
+  }
+  int per_sm = 1;
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem);
+  per_sm = std::max(per_sm, 1);
+  const int grid = std::max(1, std::min(qp.R, sm_count() * per_sm));
+  kern<<<grid, kThreads, smem, stream>>>(qp);
+  return check_launch("quant_rows_kernel");
+}
+
+fq_status check_qparams(const fq_qparams* qp, bool act) {
+  FQ_CHECK_ARG(qp != nullptr, "qparams is NULL");
+  if (qp->bits != 4) return fail(FQ_ERR_UNSUPPORTED, "bits = %d: only b = 4 is provided", qp->bits);
+  if (qp->zero_point != 8)
+    return fail(FQ_ERR_UNSUPPORTED, "zero_point = %d: only the symmetric z = 2^(b-1) = 8 is provided",
+                qp->zero_point);
+  if (qp->gran == FQ_DYNAMIC_GROUP && qp->group_size != kGroup)
+    return fail(FQ_ERR_UNSUPPORTED, "group_size = %d: only 128 is provided", qp->group_size);
+  if (qp->gran != FQ_DYNAMIC_ROW && qp->gran != FQ_DYNAMIC_GROUP && !(act && qp->gran == FQ_STATIC_CHANNEL))
+    return fail(FQ_ERR_UNSUPPORTED, "granularity %d is not provided here", int(qp->gran));
+  if (qp->gran != FQ_STATIC_CHANNEL)
+    FQ_CHECK_ARG(qp->alpha > 0.f && qp->alpha <= 1.f, "alpha = %g must lie in (0, 1]", double(qp->alpha));
+  return FQ_OK;
+}
+
+fq_status quant_common(int side, const uint16_t* X, int R, int K, const fq_qparams* qp, const fq_transform* t,
+                       const float* extra, uint8_t* Q, void* s_out, float* xhat, void* stream) {
+  clear_error();
+  fq_status st = check_qparams(qp, side == kAct);
+  if (st != FQ_OK) return st;
+  FQ_CHECK_ARG(X && Q, "X and the packed output must be non-NULL");
+  FQ_CHECK_ARG(R >= 1, "rows = %d must be >= 1", R);
+  FQ_CHECK_ARG(K >= kGroup && K <= kMaxQuantK && K % kGroup == 0, "K = %d must be a multiple of 128 in [128, %d]",
+               K, kMaxQuantK);
+  FQ_CHECK_ARG(aligned(X, 16) && aligned(Q, 16), "X and the packed output must be 16-byte aligned");
+  if (qp->gran == FQ_STATIC_CHANNEL)
+    FQ_CHECK_ARG(extra && aligned(extra, 4), "static scales [K] are required for FQ_STATIC_CHANNEL");
+  else
+    FQ_CHECK_ARG(s_out && aligned(s_out, 4), "the scale output must be non-NULL and aligned");
+  QuantParams p{};
+  p.X = reinterpret_cast<const __half*>(X);
+  p.R = R;
+  p.K = K;
+  p.gran = int(qp->gran);
+  p.alpha = qp->alpha;
+  p.Q = Q;
+  p.xhat = xhat;
+  if (qp->gran == FQ_DYNAMIC_ROW) p.s_row = static_cast<float*>(s_out);
+  if (qp->gran == FQ_DYNAMIC_GROUP) p.s_grp = static_cast<__half*>(s_out);
+  if (side == kAct && qp->gran == FQ_STATIC_CHANNEL) p.sstatic = extra;
+  if (side == kWeight) p.qsm = extra;
+  if (t) {
+    p.c = t->c;
+    if (t->c) FQ_CHECK_ARG(aligned(t->c, 4), "c must be 4-byte aligned");
+    if (t->P1) {
+      FQ_CHECK_ARG(t->P2 != nullptr, "P2 is NULL while P1 is given");
+      FQ_CHECK_ARG(t->n1 >= 1 && t->n2 >= 1 && t->n1 <= 256 && t->n2 <= 256 && t->n1 * t->n2 == K,
+                   "transform tile %d x %d must satisfy n1 * n2 = K = %d with 1 <= n1, n2 <= 256", t->n1, t->n2,
+                   K);
+      p.n1 = t->n1;
+      p.n2 = t->n2;
+      p.L = t->P1;
+      p.Rt = t->P2;
+    }
+  }
+  const bool psmem = smem_bytes(K, p.n1, p.n2, true) <= size_t(kSmemBudget);
+  if (smem_bytes(K, p.n1, p.n2, false) > size_t(kSmemBudget))
+    return fail(FQ_ERR_UNSUPPORTED, "row of K = %d does not fit in shared memory", K);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (side == kAct) return psmem ? launch_quant<kAct, true>(p, s) : launch_quant<kAct, false>(p, s);
+  return psmem ? launch_quant<kWeight, true>(p, s) : launch_quant<kWeight, false>(p, s);
+}
+
+}  // namespace
+}  // namespace fq
+
+extern "C" {
+
+fq_status fq_quant_weight(const uint16_t* W, int N, int K, const fq_qparams* qp, const fq_transform* inv,
+                          const float* qsm_scale, uint8_t* Wq, void* s_w, void* stream) {
+  return fq::quant_common(fq::kWeight, W, N, K, qp, inv, qsm_scale, Wq, s_w, nullptr, stream);
+}
+
+fq_status fq_quant_act(const uint16_t* X, int M, int K, const fq_qparams* qp, const fq_transform* t,
+                       const float* static_scale, uint8_t* Xq, void* s_x, void* stream) {
+  return fq::quant_common(fq::kAct, X, M, K, qp, t, static_scale, Xq, s_x, nullptr, stream);
+}
+
+fq_status fq_quant_act_debug(const uint16_t* X, int M, int K, const fq_qparams* qp, const fq_transform* t,
+                             const float* static_scale, uint8_t* Xq, void* s_x, float* xhat, void* stream) {
+  if (!xhat || !fq::aligned(xhat, 4)) return fq::fail(FQ_ERR_INVALID, "xhat must be non-NULL and aligned");
+  return fq::quant_common(fq::kAct, X, M, K, qp, t, static_scale, Xq, s_x, xhat, stream);
+}
+
+}  // extern "C"

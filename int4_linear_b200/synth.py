@@ -196,3 +196,28 @@ GROUP_70B_SHAPES = [(8192, 10240), (8192, 57344), (28672, 8192)]
 # Decode shapes.
 DECODE_70B_SHAPES = [(8192, 57344), (28672, 8192)]
 DECODE_TOKENS = [1, 8, 32, 64]
+
+
+# ---------------------------------------------------------------- GEMM operands
+# Packed INT4 operands for testing the GEMM on its own: every byte is a valid
+# pair of nibbles, so uniform random bytes give uniform random codes in [-8, 7].
+
+
+def random_packed(g: np.random.Generator, rows: int, k: int) -> np.ndarray:
+    """uint8 [rows, k/2], uniform random bytes (two uniform INT4 codes each)."""
+    return g.integers(0, 256, (rows, k // 2), dtype=np.uint8)
+
+
+def constant_packed(rows: int, k: int, byte: int) -> np.ndarray:
+    return np.full((rows, k // 2), byte, dtype=np.uint8)
+
+
+def random_scales(g: np.random.Generator, n: int, lo: float = 1e-3, hi: float = 1e-1) -> np.ndarray:
+    """float32 [n], log-uniform in [lo, hi]."""
+    return np.exp(g.uniform(np.log(lo), np.log(hi), n)).astype(np.float32)
+
+
+def random_group_scales(g: np.random.Generator, groups: int, rows: int, lo: float = 1e-3,
+                        hi: float = 1e-1) -> np.ndarray:
+    """float16 [groups, rows] (group-major), log-uniform in [lo, hi]."""
+    return np.exp(g.uniform(np.log(lo), np.log(hi), (groups, rows))).astype(np.float16)

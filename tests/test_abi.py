@@ -1,0 +1,131 @@
+"""The C ABI on the host: libfq.so loads, exports every entry point that
+include/fq.h declares, and rejects bad arguments before launching anything
+(these calls never reach the GPU, so they run without one)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from int4_linear_b200 import fq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fq.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(fq_[a-z0-9_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    if not os.path.exists(fq.LIB_PATH):
+        from int4_linear_b200 import build
+        build.build()
+    return fq.lib()
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for n in ["fq_quant_weight", "fq_quant_act", "fq_w4a4_gemm", "fq_linear"]:
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    for name in _declared():
+        assert hasattr(L, name), name
+
+
+def test_status_strings(L):
+    for s in range(5):
+        assert L.fq_status_string(s)
+    assert L.fq_status_string(99) == b"unknown status"
+
+
+def _qp(**kw):
+    return fq.qparams(**kw)
+
+
+# Fake, 256-byte-aligned device addresses: every case below fails validation
+# before any CUDA call, so nothing is dereferenced.
+A = 1 << 20
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(bits=3), fq.FQ_ERR_UNSUPPORTED),
+    (dict(zero_point=0), fq.FQ_ERR_UNSUPPORTED),
+    (dict(gran=fq.GROUP, group_size=64), fq.FQ_ERR_UNSUPPORTED),
+    (dict(alpha=0.0), fq.FQ_ERR_INVALID),
+    (dict(alpha=1.5), fq.FQ_ERR_INVALID),
+])
+def test_quant_act_rejects_qparams(L, kw, status):
+    qp = _qp(**kw)
+    st = L.fq_quant_act(A, 4, 256, ctypes.byref(qp), None, None, A, A, None)
+    assert st == status
+    assert L.fq_last_error()
+
+
+@pytest.mark.parametrize("m,k,x,xq,msg", [
+    (4, 100, A, A, b"K"),
+    (4, 128 * 300, A, A, b"K"),
+    (0, 256, A, A, b"rows"),
+    (4, 256, None, A, b"NULL"),
+    (4, 256, A + 8, A, b"aligned"),
+])
+def test_quant_act_rejects_sizes(L, m, k, x, xq, msg):
+    qp = _qp()
+    st = L.fq_quant_act(x, m, k, ctypes.byref(qp), None, None, xq, A, None)
+    assert st == fq.FQ_ERR_INVALID
+    assert msg in L.fq_last_error()
+
+
+def test_transform_shape_must_match_k(L):
+    qp = _qp()
+    t = fq._Transform(8, 16, A, A, None)  # 8 * 16 != 256
+    st = L.fq_quant_act(A, 4, 256, ctypes.byref(qp), ctypes.byref(t), None, A, A, None)
+    assert st == fq.FQ_ERR_INVALID and b"n1 * n2" in L.fq_last_error()
+
+
+def test_static_needs_scales(L):
+    qp = _qp(gran=fq.STATIC)
+    st = L.fq_quant_act(A, 4, 256, ctypes.byref(qp), None, None, A, None, None)
+    assert st == fq.FQ_ERR_INVALID
+    st = L.fq_quant_weight(A, 4, 256, ctypes.byref(qp), None, None, A, A, None)
+    assert st == fq.FQ_ERR_UNSUPPORTED  # weights have no static granularity
+
+
+@pytest.mark.parametrize("m,n,k", [(0, 256, 256), (4, 12, 256), (4, 256, 200), (4, 256, 131072)])
+def test_gemm_rejects_sizes(L, m, n, k):
+    st = L.fq_w4a4_gemm(A, A, A, A, m, n, k, fq.ROW, A, None, 0, None)
+    assert st == fq.FQ_ERR_INVALID
+
+
+def test_gemm_rejects_misaligned(L):
+    st = L.fq_w4a4_gemm(A + 4, A, A, A, 4, 256, 256, fq.ROW, A, None, 0, None)
+    assert st == fq.FQ_ERR_INVALID and b"aligned" in L.fq_last_error()
+    st = L.fq_w4a4_gemm(A, A, A, A, 4, 256, 256, 7, A, None, 0, None)
+    assert st == fq.FQ_ERR_UNSUPPORTED
+
+
+def test_linear_needs_workspace(L):
+    qp = _qp()
+    need = L.fq_linear_workspace_size(16, 256, 256, fq.ROW)
+    assert need >= 16 * 128 + 16 * 4
+    st = L.fq_linear(A, 16, 256, ctypes.byref(qp), None, None, A, A, 256, A, A, need - 1, None)
+    assert st == fq.FQ_ERR_INVALID and b"workspace" in L.fq_last_error()
+
+
+def test_workspace_sizes(L):
+    # prefill needs no GEMM scratch; decode with few output tiles splits K
+    assert L.fq_gemm_workspace_size(2048, 4096, 4096, fq.ROW) == 0
+    assert L.fq_gemm_workspace_size(4096, 8192, 8192, fq.GROUP) == 0
+    assert L.fq_gemm_workspace_size(8, 8192, 28672, fq.ROW) == 8 * 8192 * 4
+    ws = L.fq_linear_workspace_size(8, 8192, 28672, fq.STATIC)
+    assert ws >= 8 * 28672 // 2 + 8 * 8192 * 4
+
+
+def test_debug_timeout_rejects_limits(L):
+    assert L.fq_debug_wait_timeout(0, None) == fq.FQ_ERR_INVALID
+    assert L.fq_debug_wait_timeout(1000000, None) == fq.FQ_ERR_INVALID

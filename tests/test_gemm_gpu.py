@@ -1,0 +1,93 @@
+"""fq_w4a4_gemm on the GPU against the CPU oracle, on seeded packed operands."""
+import numpy as np
+import pytest
+import torch
+
+import gpu_checks as C
+from int4_linear_b200 import fq, synth
+from oracle import fq_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+
+def _operands(seed, m, n, k):
+    g = synth.generator(seed)
+    return synth.random_packed(g, m, k), synth.random_packed(g, n, k)
+
+
+SHAPES = [
+    (128, 256, 128),      # one tile, one K slice
+    (1, 8, 128),          # smallest
+    (200, 264, 384),      # ragged M and N tiles
+    (257, 520, 1024),     # ragged, several K slices
+    (64, 1024, 4096),     # decode-style swap path
+    (8, 8192, 28672),     # decode with split-K
+    (33, 136, 640),       # swap path with 48-wide token tile
+    (2048, 512, 4096),    # prefill, many M tiles
+]
+
+
+@pytest.mark.parametrize("m,n,k", SHAPES)
+def test_gemm_int32_exact(m, n, k):
+    a, b = _operands(m + n + k, m, n, k)
+    acc = fq.fq_w4a4_gemm_s32(C.dev(a), C.dev(b))
+    ref = O.gemm_int(C.unpack(a), C.unpack(b))
+    assert np.array_equal(C.host(acc).astype(np.int64), ref)
+
+
+def test_gemm_int32_extremes():
+    """-8 x -8 over the largest K: 64 * 65536 per output, exact in int32 and float32."""
+    m, n, k = 4, 16, 65536
+    a = synth.constant_packed(m, k, 0x88)
+    b = synth.constant_packed(n, k, 0x88)
+    acc = C.host(fq.fq_w4a4_gemm_s32(C.dev(a), C.dev(b)))
+    assert np.all(acc == 64 * k)
+    b7 = synth.constant_packed(n, k, 0x77)
+    acc = C.host(fq.fq_w4a4_gemm_s32(C.dev(a), C.dev(b7)))
+    assert np.all(acc == -56 * k)
+
+
+@pytest.mark.parametrize("m,n,k", SHAPES + [(1, 8192, 28672), (32, 8192, 28672), (64, 57344, 8192)])
+def test_gemm_row_exact(m, n, k):
+    a, b = _operands(3 * m + n + k, m, n, k)
+    g = synth.generator(m + 1)
+    sx = synth.random_scales(g, m)
+    sw = synth.random_scales(g, n)
+    y = fq.fq_w4a4_gemm(C.dev(a), C.dev(sx), C.dev(b), C.dev(sw), fq.ROW)
+    ref = O.dequant_row(O.gemm_int(C.unpack(a), C.unpack(b)), sx, sw)
+    C.check_fp16_exact(C.host(y), ref)
+
+
+@pytest.mark.parametrize("m,n,k", [(1, 8192, 28672), (8, 256, 512), (64, 57344, 8192), (300, 264, 1024)])
+def test_gemm_static_exact(m, n, k):
+    a, b = _operands(5 * m + n + k, m, n, k)
+    sw = synth.random_scales(synth.generator(m + 2), n, 1e-4, 1e-2)
+    y = fq.fq_w4a4_gemm(C.dev(a), None, C.dev(b), C.dev(sw), fq.STATIC)
+    ref = O.dequant_static(O.gemm_int(C.unpack(a), C.unpack(b)), sw)
+    C.check_fp16_exact(C.host(y), ref)
+
+
+@pytest.mark.parametrize("m,n,k", [(128, 128, 128), (200, 264, 1024), (1, 136, 2048), (512, 1024, 8192)])
+def test_gemm_group(m, n, k):
+    a, b = _operands(7 * m + n + k, m, n, k)
+    g = synth.generator(m + 3)
+    sx = synth.random_group_scales(g, k // 128, m)
+    sw = synth.random_group_scales(g, k // 128, n)
+    y = fq.fq_w4a4_gemm(C.dev(a), C.dev(sx), C.dev(b), C.dev(sw), fq.GROUP)
+    n_beyond = C.check_fp16_group(C.host(y), C.unpack(a), C.unpack(b), sx.T, sw.T)
+    print(f"group {m}x{n}x{k}: {n_beyond} outputs beyond 1 ulp (cancellation bound)")
+
+
+def test_gemm_workspace_is_reused_correctly():
+    """Two split-K calls in a row on one workspace give the same exact result."""
+    m, n, k = 8, 8192, 28672
+    a, b = _operands(99, m, n, k)
+    g = synth.generator(4)
+    sx, sw = synth.random_scales(g, m), synth.random_scales(g, n)
+    ws = torch.full((fq.fq_gemm_workspace_size(m, n, k, fq.ROW),), 0x5A, dtype=torch.uint8, device="cuda")
+    y1 = C.host(fq.fq_w4a4_gemm(C.dev(a), C.dev(sx), C.dev(b), C.dev(sw), fq.ROW, workspace=ws))
+    y2 = C.host(fq.fq_w4a4_gemm(C.dev(a), C.dev(sx), C.dev(b), C.dev(sw), fq.ROW, workspace=ws))
+    ref = O.dequant_row(O.gemm_int(C.unpack(a), C.unpack(b)), sx, sw)
+    C.check_fp16_exact(y1, ref)
+    C.check_fp16_exact(y2, ref)
+    fq.fq_check_device_error()

@@ -1,0 +1,148 @@
+"""fq_quant_act / fq_quant_weight on the GPU against the CPU oracle."""
+import numpy as np
+import pytest
+import torch
+
+import gpu_checks as C
+from int4_linear_b200 import fq, synth
+from oracle import fq_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+GRAN = {"row": (fq.ROW, O.ROW), "group": (fq.GROUP, O.GROUPED), "static": (fq.STATIC, O.STATIC)}
+
+
+def _x(seed, m, k, scale=1.0):
+    g = synth.generator(seed)
+    cs = np.ones(k)
+    cs[g.permutation(k)[: max(1, k // 100)]] = 30.0
+    return synth._draw(g, (m, k), "normal", scale, col_scale=cs)
+
+
+def _static_scales(seed, k):
+    return synth.random_scales(synth.generator(seed), k, 0.05, 2.0)
+
+
+def _gpu_scales(s, gran):
+    if s is None:
+        return None
+    s = C.host(s)
+    return s.T.astype(np.float32) if gran == fq.GROUP else s
+
+
+@pytest.mark.parametrize("gname", ["row", "group", "static"])
+@pytest.mark.parametrize("m,k", [(1, 128), (3, 256), (16, 256), (129, 4096), (64, 14336), (5, 32768)])
+@pytest.mark.parametrize("with_c", [False, True])
+def test_quant_act_exact(gname, m, k, with_c):
+    """Without the transform every step is float32 as written: bit-exact."""
+    gf, go = GRAN[gname]
+    x = _x(m * 7 + k, m, k)
+    c = synth.generator(5).uniform(0.5, 2.0, k).astype(np.float32) if with_c else None
+    ss = _static_scales(k, k) if gname == "static" else None
+    alpha = 0.9 if gname != "static" else 1.0
+    t = fq.Transform(c=C.dev(c)) if with_c else None
+    xq, sx = fq.fq_quant_act(C.dev(x), fq.qparams(gf, alpha), t, C.dev(ss) if ss is not None else None)
+    q_ref, s_ref, _ = O.quant_act(x, go, alpha, c=c, static_scale=ss)
+    assert np.array_equal(C.host(xq), O.pack_int4(q_ref))
+    if gname != "static":
+        assert np.array_equal(_gpu_scales(sx, gf), s_ref)
+
+
+def test_quant_act_tiny_workload():
+    d = synth.tiny_linear()
+    xq, sx = fq.fq_quant_act(C.dev(d["x"]), fq.qparams(fq.ROW, 1.0))
+    q_ref, s_ref, _ = O.quant_act(d["x"], O.ROW, 1.0)
+    assert np.array_equal(C.host(xq), O.pack_int4(q_ref))
+    assert np.array_equal(C.host(sx), s_ref)
+
+
+def _transform_case(d, gname, m=None):
+    gf, go = GRAN[gname]
+    x = d["x"] if m is None else d["x"][:m]
+    alpha = d.get("alpha_a", 1.0)
+    t = fq.Transform(C.dev(d["p1"]), C.dev(d["p2"]), C.dev(d["c"]) if d.get("c") is not None else None)
+    xq, sx, xhat = fq.fq_quant_act_debug(C.dev(x), fq.qparams(gf, alpha), t)
+    q_ref, s_ref, v_ref = O.quant_act(x, go, alpha, d["p1"], d["p2"], d.get("c"))
+    worst = C.check_values(C.host(xhat), v_ref, go)
+    s_gpu = _gpu_scales(sx, gf)
+    if gname == "row":
+        C.check_scales_row(s_gpu, s_ref)
+    else:
+        C.check_scales_group(s_gpu, s_ref, v_ref, alpha)
+    ex = C.exempt_mask(v_ref, s_ref, s_gpu, go)
+    n_ex, n_diff = C.check_codes(C.unpack(C.host(xq)), q_ref, ex)
+    print(f"{d['name']} {gname}: max |dv|/amax {worst:.2e}, boundary-exempt {n_ex}, differing codes {n_diff}")
+    return n_ex, n_diff
+
+
+@pytest.mark.parametrize("m", [256, 2048])
+def test_quant_act_transform_hidden(m):
+    """LLaMA-3-8B-like hidden size: Kronecker (64, 64), c, alpha 0.9, pivot token."""
+    _transform_case(synth.transform_quant(m=m), "row")
+
+
+def test_quant_act_transform_group():
+    d = synth.prefill_linear(8192, 128, m=96, transform=True)
+    d["alpha_a"] = 0.95
+    _transform_case(d, "group")
+
+
+@pytest.mark.parametrize("k", [14336, 28672])
+def test_quant_act_transform_wide(k):
+    """(112, 128) keeps the factors in shared memory; (224, 128) reads them through L1."""
+    d = synth.prefill_linear(k, 128, m=24, transform=True)
+    _transform_case(d, "row")
+    _transform_case(d, "group")
+
+
+def test_quant_act_identity_transform_is_exact():
+    d = synth.transform_quant(m=64, k=4096)
+    eye = np.eye(64, dtype=np.float32)
+    t = fq.Transform(C.dev(eye), C.dev(eye), None)
+    xq, sx = fq.fq_quant_act(C.dev(d["x"]), fq.qparams(fq.ROW, 0.9), t)
+    q_ref, s_ref, _ = O.quant_act(d["x"], O.ROW, 0.9)
+    assert np.array_equal(C.host(xq), O.pack_int4(q_ref))
+    assert np.array_equal(C.host(sx), s_ref)
+
+
+@pytest.mark.parametrize("gname", ["row", "group"])
+@pytest.mark.parametrize("qsm", [False, True])
+def test_quant_weight_exact(gname, qsm):
+    gf, go = GRAN[gname]
+    d = synth.prefill_linear(4096, 264, m=1, transform=False)
+    s_k = _static_scales(3, 4096) if qsm else None
+    wq, sw = fq.fq_quant_weight(C.dev(d["w"]), fq.qparams(gf, 0.95), None, C.dev(s_k) if qsm else None)
+    q_ref, s_ref, _ = O.quant_weight(d["w"], go, 0.95, qsm_scale=s_k)
+    assert np.array_equal(C.host(wq), O.pack_int4(q_ref))
+    assert np.array_equal(_gpu_scales(sw, gf), s_ref)
+
+
+@pytest.mark.parametrize("gname", ["row", "group"])
+def test_quant_weight_inverse_transform(gname):
+    gf, go = GRAN[gname]
+    d = synth.transform_quant(m=8, k=8192)
+    w = synth.prefill_linear(8192, 136, m=1, transform=False)["w"]
+    inv = fq.Transform(C.dev(d["p1_inv"]), C.dev(d["p2_inv"]), C.dev(d["c"]))
+    wq, sw = fq.fq_quant_weight(C.dev(w), fq.qparams(gf, 1.0), inv)
+    q_ref, s_ref, v_ref = O.quant_weight(w, go, 1.0, d["p1_inv"], d["p2_inv"], d["c"])
+    s_gpu = _gpu_scales(sw, gf)
+    if gname == "row":
+        C.check_scales_row(s_gpu, s_ref)
+    else:
+        C.check_scales_group(s_gpu, s_ref, v_ref, 1.0)
+    C.check_codes(C.unpack(C.host(wq)), q_ref, C.exempt_mask(v_ref, s_ref, s_gpu, go))
+
+
+def test_quant_act_zero_rows():
+    x = np.zeros((4, 256), np.float16)
+    x[2, 5] = 1.0
+    xq, sx = fq.fq_quant_act(C.dev(x), fq.qparams(fq.ROW, 1.0))
+    q_ref, s_ref, _ = O.quant_act(x, O.ROW, 1.0)
+    assert np.array_equal(C.host(xq), O.pack_int4(q_ref))
+    assert np.array_equal(C.host(sx), s_ref)
+    xq, sx = fq.fq_quant_act(C.dev(x), fq.qparams(fq.GROUP, 1.0))
+    q_ref, s_ref, _ = O.quant_act(x, O.GROUPED, 1.0)
+    assert np.array_equal(C.host(xq), O.pack_int4(q_ref))
+    assert np.array_equal(C.host(sx).T.astype(np.float32), s_ref)
+    torch.cuda.synchronize()
+    fq.fq_check_device_error()
