@@ -1,0 +1,420 @@
+"""Benchmark of the W4A4 linear layer on B200.
+
+One step = the four linear layers of a LLaMA-3-8B-like decoder layer at
+prefill (qkv 4096->6144, o 4096->4096, gate+up 4096->28672, down 14336->4096)
+for M = 2048 tokens: for each layer the online activation quantization
+(Kronecker transform (64,64) or (112,128), per-token INT4) and the INT4 x INT4
+tcgen05 GEMM with the per-token x per-channel fp16 epilogue.  Weights are
+quantized once beforehand (offline).  Metric: effective TOPS = sum 2 M N K /
+step time, plus the quantization kernels' GB/s.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun (N > 1) each rank runs the same step on its own GPU
+(replicas, weak scaling, no data-path collective); time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from int4_linear_b200 import synth  # noqa: E402
+
+M_TOKENS = 2048
+SHAPES = [("qkv", 4096, 6144), ("o", 4096, 4096), ("gate_up", 4096, 28672), ("down", 14336, 4096)]
+METRIC = "W4A4 linear effective TOPS + quant-kernel GB/s, % of roofline, 1xB200"
+WORKLOAD = ("llama3-8b-like decoder-layer prefill linears qkv/o/gate_up/down, M=2048 tokens, "
+            "Kronecker-transformed per-token INT4 activations (64x64 / 112x128), per-channel INT4 weights, fp16 out")
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+INT8_OVER_BF16 = 4.5 / 2.25  # nominal dense ratio (B200: 4.5 POPS int8 vs 2.25 PFLOPS bf16)
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def workload(seed=0, only=None):
+    out = []
+    for name, k, n in SHAPES:
+        if only and name != only:
+            continue
+        d = synth.prefill_linear(k, n, m=M_TOKENS, seed=seed)
+        d["layer"] = name
+        out.append(d)
+    return out
+
+
+def quant_bytes(m, k, n1, n2):
+    """Algorithmic HBM bytes of one activation-quantization launch: read X fp16,
+    write packed codes and fp32 scales, read the two factors."""
+    return m * k * 2 + m * k // 2 + m * 4 + 4 * (n1 * n1 + n2 * n2)
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, dev_id: str):
+        self.dev_id = dev_id
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.dev_id, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.1)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax = float(parts[1])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- our arm
+
+def run_ours(args, ws, rank, local):
+    import torch
+    import torch.distributed as dist
+
+    from int4_linear_b200 import fq
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    fq.lib()
+
+    layers = workload(seed=rank, only=args.only)
+    qp = fq.qparams(fq.ROW, 1.0)
+    state = []
+    for d in layers:
+        m, k, n = d["m"], d["k"], d["n"]
+        x = torch.from_numpy(d["x"]).to(dev)
+        w = torch.from_numpy(d["w"]).to(dev)
+        wq, sw = fq.fq_quant_weight(w, qp)                     # offline, not timed
+        del w
+        t = fq.Transform(torch.from_numpy(d["p1"]).to(dev), torch.from_numpy(d["p2"]).to(dev))
+        xq = torch.empty(m, k // 2, dtype=torch.uint8, device=dev)
+        sx = torch.empty(m, dtype=torch.float32, device=dev)
+        y = torch.empty(m, n, dtype=torch.float16, device=dev)
+        lws = torch.empty(max(fq.fq_linear_workspace_size(m, n, k, fq.ROW), 256), dtype=torch.uint8, device=dev)
+        state.append(dict(d=d, x=x, wq=wq, sw=sw, t=t, xq=xq, sx=sx, y=y, lws=lws, m=m, k=k, n=n))
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream(dev)
+    L = len(state)
+
+    def step(evs=None):
+        for i, s in enumerate(state):
+            if evs is not None:
+                evs[i][0].record(stream)
+            fq.fq_quant_act(s["x"], qp, s["t"], None, s["xq"], s["sx"], stream=stream)
+            if evs is not None:
+                evs[i][1].record(stream)
+            fq.fq_w4a4_gemm(s["xq"], s["sx"], s["wq"], s["sw"], fq.ROW, Y=s["y"], stream=stream)
+            if evs is not None:
+                evs[i][2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(L)] for _ in range(args.steps)]
+    dev_uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    clocks = ClockSampler(dev_uuid if dev_uuid.startswith("GPU-") else f"GPU-{dev_uuid}")
+    clocks.start()
+    time.sleep(0.3)
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for it in range(args.steps):
+        step(evs[it])
+    end.record(stream)
+    torch.cuda.synchronize()
+    if ws > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    total_ms = start.elapsed_time(end)
+
+    q_ms = [0.0] * L
+    g_ms = [0.0] * L
+    for it in range(args.steps):
+        for i in range(L):
+            q_ms[i] += evs[it][i][0].elapsed_time(evs[it][i][1])
+            g_ms[i] += evs[it][i][1].elapsed_time(evs[it][i][2])
+    q_ms = [v / args.steps for v in q_ms]
+    g_ms = [v / args.steps for v in g_ms]
+
+    if ws > 1:
+        tt = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+
+    # ------------------------------------------------ end to end through fq_linear with host buffers
+    xh = [torch.from_numpy(s["d"]["x"]).pin_memory() for s in state]
+    yh = [torch.empty(s["m"], s["n"], dtype=torch.float16).pin_memory() for s in state]
+    h2d = sum(t.numel() * 2 for t in xh)
+    d2h = sum(t.numel() * 2 for t in yh)
+
+    def e2e_step():
+        for i, s in enumerate(state):
+            s["x"].copy_(xh[i], non_blocking=True)
+            fq.fq_linear(s["x"], qp, s["wq"], s["sw"], s["t"], Y=s["y"], workspace=s["lws"], stream=stream)
+            yh[i].copy_(s["y"], non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 200))
+    for _ in range(max(3, args.warmup // 4)):
+        e2e_step()
+    torch.cuda.synchronize()
+    if ws > 1:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if ws > 1:
+        tt = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+        dist.barrier()
+        dist.destroy_process_group()
+
+    if rank != 0:
+        return None
+
+    ops_step = sum(2.0 * s["m"] * s["n"] * s["k"] for s in state)
+    ms_step = total_ms / args.steps
+    value = ops_step * ws / (ms_step * 1e-3) / 1e12
+    pk, pk_kind = peaks()
+    int8_peak = pk["bf16_tflops_sustained"] * INT8_OVER_BF16
+    g_ops = sum(2.0 * s["m"] * s["n"] * s["k"] for s in state)
+    g_time = sum(g_ms) * 1e-3
+    g_achieved = g_ops / g_time / 1e12
+    q_bytes = [quant_bytes(s["m"], s["k"], s["d"]["n1"], s["d"]["n2"]) for s in state]
+    q_gbs = sum(q_bytes) / (sum(q_ms) * 1e-3) / 1e9
+    breakdown = {}
+    for i, s in enumerate(state):
+        lo = s["d"]["layer"]
+        breakdown[lo] = {
+            "gemm_us": round(g_ms[i] * 1e3, 2),
+            "gemm_tops": round(2.0 * s["m"] * s["n"] * s["k"] / (g_ms[i] * 1e-3) / 1e12, 1),
+            "quant_us": round(q_ms[i] * 1e3, 2),
+            "quant_gbs": round(q_bytes[i] / (q_ms[i] * 1e-3) / 1e9, 1),
+            "kron": [s["d"]["n1"], s["d"]["n2"]],
+        }
+    e2e_value = ops_step * ws / (e2e_ms * 1e-3) / 1e12
+    out = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TOPS",
+        "n_gpus": ws,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "int4 (s8 tensor-core MMA, s32 accumulate), fp32 transform/scales, fp16 io",
+        "data": "synthetic (seeded Gaussian activations with outlier channels, Gaussian weights; stands in for LLaMA activations/weights)",
+        "config": {
+            "workload": WORKLOAD,
+            "tokens": M_TOKENS,
+            "layers": [{"name": s["d"]["layer"], "K": s["k"], "N": s["n"]} for s in state],
+            "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU",
+            "l2": "no flush: one step touches ~420 MB (inputs, packed weights, outputs) > 126 MB L2",
+        },
+        "quant_kernel": {"gbs": round(q_gbs, 1), "peak_gbs": pk["hbm_gbs"],
+                         "frac": round(q_gbs / pk["hbm_gbs"], 4), "peak_kind": pk_kind,
+                         "bytes_per_step": int(sum(q_bytes))},
+        "breakdown": breakdown,
+        "roofline": {
+            "kernel": "gemm_w4a4_kernel",
+            "bound": "tensor",
+            "achieved": round(g_achieved, 1),
+            "peak": round(int8_peak, 1),
+            "unit": "TOPS",
+            "frac": round(g_achieved / int8_peak, 4),
+            "peak_kind": f"{pk_kind} bf16 sustained x {INT8_OVER_BF16:g} (nominal int8/bf16 dense ratio)",
+            "traffic": None,
+            "note": "achieved = sum of algorithmic 2MNK over the GEMM launches / sum of their CUDA-event durations",
+        },
+        "e2e": {"value": round(e2e_value, 2), "unit": "TOPS", "h2d_bytes_per_step": int(h2d * ws),
+                "d2h_bytes_per_step": int(d2h * ws), "steps": e2e_steps,
+                "api": "fq_linear per layer, X copied from pinned host memory and Y read back every step"},
+        "gpu_launches": 2 * L * args.steps,
+        "clocks": clk,
+    }
+    if not args.no_cpu_baseline and ws == 1:
+        out["cpu_baseline"] = cpu_baseline(layers, budget_s=args.cpu_seconds)
+    return out
+
+
+# ---------------------------------------------------------------- the oracle on the host cores
+
+def _blas_threads():
+    try:
+        import threadpoolctl
+        n = [i["num_threads"] for i in threadpoolctl.threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_step(layers, rows_per_layer, offset, wcodes):
+    """The oracle on `rows_per_layer` token rows of every layer; returns the ops done."""
+    from oracle import fq_oracle as O
+    ops = 0.0
+    for d, (qw, sw) in zip(layers, wcodes):
+        r = (np.arange(rows_per_layer) + offset) % d["m"]
+        O.linear(d["x"][r], qw, sw, O.ROW, 1.0, d["p1"], d["p2"])
+        ops += 2.0 * rows_per_layer * d["n"] * d["k"]
+    return ops
+
+
+def oracle_weights(layers):
+    from oracle import fq_oracle as O
+    out = []
+    for d in layers:
+        qw, sw, _ = O.quant_weight(d["w"], O.ROW, 1.0)
+        out.append((qw, sw))
+    return out
+
+
+def cpu_baseline(layers, budget_s=15.0):
+    """The oracle as it stands, timed on this host's cores over a bounded sample:
+    token rows of every layer are processed in chunks until ~budget_s elapsed."""
+    wcodes = oracle_weights(layers)       # offline step, not timed
+    oracle_step(layers, 1, 0, wcodes)     # warm
+    chunk, rows, ops, dt = 8, 0, 0.0, 0.0
+    while dt < budget_s:
+        t0 = time.perf_counter()
+        ops += oracle_step(layers, chunk, rows, wcodes)
+        dt += time.perf_counter() - t0
+        rows += chunk
+    return {"value": round(ops / dt / 1e12, 6), "unit": "TOPS", "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"{rows} token rows of each of the {len(layers)} layers (full K, N), oracle quant_act (float64 "
+                      f"Kronecker transform) + exact GEMM (float64 BLAS) + dequant; weights pre-quantized; {dt:.1f} s"}
+
+
+def run_reference(args, ws, rank):
+    if rank != 0:
+        return None
+    layers = workload(seed=0)
+    wcodes = oracle_weights(layers)
+    # each step: a bounded sample sized so the whole run stays within a few minutes
+    probe_t = time.perf_counter()
+    oracle_step(layers, 1, 0, wcodes)
+    per_row = time.perf_counter() - probe_t
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    rows = max(1, int(budget / max(per_row, 1e-4)))
+    for i in range(args.warmup):
+        oracle_step(layers, rows, i * rows, wcodes)
+    t0 = time.perf_counter()
+    ops = 0.0
+    for i in range(args.steps):
+        ops += oracle_step(layers, rows, (args.warmup + i) * rows, wcodes)
+    dt = time.perf_counter() - t0
+    value = ops / dt / 1e12
+    cores = _blas_threads()
+    sample = f"{rows} token rows of each of the 4 layers per step (full K, N)"
+    return {
+        "impl": "reference",
+        "metric": METRIC, "value": round(value, 6), "unit": "TOPS", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(dt / max(1, args.steps) * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64 transform, f32 scales, exact integer GEMM",
+        "data": "synthetic", "config": {"workload": WORKLOAD, "tokens_sampled_per_step": rows},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TOPS", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", choices=[s[0] for s in SHAPES], default=None,
+                    help="run one layer only (for profiling a single launch)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    ws, rank, local = dist_env()
+    if args.impl == "reference":
+        out = run_reference(args, ws, rank)
+    else:
+        out = run_ours(args, ws, rank, local)
+    if out is not None:
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()
