@@ -140,6 +140,26 @@ fq_status fq_w4a4_gemm(const uint8_t* Xq, const void* s_x, const uint8_t* Wq, co
                        int M, int N, int K, fq_gran gran, uint16_t* Y,
                        void* workspace, size_t ws_bytes, void* stream);
 
+/* fq_w4a4_gemm for callers that cannot allocate device memory or provide
+ * scratch (a plugin inside a runtime that owns all device memory, a serving
+ * loop that forbids allocation after start-up).  The pages have no
+ * counterpart of this call; it exists for those callers only.
+ * Same arguments and results as fq_w4a4_gemm without the workspace: the
+ * split-K partial sums use a static 8 MiB device buffer inside libfq.so,
+ * which every GPU that loads the library holds until the process exits.
+ * - Sizes whose split-K scratch (fq_gemm_workspace_size) exceeds 8 MiB are
+ *   rejected with FQ_ERR_INVALID; the call enqueues nothing then.
+ * - The first call on a device that needs the buffer looks up its device
+ *   address (cudaGetSymbolAddress) with that device current; make that
+ *   first call before any stream capture.
+ * - All calls share the one buffer: calls that may overlap on the GPU (on
+ *   different streams, or from several threads) race and give wrong
+ *   results; serialize them on one stream.  Each call clears the part it
+ *   uses before use, so the previous call's contents do no harm.
+ * - Calls no allocating routine (no cudaMalloc/cudaFree). */
+fq_status fq_w4a4_gemm_noalloc(const uint8_t* Xq, const void* s_x, const uint8_t* Wq, const void* s_w,
+                               int M, int N, int K, fq_gran gran, uint16_t* Y, void* stream);
+
 /* The exact integer accumulators acc[m][n] = sum_k qx[m,k] qw[n,k] as int32
  * [M, N] (out), for checking the GEMM's integer part on its own. */
 fq_status fq_w4a4_gemm_s32(const uint8_t* Xq, const uint8_t* Wq, int M, int N, int K,

@@ -27,6 +27,7 @@
 
 #include <algorithm>
 #include <cmath>
+#include <mutex>
 
 #include "fq_device.cuh"
 #include "fq_host.h"
@@ -586,3 +587,72 @@ fq_status fq_w4a4_gemm_s32(const uint8_t* Xq, const uint8_t* Wq, int M, int N, i
 size_t fq_gemm_workspace_size(int M, int N, int K, fq_gran gran) { return fq::gemm_workspace_bytes(M, N, K, gran); }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Entry point that allocates nothing.
+//
+// Some callers cannot hand the GEMM a workspace: for example a plugin or
+// callback running inside another runtime that owns all device memory and
+// gives out none, or a serving loop that forbids device allocation after
+// start-up so that its memory use stays fixed (and because cudaMalloc may
+// synchronize the device and stall other streams).  For them the split-K
+// partial sums live in this file-scope buffer instead.  Every GPU that loads
+// the library keeps this buffer for the life of the process.
+namespace fq {
+namespace {
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB: M * N int32 partial sums
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kNoAllocMaxDevices = 64;
+void* g_noalloc_ptr[kNoAllocMaxDevices];
+std::mutex g_noalloc_mu;
+
+// Device address of the buffer on the current device, looked up once per
+// device (the host-side name of the array is not a device address).
+void* noalloc_scratch(fq_status* st) {
+  int d = -1;
+  if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= kNoAllocMaxDevices) {
+    *st = fail(FQ_ERR_CUDA, "no current CUDA device");
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[d]) {
+    void* ptr = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess || !ptr) {
+      *st = fail(FQ_ERR_CUDA, "cudaGetSymbolAddress of the static scratch failed: %s", cudaGetErrorString(e));
+      return nullptr;
+    }
+    g_noalloc_ptr[d] = ptr;
+  }
+  *st = FQ_OK;
+  return g_noalloc_ptr[d];
+}
+}  // namespace
+}  // namespace fq
+
+extern "C" fq_status fq_w4a4_gemm_noalloc(const uint8_t* Xq, const void* s_x, const uint8_t* Wq, const void* s_w,
+                                          int M, int N, int K, fq_gran gran, uint16_t* Y, void* stream) {
+  fq::clear_error();
+  int epi;
+  switch (gran) {
+    case FQ_DYNAMIC_ROW: epi = fq::kEpiRow; break;
+    case FQ_STATIC_CHANNEL: epi = fq::kEpiStatic; break;
+    case FQ_DYNAMIC_GROUP: epi = fq::kEpiGroup; break;
+    default: return fq::fail(FQ_ERR_UNSUPPORTED, "granularity %d is not provided", int(gran));
+  }
+  const size_t need = fq_gemm_workspace_size(M, N, K, gran);
+  if (need > fq::kNoAllocScratchBytes)
+    return fq::fail(FQ_ERR_INVALID,
+                    "M = %d, N = %d, K = %d needs %zu bytes of split-K scratch, more than the %zu-byte static buffer "
+                    "of fq_w4a4_gemm_noalloc; use fq_w4a4_gemm with a workspace",
+                    M, N, K, need, fq::kNoAllocScratchBytes);
+  void* ws = nullptr;
+  if (need > 0) {
+    fq_status st;
+    ws = fq::noalloc_scratch(&st);
+    if (!ws) return st;
+  }
+  return fq::gemm_impl(Xq, s_x, Wq, s_w, M, N, K, epi, Y, nullptr, ws, ws ? fq::kNoAllocScratchBytes : 0,
+                       static_cast<cudaStream_t>(stream));
+}

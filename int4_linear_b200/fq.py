@@ -83,6 +83,7 @@ def lib():
         "fq_quant_act_debug": [vp, i, i, qp, tp, vp, vp, vp, vp, vp],
         "fq_w4a4_gemm": [vp, vp, vp, vp, i, i, i, i, vp, vp, sz, vp],
         "fq_w4a4_gemm_s32": [vp, vp, i, i, i, vp, vp],
+        "fq_w4a4_gemm_noalloc": [vp, vp, vp, vp, i, i, i, i, vp, vp],
         "fq_linear": [vp, i, i, qp, tp, vp, vp, vp, i, vp, vp, sz, vp],
         "fq_check_device_error": [vp],
         "fq_debug_wait_timeout": [ctypes.c_uint, vp],
@@ -213,6 +214,23 @@ def fq_w4a4_gemm(Xq, s_x, Wq, s_w, gran: int, Y=None, workspace=None, stream=Non
     ws, wsb = _workspace(fq_gemm_workspace_size(m, n, k, gran), Xq.device, workspace)
     st = lib().fq_w4a4_gemm(Xq.data_ptr(), _p(s_x), Wq.data_ptr(), _p(s_w), m, n, k, gran, Y.data_ptr(),
                             _p(ws), wsb, _s(stream))
+    _raise(st)
+    return Y
+
+
+def fq_w4a4_gemm_noalloc(Xq, s_x, Wq, s_w, gran: int, Y=None, stream=None):
+    """fq_w4a4_gemm without a workspace, for callers that cannot allocate device
+    memory: the library's static 8 MiB scratch holds the split-K partial sums.
+    Calls that overlap on the GPU share that scratch and race; keep them on one
+    stream.  (Y is allocated here only when the caller passes none.)"""
+    _check(Xq, torch.uint8, "Xq")
+    _check(Wq, torch.uint8, "Wq")
+    m, k2 = Xq.shape
+    n = Wq.shape[0]
+    Y = torch.empty(m, n, dtype=torch.float16, device=Xq.device) if Y is None else Y
+    _check(Y, torch.float16, "Y")
+    st = lib().fq_w4a4_gemm_noalloc(Xq.data_ptr(), _p(s_x), Wq.data_ptr(), _p(s_w), m, n, 2 * k2, gran,
+                                    Y.data_ptr(), _s(stream))
     _raise(st)
     return Y
 
