@@ -446,7 +446,8 @@ fq_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmPa
                       cudaStream_t stream) {
   using C = Cfg<BN, EPI>;
   auto kern = gemm_w4a4_kernel<BN, EPI, SWAP>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess ||
+      cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
     return fail(FQ_ERR_CUDA, "cannot reserve %d bytes of shared memory for the GEMM", C::SMEM);
   kern<<<grid, kThreads, C::SMEM, stream>>>(ta, tb, gp);
   return check_launch("gemm_w4a4_kernel");

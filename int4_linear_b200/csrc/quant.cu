@@ -27,6 +27,23 @@
 
 namespace fq {
 
+struct QuantTcParams {
+  const __half* X;
+  int M, K, n1, n2, gran;
+  float alpha;
+  const float* P1;
+  const float* P2;
+  const float* c;
+  const float* sstatic;
+  uint8_t* Q;
+  float* s_row;
+  __half* s_grp;
+  float* xhat;
+  unsigned* err;
+};
+bool quant_act_tc_supported(int K, int n1, int n2);
+fq_status launch_quant_act_tc(const QuantTcParams& p, cudaStream_t stream);
+
 namespace {
 
 constexpr int kThreads = 256;
@@ -262,8 +279,9 @@ fq_status launch_quant(const QuantParams& qp, cudaStream_t stream) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
       return fail(FQ_ERR_CUDA, "cannot reserve %zu bytes of shared memory", smem);
   }
+  cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   int per_sm = 1;
-  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem);
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem) != cudaSuccess) per_sm = 1;
   per_sm = std::max(per_sm, 1);
   const int grid = std::max(1, std::min(qp.R, sm_count() * per_sm));
   kern<<<grid, kThreads, smem, stream>>>(qp);
@@ -325,10 +343,33 @@ fq_status quant_common(int side, const uint16_t* X, int R, int K, const fq_qpara
       p.Rt = t->P2;
     }
   }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (side == kAct && p.n1 > 0 && quant_act_tc_supported(K, p.n1, p.n2)) {
+    // activations with the transform: tensor-core kernel
+    unsigned* err = device_error_word();
+    if (!err) return fail(FQ_ERR_CUDA, "device error word unavailable");
+    QuantTcParams tp{};
+    tp.X = p.X;
+    tp.M = R;
+    tp.K = K;
+    tp.n1 = p.n1;
+    tp.n2 = p.n2;
+    tp.gran = p.gran;
+    tp.alpha = p.alpha;
+    tp.P1 = p.L;
+    tp.P2 = p.Rt;
+    tp.c = p.c;
+    tp.sstatic = p.sstatic;
+    tp.Q = p.Q;
+    tp.s_row = p.s_row;
+    tp.s_grp = p.s_grp;
+    tp.xhat = p.xhat;
+    tp.err = err;
+    return launch_quant_act_tc(tp, s);
+  }
   const bool psmem = smem_bytes(K, p.n1, p.n2, true) <= size_t(kSmemBudget);
   if (smem_bytes(K, p.n1, p.n2, false) > size_t(kSmemBudget))
     return fail(FQ_ERR_UNSUPPORTED, "row of K = %d does not fit in shared memory", K);
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (side == kAct) return psmem ? launch_quant<kAct, true>(p, s) : launch_quant<kAct, false>(p, s);
   return psmem ? launch_quant<kWeight, true>(p, s) : launch_quant<kWeight, false>(p, s);
 }
