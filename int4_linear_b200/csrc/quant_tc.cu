@@ -48,8 +48,9 @@ struct QuantTcParams {
 
 namespace {
 
-constexpr int kTcThreads = 256;
-constexpr int kMaxPieces = 8;  // 16-byte pieces of the X tile per thread
+constexpr int kTcThreads = 512;
+constexpr int kSplit = kTcThreads / 128;           // warps sharing one tensor-memory lane quadrant
+constexpr int kMaxPieces = 2048 / kTcThreads;      // 16-byte pieces of the X tile per thread
 
 template <int N2, int NP>
 struct TcCfg {
@@ -115,6 +116,25 @@ __device__ __forceinline__ int code_fast(float v, float s, float inv_s) {
   return static_cast<int>(fminf(fmaxf(rintf(qa), -8.0f), 7.0f));
 }
 
+// The code of v = u * up (up a power of two, exact) for scale s, given
+// f = up * (1/s) (also exact scaling of the rounded reciprocal): the quotient
+// u * f equals v * fl(1/s), so the tie test of code_fast applies unchanged.
+// Returns the code in the low 4 bits position-free (caller masks).
+__device__ __forceinline__ int code_scaled(float u, float f, float up, float s) {
+  const float qa = u * f;
+  const float r = rintf(qa);
+  const float d = fabsf(qa - r);  // distance to the nearest integer
+  if (0.5f - d <= fabsf(qa) * 9.5367431640625e-07f + 1e-30f) return code_of(u * up, s);
+  return __float2int_rn(fminf(fmaxf(r, -8.0f), 7.0f));
+}
+
+// w with bits [pos, pos + 4) replaced by the low 4 bits of q.
+__device__ __forceinline__ uint32_t put_nibble(uint32_t w, int q, int pos) {
+  uint32_t r;
+  asm("bfi.b32 %0, %1, %2, %3, 4;" : "=r"(r) : "r"(q), "r"(w), "r"(pos));
+  return r;
+}
+
 // 2^e as a float for e in [-126, 127].
 __device__ __forceinline__ float exp2i(int e) { return __int_as_float((e + 127) << 23); }
 
@@ -134,7 +154,7 @@ __device__ __forceinline__ uint32_t transpose_nibbles8(uint32_t w, int lane) {
 
 // Two CTAs per SM where the shared memory allows it (n2 = n1 = 64).
 template <int N2, int NP>
-constexpr int tc_min_blocks() { return TcCfg<N2, NP>::SMEM <= 110 * 1024 ? 2 : 1; }
+constexpr int tc_min_blocks() { return 1; }
 
 template <int N2, int NP, int GRAN>
 __global__ void __launch_bounds__(kTcThreads, tc_min_blocks<N2, NP>()) quant_act_tc_kernel(const QuantTcParams p) {
@@ -204,12 +224,15 @@ __global__ void __launch_bounds__(kTcThreads, tc_min_blocks<N2, NP>()) quant_act
     *reinterpret_cast<__half*>(sm + C::SL + C::SL_HALF + off) = lo;
   }
   // largest absolute column sum of P2 (bounds |U| by max|x| * colsum)
+  // column sums: thread tid holds part of column tid % N2; fold into 256 slots first
   float* colsum = reinterpret_cast<float*>(grpmax);
-  colsum[tid] = csum;
+  if (tid < 256) colsum[tid] = 0.f;
+  __syncthreads();
+  atomicAdd(&colsum[tid & 255], csum);  // 256 is a multiple of N2: slot keeps the column
   __syncthreads();
   float cs = 0.f;
   if (tid < N2)
-    for (int r = tid; r < kTcThreads; r += N2) cs += colsum[r];
+    for (int r = tid; r < 256; r += N2) cs += colsum[r];
   cs = warp_max_f(cs);
   __syncthreads();
   if (lane == 0) colsum[warp] = cs;
@@ -218,12 +241,12 @@ __global__ void __launch_bounds__(kTcThreads, tc_min_blocks<N2, NP>()) quant_act
   __syncthreads();
   tc_fence_after();
   float guard = 1.f;
-  for (int w = 0; w < 8; ++w) guard = fmaxf(guard, colsum[w]);
+  for (int w = 0; w < kTcThreads / 32; ++w) guard = fmaxf(guard, colsum[w]);
   const uint32_t tmem = *tslot;
   __syncthreads();
 
   const int npieces = T * K / 8;
-  const int q4 = warp & 3, half = warp >> 2;
+  const int q4 = warp & 3, part = warp >> 2;  // lane quadrant, column part (0..kSplit-1)
   const uint32_t tl = tmem + (uint32_t(q4 * 32) << 16);
   const int m = q4 * 32 + lane;  // tensor-memory lane of this thread
   constexpr uint32_t idescA = idesc_f16_m128(C::XROWS);
@@ -255,12 +278,18 @@ __global__ void __launch_bounds__(kTcThreads, tc_min_blocks<N2, NP>()) quant_act
         const int e = pc * 8, t = e / K, f = e - t * K;
         const __half2* h2 = reinterpret_cast<const __half2*>(&buf[it]);
         float mm = 0.f;
+        if (has_c) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float2 v = __half22float2(h2[j]);
-          const float a = has_c ? __fmul_rn(v.x, __ldg(p.c + f + 2 * j)) : v.x;
-          const float b = has_c ? __fmul_rn(v.y, __ldg(p.c + f + 2 * j + 1)) : v.y;
-          mm = fmaxf(mm, fmaxf(fabsf(a), fabsf(b)));
+          for (int j = 0; j < 4; ++j) {
+            const float2 v = __half22float2(h2[j]);
+            const float a = __fmul_rn(v.x, __ldg(p.c + f + 2 * j));
+            const float b = __fmul_rn(v.y, __ldg(p.c + f + 2 * j + 1));
+            mm = fmaxf(mm, fmaxf(fabsf(a), fabsf(b)));
+          }
+        } else {
+          // the max of |x| is exact in fp16
+          const __half2 m2 = __hmax2(__hmax2(__habs2(h2[0]), __habs2(h2[1])), __hmax2(__habs2(h2[2]), __habs2(h2[3])));
+          mm = fmaxf(__low2float(m2), __high2float(m2));
         }
         if (t == 0) mx0 = fmaxf(mx0, mm); else mx1 = fmaxf(mx1, mm);
       }
@@ -298,6 +327,14 @@ __global__ void __launch_bounds__(kTcThreads, tc_min_blocks<N2, NP>()) quant_act
         uint4 hi, lo;
         __half2* hh = reinterpret_cast<__half2*>(&hi);
         __half2* ll = reinterpret_cast<__half2*>(&lo);
+        if (!has_c && texp[t] >= -15 && texp[t] <= 14) {
+          // fp16 x times an fp16 power of two: exact (the result stays below 2^14)
+          const __half2 sc2 = __float2half2_rn(sc);
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj) hh[jj] = __hmul2(h2[jj], sc2);
+          *reinterpret_cast<uint4*>(sm + C::SX + off) = hi;
+          continue;
+        }
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
           float2 v = __half22float2(h2[jj]);
@@ -366,20 +403,20 @@ __global__ void __launch_bounds__(kTcThreads, tc_min_blocks<N2, NP>()) quant_act
 
     // ---- 3. U^T rows -> fp16 hi/lo, 16-byte stores (stage-B operand A: row m, K index i)
     {
-      constexpr int NC = C::XROWS / 2 / 32;  // 32-column chunks per thread
-      uint32_t ua[NC][32];
-#pragma unroll
-      for (int c = 0; c < NC; ++c) tmem_ld_32x32(tl + uint32_t(half * (C::XROWS / 2) + 32 * c), ua[c]);
+      constexpr int CW = C::XROWS / kSplit;  // columns per thread: 16 or 32
+      uint32_t u[32];
+      if (CW == 32)
+        tmem_ld_32x32(tl + uint32_t(part * CW), u);
+      else
+        tmem_ld_32x16(tl + uint32_t(part * CW), u);
       tmem_wait_ld();
-#pragma unroll
-      for (int c = 0; c < NC; ++c) {
-        const int col = half * (C::XROWS / 2) + 32 * c;  // D column = X tile row = (t, i)
-        const uint32_t* u = ua[c];
+      {
+        const int col = part * CW;  // D column = X tile row = (t, i)
         const int us = N2 == 64 ? 0 : col / NP;
         const int i0 = N2 == 64 ? col : col % NP;
         uint8_t* ub = sm + C::SX + us * (C::UKR * C::REG) + (i0 >> 6) * C::REG;
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
+        for (int g = 0; g < CW / 8; ++g) {
           uint4 hi, lo;
           __half2* hh = reinterpret_cast<__half2*>(&hi);
           __half2* ll = reinterpret_cast<__half2*>(&lo);
@@ -439,51 +476,52 @@ __global__ void __launch_bounds__(kTcThreads, tc_min_blocks<N2, NP>()) quant_act
       const bool tok_ok = tok < M;
       const float up = exp2i(texp[t]);
       const uint32_t cbase = tl + uint32_t(us * NP);
-      constexpr int NCH = NP / 16;  // 8-column chunks of this thread (chunks half, half + 2, ...)
+      constexpr int NCH = NP / 8 / kSplit;  // 8-column chunks of this thread (part, part + kSplit, ...)
       uint32_t u[NCH][8];
 #pragma unroll
-      for (int c = 0; c < NCH; ++c) tmem_ld_32x8(cbase + uint32_t((2 * c + half) * 8), u[c]);
+      for (int c = 0; c < NCH; ++c) tmem_ld_32x8(cbase + uint32_t((kSplit * c + part) * 8), u[c]);
       tmem_wait_ld();
-      // pass 1: token / group maxima
+      // pass 1: token / group maxima (rows k >= n1 and empty token slots hold zeros)
       float tm = 0.f;
 #pragma unroll
       for (int c = 0; c < NCH; ++c) {
-        const int ch = 2 * c + half;
+        const int ch = kSplit * c + part;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          const int k = ch * 8 + j;
-          const float a = (tok_ok && k < n1) ? fabsf(__uint_as_float(u[c][j])) * up : 0.f;
+          const float a = fabsf(__uint_as_float(u[c][j]));
           tm = fmaxf(tm, a);
           if (GRAN == FQ_DYNAMIC_GROUP) {
-            const float w = warp_max_f(a);
+            const int k = ch * 8 + j;
+            const float w = warp_max_f(a) * up;
             if (lane == 0 && k < n1) atomicMax(&grpmax[t * 128 + (k * N2) / kGroup], __float_as_uint(w));
           }
         }
       }
-      tm = warp_max_f(tm);
+      tm = warp_max_f(tm) * up;
       if (lane == 0) atomicMax(&tokmax[t], __float_as_uint(tm));
       __syncthreads();
       // pass 2: codes
-      float s_tok = 0.f, inv_tok = 0.f;
+      float s_tok = 0.f, f_tok = 0.f;
       if (GRAN == FQ_DYNAMIC_ROW) {
         s_tok = __fdiv_rn(__fmul_rn(__uint_as_float(tokmax[t]), p.alpha), 7.0f);
-        inv_tok = s_tok != 0.f ? 1.0f / s_tok : 0.f;
-        if (tok_ok && l == 0 && half == 0) p.s_row[tok] = s_tok;
+        f_tok = s_tok != 0.f ? (1.0f / s_tok) * up : 0.f;
+        if (tok_ok && l == 0 && part == 0) p.s_row[tok] = s_tok;
       }
 #pragma unroll
       for (int c = 0; c < NCH; ++c) {
-        const int ch = 2 * c + half;
+        const int ch = kSplit * c + part;
         uint32_t word = 0;
         float sg = 0.f, inv_g = 0.f;
         int gcur = -1;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const int k = ch * 8 + j;
-          const float v = __uint_as_float(u[c][j]) * up;
+          const float uu = __uint_as_float(u[c][j]);
+          const float v = uu * up;
           int q = 0;
           if (k < n1) {
             if (GRAN == FQ_DYNAMIC_ROW) {
-              q = code_fast(v, s_tok, inv_tok);
+              q = s_tok != 0.f ? code_scaled(uu, f_tok, up, s_tok) : 0;
             } else if (GRAN == FQ_DYNAMIC_GROUP) {
               const int g = (k * N2) / kGroup;
               if (g != gcur) {
@@ -499,7 +537,7 @@ __global__ void __launch_bounds__(kTcThreads, tc_min_blocks<N2, NP>()) quant_act
             }
             if (p.xhat && tok_ok) p.xhat[size_t(tok) * K + k * N2 + l] = v;
           }
-          word |= (uint32_t(q) & 0xFu) << (4 * j);
+          word = put_nibble(word, q, 4 * j);
         }
         word = transpose_nibbles8(word, lane);
         const int k = ch * 8 + (lane & 7);
