@@ -45,6 +45,11 @@ constexpr int kEpiWarps = 4;
 constexpr int kUnpackWarps = 8;
 constexpr int kThreads = 32 * (2 + kEpiWarps + kUnpackWarps);
 
+// Warps that unpack: the dedicated 8, plus the 4 epilogue warps when the
+// epilogue only runs after the main loop (every mode but group-128).
+template <int EPI>
+__host__ __device__ constexpr int unpack_warps() { return EPI == kEpiGroup ? kUnpackWarps : kUnpackWarps + kEpiWarps; }
+
 template <int BN, int EPI>
 struct Cfg {
   static constexpr int SP = BN >= 128 ? 4 : (BN >= 64 ? 6 : 8);
@@ -118,10 +123,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < SP; ++s) {
       mbar_init(&full_p[s], 1);
-      mbar_init(&empty_p[s], kUnpackWarps);
+      mbar_init(&empty_p[s], unpack_warps<EPI>());
     }
     for (int s = 0; s < SU; ++s) {
-      mbar_init(&full_u[s], kUnpackWarps);
+      mbar_init(&full_u[s], unpack_warps<EPI>());
       mbar_init(&empty_u[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -200,166 +205,189 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(done_bar);
       if (!mbar_wait(done_bar, 0)) record_error(p.err, kErrTimeoutDrain);
     }
-  } else if (warp < 2 + kEpiWarps) {
-    // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;  // tensor-memory lane quadrant this warp may access
-    const int rloc = q * 32 + lane;
-    const uint32_t tl = tmem + (uint32_t(q * 32) << 16);
-    const int arow = tileA * kBM + rloc;
-    const int bbase = tileB * BN;
-    if (EPI != kEpiGroup) {
-      if (!warp_wait(&acc_full[0], 0) && lane == 0) record_error(p.err, kErrTimeoutEpilogue);
-      tc_fence_after();
-      constexpr int CW = BN >= 32 ? 32 : 16;
-      for (int c0 = 0; c0 < BN; c0 += CW) {
-        uint32_t v[32];
-        if (CW == 32)
-          tmem_ld_32x32(tl + c0, v);
-        else
-          tmem_ld_32x16(tl + c0, v);
-        tmem_wait_ld();
-        if (!SWAP) {
-          // thread owns token row m = arow, columns n = bbase + c0 + j
-          const int m = arow;
-          if (m < p.M) {
-            const int n0 = bbase + c0;
-            float y[32];
-            if (EPI == kEpiRow || EPI == kEpiStatic) {
-              const float sxm = EPI == kEpiRow ? p.sx[m] : 1.0f;
+  } else {
+    // ------------------------------------------------------------ unpackers
+    // Warps 6..13 always unpack; in the modes whose epilogue runs after the
+    // main loop, warps 2..5 unpack too and then turn to the epilogue.
+    constexpr int NU = unpack_warps<EPI>();
+    const bool epi_warp = warp < 2 + kEpiWarps;
+    if (!epi_warp || EPI != kEpiGroup) {
+      const int uw = EPI == kEpiGroup ? warp - (2 + kEpiWarps) : warp - 2;
+      constexpr int kJobs = (kBM + BN) * 4;  // 16-byte packed chunks per stage (A rows, then B rows)
+      constexpr int JPT = (kJobs + NU * 32 - 1) / (NU * 32);
+      // per-lane offsets, the same in every stage: packed source, two swizzled destinations
+      uint32_t src_off[JPT], dst0[JPT], dst1[JPT];
+      bool live[JPT];
 #pragma unroll
-              for (int j = 0; j < CW; ++j) {
-                const int n = min(n0 + j, p.N - 1);
-                const float a = float(int(v[j]) >> 8);
-                y[j] = EPI == kEpiRow ? __fmul_rn(__fmul_rn(a, sxm), __ldg(p.sw + n)) : __fmul_rn(a, __ldg(p.sw + n));
-              }
-              __half* dst = p.Y + size_t(m) * p.N + n0;
-              if (n0 + CW <= p.N) {
-#pragma unroll
-                for (int j = 0; j < CW; j += 8) store_half8(dst + j, y + j);
-              } else {
-                for (int j = 0; j < CW && n0 + j < p.N; ++j) dst[j] = __float2half_rn(y[j]);
-              }
-            } else {
-              int32_t* dst = p.acc + size_t(m) * p.N + n0;
-              for (int j = 0; j < CW; ++j) {
-                if (n0 + j >= p.N) break;
-                const int32_t a = int32_t(v[j]) >> 8;
-                if (EPI == kEpiS32)
-                  dst[j] = a;
-                else
-                  atomicAdd(dst + j, a);
-              }
-            }
-          }
-        } else {
-          // swapped: thread owns output channel n = arow, columns are tokens m
-          const int n = arow;
-          if (n < p.N) {
-            const float swn = (EPI == kEpiRow || EPI == kEpiStatic) ? __ldg(p.sw + n) : 0.f;
-            for (int j = 0; j < CW; ++j) {
-              const int m = bbase + c0 + j;
-              if (m >= p.M) break;
-              const int32_t ai = int32_t(v[j]) >> 8;
-              if (EPI == kEpiRow) {
-                p.Y[size_t(m) * p.N + n] = __float2half_rn(__fmul_rn(__fmul_rn(float(ai), __ldg(p.sx + m)), swn));
-              } else if (EPI == kEpiStatic) {
-                p.Y[size_t(m) * p.N + n] = __float2half_rn(__fmul_rn(float(ai), swn));
-              } else if (EPI == kEpiS32) {
-                p.acc[size_t(m) * p.N + n] = ai;
-              } else {
-                atomicAdd(p.acc + size_t(m) * p.N + n, ai);
-              }
-            }
-          }
-        }
+      for (int it = 0; it < JPT; ++it) {
+        const int j = (it * NU + uw) * 32 + lane;
+        live[it] = j < kJobs;
+        const int row = live[it] ? (j >> 2) : 0, c = j & 3, r7 = row & 7;
+        src_off[it] = uint32_t(row * kPK + c * 16);
+        const uint32_t rb = uint32_t((row >> 3) * 1024 + r7 * 128);
+        dst0[it] = rb + uint32_t(((2 * c) ^ r7) << 4);
+        dst1[it] = rb + uint32_t(((2 * c + 1) ^ r7) << 4);
       }
-    } else {
-      // group-128: one accumulator per K slice, double-buffered in tensor
-      // memory; the running float32 sum lives in columns [2 BN, 3 BN).
-      float* sbuf = reinterpret_cast<float*>(smem + C::OFF_SCALE) + (warp - 2) * BN;
-      const uint32_t tsum = tl + uint32_t(2 * BN);
-      const int m = arow;
-      const bool mok = m < p.M;
       for (int i = 0; i < nkb; ++i) {
-        const int g = kb0 + i, b = i & 1;
-        for (int c = lane; c < BN; c += 32) {
-          const int n = bbase + c;
-          sbuf[c] = n < p.N ? __half2float(p.gsw[size_t(g) * p.N + n]) : 0.f;
-        }
-        const float sxg = mok ? __half2float(p.gsx[size_t(g) * p.M + m]) : 0.f;
-        __syncwarp();
-        if (!warp_wait(&acc_full[b], (i >> 1) & 1)) {
-          if (lane == 0) record_error(p.err, kErrTimeoutEpilogue);
+        const int sp = i % SP, su = i % SU;
+        if (!warp_wait(&full_p[sp], (i / SP) & 1) || !warp_wait(&empty_u[su], ((i / SU) & 1) ^ 1)) {
+          if (lane == 0) record_error(p.err, kErrTimeoutUnpack);
           break;
         }
-        tc_fence_after();
-        for (int c0 = 0; c0 < BN; c0 += 32) {
-          uint32_t v[32], s[32];
-          tmem_ld_32x32(tl + uint32_t(b * BN + c0), v);
-          if (i > 0) tmem_ld_32x32(tsum + c0, s);
-          tmem_wait_ld();
+        const uint8_t* pk = smem + C::OFF_PACK + sp * C::PACK_STAGE;
+        uint8_t* uk = smem + C::OFF_UNP + su * C::UNP_STAGE;
+        uint4 w[JPT];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const float prev = i > 0 ? __uint_as_float(s[j]) : 0.f;
-            const float t = __fmul_rn(sxg, sbuf[c0 + j]);
-            s[j] = __float_as_uint(fmaf(float(int32_t(v[j]) >> 8), t, prev));
-          }
-          tmem_st_32x32(tsum + c0, s);
+        for (int it = 0; it < JPT; ++it)
+          if (live[it]) w[it] = *reinterpret_cast<const uint4*>(pk + src_off[it]);
+#pragma unroll
+        for (int it = 0; it < JPT; ++it) {
+          if (!live[it]) continue;
+          uint4 o0, o1;
+          unpack8_hi(w[it].x, o0.x, o0.y);
+          unpack8_hi(w[it].y, o0.z, o0.w);
+          unpack8_hi(w[it].z, o1.x, o1.y);
+          unpack8_hi(w[it].w, o1.z, o1.w);
+          *reinterpret_cast<uint4*>(uk + dst0[it]) = o0;
+          *reinterpret_cast<uint4*>(uk + dst1[it]) = o1;
         }
-        tmem_wait_st();
-        tc_fence_before();
+        fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&acc_empty[b]);
-      }
-      for (int c0 = 0; c0 < BN; c0 += 32) {
-        uint32_t s[32];
-        tmem_ld_32x32(tsum + c0, s);
-        tmem_wait_ld();
-        if (mok) {
-          const int n0 = bbase + c0;
-          float y[32];
-#pragma unroll
-          for (int j = 0; j < 32; ++j) y[j] = nkb > 0 ? __uint_as_float(s[j]) : 0.f;
-          __half* dst = p.Y + size_t(m) * p.N + n0;
-          if (n0 + 32 <= p.N) {
-#pragma unroll
-            for (int j = 0; j < 32; j += 8) store_half8(dst + j, y + j);
-          } else {
-            for (int j = 0; j < 32 && n0 + j < p.N; ++j) dst[j] = __float2half_rn(y[j]);
-          }
+        if (lane == 0) {
+          mbar_arrive(&full_u[su]);
+          mbar_arrive(&empty_p[sp]);
         }
       }
     }
-  } else {
-    // ------------------------------------------------------------ unpackers
-    const int uw = warp - (2 + kEpiWarps);
-    constexpr int kJobs = (kBM + BN) * 4;  // 16-byte packed chunks per stage (A rows, then B rows)
-    for (int i = 0; i < nkb; ++i) {
-      const int sp = i % SP, su = i % SU;
-      if (!warp_wait(&full_p[sp], (i / SP) & 1) || !warp_wait(&empty_u[su], ((i / SU) & 1) ^ 1)) {
-        if (lane == 0) record_error(p.err, kErrTimeoutUnpack);
-        break;
-      }
-      const uint8_t* pk = smem + C::OFF_PACK + sp * C::PACK_STAGE;
-      uint8_t* uk = smem + C::OFF_UNP + su * C::UNP_STAGE;
-      for (int j = uw * 32 + lane; j < kJobs; j += kUnpackWarps * 32) {
-        const int row = j >> 2, c = j & 3;
-        const uint4 w = *reinterpret_cast<const uint4*>(pk + row * kPK + c * 16);
-        uint4 o0, o1;
-        unpack8_hi(w.x, o0.x, o0.y);
-        unpack8_hi(w.y, o0.z, o0.w);
-        unpack8_hi(w.z, o1.x, o1.y);
-        unpack8_hi(w.w, o1.z, o1.w);
-        uint8_t* rb = uk + (row >> 3) * 1024 + (row & 7) * 128;
-        const int r7 = row & 7;
-        *reinterpret_cast<uint4*>(rb + (((2 * c) ^ r7) << 4)) = o0;
-        *reinterpret_cast<uint4*>(rb + (((2 * c + 1) ^ r7) << 4)) = o1;
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&full_u[su]);
-        mbar_arrive(&empty_p[sp]);
+    if (epi_warp) {
+    // ------------------------------------------------------------ epilogue
+      const int q = warp & 3;  // tensor-memory lane quadrant this warp may access
+      const int rloc = q * 32 + lane;
+      const uint32_t tl = tmem + (uint32_t(q * 32) << 16);
+      const int arow = tileA * kBM + rloc;
+      const int bbase = tileB * BN;
+      if (EPI != kEpiGroup) {
+        if (!warp_wait(&acc_full[0], 0) && lane == 0) record_error(p.err, kErrTimeoutEpilogue);
+        tc_fence_after();
+        constexpr int CW = BN >= 32 ? 32 : 16;
+        for (int c0 = 0; c0 < BN; c0 += CW) {
+          uint32_t v[32];
+          if (CW == 32)
+            tmem_ld_32x32(tl + c0, v);
+          else
+            tmem_ld_32x16(tl + c0, v);
+          tmem_wait_ld();
+          if (!SWAP) {
+            // thread owns token row m = arow, columns n = bbase + c0 + j
+            const int m = arow;
+            if (m < p.M) {
+              const int n0 = bbase + c0;
+              float y[32];
+              if (EPI == kEpiRow || EPI == kEpiStatic) {
+                const float sxm = EPI == kEpiRow ? p.sx[m] : 1.0f;
+  #pragma unroll
+                for (int j = 0; j < CW; ++j) {
+                  const int n = min(n0 + j, p.N - 1);
+                  const float a = float(int(v[j]) >> 8);
+                  y[j] = EPI == kEpiRow ? __fmul_rn(__fmul_rn(a, sxm), __ldg(p.sw + n)) : __fmul_rn(a, __ldg(p.sw + n));
+                }
+                __half* dst = p.Y + size_t(m) * p.N + n0;
+                if (n0 + CW <= p.N) {
+  #pragma unroll
+                  for (int j = 0; j < CW; j += 8) store_half8(dst + j, y + j);
+                } else {
+                  for (int j = 0; j < CW && n0 + j < p.N; ++j) dst[j] = __float2half_rn(y[j]);
+                }
+              } else {
+                int32_t* dst = p.acc + size_t(m) * p.N + n0;
+                for (int j = 0; j < CW; ++j) {
+                  if (n0 + j >= p.N) break;
+                  const int32_t a = int32_t(v[j]) >> 8;
+                  if (EPI == kEpiS32)
+                    dst[j] = a;
+                  else
+                    atomicAdd(dst + j, a);
+                }
+              }
+            }
+          } else {
+            // swapped: thread owns output channel n = arow, columns are tokens m
+            const int n = arow;
+            if (n < p.N) {
+              const float swn = (EPI == kEpiRow || EPI == kEpiStatic) ? __ldg(p.sw + n) : 0.f;
+              for (int j = 0; j < CW; ++j) {
+                const int m = bbase + c0 + j;
+                if (m >= p.M) break;
+                const int32_t ai = int32_t(v[j]) >> 8;
+                if (EPI == kEpiRow) {
+                  p.Y[size_t(m) * p.N + n] = __float2half_rn(__fmul_rn(__fmul_rn(float(ai), __ldg(p.sx + m)), swn));
+                } else if (EPI == kEpiStatic) {
+                  p.Y[size_t(m) * p.N + n] = __float2half_rn(__fmul_rn(float(ai), swn));
+                } else if (EPI == kEpiS32) {
+                  p.acc[size_t(m) * p.N + n] = ai;
+                } else {
+                  atomicAdd(p.acc + size_t(m) * p.N + n, ai);
+                }
+              }
+            }
+          }
+        }
+      } else {
+        // group-128: one accumulator per K slice, double-buffered in tensor
+        // memory; the running float32 sum lives in columns [2 BN, 3 BN).
+        float* sbuf = reinterpret_cast<float*>(smem + C::OFF_SCALE) + (warp - 2) * BN;
+        const uint32_t tsum = tl + uint32_t(2 * BN);
+        const int m = arow;
+        const bool mok = m < p.M;
+        for (int i = 0; i < nkb; ++i) {
+          const int g = kb0 + i, b = i & 1;
+          for (int c = lane; c < BN; c += 32) {
+            const int n = bbase + c;
+            sbuf[c] = n < p.N ? __half2float(p.gsw[size_t(g) * p.N + n]) : 0.f;
+          }
+          const float sxg = mok ? __half2float(p.gsx[size_t(g) * p.M + m]) : 0.f;
+          __syncwarp();
+          if (!warp_wait(&acc_full[b], (i >> 1) & 1)) {
+            if (lane == 0) record_error(p.err, kErrTimeoutEpilogue);
+            break;
+          }
+          tc_fence_after();
+          for (int c0 = 0; c0 < BN; c0 += 32) {
+            uint32_t v[32], s[32];
+            tmem_ld_32x32(tl + uint32_t(b * BN + c0), v);
+            if (i > 0) tmem_ld_32x32(tsum + c0, s);
+            tmem_wait_ld();
+  #pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const float prev = i > 0 ? __uint_as_float(s[j]) : 0.f;
+              const float t = __fmul_rn(sxg, sbuf[c0 + j]);
+              s[j] = __float_as_uint(fmaf(float(int32_t(v[j]) >> 8), t, prev));
+            }
+            tmem_st_32x32(tsum + c0, s);
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[b]);
+        }
+        for (int c0 = 0; c0 < BN; c0 += 32) {
+          uint32_t s[32];
+          tmem_ld_32x32(tsum + c0, s);
+          tmem_wait_ld();
+          if (mok) {
+            const int n0 = bbase + c0;
+            float y[32];
+  #pragma unroll
+            for (int j = 0; j < 32; ++j) y[j] = nkb > 0 ? __uint_as_float(s[j]) : 0.f;
+            __half* dst = p.Y + size_t(m) * p.N + n0;
+            if (n0 + 32 <= p.N) {
+  #pragma unroll
+              for (int j = 0; j < 32; j += 8) store_half8(dst + j, y + j);
+            } else {
+              for (int j = 0; j < 32 && n0 + j < p.N; ++j) dst[j] = __float2half_rn(y[j]);
+            }
+          }
+        }
       }
     }
   }
