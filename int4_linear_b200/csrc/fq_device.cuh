@@ -279,15 +279,14 @@ __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.
 // Four packed bytes (codes e0..e7, e(2j) in the low nibble of byte j) to
 // eight int8 bytes holding 16 * e: the nibble is moved to the high half of
 // its byte, which makes it a signed int8 without a sign-extension step.
+// The bytes come out as [e0 e2 e4 e6] [e1 e3 e5 e7]: a fixed permutation of
+// K inside each 128-deep slice, applied identically to both GEMM operands,
+// leaves every dot product unchanged and saves the byte interleaving.
 // The MMA then accumulates 256 * (sum of code products), removed exactly by
 // an arithmetic shift in the epilogue.
 __device__ __forceinline__ void unpack8_hi(uint32_t w, uint32_t& lo4, uint32_t& hi4) {
-  const uint32_t s = w << 4;
-  uint32_t a, b;
-  asm("prmt.b32 %0, %1, %2, 0x5140;" : "=r"(a) : "r"(s), "r"(w));
-  asm("prmt.b32 %0, %1, %2, 0x7362;" : "=r"(b) : "r"(s), "r"(w));
-  lo4 = a & 0xF0F0F0F0u;
-  hi4 = b & 0xF0F0F0F0u;
+  lo4 = (w << 4) & 0xF0F0F0F0u;
+  hi4 = w & 0xF0F0F0F0u;
 }
 
 }  // namespace fq

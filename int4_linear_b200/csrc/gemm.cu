@@ -6,13 +6,19 @@
 // 核心思想: Y ~ Q(XP) Q(P^-1 W^T) with integer accumulation).
 //
 // Warp roles inside one CTA (one 128 x BN output tile, a K range):
-//   warp 0      TMA producer: packed A/B slices into a ring of SP stages
 //   warp 1      tensor-memory allocation and the single MMA-issuing thread
 //   warps 2-5   epilogue: tcgen05.ld of the accumulator, dequantization, stores
-//   warps 6-13  unpackers: packed stage -> int8 stage in the 128-byte
-//               swizzled K-major layout the MMA descriptors describe
-// Stages are handed over with mbarriers; every wait is bounded and a wait
-// that gives up records a timeout code in the device error word.
+//               (outside group mode they first unpack with the others)
+//   warps 6-13  unpackers: each lane owns fixed 16-byte packed pieces of the
+//               A/B slices, loads them from global memory several K slices
+//               ahead into registers, and writes them as int8 into a ring of
+//               SU stages in the 128-byte swizzled K-major layout that the
+//               MMA descriptors describe.
+// The packed operands never pass through shared memory: shared-memory
+// bandwidth (unpacked writes plus the tensor core's operand reads) is what
+// bounds this kernel, so the packed round trip a TMA stage would add is left
+// out.  Stages are handed over with mbarriers; every wait is bounded and a
+// wait that gives up records a timeout code in the device error word.
 //
 // The nibble is unpacked into the high half of its byte (16 q, see
 // unpack8_hi), so the tensor core accumulates 256 * sum(qx qw); the epilogue
@@ -52,30 +58,29 @@ __host__ __device__ constexpr int unpack_warps() { return EPI == kEpiGroup ? kUn
 
 template <int BN, int EPI>
 struct Cfg {
-  static constexpr int SP = BN >= 128 ? 4 : (BN >= 64 ? 6 : 8);
-  static constexpr int SU = EPI == kEpiGroup ? 3 : 2;
-  static constexpr int A_PACK = kBM * kPK;
-  static constexpr int B_PACK = BN * kPK;
+  static constexpr int SU = 4;                 // unpacked stages
   static constexpr int A_UNP = kBM * kBK;
   static constexpr int B_UNP = BN * kBK;
   static constexpr int TMEM_COLS = EPI == kEpiGroup ? 512 : (BN < 32 ? 32 : BN);
   static constexpr int UNP_STAGE = A_UNP + B_UNP;
-  static constexpr int PACK_STAGE = A_PACK + B_PACK;
   static constexpr int OFF_UNP = 0;
-  static constexpr int OFF_PACK = OFF_UNP + SU * UNP_STAGE;
-  static constexpr int OFF_SCALE = OFF_PACK + SP * PACK_STAGE;
+  static constexpr int OFF_SCALE = OFF_UNP + SU * UNP_STAGE;
   static constexpr int SCALE_BYTES = EPI == kEpiGroup ? kEpiWarps * BN * 4 : 0;
   static constexpr int OFF_BAR = OFF_SCALE + SCALE_BYTES;
-  static constexpr int NBAR = 2 * SP + 2 * SU + 5;
+  static constexpr int NBAR = 2 * SU + 5;
   static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
   static constexpr int SMEM = OFF_TMEM + 16 + 1024;  // + slack to align the base to 1024
+  // the fp16 output tile is staged in the (then idle) unpacked ring, rows padded by 16 bytes
+  static constexpr int OUT_PITCH = 2 * BN + 16;
   static_assert(UNP_STAGE % 1024 == 0, "unpacked stages must keep 1024-byte alignment");
-  static_assert(PACK_STAGE % 128 == 0, "packed stages must keep 128-byte alignment");
+  static_assert(kBM * OUT_PITCH <= SU * UNP_STAGE, "output tile fits in the ring");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
   static_assert(EPI != kEpiGroup || 3 * BN <= 512, "group epilogue needs 3 x BN tensor-memory columns");
 };
 
 struct GemmParams {
+  const uint8_t* A;   // packed operand on the 128-row side: [rowsA][K/2]
+  const uint8_t* B;   // packed operand on the BN-row side:  [rowsB][K/2]
   int M, N, K;        // Y is [M][N]
   int rowsA, rowsB;   // rows of the A (128-row tiles) and B (BN-row tiles) operands
   int num_kb;         // K / 128
@@ -98,17 +103,13 @@ __device__ __forceinline__ void store_half8(__half* dst, const float* v) {
 }
 
 template <int BN, int EPI, bool SWAP>
-__global__ void __launch_bounds__(kThreads, 1)
-    gemm_w4a4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                     const GemmParams p) {
+__global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(const GemmParams p) {
   using C = Cfg<BN, EPI>;
-  constexpr int SP = C::SP, SU = C::SU;
+  constexpr int SU = C::SU;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-  uint64_t* full_p = bars;
-  uint64_t* empty_p = full_p + SP;
-  uint64_t* full_u = empty_p + SP;
+  uint64_t* full_u = bars;
   uint64_t* empty_u = full_u + SU;
   uint64_t* acc_full = empty_u + SU;
   uint64_t* acc_empty = acc_full + 2;
@@ -121,10 +122,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nkb = max(0, min(p.num_kb, kb0 + p.kb_per_split) - kb0);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < SP; ++s) {
-      mbar_init(&full_p[s], 1);
-      mbar_init(&empty_p[s], unpack_warps<EPI>());
-    }
     for (int s = 0; s < SU; ++s) {
       mbar_init(&full_u[s], unpack_warps<EPI>());
       mbar_init(&empty_u[s], 1);
@@ -136,10 +133,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(done_bar, 1);
     fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) {
-    prefetch_tensormap(&tmA);
-    prefetch_tensormap(&tmB);
-  }
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
@@ -150,26 +143,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      int issued = 0;
-      for (int i = 0; i < nkb; ++i) {
-        const int s = i % SP;
-        if (!mbar_wait(&empty_p[s], ((i / SP) & 1) ^ 1)) {
-          record_error(p.err, kErrTimeoutProducer);
-          break;
-        }
-        uint8_t* pa = smem + C::OFF_PACK + s * C::PACK_STAGE;
-        mbar_arrive_expect_tx(&full_p[s], C::PACK_STAGE);
-        const int kx = (kb0 + i) * kPK;
-        tma_load_2d(pa, &tmA, &full_p[s], kx, tileA * kBM);
-        tma_load_2d(pa + C::A_PACK, &tmB, &full_p[s], kx, tileB * BN);
-        ++issued;
-      }
-      // Every load this thread issued has landed before the CTA can exit.
-      for (int i = max(0, issued - SP); i < issued; ++i)
-        if (!mbar_wait(&full_p[i % SP], (i / SP) & 1)) record_error(p.err, kErrTimeoutDrain);
-    }
+    // idle: joins the final barrier
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -213,49 +187,77 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool epi_warp = warp < 2 + kEpiWarps;
     if (!epi_warp || EPI != kEpiGroup) {
       const int uw = EPI == kEpiGroup ? warp - (2 + kEpiWarps) : warp - 2;
-      constexpr int kJobs = (kBM + BN) * 4;  // 16-byte packed chunks per stage (A rows, then B rows)
+      constexpr int kJobs = (kBM + BN) * 4;  // 16-byte packed pieces per stage (A rows, then B rows)
       constexpr int JPT = (kJobs + NU * 32 - 1) / (NU * 32);
-      // per-lane offsets, the same in every stage: packed source, two swizzled destinations
-      uint32_t src_off[JPT], dst0[JPT], dst1[JPT];
-      bool live[JPT];
+      constexpr int D = SWAP ? 6 : 3;  // K slices of packed data in flight per thread
+      // per-lane pieces, the same in every stage: global source row, two swizzled destinations
+      const uint8_t* gsrc[JPT];
+      uint32_t dst0[JPT], dst1[JPT];
+      bool live[JPT], load_ok[JPT];
+      const size_t ld = size_t(p.K) / 2;
 #pragma unroll
       for (int it = 0; it < JPT; ++it) {
         const int j = (it * NU + uw) * 32 + lane;
         live[it] = j < kJobs;
         const int row = live[it] ? (j >> 2) : 0, c = j & 3, r7 = row & 7;
-        src_off[it] = uint32_t(row * kPK + c * 16);
         const uint32_t rb = uint32_t((row >> 3) * 1024 + r7 * 128);
         dst0[it] = rb + uint32_t(((2 * c) ^ r7) << 4);
         dst1[it] = rb + uint32_t(((2 * c + 1) ^ r7) << 4);
-      }
-      for (int i = 0; i < nkb; ++i) {
-        const int sp = i % SP, su = i % SU;
-        if (!warp_wait(&full_p[sp], (i / SP) & 1) || !warp_wait(&empty_u[su], ((i / SU) & 1) ^ 1)) {
-          if (lane == 0) record_error(p.err, kErrTimeoutUnpack);
-          break;
+        int grow;
+        const uint8_t* base;
+        if (row < kBM) {
+          grow = tileA * kBM + row;
+          base = p.A;
+          load_ok[it] = live[it] && grow < p.rowsA;
+        } else {
+          grow = tileB * BN + (row - kBM);
+          base = p.B;
+          load_ok[it] = live[it] && grow < p.rowsB;
         }
-        const uint8_t* pk = smem + C::OFF_PACK + sp * C::PACK_STAGE;
-        uint8_t* uk = smem + C::OFF_UNP + su * C::UNP_STAGE;
-        uint4 w[JPT];
+        gsrc[it] = base + (load_ok[it] ? size_t(grow) * ld : 0) + size_t(kb0) * kPK + c * 16;
+      }
+      uint4 w[D][JPT];
+#pragma unroll
+      for (int d = 0; d < D; ++d) {
 #pragma unroll
         for (int it = 0; it < JPT; ++it)
-          if (live[it]) w[it] = *reinterpret_cast<const uint4*>(pk + src_off[it]);
+          w[d][it] = (d < nkb && load_ok[it]) ? __ldg(reinterpret_cast<const uint4*>(gsrc[it] + d * kPK))
+                                              : make_uint4(0, 0, 0, 0);
+      }
+      bool ok = true;
+      for (int i0 = 0; i0 < nkb && ok; i0 += D) {
 #pragma unroll
-        for (int it = 0; it < JPT; ++it) {
-          if (!live[it]) continue;
-          uint4 o0, o1;
-          unpack8_hi(w[it].x, o0.x, o0.y);
-          unpack8_hi(w[it].y, o0.z, o0.w);
-          unpack8_hi(w[it].z, o1.x, o1.y);
-          unpack8_hi(w[it].w, o1.z, o1.w);
-          *reinterpret_cast<uint4*>(uk + dst0[it]) = o0;
-          *reinterpret_cast<uint4*>(uk + dst1[it]) = o1;
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&full_u[su]);
-          mbar_arrive(&empty_p[sp]);
+        for (int d = 0; d < D; ++d) {
+          const int i = i0 + d;
+          if (i >= nkb) break;
+          const int su = i % SU;
+          if (!warp_wait(&empty_u[su], ((i / SU) & 1) ^ 1)) {
+            if (lane == 0) record_error(p.err, kErrTimeoutUnpack);
+            ok = false;
+            break;
+          }
+          uint8_t* uk = smem + C::OFF_UNP + su * C::UNP_STAGE;
+#pragma unroll
+          for (int it = 0; it < JPT; ++it) {
+            if (!live[it]) continue;
+            uint4 o0, o1;
+            unpack8_hi(w[d][it].x, o0.x, o0.y);
+            unpack8_hi(w[d][it].y, o0.z, o0.w);
+            unpack8_hi(w[d][it].z, o1.x, o1.y);
+            unpack8_hi(w[d][it].w, o1.z, o1.w);
+            *reinterpret_cast<uint4*>(uk + dst0[it]) = o0;
+            *reinterpret_cast<uint4*>(uk + dst1[it]) = o1;
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&full_u[su]);
+          // refill this register slot with the slice D steps ahead
+          if (i + D < nkb) {
+#pragma unroll
+            for (int it = 0; it < JPT; ++it)
+              w[d][it] = load_ok[it] ? __ldg(reinterpret_cast<const uint4*>(gsrc[it] + (i + D) * kPK))
+                                     : make_uint4(0, 0, 0, 0);
+          }
         }
       }
     }
@@ -291,13 +293,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                   const float a = float(int(v[j]) >> 8);
                   y[j] = EPI == kEpiRow ? __fmul_rn(__fmul_rn(a, sxm), __ldg(p.sw + n)) : __fmul_rn(a, __ldg(p.sw + n));
                 }
-                __half* dst = p.Y + size_t(m) * p.N + n0;
-                if (n0 + CW <= p.N) {
+                // staged in shared memory; written out coalesced after the barrier below
+                __half* dst = reinterpret_cast<__half*>(smem + C::OFF_UNP + rloc * C::OUT_PITCH) + c0;
   #pragma unroll
-                  for (int j = 0; j < CW; j += 8) store_half8(dst + j, y + j);
-                } else {
-                  for (int j = 0; j < CW && n0 + j < p.N; ++j) dst[j] = __float2half_rn(y[j]);
-                }
+                for (int j = 0; j < CW; j += 8) store_half8(dst + j, y + j);
               } else {
                 int32_t* dst = p.acc + size_t(m) * p.N + n0;
                 for (int j = 0; j < CW; ++j) {
@@ -374,21 +373,32 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t s[32];
           tmem_ld_32x32(tsum + c0, s);
           tmem_wait_ld();
-          if (mok) {
-            const int n0 = bbase + c0;
+          {
             float y[32];
   #pragma unroll
             for (int j = 0; j < 32; ++j) y[j] = nkb > 0 ? __uint_as_float(s[j]) : 0.f;
-            __half* dst = p.Y + size_t(m) * p.N + n0;
-            if (n0 + 32 <= p.N) {
+            __half* dst = reinterpret_cast<__half*>(smem + C::OFF_UNP + rloc * C::OUT_PITCH) + c0;
   #pragma unroll
-              for (int j = 0; j < 32; j += 8) store_half8(dst + j, y + j);
-            } else {
-              for (int j = 0; j < 32 && n0 + j < p.N; ++j) dst[j] = __float2half_rn(y[j]);
-            }
+            for (int j = 0; j < 32; j += 8) store_half8(dst + j, y + j);
           }
         }
       }
+    }
+  }
+
+  // fp16 tiles staged in shared memory leave as whole 512-byte row segments
+  constexpr bool kStaged = !SWAP && (EPI == kEpiRow || EPI == kEpiStatic || EPI == kEpiGroup);
+  if (kStaged) {
+    __syncthreads();
+    const int n0 = tileB * BN;
+    const int chunks = max(0, min(BN, p.N - n0)) / 8;  // 16-byte chunks per row (N % 8 == 0)
+    for (int r = warp; r < kBM; r += kThreads / 32) {
+      const int m = tileA * kBM + r;
+      if (m >= p.M) break;
+      const uint8_t* src = smem + C::OFF_UNP + r * C::OUT_PITCH;
+      __half* dst = p.Y + size_t(m) * p.N + n0;
+      for (int c = lane; c < chunks; c += 32)
+        *reinterpret_cast<uint4*>(dst + c * 8) = *reinterpret_cast<const uint4*>(src + c * 16);
     }
   }
 
@@ -470,34 +480,32 @@ Plan make_plan(int M, int N, int K, int epi_final, int sms) {
 }
 
 template <int BN, int EPI, bool SWAP>
-fq_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& gp, dim3 grid,
-                      cudaStream_t stream) {
+fq_status launch_gemm(const GemmParams& gp, dim3 grid, cudaStream_t stream) {
   using C = Cfg<BN, EPI>;
   auto kern = gemm_w4a4_kernel<BN, EPI, SWAP>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess ||
       cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
     return fail(FQ_ERR_CUDA, "cannot reserve %d bytes of shared memory for the GEMM", C::SMEM);
-  kern<<<grid, kThreads, C::SMEM, stream>>>(ta, tb, gp);
+  kern<<<grid, kThreads, C::SMEM, stream>>>(gp);
   return check_launch("gemm_w4a4_kernel");
 }
 
-fq_status dispatch(const Plan& pl, const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& gp, dim3 grid,
-                   cudaStream_t s) {
+fq_status dispatch(const Plan& pl, const GemmParams& gp, dim3 grid, cudaStream_t s) {
   if (!pl.swap) {
     switch (pl.epi) {
-      case kEpiRow: return launch_gemm<256, kEpiRow, false>(ta, tb, gp, grid, s);
-      case kEpiStatic: return launch_gemm<256, kEpiStatic, false>(ta, tb, gp, grid, s);
-      case kEpiS32: return launch_gemm<256, kEpiS32, false>(ta, tb, gp, grid, s);
-      case kEpiGroup: return launch_gemm<128, kEpiGroup, false>(ta, tb, gp, grid, s);
+      case kEpiRow: return launch_gemm<256, kEpiRow, false>(gp, grid, s);
+      case kEpiStatic: return launch_gemm<256, kEpiStatic, false>(gp, grid, s);
+      case kEpiS32: return launch_gemm<256, kEpiS32, false>(gp, grid, s);
+      case kEpiGroup: return launch_gemm<128, kEpiGroup, false>(gp, grid, s);
       default: break;
     }
   } else {
 #define FQ_SWAP_CASES(BNV)                                                           \
   if (pl.bn == BNV) {                                                                \
     switch (pl.epi) {                                                                \
-      case kEpiRow: return launch_gemm<BNV, kEpiRow, true>(ta, tb, gp, grid, s);       \
-      case kEpiStatic: return launch_gemm<BNV, kEpiStatic, true>(ta, tb, gp, grid, s); \
-      case kEpiAtomic: return launch_gemm<BNV, kEpiAtomic, true>(ta, tb, gp, grid, s); \
+      case kEpiRow: return launch_gemm<BNV, kEpiRow, true>(gp, grid, s);       \
+      case kEpiStatic: return launch_gemm<BNV, kEpiStatic, true>(gp, grid, s); \
+      case kEpiAtomic: return launch_gemm<BNV, kEpiAtomic, true>(gp, grid, s); \
       default: break;                                                                \
     }                                                                                \
   }
@@ -552,23 +560,16 @@ fq_status gemm_impl(const uint8_t* Xq, const void* s_x, const uint8_t* Wq, const
   }
   gp.acc = epi_final == kEpiS32 ? acc_out : (pl.splits > 1 ? static_cast<int32_t*>(ws) : nullptr);
 
-  const uint8_t* A = pl.swap ? Wq : Xq;
-  const uint8_t* B = pl.swap ? Xq : Wq;
+  gp.A = pl.swap ? Wq : Xq;
+  gp.B = pl.swap ? Xq : Wq;
   gp.rowsA = pl.swap ? N : M;
   gp.rowsB = pl.swap ? M : N;
-  CUtensorMap ta, tb;
-  st = make_tmap_2d(&ta, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, uint64_t(K / 2), uint64_t(gp.rowsA), uint64_t(K / 2),
-                    kPK, kBM);
-  if (st != FQ_OK) return st;
-  st = make_tmap_2d(&tb, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, uint64_t(K / 2), uint64_t(gp.rowsB), uint64_t(K / 2),
-                    kPK, uint32_t(pl.bn));
-  if (st != FQ_OK) return st;
 
   const dim3 grid((gp.rowsA + kBM - 1) / kBM, (gp.rowsB + pl.bn - 1) / pl.bn, pl.splits);
   if (pl.splits > 1) {
     if (cudaMemsetAsync(ws, 0, need, stream) != cudaSuccess) return fail(FQ_ERR_CUDA, "workspace clear failed");
   }
-  st = dispatch(pl, ta, tb, gp, grid, stream);
+  st = dispatch(pl, gp, grid, stream);
   if (st != FQ_OK) return st;
   if (pl.splits > 1) {
     const int threads = 256;
