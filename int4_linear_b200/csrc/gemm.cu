@@ -51,18 +51,26 @@ constexpr int kEpiWarps = 4;
 constexpr int kUnpackWarps = 8;
 constexpr int kThreads = 32 * (2 + kEpiWarps + kUnpackWarps);
 
-// Warps that unpack: the dedicated 8, plus the 4 epilogue warps when the
-// epilogue only runs after the main loop (every mode but group-128).
+// Warps that feed a stage: 4 A-warps (one per tensor-memory lane quadrant)
+// write the unpacked A rows into tensor memory; the B-warps write the
+// unpacked B rows into shared memory.  Outside group mode the A-warps are
+// the epilogue warps (the epilogue runs after the main loop); in group mode
+// the epilogue runs alongside, so warps 6..9 take A and 10..13 take B.
 template <int EPI>
-__host__ __device__ constexpr int unpack_warps() { return EPI == kEpiGroup ? kUnpackWarps : kUnpackWarps + kEpiWarps; }
+__host__ __device__ constexpr int b_warps() { return EPI == kEpiGroup ? kUnpackWarps - 4 : kUnpackWarps; }
+template <int EPI>
+__host__ __device__ constexpr int feed_warps() { return 4 + b_warps<EPI>(); }
 
-template <int BN, int EPI>
+template <int BN, int EPI, bool SWAP>
 struct Cfg {
-  static constexpr int SU = 4;                 // unpacked stages
-  static constexpr int A_UNP = kBM * kBK;
+  static constexpr int SU = 4;                 // unpacked stages (A in tensor memory, B in shared memory)
   static constexpr int B_UNP = BN * kBK;
-  static constexpr int TMEM_COLS = EPI == kEpiGroup ? 512 : (BN < 32 ? 32 : BN);
-  static constexpr int UNP_STAGE = A_UNP + B_UNP;
+  static constexpr int ACC_COLS = EPI == kEpiGroup ? 3 * BN : BN;
+  static constexpr int A_COL0 = ((ACC_COLS + 31) / 32) * 32;   // tensor-memory columns of the A ring
+  static constexpr int A_STAGE_COLS = kBK / 4;                 // 4 int8 per 32-bit column
+  static constexpr int TMEM_NEED = A_COL0 + SU * A_STAGE_COLS;
+  static constexpr int TMEM_COLS = TMEM_NEED <= 64 ? 64 : (TMEM_NEED <= 128 ? 128 : (TMEM_NEED <= 256 ? 256 : 512));
+  static constexpr int UNP_STAGE = B_UNP;
   static constexpr int OFF_UNP = 0;
   static constexpr int OFF_SCALE = OFF_UNP + SU * UNP_STAGE;
   static constexpr int SCALE_BYTES = EPI == kEpiGroup ? kEpiWarps * BN * 4 : 0;
@@ -73,7 +81,8 @@ struct Cfg {
   // the fp16 output tile is staged in the (then idle) unpacked ring, rows padded by 16 bytes
   static constexpr int OUT_PITCH = 2 * BN + 16;
   static_assert(UNP_STAGE % 1024 == 0, "unpacked stages must keep 1024-byte alignment");
-  static_assert(kBM * OUT_PITCH <= SU * UNP_STAGE, "output tile fits in the ring");
+  static_assert(SWAP || kBM * OUT_PITCH <= SU * UNP_STAGE, "output tile fits in the ring");
+  static_assert(TMEM_NEED <= 512, "tensor memory");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
   static_assert(EPI != kEpiGroup || 3 * BN <= 512, "group epilogue needs 3 x BN tensor-memory columns");
 };
@@ -104,7 +113,7 @@ __device__ __forceinline__ void store_half8(__half* dst, const float* v) {
 
 template <int BN, int EPI, bool SWAP>
 __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(const GemmParams p) {
-  using C = Cfg<BN, EPI>;
+  using C = Cfg<BN, EPI, SWAP>;
   constexpr int SU = C::SU;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -123,7 +132,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(const GemmParams
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < SU; ++s) {
-      mbar_init(&full_u[s], unpack_warps<EPI>());
+      mbar_init(&full_u[s], feed_warps<EPI>());
       mbar_init(&empty_u[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -165,12 +174,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(const GemmParams
           break;
         }
         tc_fence_after();
-        const uint32_t a0 = smem_u32(smem + C::OFF_UNP + su * C::UNP_STAGE);
-        const uint32_t b0 = a0 + C::A_UNP;
+        const uint32_t a0 = tmem + uint32_t(C::A_COL0 + su * C::A_STAGE_COLS);
+        const uint32_t b0 = smem_u32(smem + C::OFF_UNP + su * C::UNP_STAGE);
 #pragma unroll
         for (int k = 0; k < kBK / 32; ++k) {
           const uint32_t accum = EPI == kEpiGroup ? uint32_t(k > 0) : uint32_t(i > 0 || k > 0);
-          mma_i8(d, sdesc_k128_sw128(a0 + 32 * k), sdesc_k128_sw128(b0 + 32 * k), idesc, accum);
+          mma_i8_ts(d, a0 + uint32_t(8 * k), sdesc_k128_sw128(b0 + 32 * k), idesc, accum);
         }
         mma_commit(&empty_u[su]);
         if (EPI == kEpiGroup) mma_commit(&acc_full[i & 1]);
@@ -180,41 +189,82 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(const GemmParams
       if (!mbar_wait(done_bar, 0)) record_error(p.err, kErrTimeoutDrain);
     }
   } else {
-    // ------------------------------------------------------------ unpackers
-    // Warps 6..13 always unpack; in the modes whose epilogue runs after the
-    // main loop, warps 2..5 unpack too and then turn to the epilogue.
-    constexpr int NU = unpack_warps<EPI>();
+    // ------------------------------------------------------------ feeders
+    constexpr int NB = b_warps<EPI>();
     const bool epi_warp = warp < 2 + kEpiWarps;
-    if (!epi_warp || EPI != kEpiGroup) {
-      const int uw = EPI == kEpiGroup ? warp - (2 + kEpiWarps) : warp - 2;
-      constexpr int kJobs = (kBM + BN) * 4;  // 16-byte packed pieces per stage (A rows, then B rows)
-      constexpr int JPT = (kJobs + NU * 32 - 1) / (NU * 32);
-      constexpr int D = SWAP ? 6 : 3;  // K slices of packed data in flight per thread
+    const bool a_warp = EPI == kEpiGroup ? (warp >= 6 && warp < 10) : epi_warp;
+    const bool b_warp = EPI == kEpiGroup ? (warp >= 10) : (warp >= 6);
+    const size_t ld = size_t(p.K) / 2;
+    if (a_warp) {
+      constexpr int D = SWAP ? 4 : 3;  // K slices of packed A in flight per thread
+      // one A row per thread (its tensor-memory lane): 64 packed bytes per slice
+      const int q = warp & 3;
+      const int row = q * 32 + lane;
+      const int grow = tileA * kBM + row;
+      const bool ok_row = grow < p.rowsA;
+      const uint8_t* src = p.A + (ok_row ? size_t(grow) * ld : 0) + size_t(kb0) * kPK;
+      const uint32_t ta = tmem + (uint32_t(q * 32) << 16) + uint32_t(C::A_COL0);
+      uint4 w[D][4];
+#pragma unroll
+      for (int d = 0; d < D; ++d)
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          w[d][c] = (d < nkb && ok_row) ? __ldg(reinterpret_cast<const uint4*>(src + d * kPK + c * 16))
+                                        : make_uint4(0, 0, 0, 0);
+      bool ok = true;
+      for (int i0 = 0; i0 < nkb && ok; i0 += D) {
+#pragma unroll
+        for (int d = 0; d < D; ++d) {
+          const int i = i0 + d;
+          if (i >= nkb) break;
+          const int su = i % SU;
+          if (!warp_wait(&empty_u[su], ((i / SU) & 1) ^ 1)) {
+            if (lane == 0) record_error(p.err, kErrTimeoutUnpack);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          uint32_t r[32];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            unpack8_hi(w[d][c].x, r[8 * c + 0], r[8 * c + 1]);
+            unpack8_hi(w[d][c].y, r[8 * c + 2], r[8 * c + 3]);
+            unpack8_hi(w[d][c].z, r[8 * c + 4], r[8 * c + 5]);
+            unpack8_hi(w[d][c].w, r[8 * c + 6], r[8 * c + 7]);
+          }
+          tmem_st_32x32(ta + uint32_t(su * C::A_STAGE_COLS), r);
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&full_u[su]);
+          if (i + D < nkb) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+              w[d][c] = ok_row ? __ldg(reinterpret_cast<const uint4*>(src + (i + D) * kPK + c * 16))
+                               : make_uint4(0, 0, 0, 0);
+          }
+        }
+      }
+    } else if (b_warp) {
+      constexpr int D = SWAP ? 6 : 3;  // K slices of packed B in flight per thread
+      const int uw = EPI == kEpiGroup ? warp - 10 : warp - 6;
+      constexpr int kJobs = BN * 4;  // 16-byte packed pieces of B per stage
+      constexpr int JPT = (kJobs + NB * 32 - 1) / (NB * 32);
       // per-lane pieces, the same in every stage: global source row, two swizzled destinations
       const uint8_t* gsrc[JPT];
       uint32_t dst0[JPT], dst1[JPT];
       bool live[JPT], load_ok[JPT];
-      const size_t ld = size_t(p.K) / 2;
 #pragma unroll
       for (int it = 0; it < JPT; ++it) {
-        const int j = (it * NU + uw) * 32 + lane;
+        const int j = (it * NB + uw) * 32 + lane;
         live[it] = j < kJobs;
         const int row = live[it] ? (j >> 2) : 0, c = j & 3, r7 = row & 7;
         const uint32_t rb = uint32_t((row >> 3) * 1024 + r7 * 128);
         dst0[it] = rb + uint32_t(((2 * c) ^ r7) << 4);
         dst1[it] = rb + uint32_t(((2 * c + 1) ^ r7) << 4);
-        int grow;
-        const uint8_t* base;
-        if (row < kBM) {
-          grow = tileA * kBM + row;
-          base = p.A;
-          load_ok[it] = live[it] && grow < p.rowsA;
-        } else {
-          grow = tileB * BN + (row - kBM);
-          base = p.B;
-          load_ok[it] = live[it] && grow < p.rowsB;
-        }
-        gsrc[it] = base + (load_ok[it] ? size_t(grow) * ld : 0) + size_t(kb0) * kPK + c * 16;
+        const int grow = tileB * BN + row;
+        load_ok[it] = live[it] && grow < p.rowsB;
+        gsrc[it] = p.B + (load_ok[it] ? size_t(grow) * ld : 0) + size_t(kb0) * kPK + c * 16;
       }
       uint4 w[D][JPT];
 #pragma unroll
@@ -481,7 +531,7 @@ Plan make_plan(int M, int N, int K, int epi_final, int sms) {
 
 template <int BN, int EPI, bool SWAP>
 fq_status launch_gemm(const GemmParams& gp, dim3 grid, cudaStream_t stream) {
-  using C = Cfg<BN, EPI>;
+  using C = Cfg<BN, EPI, SWAP>;
   auto kern = gemm_w4a4_kernel<BN, EPI, SWAP>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess ||
       cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
