@@ -83,6 +83,7 @@ class ClockSampler:
         self.dev_id = dev_id
         self.proc = None
         self.lines = []
+        self.active = True  # samples are kept only while active (the timed regions)
 
     def start(self):
         try:
@@ -96,7 +97,8 @@ class ClockSampler:
 
     def _read(self):
         for ln in self.proc.stdout:
-            self.lines.append(ln.strip())
+            if self.active:
+                self.lines.append(ln.strip())
 
     def stop(self):
         if self.proc is None:
@@ -314,6 +316,185 @@ def run_ours(args, ws, rank, local):
     return out
 
 
+# ---------------------------------------------------------------- the other workloads, one line each
+#
+# --workload transform_quant | group | decode measures one kernel family on
+# its own workload against its own roofline.  Each launch is timed by its own
+# CUDA-event pair with an L2 flush (a 256 MiB write) between launches, outside
+# the timed pair, because these inputs alone may fit in the 126 MB L2.
+
+class LaunchTimer:
+    def __init__(self, dev, stream, clocks):
+        import torch
+        self.torch = torch
+        self.stream = stream
+        self.clocks = clocks
+        clocks.active = False
+        self.flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def time(self, fn, steps, warmup):
+        torch = self.torch
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        self.clocks.active = True
+        for a, b in evs:
+            self.flush_buf.fill_(1)
+            a.record(self.stream)
+            fn()
+            b.record(self.stream)
+        torch.cuda.synchronize()
+        self.clocks.active = False
+        ms = sorted(a.elapsed_time(b) for a, b in evs)
+        return ms[len(ms) // 2]
+
+
+def _suite_common(args, dev_index):
+    import torch
+
+    from int4_linear_b200 import fq
+    torch.cuda.set_device(dev_index)
+    dev = torch.device("cuda", dev_index)
+    fq.lib()
+    stream = torch.cuda.current_stream(dev)
+    dev_uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    clocks = ClockSampler(dev_uuid if dev_uuid.startswith("GPU-") else f"GPU-{dev_uuid}")
+    return torch, fq, dev, stream, clocks
+
+
+def run_transform_quant(args, dev_index):
+    """The transform + per-token quantization workload on its own: X [2048, 4096]
+    with 1% outlier channels x30 and a x100 pivot token, Kronecker (64, 64),
+    c ~ U[0.5, 2], alpha_a = 0.9.  Roofline: HBM."""
+    torch, fq, dev, stream, clocks = _suite_common(args, dev_index)
+    d = synth.transform_quant()
+    x = torch.from_numpy(d["x"]).to(dev)
+    t = fq.Transform(torch.from_numpy(d["p1"]).to(dev), torch.from_numpy(d["p2"]).to(dev),
+                     torch.from_numpy(d["c"]).to(dev))
+    qp = fq.qparams(fq.ROW, d["alpha_a"])
+    xq = torch.empty(d["m"], d["k"] // 2, dtype=torch.uint8, device=dev)
+    sx = torch.empty(d["m"], dtype=torch.float32, device=dev)
+    timer = LaunchTimer(dev, stream, clocks)
+    clocks.start()
+    ms = timer.time(lambda: fq.fq_quant_act(x, qp, t, None, xq, sx, stream=stream), args.steps, args.warmup)
+    clk = clocks.stop()
+    nbytes = quant_bytes(d["m"], d["k"], d["n1"], d["n2"]) + 4 * d["k"]  # + c
+    pk, pk_kind = peaks()
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {
+        "metric": METRIC, "workload": "transform_quant", "value": round(gbs, 1), "unit": "GB/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
+        "higher_is_better": True, "dtype": "fp16 in, fp32 transform (fp16 hi/lo tensor-core products), int4 out",
+        "data": "synthetic",
+        "config": {"workload": "transform+quant, X [2048, 4096], 1% outlier channels x30, token 0 x100, "
+                               "Kronecker (64, 64), c ~ U[0.5, 2], alpha_a = 0.9, per-token INT4 + fp32 scales",
+                   "l2": "256 MiB flush between launches; median of the launches"},
+        "roofline": {"kernel": "quant_act_tc_kernel", "bound": "hbm", "achieved": round(gbs, 1),
+                     "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": round(gbs / pk["hbm_gbs"], 4),
+                     "peak_kind": pk_kind, "algorithmic_bytes": int(nbytes), "traffic": None},
+        "clocks": clk,
+    }
+
+
+def run_group(args, dev_index):
+    """Group-128 linears at M = 4096: (K, N) = (8192, 10240), (8192, 57344),
+    (28672, 8192); group scales on both sides, Student-t weights, Kronecker
+    transform on the activations.  Roofline: tensor (INT8)."""
+    torch, fq, dev, stream, clocks = _suite_common(args, dev_index)
+    qp = fq.qparams(fq.GROUP, 1.0)
+    rows, timer = [], LaunchTimer(dev, stream, clocks)
+    pk, pk_kind = peaks()
+    int8_peak = pk["bf16_tflops_sustained"] * INT8_OVER_BF16
+    clocks.start()
+    for k, n in synth.GROUP_70B_SHAPES:
+        d = synth.prefill_linear(k, n, m=4096, w_kind="t")
+        w = torch.from_numpy(d["w"]).to(dev)
+        wq, sw = fq.fq_quant_weight(w, qp)
+        del w
+        x = torch.from_numpy(d["x"]).to(dev)
+        t = fq.Transform(torch.from_numpy(d["p1"]).to(dev), torch.from_numpy(d["p2"]).to(dev))
+        xq, sx = fq.fq_quant_act(x, qp, t)
+        y = torch.empty(d["m"], n, dtype=torch.float16, device=dev)
+        ws = torch.empty(max(fq.fq_gemm_workspace_size(d["m"], n, k, fq.GROUP), 256), dtype=torch.uint8, device=dev)
+        q_ms = timer.time(lambda: fq.fq_quant_act(x, qp, t, None, xq, sx, stream=stream), args.steps, args.warmup)
+        g_ms = timer.time(lambda: fq.fq_w4a4_gemm(xq, sx, wq, sw, fq.GROUP, Y=y, workspace=ws, stream=stream),
+                          args.steps, args.warmup)
+        ops = 2.0 * d["m"] * n * k
+        qb = d["m"] * k * 2 + d["m"] * k // 2 + 2 * d["m"] * (k // 128) + 4 * (d["n1"] ** 2 + d["n2"] ** 2)
+        rows.append({"K": k, "N": n, "kron": [d["n1"], d["n2"]], "gemm_us": round(g_ms * 1e3, 2),
+                     "gemm_tops": round(ops / (g_ms * 1e-3) / 1e12, 1), "quant_us": round(q_ms * 1e3, 2),
+                     "quant_gbs": round(qb / (q_ms * 1e-3) / 1e9, 1), "ops": ops})
+        del d, x, xq, sx, y, wq, sw, ws
+        torch.cuda.empty_cache()
+    clk = clocks.stop()
+    ops = sum(r.pop("ops") for r in rows)
+    g_s = sum(r["gemm_us"] for r in rows) * 1e-6
+    tops = ops / g_s / 1e12
+    return {
+        "metric": METRIC, "workload": "group", "value": round(tops, 1), "unit": "TOPS", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(g_s * 1e3, 4), "higher_is_better": True,
+        "dtype": "int4 (s8 tensor-core MMA, s32 per-group partials, fp32 running sum), fp16 io", "data": "synthetic",
+        "config": {"workload": "group-128 linears, M=4096, (K, N) = (8192, 10240), (8192, 57344), (28672, 8192), "
+                               "Student-t(5) x 0.02 weights, Kronecker-transformed group-quantized activations",
+                   "l2": "256 MiB flush between launches; median of the launches"},
+        "rows": rows,
+        "roofline": {"kernel": "gemm_w4a4_kernel<128, group>", "bound": "tensor", "achieved": round(tops, 1),
+                     "peak": round(int8_peak, 1), "unit": "TOPS", "frac": round(tops / int8_peak, 4),
+                     "peak_kind": f"{pk_kind} bf16 sustained x {INT8_OVER_BF16:g}", "traffic": None},
+        "clocks": clk,
+    }
+
+
+def run_decode(args, dev_index):
+    """Decode with static (QSM-folded) activation scales: M in {1, 8, 32, 64}
+    against (K, N) = (8192, 57344) and (28672, 8192) per-channel INT4 weights.
+    Roofline: HBM (the packed weights dominate the bytes)."""
+    torch, fq, dev, stream, clocks = _suite_common(args, dev_index)
+    rows, timer = [], LaunchTimer(dev, stream, clocks)
+    pk, pk_kind = peaks()
+    clocks.start()
+    for k, n in synth.DECODE_70B_SHAPES:
+        d0 = synth.decode_static(synth.DECODE_TOKENS[-1], k, n)
+        s_k = torch.from_numpy(d0["static_scale"]).to(dev)
+        w = torch.from_numpy(d0["w"]).to(dev)
+        wq, sw = fq.fq_quant_weight(w, fq.qparams(fq.ROW, 1.0), None, s_k)
+        del w
+        qs = fq.qparams(fq.STATIC)
+        for m in synth.DECODE_TOKENS:
+            x = torch.from_numpy(d0["x"][:m].copy()).to(dev)
+            xq, _ = fq.fq_quant_act(x, qs, None, s_k)
+            y = torch.empty(m, n, dtype=torch.float16, device=dev)
+            ws = torch.empty(max(fq.fq_gemm_workspace_size(m, n, k, fq.STATIC), 256), dtype=torch.uint8, device=dev)
+            q_ms = timer.time(lambda: fq.fq_quant_act(x, qs, None, s_k, xq, None, stream=stream), args.steps,
+                              args.warmup)
+            g_ms = timer.time(lambda: fq.fq_w4a4_gemm(xq, None, wq, sw, fq.STATIC, Y=y, workspace=ws, stream=stream),
+                              args.steps, args.warmup)
+            gb = n * k // 2 + 4 * n + m * k // 2 + 2 * m * n
+            rows.append({"M": m, "K": k, "N": n, "gemm_us": round(g_ms * 1e3, 2),
+                         "gemm_gbs": round(gb / (g_ms * 1e-3) / 1e9, 1), "quant_us": round(q_ms * 1e3, 2),
+                         "bytes": gb})
+        del wq, sw, s_k, d0
+        torch.cuda.empty_cache()
+    clk = clocks.stop()
+    nbytes = sum(r.pop("bytes") for r in rows)
+    g_s = sum(r["gemm_us"] for r in rows) * 1e-6
+    gbs = nbytes / g_s / 1e9
+    return {
+        "metric": METRIC, "workload": "decode", "value": round(gbs, 1), "unit": "GB/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(g_s * 1e3, 4), "higher_is_better": True,
+        "dtype": "int4 (s8 tensor-core MMA, swap-AB, split-K int32), fp16 io", "data": "synthetic",
+        "config": {"workload": "decode M in {1, 8, 32, 64} x (K, N) in {(8192, 57344), (28672, 8192)}, static "
+                               "per-channel activation scales folded into per-channel INT4 weights",
+                   "l2": "256 MiB flush between launches; median of the launches"},
+        "rows": rows,
+        "roofline": {"kernel": "gemm_w4a4_kernel swap-AB (+ splitk_finalize_kernel)", "bound": "hbm",
+                     "achieved": round(gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                     "frac": round(gbs / pk["hbm_gbs"], 4), "peak_kind": pk_kind, "traffic": None},
+        "clocks": clk,
+    }
+
+
 # ---------------------------------------------------------------- the oracle on the host cores
 
 def _blas_threads():
@@ -404,12 +585,18 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", choices=[s[0] for s in SHAPES], default=None,
                     help="run one layer only (for profiling a single launch)")
+    ap.add_argument("--workload", choices=["prefill", "transform_quant", "group", "decode"], default="prefill",
+                    help="prefill (default): the decoder-layer prefill step; the others time one kernel family "
+                         "on its own workload (1 GPU)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     ws, rank, local = dist_env()
     if args.impl == "reference":
         out = run_reference(args, ws, rank)
+    elif args.workload != "prefill":
+        suite = {"transform_quant": run_transform_quant, "group": run_group, "decode": run_decode}[args.workload]
+        out = suite(args, local) if rank == 0 else None
     else:
         out = run_ours(args, ws, rank, local)
     if out is not None:
