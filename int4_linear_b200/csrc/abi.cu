@@ -73,7 +73,7 @@ fq_status check_launch(const char* what) {
 }
 
 fq_status make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, uint64_t inner, uint64_t rows,
-                       uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows) {
+                       uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle swizzle) {
   {
     std::lock_guard<std::mutex> lk(g_mu);
     if (!g_encode) {
@@ -90,7 +90,7 @@ fq_status make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType d
   const cuuint32_t box[2] = {box_inner, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r = g_encode(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
-                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS)
     return fail(FQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d) for %llu x %llu, box %u x %u", int(r),

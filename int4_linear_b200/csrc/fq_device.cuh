@@ -301,4 +301,17 @@ __device__ __forceinline__ void unpack8_hi(uint32_t w, uint32_t& lo4, uint32_t& 
   hi4 = w & 0xF0F0F0F0u;
 }
 
+// ------------------------------------------------------------------ packed float32 pairs
+
+// d = a * b + c on two float32 lanes with one rounding each (fma.rn.f32x2).
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+
 }  // namespace fq

@@ -33,7 +33,8 @@ inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_
 // out-of-range boxes).  inner = elements per row, rows = rows,
 // row_bytes = stride, box = {box_inner, box_rows}.
 fq_status make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, uint64_t inner,
-                       uint64_t rows, uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows);
+                       uint64_t rows, uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows,
+                       CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_NONE);
 
 constexpr int kGroup = 128;
 constexpr int kMaxK = 65536;

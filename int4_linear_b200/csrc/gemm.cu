@@ -73,9 +73,14 @@ struct Cfg {
   static constexpr int UNP_STAGE = B_UNP;
   static constexpr int OFF_UNP = 0;
   static constexpr int OFF_SCALE = OFF_UNP + SU * UNP_STAGE;
-  static constexpr int SCALE_BYTES = EPI == kEpiGroup ? kEpiWarps * BN * 4 : 0;
+  // group mode: a ring of SS per-slice scale stages written by warp 0: the
+  // weight scales as {s, s, -1.5*2^23*s, -1.5*2^23*s} pairs for BN columns,
+  // then the activation scales of the 128 rows
+  static constexpr int SS = 8;
+  static constexpr int SC_STAGE = BN * 8 + kBM * 4;
+  static constexpr int SCALE_BYTES = EPI == kEpiGroup ? SS * SC_STAGE : 0;
   static constexpr int OFF_BAR = OFF_SCALE + SCALE_BYTES;
-  static constexpr int NBAR = 2 * SU + 5;
+  static constexpr int NBAR = 2 * SU + 5 + (EPI == kEpiGroup ? 2 * SS : 0);
   static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
   static constexpr int SMEM = OFF_TMEM + 16 + 1024;  // + slack to align the base to 1024
   // the fp16 output tile is staged in the (then idle) unpacked ring, rows padded by 16 bytes
@@ -123,6 +128,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(const GemmParams
   uint64_t* acc_full = empty_u + SU;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* done_bar = acc_empty + 2;
+  uint64_t* sfull = done_bar + 1;   // group mode: scale stages
+  uint64_t* sempty = sfull + C::SS;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -140,6 +147,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(const GemmParams
       mbar_init(&acc_empty[b], kEpiWarps);
     }
     mbar_init(done_bar, 1);
+    if (EPI == kEpiGroup) {
+      for (int s = 0; s < C::SS; ++s) {
+        mbar_init(&sfull[s], 1);
+        mbar_init(&sempty[s], kEpiWarps);
+      }
+    }
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -152,7 +165,58 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(const GemmParams
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    // idle: joins the final barrier
+    if (EPI == kEpiGroup) {
+      // ------------------------------------------------------------ group scales -> shared-memory ring
+      // Loads run D slices ahead in registers, so their latency is paid once.
+      constexpr int D = 4;
+      constexpr int NP2 = BN / 64;  // column pairs per lane
+      constexpr float kMagicF = 12582912.0f;  // 1.5 * 2^23 (see the group epilogue)
+      const int bbase = tileB * BN, abase = tileA * kBM;
+      __half2 wv[D][NP2];
+      __half xv[D][4];
+      auto load = [&](int d, int i) {
+        const int g = kb0 + i;
+#pragma unroll
+        for (int t = 0; t < NP2; ++t) {
+          const int n = bbase + 2 * (lane + 32 * t);  // N is a multiple of 8: both columns or neither
+          wv[d][t] = (i < nkb && n < p.N) ? *reinterpret_cast<const __half2*>(p.gsw + size_t(g) * p.N + n)
+                                          : __floats2half2_rn(0.f, 0.f);
+        }
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const int m = abase + lane + 32 * t;
+          xv[d][t] = (i < nkb && m < p.M) ? p.gsx[size_t(g) * p.M + m] : __float2half_rn(0.f);
+        }
+      };
+#pragma unroll
+      for (int d = 0; d < D; ++d) load(d, d);
+      bool ok = true;
+      for (int i0 = 0; i0 < nkb && ok; i0 += D) {
+#pragma unroll
+        for (int d = 0; d < D; ++d) {
+          const int i = i0 + d;
+          if (i >= nkb) break;
+          const int st = i % C::SS;
+          if (!warp_wait(&sempty[st], ((i / C::SS) & 1) ^ 1)) {
+            if (lane == 0) record_error(p.err, kErrTimeoutProducer);
+            ok = false;
+            break;
+          }
+          uint8_t* sc = smem + C::OFF_SCALE + st * C::SC_STAGE;
+#pragma unroll
+          for (int t = 0; t < NP2; ++t) {
+            const float2 w = __half22float2(wv[d][t]);
+            const float a = w.x * 0.00390625f, b = w.y * 0.00390625f;  // / 256, exact
+            reinterpret_cast<float4*>(sc)[lane + 32 * t] = make_float4(a, b, -kMagicF * a, -kMagicF * b);
+          }
+#pragma unroll
+          for (int t = 0; t < 4; ++t) reinterpret_cast<float*>(sc + BN * 8)[lane + 32 * t] = __half2float(xv[d][t]);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sfull[st]);
+          load(d, i + D);
+        }
+      }
+    }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -161,8 +225,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(const GemmParams
         const int su = i % SU;
         uint32_t d = tmem;
         if (EPI == kEpiGroup) {
+          // phase 0 of acc_empty[b] is the epilogue priming buffer b
           const int b = i & 1;
-          if (!mbar_wait(&acc_empty[b], ((i >> 1) & 1) ^ 1)) {
+          if (!mbar_wait(&acc_empty[b], (i >> 1) & 1)) {
             record_error(p.err, kErrTimeoutMma);
             break;
           }
@@ -178,7 +243,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(const GemmParams
         const uint32_t b0 = smem_u32(smem + C::OFF_UNP + su * C::UNP_STAGE);
 #pragma unroll
         for (int k = 0; k < kBK / 32; ++k) {
-          const uint32_t accum = EPI == kEpiGroup ? uint32_t(k > 0) : uint32_t(i > 0 || k > 0);
+          // group mode accumulates onto the primed offset (see the group epilogue)
+          const uint32_t accum = EPI == kEpiGroup ? 1u : uint32_t(i > 0 || k > 0);
           mma_i8_ts(d, a0 + uint32_t(8 * k), sdesc_k128_sw128(b0 + 32 * k), idesc, accum);
         }
         mma_commit(&empty_u[su]);
@@ -384,18 +450,40 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(const GemmParams
       } else {
         // group-128: one accumulator per K slice, double-buffered in tensor
         // memory; the running float32 sum lives in columns [2 BN, 3 BN).
-        float* sbuf = reinterpret_cast<float*>(smem + C::OFF_SCALE) + (warp - 2) * BN;
+        // Each accumulator buffer is primed with the integer 0x4B400000 (the
+        // bits of 1.5 * 2^23) before the MMAs add 256 * sum(qx qw) (|.| <
+        // 2^22) to it, so its bits read as the float 1.5 * 2^23 + acc
+        // exactly, with no int-to-float conversion.  Then one fused
+        // multiply-add, fma(f, s', -1.5 * 2^23 * s') with s' = s_w / 256
+        // (both exact in float32), gives fl(sum * s_w) with a single
+        // rounding, and a second one adds it times s_x into the running sum;
+        // both run two columns per instruction (fma.rn.f32x2).  Warp 0 has
+        // the slice's s' and -1.5 * 2^23 * s' pairs and the row scales ready
+        // in a shared-memory ring.
+        constexpr uint32_t kMagic = 0x4B400000u;
         const uint32_t tsum = tl + uint32_t(2 * BN);
-        const int m = arow;
-        const bool mok = m < p.M;
+        uint32_t mg[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) mg[j] = kMagic;
+#pragma unroll
+        for (int b = 0; b < 2; ++b)
+          for (int c0 = 0; c0 < BN; c0 += 32) tmem_st_32x32(tl + uint32_t(b * BN + c0), mg);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&acc_empty[0]);
+          mbar_arrive(&acc_empty[1]);
+        }
         for (int i = 0; i < nkb; ++i) {
-          const int g = kb0 + i, b = i & 1;
-          for (int c = lane; c < BN; c += 32) {
-            const int n = bbase + c;
-            sbuf[c] = n < p.N ? __half2float(p.gsw[size_t(g) * p.N + n]) : 0.f;
+          const int b = i & 1, st = i % C::SS;
+          if (!warp_wait(&sfull[st], (i / C::SS) & 1)) {
+            if (lane == 0) record_error(p.err, kErrTimeoutEpilogue);
+            break;
           }
-          const float sxg = mok ? __half2float(p.gsx[size_t(g) * p.M + m]) : 0.f;
-          __syncwarp();
+          const float4* sbuf = reinterpret_cast<const float4*>(smem + C::OFF_SCALE + st * C::SC_STAGE);
+          const float sxg = reinterpret_cast<const float*>(smem + C::OFF_SCALE + st * C::SC_STAGE + BN * 8)[rloc];
+          const float2 sx2 = make_float2(sxg, sxg);
           if (!warp_wait(&acc_full[b], (i >> 1) & 1)) {
             if (lane == 0) record_error(p.err, kErrTimeoutEpilogue);
             break;
@@ -407,17 +495,26 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(const GemmParams
             if (i > 0) tmem_ld_32x32(tsum + c0, s);
             tmem_wait_ld();
   #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const float prev = i > 0 ? __uint_as_float(s[j]) : 0.f;
-              const float t = __fmul_rn(sxg, sbuf[c0 + j]);
-              s[j] = __float_as_uint(fmaf(float(int32_t(v[j]) >> 8), t, prev));
+            for (int j = 0; j < 32; j += 2) {
+              const float4 q = sbuf[(c0 + j) / 2];
+              const float2 u = ffma2(make_float2(__uint_as_float(v[j]), __uint_as_float(v[j + 1])),
+                                     make_float2(q.x, q.y), make_float2(q.z, q.w));
+              const float2 prev = i > 0 ? make_float2(__uint_as_float(s[j]), __uint_as_float(s[j + 1]))
+                                        : make_float2(0.f, 0.f);
+              const float2 r = ffma2(u, sx2, prev);
+              s[j] = __float_as_uint(r.x);
+              s[j + 1] = __float_as_uint(r.y);
             }
             tmem_st_32x32(tsum + c0, s);
+            tmem_st_32x32(tl + uint32_t(b * BN + c0), mg);  // re-prime for slice i + 2
           }
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&acc_empty[b]);
+          if (lane == 0) {
+            mbar_arrive(&acc_empty[b]);
+            mbar_arrive(&sempty[st]);
+          }
         }
         for (int c0 = 0; c0 < BN; c0 += 32) {
           uint32_t s[32];
@@ -473,6 +570,286 @@ __global__ void splitk_finalize_kernel(const int32_t* __restrict__ acc, const fl
   }
 }
 
+// ---------------------------------------------------------------- decode
+//
+// Few tokens (M <= 64): the GEMM is a stream of the packed weights, so the
+// kernel is built around keeping enough of that stream in flight.  The
+// weights take the 128-row MMA side (one CTA = 128 output channels x a K
+// range), the tokens the N side (BN = 16, 32 or 64).
+//   warp 0      one thread issues TMA loads of packed 128 x 64-byte weight
+//               slices into a ring of SP stages (64-byte swizzle, so that
+//               the row-per-thread reads below are free of bank conflicts)
+//   warp 1      tensor-memory allocation and the MMA-issuing thread
+//   warps 2-5   read one weight row each from the ring, unpack it and store
+//               it into a tensor-memory A ring (SU stages); afterwards the
+//               epilogue (thread = output channel, columns = tokens)
+//   warps 6-7   unpack the tokens' packed slices (L2-resident) into the
+//               128-byte swizzled shared-memory B ring
+// 256 threads and under 100 KB of shared memory, so two CTAs share an SM
+// and up to 2 x SP x 8 KB of the weight stream are in flight per SM.
+constexpr int kDecThreads = 256;
+
+template <int BN>
+struct DecCfg {
+  static constexpr int SP = 8;                    // packed weight stages (TMA ring)
+  static constexpr int SU = 4;                    // unpacked stages
+  static constexpr int P_STAGE = kBM * kPK;       // 128 rows x 64 bytes
+  static constexpr int B_STAGE = BN * kBK;        // BN rows x 128 int8, 128-byte swizzle
+  static constexpr int OFF_P = 0;
+  static constexpr int OFF_B = OFF_P + SP * P_STAGE;
+  static constexpr int OFF_BAR = OFF_B + SU * B_STAGE;
+  static constexpr int NBAR = 2 * SP + 2 * SU + 2;
+  static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
+  // at least 80 KB, so that no more than two CTAs (2 x 256 tensor-memory
+  // columns) are resident on one SM
+  static constexpr int SMEM = (OFF_TMEM + 16 + 1024) > 80 * 1024 ? (OFF_TMEM + 16 + 1024) : 80 * 1024;
+  static constexpr int A_COL0 = BN < 32 ? 32 : BN;  // accumulator in columns [0, BN)
+  static constexpr int A_STAGE_COLS = kBK / 4;
+  static constexpr int TMEM_NEED = A_COL0 + SU * A_STAGE_COLS;
+  static constexpr int TMEM_COLS = TMEM_NEED <= 128 ? 128 : 256;
+  static_assert(B_STAGE % 1024 == 0 && P_STAGE % 1024 == 0, "stage alignment");
+  static_assert(TMEM_NEED <= 256, "two CTAs per SM share the tensor memory");
+};
+
+template <int BN, int EPI>
+__global__ void __launch_bounds__(kDecThreads, 2)
+    gemm_decode_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tmA) {
+  using C = DecCfg<BN>;
+  constexpr int SP = C::SP, SU = C::SU;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* pfull = bars;
+  uint64_t* pempty = pfull + SP;
+  uint64_t* ufull = pempty + SP;
+  uint64_t* uempty = ufull + SU;
+  uint64_t* acc_full = uempty + SU;
+  uint64_t* done_bar = acc_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tileA = blockIdx.x;
+  const int kb0 = blockIdx.z * p.kb_per_split;
+  const int nkb = max(0, min(p.num_kb, kb0 + p.kb_per_split) - kb0);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < SP; ++s) {
+      mbar_init(&pfull[s], 1);
+      mbar_init(&pempty[s], 4);
+    }
+    for (int s = 0; s < SU; ++s) {
+      mbar_init(&ufull[s], 6);
+      mbar_init(&uempty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(done_bar, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tensormap(&tmA);
+      const uint64_t pol = policy_evict_first();  // the weights are read once
+      int issued = 0;
+      for (int i = 0; i < nkb; ++i) {
+        const int sp = i % SP;
+        if (!mbar_wait(&pempty[sp], ((i / SP) & 1) ^ 1)) {
+          record_error(p.err, kErrTimeoutProducer);
+          break;
+        }
+        mbar_arrive_expect_tx(&pfull[sp], C::P_STAGE);
+        tma_load_2d_hint(smem + C::OFF_P + sp * C::P_STAGE, &tmA, &pfull[sp], (kb0 + i) * kPK, tileA * kBM, pol);
+        ++issued;
+      }
+      // every issued copy has landed before the CTA may leave (normally the
+      // unpacking warps already waited for each of them)
+      for (int i = max(0, issued - SP); i < issued; ++i)
+        if (!mbar_wait(&pfull[i % SP], (i / SP) & 1)) {
+          record_error(p.err, kErrTimeoutDrain);
+          break;
+        }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_i8_m128(BN);
+      for (int i = 0; i < nkb; ++i) {
+        const int su = i % SU;
+        if (!mbar_wait(&ufull[su], (i / SU) & 1)) {
+          record_error(p.err, kErrTimeoutMma);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a0 = tmem + uint32_t(C::A_COL0 + su * C::A_STAGE_COLS);
+        const uint32_t b0 = smem_u32(smem + C::OFF_B + su * C::B_STAGE);
+#pragma unroll
+        for (int k = 0; k < kBK / 32; ++k)
+          mma_i8_ts(tmem, a0 + uint32_t(8 * k), sdesc_k128_sw128(b0 + 32 * k), idesc, uint32_t(i > 0 || k > 0));
+        mma_commit(&uempty[su]);
+      }
+      mma_commit(acc_full);
+      mma_commit(done_bar);
+      if (!mbar_wait(done_bar, 0)) record_error(p.err, kErrTimeoutDrain);
+    }
+  } else if (warp < 6) {
+    // ------------------------------------------------------------ weight rows -> tensor memory
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    const uint32_t ta = tmem + (uint32_t(q * 32) << 16) + uint32_t(C::A_COL0);
+    const int sw = (row >> 1) & 3;  // 64-byte swizzle: chunk c of this row sits at chunk c ^ sw
+    bool ok = true;
+    for (int i = 0; i < nkb; ++i) {
+      const int sp = i % SP, su = i % SU;
+      if (!warp_wait(&pfull[sp], (i / SP) & 1)) {
+        ok = false;
+        break;
+      }
+      const uint8_t* src = smem + C::OFF_P + sp * C::P_STAGE + row * kPK;
+      uint4 w[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) w[c] = *reinterpret_cast<const uint4*>(src + ((c ^ sw) << 4));
+      if (!warp_wait(&uempty[su], ((i / SU) & 1) ^ 1)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t r[32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        unpack8_hi(w[c].x, r[8 * c + 0], r[8 * c + 1]);
+        unpack8_hi(w[c].y, r[8 * c + 2], r[8 * c + 3]);
+        unpack8_hi(w[c].z, r[8 * c + 4], r[8 * c + 5]);
+        unpack8_hi(w[c].w, r[8 * c + 6], r[8 * c + 7]);
+      }
+      tmem_st_32x32(ta + uint32_t(su * C::A_STAGE_COLS), r);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      // The packed stage goes back to the TMA producer only now, after the
+      // tensor-memory store has consumed the registers it was read into: a
+      // release right after issuing the shared-memory loads let the refill
+      // overwrite rows whose reads had not completed yet.
+      if (lane == 0) {
+        mbar_arrive(&pempty[sp]);
+        mbar_arrive(&ufull[su]);
+      }
+    }
+    if (!ok && lane == 0) record_error(p.err, kErrTimeoutUnpack);
+  } else {
+    // ------------------------------------------------------------ token rows -> shared memory
+    constexpr int D = 6;                           // K slices of packed tokens in flight per thread
+    constexpr int kJobs = BN * 4;                  // 16-byte packed pieces per stage
+    constexpr int JPT = (kJobs + 63) / 64;         // per thread (two warps)
+    const int t = (warp - 6) * 32 + lane;
+    const size_t ld = size_t(p.K) / 2;
+    const uint8_t* gsrc[JPT];
+    uint32_t dst0[JPT], dst1[JPT];
+    bool live[JPT], load_ok[JPT];
+#pragma unroll
+    for (int it = 0; it < JPT; ++it) {
+      const int j = it * 64 + t;
+      live[it] = j < kJobs;
+      const int brow = live[it] ? (j >> 2) : 0, c = j & 3, r7 = brow & 7;
+      const uint32_t rb = uint32_t((brow >> 3) * 1024 + r7 * 128);
+      dst0[it] = rb + uint32_t(((2 * c) ^ r7) << 4);
+      dst1[it] = rb + uint32_t(((2 * c + 1) ^ r7) << 4);
+      load_ok[it] = live[it] && brow < p.rowsB;
+      gsrc[it] = p.B + (load_ok[it] ? size_t(brow) * ld : 0) + size_t(kb0) * kPK + c * 16;
+    }
+    uint4 w[D][JPT];
+#pragma unroll
+    for (int d = 0; d < D; ++d)
+#pragma unroll
+      for (int it = 0; it < JPT; ++it)
+        w[d][it] = (d < nkb && load_ok[it]) ? __ldg(reinterpret_cast<const uint4*>(gsrc[it] + d * kPK))
+                                            : make_uint4(0, 0, 0, 0);
+    bool ok = true;
+    for (int i0 = 0; i0 < nkb && ok; i0 += D) {
+#pragma unroll
+      for (int d = 0; d < D; ++d) {
+        const int i = i0 + d;
+        if (i >= nkb) break;
+        const int su = i % SU;
+        if (!warp_wait(&uempty[su], ((i / SU) & 1) ^ 1)) {
+          if (lane == 0) record_error(p.err, kErrTimeoutUnpack);
+          ok = false;
+          break;
+        }
+        uint8_t* uk = smem + C::OFF_B + su * C::B_STAGE;
+#pragma unroll
+        for (int it = 0; it < JPT; ++it) {
+          if (!live[it]) continue;
+          uint4 o0, o1;
+          unpack8_hi(w[d][it].x, o0.x, o0.y);
+          unpack8_hi(w[d][it].y, o0.z, o0.w);
+          unpack8_hi(w[d][it].z, o1.x, o1.y);
+          unpack8_hi(w[d][it].w, o1.z, o1.w);
+          *reinterpret_cast<uint4*>(uk + dst0[it]) = o0;
+          *reinterpret_cast<uint4*>(uk + dst1[it]) = o1;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ufull[su]);
+        if (i + D < nkb) {
+#pragma unroll
+          for (int it = 0; it < JPT; ++it)
+            w[d][it] = load_ok[it] ? __ldg(reinterpret_cast<const uint4*>(gsrc[it] + (i + D) * kPK))
+                                   : make_uint4(0, 0, 0, 0);
+        }
+      }
+    }
+  }
+
+  if (warp >= 2 && warp < 6) {
+    // ------------------------------------------------------------ epilogue: thread = output channel n
+    const int q = warp & 3;
+    const int n = tileA * kBM + q * 32 + lane;
+    const uint32_t tl = tmem + (uint32_t(q * 32) << 16);
+    if (!warp_wait(acc_full, 0) && lane == 0) record_error(p.err, kErrTimeoutEpilogue);
+    tc_fence_after();
+    const float swn = (EPI == kEpiRow || EPI == kEpiStatic) && n < p.N ? __ldg(p.sw + n) : 0.f;
+    constexpr int CW = BN >= 32 ? 32 : 16;
+    for (int c0 = 0; c0 < BN; c0 += CW) {
+      uint32_t v[32];
+      if (CW == 32)
+        tmem_ld_32x32(tl + uint32_t(c0), v);
+      else
+        tmem_ld_32x16(tl + uint32_t(c0), v);
+      tmem_wait_ld();
+      if (n < p.N) {
+#pragma unroll
+        for (int j = 0; j < CW; ++j) {
+          const int m = c0 + j;
+          if (m >= p.M) break;
+          const int32_t ai = int32_t(v[j]) >> 8;
+          if (EPI == kEpiRow)
+            p.Y[size_t(m) * p.N + n] = __float2half_rn(__fmul_rn(__fmul_rn(float(ai), __ldg(p.sx + m)), swn));
+          else if (EPI == kEpiStatic)
+            p.Y[size_t(m) * p.N + n] = __float2half_rn(__fmul_rn(float(ai), swn));
+          else
+            atomicAdd(p.acc + size_t(m) * p.N + n, ai);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
 struct Plan {
   bool swap;
   int bn;
@@ -505,7 +882,7 @@ Plan make_plan(int M, int N, int K, int epi_final, int sms) {
   pl.bn = pick_bn_swap(M);
   pl.epi = epi_final;
   const int tiles = (N + kBM - 1) / kBM;
-  const int per_sm = pl.bn <= 16 ? 2 : 1;
+  const int per_sm = 2;  // decode CTAs resident per SM
   const int slots = sms * per_sm;
   double best = -1.0;
   int best_s = 1;
@@ -540,6 +917,21 @@ fq_status launch_gemm(const GemmParams& gp, dim3 grid, cudaStream_t stream) {
   return check_launch("gemm_w4a4_kernel");
 }
 
+template <int BN, int EPI>
+fq_status launch_decode(const GemmParams& gp, dim3 grid, cudaStream_t stream) {
+  using C = DecCfg<BN>;
+  CUtensorMap tm;
+  const fq_status st = make_tmap_2d(&tm, gp.A, CU_TENSOR_MAP_DATA_TYPE_UINT8, uint64_t(gp.K) / 2, uint64_t(gp.rowsA),
+                                    uint64_t(gp.K) / 2, uint32_t(kPK), uint32_t(kBM), CU_TENSOR_MAP_SWIZZLE_64B);
+  if (st != FQ_OK) return st;
+  auto kern = gemm_decode_kernel<BN, EPI>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess ||
+      cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
+    return fail(FQ_ERR_CUDA, "cannot reserve %d bytes of shared memory for the decode GEMM", C::SMEM);
+  kern<<<grid, kDecThreads, C::SMEM, stream>>>(gp, tm);
+  return check_launch("gemm_decode_kernel");
+}
+
 fq_status dispatch(const Plan& pl, const GemmParams& gp, dim3 grid, cudaStream_t s) {
   if (!pl.swap) {
     switch (pl.epi) {
@@ -550,14 +942,14 @@ fq_status dispatch(const Plan& pl, const GemmParams& gp, dim3 grid, cudaStream_t
       default: break;
     }
   } else {
-#define FQ_SWAP_CASES(BNV)                                                           \
-  if (pl.bn == BNV) {                                                                \
-    switch (pl.epi) {                                                                \
-      case kEpiRow: return launch_gemm<BNV, kEpiRow, true>(gp, grid, s);       \
-      case kEpiStatic: return launch_gemm<BNV, kEpiStatic, true>(gp, grid, s); \
-      case kEpiAtomic: return launch_gemm<BNV, kEpiAtomic, true>(gp, grid, s); \
-      default: break;                                                                \
-    }                                                                                \
+#define FQ_SWAP_CASES(BNV)                                                     \
+  if (pl.bn == BNV) {                                                          \
+    switch (pl.epi) {                                                          \
+      case kEpiRow: return launch_decode<BNV, kEpiRow>(gp, grid, s);           \
+      case kEpiStatic: return launch_decode<BNV, kEpiStatic>(gp, grid, s);     \
+      case kEpiAtomic: return launch_decode<BNV, kEpiAtomic>(gp, grid, s);     \
+      default: break;                                                          \
+    }                                                                          \
   }
     FQ_SWAP_CASES(16)
     FQ_SWAP_CASES(32)

@@ -265,6 +265,54 @@ __global__ void __launch_bounds__(kThreads) quant_rows_kernel(QuantParams p) {
   }
 }
 
+// Static per-channel activation scales with no Kronecker transform: every
+// element is independent (q = clamp(rint(x c / s_k))), so the elements are
+// spread over the whole grid, 8 per thread-iteration (one 16-byte load, one
+// 32-bit packed store), instead of one CTA per token row.
+__global__ void __launch_bounds__(kThreads) quant_static_kernel(QuantParams p) {
+  const size_t pieces = size_t(p.R) * (p.K / 8);
+  const int kp = p.K / 8;
+  for (size_t pc = blockIdx.x * size_t(kThreads) + threadIdx.x; pc < pieces; pc += size_t(gridDim.x) * kThreads) {
+    const int r = int(pc / kp), e0 = int(pc % kp) * 8;
+    const uint4 raw = *reinterpret_cast<const uint4*>(p.X + size_t(r) * p.K + e0);
+    const __half2* h2 = reinterpret_cast<const __half2*>(&raw);
+    const float4 s0 = __ldg(reinterpret_cast<const float4*>(p.sstatic + e0));
+    const float4 s1 = __ldg(reinterpret_cast<const float4*>(p.sstatic + e0 + 4));
+    const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+    float v[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = __half22float2(h2[j]);
+      v[2 * j] = f.x;
+      v[2 * j + 1] = f.y;
+    }
+    if (p.c) {
+      const float4 c0 = __ldg(reinterpret_cast<const float4*>(p.c + e0));
+      const float4 c1 = __ldg(reinterpret_cast<const float4*>(p.c + e0 + 4));
+      const float cv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = __fmul_rn(v[j], cv[j]);
+    }
+    uint32_t word = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) word |= (uint32_t(rtn_code(v[j], sv[j])) & 0xFu) << (4 * j);
+    reinterpret_cast<uint32_t*>(p.Q + size_t(r) * (p.K / 2))[e0 / 8] = word;
+    if (p.xhat) {
+      float4* xo = reinterpret_cast<float4*>(p.xhat + size_t(r) * p.K + e0);
+      xo[0] = make_float4(v[0], v[1], v[2], v[3]);
+      xo[1] = make_float4(v[4], v[5], v[6], v[7]);
+    }
+  }
+}
+
+fq_status launch_quant_static(const QuantParams& qp, cudaStream_t stream) {
+  const size_t pieces = size_t(qp.R) * (qp.K / 8);
+  const size_t want = (pieces + kThreads - 1) / kThreads;
+  const int grid = int(std::max<size_t>(1, std::min<size_t>(want, size_t(sm_count()) * 8)));
+  quant_static_kernel<<<grid, kThreads, 0, stream>>>(qp);
+  return check_launch("quant_static_kernel");
+}
+
 size_t smem_bytes(int K, int n1, int n2, bool psmem) {
   const size_t row = n1 > 0 ? size_t(n1) * (n2 + 1) : size_t(K);
   const size_t pm = (psmem && n1 > 0) ? size_t(n1) * n1 + size_t(n2) * n2 : 0;
@@ -367,6 +415,11 @@ fq_status quant_common(int side, const uint16_t* X, int R, int K, const fq_qpara
     tp.err = err;
     return launch_quant_act_tc(tp, s);
   }
+  // static scales without a transform: element-parallel kernel (its vector
+  // loads need 16-byte aligned scales and c; otherwise the row kernel runs)
+  if (side == kAct && qp->gran == FQ_STATIC_CHANNEL && p.n1 == 0 && aligned(extra, 16) &&
+      (!p.c || aligned(p.c, 16)))
+    return launch_quant_static(p, s);
   const bool psmem = smem_bytes(K, p.n1, p.n2, true) <= size_t(kSmemBudget);
   if (smem_bytes(K, p.n1, p.n2, false) > size_t(kSmemBudget))
     return fail(FQ_ERR_UNSUPPORTED, "row of K = %d does not fit in shared memory", K);

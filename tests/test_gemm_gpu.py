@@ -78,6 +78,20 @@ def test_gemm_group(m, n, k):
     print(f"group {m}x{n}x{k}: {n_beyond} outputs beyond 1 ulp (cancellation bound)")
 
 
+@pytest.mark.parametrize("m", [17, 32, 64])
+def test_gemm_decode_split_k_repeatable(m):
+    """Decode shapes with split-K over a long K, run several times: every run
+    bit-exact (a stage handed back too early corrupts random rows in some runs)."""
+    n, k = 8192, 28672
+    a, b = _operands(11 * m, m, n, k)
+    sw = synth.random_scales(synth.generator(m + 5), n, 1e-4, 1e-2)
+    ref = O.dequant_static(O.gemm_int(C.unpack(a), C.unpack(b)), sw)
+    A, B, S = C.dev(a), C.dev(b), C.dev(sw)
+    for _ in range(4):
+        C.check_fp16_exact(C.host(fq.fq_w4a4_gemm(A, None, B, S, fq.STATIC)), ref)
+    fq.fq_check_device_error()
+
+
 def test_gemm_workspace_is_reused_correctly():
     """Two split-K calls in a row on one workspace give the same exact result."""
     m, n, k = 8, 8192, 28672

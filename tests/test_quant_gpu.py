@@ -48,6 +48,26 @@ def test_quant_act_exact(gname, m, k, with_c):
         assert np.array_equal(_gpu_scales(sx, gf), s_ref)
 
 
+@pytest.mark.parametrize("with_c", [False, True])
+def test_quant_act_static_4byte_aligned_scales(with_c):
+    """Static scales (and c) that are only 4-byte aligned take the row kernel
+    instead of the element-parallel one; the codes are the same."""
+    m, k = 37, 1024
+    x = _x(11, m, k)
+    ss = _static_scales(12, k)
+    c = synth.generator(13).uniform(0.5, 2.0, k).astype(np.float32) if with_c else None
+    ss_buf = torch.zeros(k + 1, dtype=torch.float32, device="cuda")
+    ss_buf[1:] = torch.from_numpy(ss).cuda()
+    t = None
+    if with_c:
+        c_buf = torch.zeros(k + 1, dtype=torch.float32, device="cuda")
+        c_buf[1:] = torch.from_numpy(c).cuda()
+        t = fq.Transform(c=c_buf[1:])
+    xq, _ = fq.fq_quant_act(C.dev(x), fq.qparams(fq.STATIC), t, ss_buf[1:])
+    q_ref, _, _ = O.quant_act(x, O.STATIC, 1.0, c=c, static_scale=ss)
+    assert np.array_equal(C.host(xq), O.pack_int4(q_ref))
+
+
 def test_quant_act_tiny_workload():
     d = synth.tiny_linear()
     xq, sx = fq.fq_quant_act(C.dev(d["x"]), fq.qparams(fq.ROW, 1.0))
