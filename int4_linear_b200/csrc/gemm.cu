@@ -591,12 +591,14 @@ constexpr int kDecThreads = 256;
 
 template <int BN>
 struct DecCfg {
-  static constexpr int SP = 8;                    // packed weight stages (TMA ring)
+  static constexpr int SP = BN == 64 ? 6 : 8;     // packed stages (TMA ring: weights + tokens)
   static constexpr int SU = 4;                    // unpacked stages
-  static constexpr int P_STAGE = kBM * kPK;       // 128 rows x 64 bytes
+  static constexpr int P_STAGE = kBM * kPK;       // weights: 128 rows x 64 bytes
+  static constexpr int X_STAGE = BN * kPK;        // tokens: BN rows x 64 bytes
   static constexpr int B_STAGE = BN * kBK;        // BN rows x 128 int8, 128-byte swizzle
   static constexpr int OFF_P = 0;
-  static constexpr int OFF_B = OFF_P + SP * P_STAGE;
+  static constexpr int OFF_X = OFF_P + SP * P_STAGE;
+  static constexpr int OFF_B = OFF_X + SP * X_STAGE;
   static constexpr int OFF_BAR = OFF_B + SU * B_STAGE;
   static constexpr int NBAR = 2 * SP + 2 * SU + 2;
   static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
@@ -607,13 +609,15 @@ struct DecCfg {
   static constexpr int A_STAGE_COLS = kBK / 4;
   static constexpr int TMEM_NEED = A_COL0 + SU * A_STAGE_COLS;
   static constexpr int TMEM_COLS = TMEM_NEED <= 128 ? 128 : 256;
-  static_assert(B_STAGE % 1024 == 0 && P_STAGE % 1024 == 0, "stage alignment");
+  static_assert(B_STAGE % 1024 == 0 && P_STAGE % 1024 == 0 && X_STAGE % 1024 == 0, "stage alignment");
   static_assert(TMEM_NEED <= 256, "two CTAs per SM share the tensor memory");
+  static_assert(2 * (SMEM + 1024) <= 228 * 1024, "two CTAs per SM");
 };
 
 template <int BN, int EPI>
 __global__ void __launch_bounds__(kDecThreads, 2)
-    gemm_decode_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tmA) {
+    gemm_decode_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tmA,
+                       const __grid_constant__ CUtensorMap tmX) {
   using C = DecCfg<BN>;
   constexpr int SP = C::SP, SU = C::SU;
   extern __shared__ uint8_t smem_raw[];
@@ -635,7 +639,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
   if (threadIdx.x == 0) {
     for (int s = 0; s < SP; ++s) {
       mbar_init(&pfull[s], 1);
-      mbar_init(&pempty[s], 4);
+      mbar_init(&pempty[s], 6);  // 4 weight-row warps + 2 token warps
     }
     for (int s = 0; s < SU; ++s) {
       mbar_init(&ufull[s], 6);
@@ -658,7 +662,9 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       prefetch_tensormap(&tmA);
+      prefetch_tensormap(&tmX);
       const uint64_t pol = policy_evict_first();  // the weights are read once
+      const uint64_t pol_x = policy_evict_last();  // the tokens are read by every CTA
       int issued = 0;
       for (int i = 0; i < nkb; ++i) {
         const int sp = i % SP;
@@ -666,8 +672,9 @@ __global__ void __launch_bounds__(kDecThreads, 2)
           record_error(p.err, kErrTimeoutProducer);
           break;
         }
-        mbar_arrive_expect_tx(&pfull[sp], C::P_STAGE);
+        mbar_arrive_expect_tx(&pfull[sp], C::P_STAGE + C::X_STAGE);
         tma_load_2d_hint(smem + C::OFF_P + sp * C::P_STAGE, &tmA, &pfull[sp], (kb0 + i) * kPK, tileA * kBM, pol);
+        tma_load_2d_hint(smem + C::OFF_X + sp * C::X_STAGE, &tmX, &pfull[sp], (kb0 + i) * kPK, 0, pol_x);
         ++issued;
       }
       // every issued copy has landed before the CTA may leave (normally the
@@ -746,14 +753,14 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     if (!ok && lane == 0) record_error(p.err, kErrTimeoutUnpack);
   } else {
     // ------------------------------------------------------------ token rows -> shared memory
-    constexpr int D = 6;                           // K slices of packed tokens in flight per thread
+    // The packed token slice arrives with the weights in the TMA ring; each
+    // lane unpacks fixed 16-byte pieces (consecutive lanes read consecutive
+    // pieces, so the reads are free of bank conflicts).
     constexpr int kJobs = BN * 4;                  // 16-byte packed pieces per stage
     constexpr int JPT = (kJobs + 63) / 64;         // per thread (two warps)
     const int t = (warp - 6) * 32 + lane;
-    const size_t ld = size_t(p.K) / 2;
-    const uint8_t* gsrc[JPT];
     uint32_t dst0[JPT], dst1[JPT];
-    bool live[JPT], load_ok[JPT];
+    bool live[JPT];
 #pragma unroll
     for (int it = 0; it < JPT; ++it) {
       const int j = it * 64 + t;
@@ -762,51 +769,44 @@ __global__ void __launch_bounds__(kDecThreads, 2)
       const uint32_t rb = uint32_t((brow >> 3) * 1024 + r7 * 128);
       dst0[it] = rb + uint32_t(((2 * c) ^ r7) << 4);
       dst1[it] = rb + uint32_t(((2 * c + 1) ^ r7) << 4);
-      load_ok[it] = live[it] && brow < p.rowsB;
-      gsrc[it] = p.B + (load_ok[it] ? size_t(brow) * ld : 0) + size_t(kb0) * kPK + c * 16;
     }
-    uint4 w[D][JPT];
-#pragma unroll
-    for (int d = 0; d < D; ++d)
+    bool ok = true;
+    for (int i = 0; i < nkb; ++i) {
+      const int sp = i % SP, su = i % SU;
+      if (!warp_wait(&pfull[sp], (i / SP) & 1)) {
+        ok = false;
+        break;
+      }
+      const uint8_t* xs = smem + C::OFF_X + sp * C::X_STAGE;
+      uint4 w[JPT];
 #pragma unroll
       for (int it = 0; it < JPT; ++it)
-        w[d][it] = (d < nkb && load_ok[it]) ? __ldg(reinterpret_cast<const uint4*>(gsrc[it] + d * kPK))
-                                            : make_uint4(0, 0, 0, 0);
-    bool ok = true;
-    for (int i0 = 0; i0 < nkb && ok; i0 += D) {
+        w[it] = live[it] ? *reinterpret_cast<const uint4*>(xs + (it * 64 + t) * 16) : make_uint4(0, 0, 0, 0);
+      if (!warp_wait(&uempty[su], ((i / SU) & 1) ^ 1)) {
+        ok = false;
+        break;
+      }
+      uint8_t* uk = smem + C::OFF_B + su * C::B_STAGE;
 #pragma unroll
-      for (int d = 0; d < D; ++d) {
-        const int i = i0 + d;
-        if (i >= nkb) break;
-        const int su = i % SU;
-        if (!warp_wait(&uempty[su], ((i / SU) & 1) ^ 1)) {
-          if (lane == 0) record_error(p.err, kErrTimeoutUnpack);
-          ok = false;
-          break;
-        }
-        uint8_t* uk = smem + C::OFF_B + su * C::B_STAGE;
-#pragma unroll
-        for (int it = 0; it < JPT; ++it) {
-          if (!live[it]) continue;
-          uint4 o0, o1;
-          unpack8_hi(w[d][it].x, o0.x, o0.y);
-          unpack8_hi(w[d][it].y, o0.z, o0.w);
-          unpack8_hi(w[d][it].z, o1.x, o1.y);
-          unpack8_hi(w[d][it].w, o1.z, o1.w);
-          *reinterpret_cast<uint4*>(uk + dst0[it]) = o0;
-          *reinterpret_cast<uint4*>(uk + dst1[it]) = o1;
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&ufull[su]);
-        if (i + D < nkb) {
-#pragma unroll
-          for (int it = 0; it < JPT; ++it)
-            w[d][it] = load_ok[it] ? __ldg(reinterpret_cast<const uint4*>(gsrc[it] + (i + D) * kPK))
-                                   : make_uint4(0, 0, 0, 0);
-        }
+      for (int it = 0; it < JPT; ++it) {
+        if (!live[it]) continue;
+        uint4 o0, o1;
+        unpack8_hi(w[it].x, o0.x, o0.y);
+        unpack8_hi(w[it].y, o0.z, o0.w);
+        unpack8_hi(w[it].z, o1.x, o1.y);
+        unpack8_hi(w[it].w, o1.z, o1.w);
+        *reinterpret_cast<uint4*>(uk + dst0[it]) = o0;
+        *reinterpret_cast<uint4*>(uk + dst1[it]) = o1;
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      // both stages are released after the stores consumed the loaded registers
+      if (lane == 0) {
+        mbar_arrive(&pempty[sp]);
+        mbar_arrive(&ufull[su]);
       }
     }
+    if (!ok && lane == 0) record_error(p.err, kErrTimeoutUnpack);
   }
 
   if (warp >= 2 && warp < 6) {
@@ -920,15 +920,18 @@ fq_status launch_gemm(const GemmParams& gp, dim3 grid, cudaStream_t stream) {
 template <int BN, int EPI>
 fq_status launch_decode(const GemmParams& gp, dim3 grid, cudaStream_t stream) {
   using C = DecCfg<BN>;
-  CUtensorMap tm;
-  const fq_status st = make_tmap_2d(&tm, gp.A, CU_TENSOR_MAP_DATA_TYPE_UINT8, uint64_t(gp.K) / 2, uint64_t(gp.rowsA),
-                                    uint64_t(gp.K) / 2, uint32_t(kPK), uint32_t(kBM), CU_TENSOR_MAP_SWIZZLE_64B);
+  CUtensorMap tm, tx;
+  fq_status st = make_tmap_2d(&tm, gp.A, CU_TENSOR_MAP_DATA_TYPE_UINT8, uint64_t(gp.K) / 2, uint64_t(gp.rowsA),
+                              uint64_t(gp.K) / 2, uint32_t(kPK), uint32_t(kBM), CU_TENSOR_MAP_SWIZZLE_64B);
+  if (st != FQ_OK) return st;
+  st = make_tmap_2d(&tx, gp.B, CU_TENSOR_MAP_DATA_TYPE_UINT8, uint64_t(gp.K) / 2, uint64_t(gp.rowsB), uint64_t(gp.K) / 2,
+                    uint32_t(kPK), uint32_t(BN));
   if (st != FQ_OK) return st;
   auto kern = gemm_decode_kernel<BN, EPI>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess ||
       cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
     return fail(FQ_ERR_CUDA, "cannot reserve %d bytes of shared memory for the decode GEMM", C::SMEM);
-  kern<<<grid, kDecThreads, C::SMEM, stream>>>(gp, tm);
+  kern<<<grid, kDecThreads, C::SMEM, stream>>>(gp, tm, tx);
   return check_launch("gemm_decode_kernel");
 }
 

@@ -2,25 +2,32 @@
 // cores (FlatQuant notes, 高效 Kernel 设计: transform and quantization fused,
 // intermediates kept on chip; Kronecker 分解: X̂ = P1^T Xbar P2 per token).
 //
-// Each token row is viewed as Xbar (n1 x n2).  Per tile of T tokens a CTA runs:
-//   1. load the fp16 rows (128-bit, coalesced), scale them by c and by a
-//      per-token power of two 2^-e (exact; every fp16 operand and the
-//      intermediate stay below 2^14), split into fp16 hi (+ lo when c is
-//      given; fp16 inputs times 2^-e are exact in fp16) and store them as the
-//      K-major B operand "rows i, K = j" in the 128-byte swizzle;
-//   2. stage A on the tensor cores: U^T = P2^T Xbar^T, i.e. D[l][i] =
-//      sum_j P2[j][l] Xbar[i][j] (tcgen05.mma kind::f16, float32 in tensor
-//      memory).  For n2 = 64 two tokens share one MMA through a
-//      block-diagonal P2^T (token s in K half s, D rows (s, l));
-//   3. U^T is read back row by row (thread = row (s, l), contiguous i), split
-//      into fp16 hi + lo and stored with 16-byte stores as the A operand of
-//   4. stage B: D[(s, l)][k] = sum_i U^T[(s, l)][i] P1[i][k] = X̂_s[k][l],
-//      three passes (hi*hi + hi*lo + lo*hi);
-//   5. thread = column l of X̂ of one token: per-token / per-group absmax via
-//      warp reductions and shared atomics, scale, round-half-even (multiply by
-//      1/s, IEEE division next to ties), clamp, and the codes of 8 x 8 blocks
-//      are packed with a 3-step shuffle transpose into 32-bit stores.
-// Products of fp16 hi/lo parts keep ~22 bits of every operand, so the
+// Each token row is viewed as Xbar (n1 x n2, row-major).  A CTA runs P
+// independent pipelines (4 when the padded n1 is 64, else 2; 1 when c is
+// given with n1 > 64), each with its own tensor-memory region, shared-memory
+// X tile, mbarriers and named barrier, so that one pipeline's tensor-core
+// round trips overlap another's SIMT work.  A pipeline handles one "group"
+// of G tokens at a time (G = 2 for n2 = 64: two tokens share the 128 MMA
+// rows through a block-diagonal P2^T; G = 1 for n2 = 128):
+//   1. the X tile: without c, the fp16 rows land by TMA directly in the
+//      128-byte-swizzled K-major layout of the MMA's B operand (rows i of
+//      Xbar, K = j); with c, the threads form x * c in float32, scale each
+//      row i by a power of two 2^-e_i and store fp16 hi and lo parts;
+//   2. stage A: D[row][i] = sum_j P2[j][l] Xbar[i][j] (row = (s, l) for token
+//      s of the group), P2^T as fp16 hi + lo, float32 accumulation in tensor
+//      memory (kind::f16);
+//   3. thread = row: U^T row = D row (times 2^e_i with c), scaled by a power
+//      of two 2^-e_row that brings its largest entry into [2^13, 2^14), split
+//      into fp16 hi + lo and stored back into tensor memory as the A operand
+//      of
+//   4. stage B: D[row][k] = sum_i U^T[row][i] P1[i][k] (three products
+//      hi*hi + hi*lo + lo*hi, A read from tensor memory);
+//   5. thread = row = column l of token s: X̂[k][l] = D[row][k] * 2^e_row;
+//      per-token (warp max reductions) or per-group maxima, scales,
+//      round-half-even codes (multiply by 1/s, IEEE division next to ties),
+//      and a 3-step shuffle transpose that packs 8 x 8 code blocks into
+//      32-bit stores.
+// Products of fp16 hi/lo parts keep about 22 bits of every operand, so the
 // transform is accurate to float32 level.
 #include <cuda_fp16.h>
 
@@ -49,48 +56,54 @@ struct QuantTcParams {
 namespace {
 
 constexpr int kTcThreads = 512;
-constexpr int kSplit = kTcThreads / 128;           // warps sharing one tensor-memory lane quadrant
-constexpr int kMaxPieces = 2048 / kTcThreads;      // 16-byte pieces of the X tile per thread
+constexpr int kTcWarps = kTcThreads / 32;
 
-template <int N2, int NP>
+template <int N2, int NP, bool HAS_C>
 struct TcCfg {
-  // tokens per tile: n2 = 64 pairs two tokens in K; n2 = 128 stacks 128/NP tokens in N
-  static constexpr int T = N2 == 64 ? 2 : 128 / NP;
-  static constexpr int XROWS = N2 == 64 ? NP : 128;  // rows of the X tile operand (= stage-A N)
-  static constexpr int XKR = 2;                      // 64-wide K regions of the X tile
-  static constexpr int USETS = N2 == 64 ? 1 : T;     // stage-B A operands (one per token when n2 = 128)
-  static constexpr int UKR = NP / 64;                // K regions of the stage-B operands (K = n1 padded)
-  static constexpr int REG = 128 * 128;              // one 128-row x 128-byte region
-  // stage-A A operand P2^T: n2 = 64 keeps [0; P2^T; 0] (192 rows) so that the
-  // two K halves see [P2^T; 0] and [0; P2^T]; n2 = 128 keeps two K regions
+  static constexpr int G = N2 == 64 ? 2 : 1;                // tokens per group (128 MMA rows)
+  static constexpr int P = NP == 64 ? 4 : (HAS_C ? 1 : 2);  // pipelines per CTA
+  static constexpr int WPP = kTcWarps / P;                  // warps per pipeline
+  static constexpr int TPP = WPP * 32;                      // threads per pipeline
+  static constexpr int KSPLIT = WPP / 4;                    // warps sharing a lane quadrant
+  static constexpr int COLS = NP / KSPLIT;                  // D columns per thread (64 or 32)
+  static constexpr int TMEM_PIPE = 2 * NP;                  // D (stage A, then B) + U^T (hi, lo)
+  static constexpr int REG = 128 * 128;                     // one 128-row x 128-byte region
+  // stage-A A operand P2^T hi/lo: n2 = 64 keeps [0; P2^T; 0] (192 rows) so
+  // that the two K halves see [P2^T; 0] and [0; P2^T]; n2 = 128 two K regions
   static constexpr int SA_HALF = (N2 == 64 ? 192 : 256) * 128;
-  static constexpr int SA = 0;
-  static constexpr int SX = SA + 2 * SA_HALF;
-  static constexpr int SX_XHALF = XKR * XROWS * 128;      // X tile hi (lo follows)
-  static constexpr int SX_UHALF = USETS * UKR * REG;      // U^T hi (lo follows)
-  static constexpr int SX_BYTES = (2 * SX_XHALF > 2 * SX_UHALF) ? 2 * SX_XHALF : 2 * SX_UHALF;
-  static constexpr int SL = SX + SX_BYTES;                 // stage-B B operand P1: rows k, K = i
-  static constexpr int SL_HALF = UKR * NP * 128;
-  static constexpr int STG = SL + 2 * SL_HALF;             // fp16 staging of the next tile's rows
-  static constexpr int STG_BYTES = T * NP * N2 * 2;        // (T tokens of at most NP x N2)
-  static constexpr int OFF_MAX = STG + STG_BYTES;          // uint [2] token max, [2][128] group max
-  static constexpr int OFF_BAR = OFF_MAX + 4 * (2 + 256) + 8;
-  static constexpr int OFF_SLOT = OFF_BAR + 24;
+  // X tile: two K regions of NP rows (n2 = 64: one per token; n2 = 128: j halves)
+  static constexpr int X_REG = NP * 128;
+  static constexpr int X_HALF = 2 * X_REG;
+  static constexpr int X_BYTES = HAS_C ? 2 * X_HALF : X_HALF;  // hi (+ lo)
+  // stage-B B operand P1 hi/lo: rows k, K = i in 64-wide regions
+  static constexpr int SL_HALF = (NP / 64) * NP * 128;
+  // per-pipeline scratch (floats): row-max parts [KSPLIT][128], token-max
+  // parts [WPP], group maxima [G][128] (uint), group scales and inverses
+  // [G][128] each, row exponents of the X tile [G][NP] (int, with c)
+  static constexpr int R_RMAX = 0;
+  static constexpr int R_TMAX = R_RMAX + KSPLIT * 128;
+  static constexpr int R_GMAX = R_TMAX + 16;
+  static constexpr int R_SG = R_GMAX + G * 128;
+  static constexpr int R_SINV = R_SG + G * 128;
+  static constexpr int R_XEXP = R_SINV + G * 128;
+  static constexpr int RED_FLOATS = R_XEXP + G * NP;
+  static constexpr int OFF_SA = 0;
+  static constexpr int OFF_SL = OFF_SA + 2 * SA_HALF;
+  static constexpr int OFF_X = OFF_SL + 2 * SL_HALF;
+  static constexpr int OFF_RED = OFF_X + P * X_BYTES;
+  static constexpr int OFF_BAR = OFF_RED + P * RED_FLOATS * 4;
+  static constexpr int OFF_SLOT = OFF_BAR + 3 * P * 8;
   static constexpr int SMEM = OFF_SLOT + 16 + 1024;
-  static constexpr int TMEM_COLS = 128;
   static_assert(N2 == 64 || N2 == 128, "n2");
-  static_assert(NP == 64 || NP == 128, "n1 padding");
-  static_assert((OFF_BAR & 7) == 0, "barrier alignment");
+  static_assert(NP == 64 || NP == 128, "padded n1");
+  static_assert(COLS == 64 || COLS == 32, "columns per thread");
+  static_assert(P * TMEM_PIPE <= 512, "tensor memory");
+  static_assert(SMEM <= 227 * 1024, "shared memory");
+  static_assert((OFF_X % 1024) == 0 && (X_REG % 1024) == 0 && (OFF_BAR % 8) == 0, "alignment");
 };
 
-__device__ __forceinline__ float warp_max_f(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
-}
-
-// Kept out of line: it is the rare path of code_fast and the static path,
-// and inlining its division everywhere bloats the kernel's instruction stream.
+// Kept out of line: it is the rare path of code_scaled / code_fast and the
+// static path, and inlining its division everywhere bloats the kernel.
 __device__ __noinline__ int code_of(float v, float s) {
   if (s == 0.0f) return 0;
   const float r = rintf(__fdiv_rn(v, s));
@@ -110,21 +123,19 @@ __device__ __noinline__ __half group_scale(float amax, float alpha) {
 __device__ __forceinline__ int code_fast(float v, float s, float inv_s) {
   if (s == 0.0f) return 0;
   const float qa = v * inv_s;
-  const float f = qa - floorf(qa);
-  if (fabsf(f - 0.5f) <= fabsf(qa) * 9.5367431640625e-07f + 1e-30f)  // 2^-20 relative margin
+  const float r = rintf(qa);
+  if (0.5f - fabsf(qa - r) <= fabsf(qa) * 9.5367431640625e-07f + 1e-30f)  // 2^-20 relative margin
     return code_of(v, s);
-  return static_cast<int>(fminf(fmaxf(rintf(qa), -8.0f), 7.0f));
+  return __float2int_rn(fminf(fmaxf(r, -8.0f), 7.0f));
 }
 
 // The code of v = u * up (up a power of two, exact) for scale s, given
 // f = up * (1/s) (also exact scaling of the rounded reciprocal): the quotient
 // u * f equals v * fl(1/s), so the tie test of code_fast applies unchanged.
-// Returns the code in the low 4 bits position-free (caller masks).
 __device__ __forceinline__ int code_scaled(float u, float f, float up, float s) {
   const float qa = u * f;
   const float r = rintf(qa);
-  const float d = fabsf(qa - r);  // distance to the nearest integer
-  if (0.5f - d <= fabsf(qa) * 9.5367431640625e-07f + 1e-30f) return code_of(u * up, s);
+  if (0.5f - fabsf(qa - r) <= fabsf(qa) * 9.5367431640625e-07f + 1e-30f) return code_of(u * up, s);
   return __float2int_rn(fminf(fmaxf(r, -8.0f), 7.0f));
 }
 
@@ -137,6 +148,14 @@ __device__ __forceinline__ uint32_t put_nibble(uint32_t w, int q, int pos) {
 
 // 2^e as a float for e in [-126, 127].
 __device__ __forceinline__ float exp2i(int e) { return __int_as_float((e + 127) << 23); }
+
+// Exponent e with 2^-e * mx in [2^13, 2^14) (0 for mx == 0), clamped so that
+// 2^-e and 2^e stay normal floats.
+__device__ __forceinline__ int row_exponent(float mx) {
+  if (!(mx > 0.f)) return 0;
+  const int e = ((__float_as_int(mx) >> 23) & 0xFF) - 127 - 13;
+  return min(max(e, -100), 100);
+}
 
 // Lanes 8g..8g+7 each hold 8 nibbles (nibble b = code of row k0 + b, column
 // l0 + a for lane a of the group); afterwards lane a holds the 8 codes of row
@@ -152,437 +171,409 @@ __device__ __forceinline__ uint32_t transpose_nibbles8(uint32_t w, int lane) {
   return w;
 }
 
-// Two CTAs per SM where the shared memory allows it (n2 = n1 = 64).
-template <int N2, int NP>
-constexpr int tc_min_blocks() { return 1; }
-
-template <int N2, int NP, int GRAN>
-__global__ void __launch_bounds__(kTcThreads, tc_min_blocks<N2, NP>()) quant_act_tc_kernel(const QuantTcParams p) {
-  using C = TcCfg<N2, NP>;
-  constexpr int T = C::T;
+template <int N2, int NP, int GRAN, bool HAS_C>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    quant_act_tc_kernel(const QuantTcParams p, const __grid_constant__ CUtensorMap tmX) {
+  using C = TcCfg<N2, NP, HAS_C>;
+  constexpr int G = C::G, COLS = C::COLS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  unsigned* tokmax = reinterpret_cast<unsigned*>(sm + C::OFF_MAX);  // [2] float bits
-  unsigned* grpmax = tokmax + 2;                                     // [2][128] float bits
-  uint64_t* barA = reinterpret_cast<uint64_t*>(sm + C::OFF_BAR);
-  uint64_t* barB = barA + 1;
-  uint64_t* barX = barA + 2;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + C::OFF_SLOT);
-
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int pipe = warp / C::WPP, pw = warp % C::WPP;  // pipeline, warp within it
+  const int ptid = tid - pipe * C::TPP;
+  const int q4 = warp & 3;                             // tensor-memory lane quadrant
+  const int part = pw >> 2;                            // column part of the row
+  const int m = q4 * 32 + lane;                        // D row of this thread
   const int n1 = p.n1, K = p.K, M = p.M;
-  const bool has_c = p.c != nullptr;
-  const int ntiles = (M + T - 1) / T;
-
-  // rows of tile `tile` -> staging buffer (bulk copy, async proxy)
-  auto issue_tile = [&](int tile) {
-    if (tile < ntiles) {
-      const int tok0 = tile * T;
-      const int ntok = min(T, M - tok0);
-      const uint32_t bytes = uint32_t(ntok) * uint32_t(K) * 2u;
-      mbar_arrive_expect_tx(barX, bytes);
-      bulk_load(sm + C::STG, p.X + size_t(tok0) * K, bytes, barX);
-    }
-  };
+  const int ngroups = (M + G - 1) / G;
+  uint64_t* xfull = reinterpret_cast<uint64_t*>(sm + C::OFF_BAR) + 3 * pipe;
+  uint64_t* mmaA = xfull + 1;
+  uint64_t* mmaB = xfull + 2;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + C::OFF_SLOT);
+  float* red = reinterpret_cast<float*>(sm + C::OFF_RED) + pipe * C::RED_FLOATS;
+  uint32_t* gmax = reinterpret_cast<uint32_t*>(red + C::R_GMAX);
+  int* xexp = reinterpret_cast<int*>(red + C::R_XEXP);
+  uint8_t* xt = sm + C::OFF_X + pipe * C::X_BYTES;
 
   if (tid == 0) {
-    mbar_init(barA, 1);
-    mbar_init(barB, 1);
-    mbar_init(barX, 1);
+    for (int b = 0; b < 3 * C::P; ++b) mbar_init(reinterpret_cast<uint64_t*>(sm + C::OFF_BAR) + b, 1);
     fence_mbar_init();
-    issue_tile(blockIdx.x);
   }
   if (warp == 0) {
-    tmem_alloc(tslot, C::TMEM_COLS);
+    tmem_alloc(tslot, 512);
     tmem_relinquish();
   }
-  // ---- factors -> fp16 hi/lo operands, once per CTA (zero-filled first)
-  for (int c = tid; c < (2 * C::SA_HALF) / 16; c += kTcThreads)
-    *reinterpret_cast<uint4*>(sm + C::SA + c * 16) = make_uint4(0, 0, 0, 0);
-  for (int c = tid; c < (2 * C::SL_HALF) / 16; c += kTcThreads)
-    *reinterpret_cast<uint4*>(sm + C::SL + c * 16) = make_uint4(0, 0, 0, 0);
+  // operands and scratch start at zero (padding rows and columns stay zero)
+  for (int c = tid; c < C::OFF_BAR / 16; c += kTcThreads)
+    reinterpret_cast<uint4*>(sm)[c] = make_uint4(0, 0, 0, 0);
   __syncthreads();
-  float csum = 0.f;  // part of the |P2| column sum of column tid % N2
+  // ---- factors -> fp16 hi/lo operands, once per CTA
   for (int e = tid; e < N2 * N2; e += kTcThreads) {
-    const int j = e / N2, l = e % N2;  // A operand of stage A: row l, K index j, value P2[j][l]
+    const int j = e / N2, l = e % N2;  // stage-A A operand: row l, K index j, value P2[j][l]
     const float v = __ldg(p.P2 + e);
-    csum += fabsf(v);
     const __half hi = __float2half_rn(v);
     const __half lo = __float2half_rn(v - __half2float(hi));
     const int row = N2 == 64 ? 64 + l : l;
     const uint32_t off = (N2 == 64 ? 0u : uint32_t(j >> 6) * C::REG) + sw128_offset(row, (j & 63) * 2);
-    *reinterpret_cast<__half*>(sm + C::SA + off) = hi;
-    *reinterpret_cast<__half*>(sm + C::SA + C::SA_HALF + off) = lo;
+    *reinterpret_cast<__half*>(sm + C::OFF_SA + off) = hi;
+    *reinterpret_cast<__half*>(sm + C::OFF_SA + C::SA_HALF + off) = lo;
   }
   for (int e = tid; e < n1 * n1; e += kTcThreads) {
-    const int i = e / n1, k = e % n1;  // B operand of stage B: row k, K index i, value P1[i][k]
+    const int i = e / n1, k = e % n1;  // stage-B B operand: row k, K index i, value P1[i][k]
     const float v = __ldg(p.P1 + e);
     const __half hi = __float2half_rn(v);
     const __half lo = __float2half_rn(v - __half2float(hi));
     const uint32_t off = uint32_t(i >> 6) * (NP * 128) + sw128_offset(k, (i & 63) * 2);
-    *reinterpret_cast<__half*>(sm + C::SL + off) = hi;
-    *reinterpret_cast<__half*>(sm + C::SL + C::SL_HALF + off) = lo;
+    *reinterpret_cast<__half*>(sm + C::OFF_SL + off) = hi;
+    *reinterpret_cast<__half*>(sm + C::OFF_SL + C::SL_HALF + off) = lo;
   }
-  // largest absolute column sum of P2 (bounds |U| by max|x| * colsum)
-  // column sums: thread tid holds part of column tid % N2; fold into 256 slots first
-  float* colsum = reinterpret_cast<float*>(grpmax);
-  if (tid < 256) colsum[tid] = 0.f;
-  __syncthreads();
-  atomicAdd(&colsum[tid & 255], csum);  // 256 is a multiple of N2: slot keeps the column
-  __syncthreads();
-  float cs = 0.f;
-  if (tid < N2)
-    for (int r = tid; r < 256; r += N2) cs += colsum[r];
-  cs = warp_max_f(cs);
-  __syncthreads();
-  if (lane == 0) colsum[warp] = cs;
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  float guard = 1.f;
-  for (int w = 0; w < kTcThreads / 32; ++w) guard = fmaxf(guard, colsum[w]);
+
   const uint32_t tmem = *tslot;
-  __syncthreads();
+  const uint32_t tD = tmem + uint32_t(pipe * C::TMEM_PIPE);  // D: stage A, then stage B
+  const uint32_t tU = tD + uint32_t(NP);                      // U^T: hi [0, NP/2), lo [NP/2, NP)
+  const uint32_t lane_off = uint32_t(q4 * 32) << 16;
+  const int bar_id = 1 + pipe;
+  const bool leader = pw == 0 && lane == 0;
+  const uint32_t idesc = idesc_f16_m128(NP);
+  const bool c_vec = HAS_C && (reinterpret_cast<uintptr_t>(p.c) & 15u) == 0;  // c in 16-byte pieces
+  const int s_of_row = N2 == 64 ? (m >> 6) : 0;  // token of this D row within the group
+  const int l_of_row = N2 == 64 ? (m & 63) : m;  // column l of X̂ this row holds
 
-  const int npieces = T * K / 8;
-  const int q4 = warp & 3, part = warp >> 2;  // lane quadrant, column part (0..kSplit-1)
-  const uint32_t tl = tmem + (uint32_t(q4 * 32) << 16);
-  const int m = q4 * 32 + lane;  // tensor-memory lane of this thread
-  constexpr uint32_t idescA = idesc_f16_m128(C::XROWS);
-  constexpr uint32_t idescB = idesc_f16_m128(NP);
-
-  uint32_t phase = 0;
-  bool inflight = blockIdx.x < ntiles;  // a bulk copy into the staging buffer is outstanding
-  uint32_t inflight_parity = 0;
-  for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-    const int tok0 = tile * T;
-    if (tid < 2) tokmax[tid] = 0u;
-    for (int i = tid; i < 256; i += kTcThreads) grpmax[i] = 0u;
-    bool okx = warp_wait(barX, phase);  // this tile's rows are in the staging buffer
-    inflight = false;
-
-    // ---- 1a. per-token max of c * x
-    uint4 buf[kMaxPieces];
-    float mx0 = 0.f, mx1 = 0.f;
-#pragma unroll
-    for (int it = 0; it < kMaxPieces; ++it) {
-      const int pc = tid + kTcThreads * it;
-      buf[it] = make_uint4(0, 0, 0, 0);
-      if (pc < npieces && tok0 + (pc * 8) / K < M) buf[it] = *reinterpret_cast<const uint4*>(sm + C::STG + pc * 16);
+  // TMA of the fp16 X tile of group grp (rows i of Xbar, K = j)
+  auto issue_x = [&](int grp) {
+    const int tok0 = grp * G;
+    mbar_arrive_expect_tx(xfull, uint32_t(256 * n1));
+    if (N2 == 64) {
+      tma_load_2d(xt, &tmX, xfull, 0, tok0 * n1);
+      tma_load_2d(xt + C::X_REG, &tmX, xfull, 0, (tok0 + 1) * n1);
+    } else {
+      tma_load_2d(xt, &tmX, xfull, 0, tok0 * n1);
+      tma_load_2d(xt + C::X_REG, &tmX, xfull, 64, tok0 * n1);
     }
-#pragma unroll
-    for (int it = 0; it < kMaxPieces; ++it) {
-      const int pc = tid + kTcThreads * it;
-      if (pc < npieces) {
-        const int e = pc * 8, t = e / K, f = e - t * K;
-        const __half2* h2 = reinterpret_cast<const __half2*>(&buf[it]);
-        float mm = 0.f;
-        if (has_c) {
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const float2 v = __half22float2(h2[j]);
-            const float a = __fmul_rn(v.x, __ldg(p.c + f + 2 * j));
-            const float b = __fmul_rn(v.y, __ldg(p.c + f + 2 * j + 1));
-            mm = fmaxf(mm, fmaxf(fabsf(a), fabsf(b)));
-          }
+  };
+
+  const int gstride = gridDim.x * C::P;
+  int grp = blockIdx.x * C::P + pipe;
+  bool x_pending = false;  // (leader) a TMA into the X tile has not been waited for
+  if (!HAS_C && leader && grp < ngroups) {
+    prefetch_tensormap(&tmX);
+    issue_x(grp);
+    x_pending = true;
+  }
+  uint32_t ph = 0;
+  bool bad = false;
+  for (; grp < ngroups; grp += gstride, ph ^= 1u) {
+    const int tok0 = grp * G;
+
+    // ---- 1. X tile
+    if (HAS_C) {
+      constexpr int PPR = N2 / 8;  // 16-byte pieces per row i of Xbar
+      const int npieces = G * K / 8;
+      for (int pc = ptid; pc < npieces; pc += C::TPP) {
+        const int t = pc / (K / 8), f = (pc - t * (K / 8)) * 8;
+        const int i = f / N2, j0 = f % N2;
+        const int tok = tok0 + t;
+        uint4 raw = make_uint4(0, 0, 0, 0);
+        if (tok < M) raw = *reinterpret_cast<const uint4*>(p.X + size_t(tok) * K + f);
+        float cv[8];
+        if (c_vec) {
+          const float4 c0 = __ldg(reinterpret_cast<const float4*>(p.c + f));
+          const float4 c1 = __ldg(reinterpret_cast<const float4*>(p.c + f + 4));
+          cv[0] = c0.x, cv[1] = c0.y, cv[2] = c0.z, cv[3] = c0.w;
+          cv[4] = c1.x, cv[5] = c1.y, cv[6] = c1.z, cv[7] = c1.w;
         } else {
-          // the max of |x| is exact in fp16
-          const __half2 m2 = __hmax2(__hmax2(__habs2(h2[0]), __habs2(h2[1])), __hmax2(__habs2(h2[2]), __habs2(h2[3])));
-          mm = fmaxf(__low2float(m2), __high2float(m2));
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj) cv[jj] = __ldg(p.c + f + jj);
         }
-        if (t == 0) mx0 = fmaxf(mx0, mm); else mx1 = fmaxf(mx1, mm);
-      }
-    }
-    mx0 = warp_max_f(mx0);
-    mx1 = warp_max_f(mx1);
-    __syncthreads();  // maxima cleared, previous tile finished
-    if (lane == 0) {
-      atomicMax(&tokmax[0], __float_as_uint(mx0));
-      atomicMax(&tokmax[1], __float_as_uint(mx1));
-    }
-    __syncthreads();
-    int texp[2];
+        const __half2* h2 = reinterpret_cast<const __half2*>(&raw);
+        float v[8];
+        float mx = 0.f;
 #pragma unroll
-    for (int t = 0; t < 2; ++t) {
-      const float mt = __uint_as_float(tokmax[t]);
-      int E = 0;
-      if (mt > 0.f) frexpf(mt * guard, &E);
-      texp[t] = mt > 0.f ? min(max(E - 14, -100), 100) : 0;  // scaled max * guard <= 2^14
-    }
-    __syncthreads();  // everyone has read the token maxima
-    if (tid < 2) tokmax[tid] = 0u;  // reused for the maxima of the transformed values
-    // ---- 1b. scaled X tile: element (token t, row i, column j) -> operand row, K index
+        for (int jj = 0; jj < 4; ++jj) {
+          const float2 x2 = __half22float2(h2[jj]);
+          v[2 * jj] = __fmul_rn(x2.x, cv[2 * jj]);
+          v[2 * jj + 1] = __fmul_rn(x2.y, cv[2 * jj + 1]);
+          mx = fmaxf(mx, fmaxf(fabsf(v[2 * jj]), fabsf(v[2 * jj + 1])));
+        }
+        // max over the row's PPR pieces (consecutive lanes)
 #pragma unroll
-    for (int it = 0; it < kMaxPieces; ++it) {
-      const int pc = tid + kTcThreads * it;
-      if (pc < npieces) {
-        const int e = pc * 8, t = e / K, f = e - t * K;
-        const int i = f / N2, j = f % N2;
-        const int row = N2 == 64 ? i : t * NP + i;
-        const int kidx = N2 == 64 ? t * 64 + j : j;
-        const uint32_t off = uint32_t(kidx >> 6) * (C::XROWS * 128) + sw128_offset(row, (kidx & 63) * 2);
-        const float sc = exp2i(-texp[t]);
-        const __half2* h2 = reinterpret_cast<const __half2*>(&buf[it]);
+        for (int o = 1; o < PPR; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        const int e = row_exponent(mx);
+        const float sc = exp2i(-e);
+        if (j0 == 0) xexp[t * NP + i] = e;
         uint4 hi, lo;
         __half2* hh = reinterpret_cast<__half2*>(&hi);
         __half2* ll = reinterpret_cast<__half2*>(&lo);
-        if (!has_c && texp[t] >= -15 && texp[t] <= 14) {
-          // fp16 x times an fp16 power of two: exact (the result stays below 2^14)
-          const __half2 sc2 = __float2half2_rn(sc);
-#pragma unroll
-          for (int jj = 0; jj < 4; ++jj) hh[jj] = __hmul2(h2[jj], sc2);
-          *reinterpret_cast<uint4*>(sm + C::SX + off) = hi;
-          continue;
-        }
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
-          float2 v = __half22float2(h2[jj]);
-          if (has_c) {
-            v.x = __fmul_rn(v.x, __ldg(p.c + f + 2 * jj));
-            v.y = __fmul_rn(v.y, __ldg(p.c + f + 2 * jj + 1));
-          }
-          v.x *= sc;
-          v.y *= sc;
-          const __half2 a = __floats2half2_rn(v.x, v.y);
-          const float2 af = __half22float2(a);
-          hh[jj] = a;
-          ll[jj] = __floats2half2_rn(v.x - af.x, v.y - af.y);
+          const float a = v[2 * jj] * sc, b = v[2 * jj + 1] * sc;
+          const __half2 h = __floats2half2_rn(a, b);
+          const float2 hf = __half22float2(h);
+          hh[jj] = h;
+          ll[jj] = __floats2half2_rn(a - hf.x, b - hf.y);
         }
-        *reinterpret_cast<uint4*>(sm + C::SX + off) = hi;
-        if (has_c) *reinterpret_cast<uint4*>(sm + C::SX + C::SX_XHALF + off) = lo;
+        const int region = N2 == 64 ? t : (j0 >> 6);
+        const uint32_t off = uint32_t(region) * C::X_REG + sw128_offset(i, (j0 & 63) * 2);
+        *reinterpret_cast<uint4*>(xt + off) = hi;
+        *reinterpret_cast<uint4*>(xt + C::X_HALF + off) = lo;
+      }
+      fence_proxy_async_smem();
+      named_barrier(bar_id, C::TPP);
+    } else if (leader) {
+      if (mbar_wait(xfull, ph)) {
+        x_pending = false;
+      } else {
+        record_error(p.err, kErrTimeoutProducer);
+        bad = true;
       }
     }
-    // zero the padding rows i >= n1 of every token slot (all rows of an empty slot)
-    {
-      constexpr int kRegPerRow = N2 == 64 ? 1 : 2;  // K regions a token row spans
-      constexpr int chunks = 8 * kRegPerRow;       // 16-byte chunks per padded row
-      for (int t = 0; t < T; ++t) {
-        const int i0 = (tok0 + t < M) ? n1 : 0;
-        const int total = (NP - i0) * chunks;
-        for (int cidx = tid; cidx < total; cidx += kTcThreads) {
-          const int r = cidx / chunks, rem = cidx % chunks;
-          const int kidx = (N2 == 64 ? t * 64 : (rem / 8) * 64) + (rem % 8) * 8;
-          const int row = N2 == 64 ? i0 + r : t * NP + i0 + r;
-          const uint32_t off = uint32_t(kidx >> 6) * (C::XROWS * 128) + sw128_offset(row, (kidx & 63) * 2);
-          *reinterpret_cast<uint4*>(sm + C::SX + off) = make_uint4(0, 0, 0, 0);
-          if (has_c) *reinterpret_cast<uint4*>(sm + C::SX + C::SX_XHALF + off) = make_uint4(0, 0, 0, 0);
-        }
-      }
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    if (__syncthreads_or(!okx)) {
-      if (tid == 0) record_error(p.err, kErrTimeoutUnpack);
-      break;
-    }
-    if (tid == 0) issue_tile(tile + gridDim.x);  // the next tile's rows land during this one
-    inflight = tile + int(gridDim.x) < ntiles;
-    inflight_parity = phase ^ 1u;
 
-    // ---- 2. stage A: D[l][i] = sum_j P2^T[l][j] Xbar[i][j]
-    if (tid == 0) {
+    // ---- 2. stage A: D[row][i] = sum_j P2^T[l][j] Xbar_s[i][j]
+    if (leader && !bad) {
       tc_fence_after();
-      const uint32_t sa = smem_u32(sm + C::SA), sx = smem_u32(sm + C::SX);
+      const uint32_t sa = smem_u32(sm + C::OFF_SA), sx = smem_u32(xt);
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         const int kr = kk >> 2;
         const uint32_t oa =
             (N2 == 64 ? uint32_t(kr == 0 ? 64 : 0) * 128u : uint32_t(kr) * C::REG) + uint32_t(kk & 3) * 32u;
-        const uint32_t ob = uint32_t(kr) * (C::XROWS * 128) + uint32_t(kk & 3) * 32u;
+        const uint32_t ob = uint32_t(kr) * C::X_REG + uint32_t(kk & 3) * 32u;
         const uint64_t ahi = sdesc_k128_sw128(sa + oa), alo = sdesc_k128_sw128(sa + C::SA_HALF + oa);
         const uint64_t bhi = sdesc_k128_sw128(sx + ob);
-        mma_f16(tmem, ahi, bhi, idescA, kk > 0);
-        mma_f16(tmem, alo, bhi, idescA, 1);
-        if (has_c) mma_f16(tmem, ahi, sdesc_k128_sw128(sx + C::SX_XHALF + ob), idescA, 1);
+        mma_f16(tD, ahi, bhi, idesc, kk > 0);
+        mma_f16(tD, alo, bhi, idesc, 1);
+        if (HAS_C) mma_f16(tD, ahi, sdesc_k128_sw128(sx + C::X_HALF + ob), idesc, 1);
       }
-      mma_commit(barA);
+      mma_commit(mmaA);
     }
-    bool ok = warp_wait(barA, phase);
+    if (!warp_wait(mmaA, ph)) bad = true;
     tc_fence_after();
+    // the X tile is free again: the next group's rows land during steps 3-5
+    if (!HAS_C && leader && !bad && grp + gstride < ngroups) {
+      issue_x(grp + gstride);
+      x_pending = true;
+    }
 
-    // ---- 3. U^T rows -> fp16 hi/lo, 16-byte stores (stage-B operand A: row m, K index i)
+    // ---- 3. U^T rows: D row (times 2^e_i with c), row scale 2^-e_row, fp16 hi/lo -> tensor memory
+    int e_row;
     {
-      constexpr int CW = C::XROWS / kSplit;  // columns per thread: 16 or 32
-      uint32_t u[32];
-      if (CW == 32)
-        tmem_ld_32x32(tl + uint32_t(part * CW), u);
-      else
-        tmem_ld_32x16(tl + uint32_t(part * CW), u);
-      tmem_wait_ld();
-      {
-        const int col = part * CW;  // D column = X tile row = (t, i)
-        const int us = N2 == 64 ? 0 : col / NP;
-        const int i0 = N2 == 64 ? col : col % NP;
-        uint8_t* ub = sm + C::SX + us * (C::UKR * C::REG) + (i0 >> 6) * C::REG;
+      float mx = 0.f;
 #pragma unroll
-        for (int g = 0; g < CW / 8; ++g) {
-          uint4 hi, lo;
-          __half2* hh = reinterpret_cast<__half2*>(&hi);
-          __half2* ll = reinterpret_cast<__half2*>(&lo);
+      for (int c = 0; c < COLS / 32; ++c) {
+        uint32_t u[32];
+        tmem_ld_32x32(tD + lane_off + uint32_t(part * COLS + 32 * c), u);
+        tmem_wait_ld();
 #pragma unroll
-          for (int jj = 0; jj < 4; ++jj) {
-            const float a = __uint_as_float(u[g * 8 + 2 * jj]), b = __uint_as_float(u[g * 8 + 2 * jj + 1]);
-            const __half2 h = __floats2half2_rn(a, b);
-            const float2 hf = __half22float2(h);
-            hh[jj] = h;
-            ll[jj] = __floats2half2_rn(a - hf.x, b - hf.y);
+        for (int j = 0; j < 32; ++j) {
+          float v = __uint_as_float(u[j]);
+          if (HAS_C) v *= exp2i(xexp[s_of_row * NP + part * COLS + 32 * c + j]);
+          mx = fmaxf(mx, fabsf(v));
+        }
+      }
+      if (C::KSPLIT > 1) {
+        red[C::R_RMAX + part * 128 + m] = mx;
+        named_barrier(bar_id, C::TPP);
+#pragma unroll
+        for (int pp = 0; pp < C::KSPLIT; ++pp) mx = fmaxf(mx, red[C::R_RMAX + pp * 128 + m]);
+      }
+      e_row = row_exponent(mx);
+      const float sc = exp2i(-e_row);
+#pragma unroll
+      for (int c = 0; c < COLS / 32; ++c) {
+        uint32_t u[32];
+        tmem_ld_32x32(tD + lane_off + uint32_t(part * COLS + 32 * c), u);
+        tmem_wait_ld();
+        uint32_t hi[16], lo[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          float a = __uint_as_float(u[2 * j]), b = __uint_as_float(u[2 * j + 1]);
+          if (HAS_C) {
+            a *= exp2i(xexp[s_of_row * NP + part * COLS + 32 * c + 2 * j]);
+            b *= exp2i(xexp[s_of_row * NP + part * COLS + 32 * c + 2 * j + 1]);
           }
-          const uint32_t off = sw128_offset(m, ((i0 & 63) + g * 8) * 2);
-          *reinterpret_cast<uint4*>(ub + off) = hi;
-          *reinterpret_cast<uint4*>(ub + C::SX_UHALF + off) = lo;
+          a *= sc;
+          b *= sc;
+          const __half2 h = __floats2half2_rn(a, b);
+          const float2 hf = __half22float2(h);
+          const __half2 l2 = __floats2half2_rn(a - hf.x, b - hf.y);
+          hi[j] = *reinterpret_cast<const uint32_t*>(&h);
+          lo[j] = *reinterpret_cast<const uint32_t*>(&l2);
         }
+        const uint32_t col = uint32_t(part * COLS / 2 + 16 * c);
+        tmem_st_32x16(tU + lane_off + col, hi);
+        tmem_st_32x16(tU + lane_off + uint32_t(NP / 2) + col, lo);
       }
     }
-    fence_proxy_async_smem();
+    // the group maxima of step 5 start from zero
+    if (GRAN == FQ_DYNAMIC_GROUP)
+      for (int e = ptid; e < G * 128; e += C::TPP) gmax[e] = 0u;
+    tmem_wait_st();
     tc_fence_before();
-    if (__syncthreads_or(!ok)) {
-      if (tid == 0) record_error(p.err, kErrTimeoutMma);
-      break;
-    }
+    bad = named_barrier_or(bar_id, C::TPP, bad);
+    if (bad) break;
 
-    // ---- 4. stage B: D[(s, l)][k] = sum_i U^T[(s, l)][i] P1[i][k]
-    if (tid == 0) {
+    // ---- 4. stage B: D[row][k] = sum_i U^T[row][i] P1[i][k]
+    if (leader) {
       tc_fence_after();
-      const uint32_t sx = smem_u32(sm + C::SX), sl = smem_u32(sm + C::SL);
+      const uint32_t sl = smem_u32(sm + C::OFF_SL);
 #pragma unroll
-      for (int us = 0; us < C::USETS; ++us) {
-#pragma unroll
-        for (int kk = 0; kk < NP / 16; ++kk) {
-          const uint32_t oa = uint32_t(us * C::UKR + (kk >> 2)) * C::REG + uint32_t(kk & 3) * 32u;
-          const uint32_t ob = uint32_t(kk >> 2) * (NP * 128) + uint32_t(kk & 3) * 32u;
-          const uint64_t ahi = sdesc_k128_sw128(sx + oa), alo = sdesc_k128_sw128(sx + C::SX_UHALF + oa);
-          const uint64_t bhi = sdesc_k128_sw128(sl + ob), blo = sdesc_k128_sw128(sl + C::SL_HALF + ob);
-          const uint32_t d = tmem + uint32_t(us * NP);
-          mma_f16(d, ahi, bhi, idescB, kk > 0);
-          mma_f16(d, ahi, blo, idescB, 1);
-          mma_f16(d, alo, bhi, idescB, 1);
-        }
+      for (int kk = 0; kk < NP / 16; ++kk) {
+        const uint32_t ob = uint32_t(kk >> 2) * (NP * 128) + uint32_t(kk & 3) * 32u;
+        const uint64_t bhi = sdesc_k128_sw128(sl + ob), blo = sdesc_k128_sw128(sl + C::SL_HALF + ob);
+        const uint32_t ahi = tU + uint32_t(8 * kk), alo = tU + uint32_t(NP / 2 + 8 * kk);
+        mma_f16_ts(tD, ahi, bhi, idesc, kk > 0);
+        mma_f16_ts(tD, ahi, blo, idesc, 1);
+        mma_f16_ts(tD, alo, bhi, idesc, 1);
       }
-      mma_commit(barB);
+      mma_commit(mmaB);
     }
-    ok = warp_wait(barB, phase);
+    if (!warp_wait(mmaB, ph)) bad = true;
     tc_fence_after();
-    if (__syncthreads_or(!ok)) {
-      if (tid == 0) record_error(p.err, kErrTimeoutMma);
-      break;
-    }
 
-    // ---- 5. quantize: thread = column l of X̂ of one token, columns k in chunks of 8
-    for (int us = 0; us < C::USETS; ++us) {
-      const int t = N2 == 64 ? (m >> 6) : us;  // token slot of this thread
-      const int l = N2 == 64 ? (m & 63) : m;
-      const int tok = tok0 + t;
+    // ---- 5. quantize: thread = row (s, l), columns k of this part
+    {
+      const int s = s_of_row, l = l_of_row;
+      const int tok = tok0 + s;
       const bool tok_ok = tok < M;
-      const float up = exp2i(texp[t]);
-      const uint32_t cbase = tl + uint32_t(us * NP);
-      constexpr int NCH = NP / 8 / kSplit;  // 8-column chunks of this thread (part, part + kSplit, ...)
-      uint32_t u[NCH][8];
-#pragma unroll
-      for (int c = 0; c < NCH; ++c) tmem_ld_32x8(cbase + uint32_t((kSplit * c + part) * 8), u[c]);
-      tmem_wait_ld();
-      // pass 1: token / group maxima (rows k >= n1 and empty token slots hold zeros)
+      const float up = exp2i(e_row);
+      // pass 1: maxima (columns k >= n1 and empty token slots hold zeros)
       float tm = 0.f;
 #pragma unroll
-      for (int c = 0; c < NCH; ++c) {
-        const int ch = kSplit * c + part;
+      for (int c = 0; c < COLS / 32; ++c) {
+        uint32_t u[32];
+        tmem_ld_32x32(tD + lane_off + uint32_t(part * COLS + 32 * c), u);
+        tmem_wait_ld();
+        if (GRAN == FQ_DYNAMIC_GROUP) {
+          // group of element (k, l): (k * n2 + l) / 128, i.e. k (n2 = 128) or k / 2 (n2 = 64)
+          constexpr int KPG = 128 / N2;  // columns k per group
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float a = fabsf(__uint_as_float(u[c][j]));
-          tm = fmaxf(tm, a);
-          if (GRAN == FQ_DYNAMIC_GROUP) {
-            const int k = ch * 8 + j;
-            const float w = warp_max_f(a) * up;
-            if (lane == 0 && k < n1) atomicMax(&grpmax[t * 128 + (k * N2) / kGroup], __float_as_uint(w));
+          for (int j = 0; j < 32; j += KPG) {
+            float a = fabsf(__uint_as_float(u[j]));
+            if (KPG == 2) a = fmaxf(a, fabsf(__uint_as_float(u[j + 1])));
+            const uint32_t r = warp_max_u32(__float_as_uint(a * up));
+            const int g = (part * COLS + 32 * c + j) / KPG;
+            if (lane == 0) atomicMax(&gmax[s * 128 + g], r);
           }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) tm = fmaxf(tm, fabsf(__uint_as_float(u[j])));
         }
       }
-      tm = warp_max_f(tm) * up;
-      if (lane == 0) atomicMax(&tokmax[t], __float_as_uint(tm));
-      __syncthreads();
-      // pass 2: codes
       float s_tok = 0.f, f_tok = 0.f;
       if (GRAN == FQ_DYNAMIC_ROW) {
-        s_tok = __fdiv_rn(__fmul_rn(__uint_as_float(tokmax[t]), p.alpha), 7.0f);
+        const uint32_t r = warp_max_u32(__float_as_uint(tm * up));
+        if (lane == 0) red[C::R_TMAX + pw] = __uint_as_float(r);
+        named_barrier(bar_id, C::TPP);
+        // warps holding the rows of token s: quadrants 2s, 2s + 1 (n2 = 64) or all four
+        float amax = 0.f;
+#pragma unroll
+        for (int pp = 0; pp < C::KSPLIT; ++pp) {
+          if (N2 == 64) {
+            amax = fmaxf(amax, red[C::R_TMAX + pp * 4 + 2 * s]);
+            amax = fmaxf(amax, red[C::R_TMAX + pp * 4 + 2 * s + 1]);
+          } else {
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq) amax = fmaxf(amax, red[C::R_TMAX + pp * 4 + qq]);
+          }
+        }
+        s_tok = __fdiv_rn(__fmul_rn(amax, p.alpha), 7.0f);
         f_tok = s_tok != 0.f ? (1.0f / s_tok) * up : 0.f;
         if (tok_ok && l == 0 && part == 0) p.s_row[tok] = s_tok;
-      }
-#pragma unroll
-      for (int c = 0; c < NCH; ++c) {
-        const int ch = kSplit * c + part;
-        uint32_t word = 0;
-        float sg = 0.f, inv_g = 0.f;
-        int gcur = -1;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int k = ch * 8 + j;
-          const float uu = __uint_as_float(u[c][j]);
-          const float v = uu * up;
-          int q = 0;
-          if (k < n1) {
-            if (GRAN == FQ_DYNAMIC_ROW) {
-              q = s_tok != 0.f ? code_scaled(uu, f_tok, up, s_tok) : 0;
-            } else if (GRAN == FQ_DYNAMIC_GROUP) {
-              const int g = (k * N2) / kGroup;
-              if (g != gcur) {
-                gcur = g;
-                const __half sh = group_scale(__uint_as_float(grpmax[t * 128 + g]), p.alpha);
-                sg = __half2float(sh);
-                inv_g = sg != 0.f ? 1.0f / sg : 0.f;
-                if (tok_ok && l == 0 && (k * N2) % kGroup == 0) p.s_grp[size_t(g) * M + tok] = sh;
-              }
-              q = code_fast(v, sg, inv_g);
-            } else {
-              q = code_of(v, __ldg(p.sstatic + k * N2 + l));
-            }
-            if (p.xhat && tok_ok) p.xhat[size_t(tok) * K + k * N2 + l] = v;
-          }
-          word = put_nibble(word, q, 4 * j);
+      } else if (GRAN == FQ_DYNAMIC_GROUP) {
+        named_barrier(bar_id, C::TPP);
+        const int ngr = n1 * N2 / 128;  // groups per token
+        for (int e = ptid; e < G * ngr; e += C::TPP) {
+          const int ts = e / ngr, g = e - ts * ngr;
+          const __half sh = group_scale(__uint_as_float(gmax[ts * 128 + g]), p.alpha);
+          const float sg = __half2float(sh);
+          red[C::R_SG + ts * 128 + g] = sg;
+          red[C::R_SINV + ts * 128 + g] = sg != 0.f ? 1.0f / sg : 0.f;
+          if (tok0 + ts < M) p.s_grp[size_t(g) * M + tok0 + ts] = sh;
         }
-        word = transpose_nibbles8(word, lane);
-        const int k = ch * 8 + (lane & 7);
-        const int l0 = l & ~7;
-        if (tok_ok && k < n1)
-          *reinterpret_cast<uint32_t*>(p.Q + size_t(tok) * (K / 2) + (k * N2 + l0) / 2) = word;
+        named_barrier(bar_id, C::TPP);
       }
-      __syncthreads();
+      // pass 2: codes, 8 columns k per 32-bit word, transposed to 8 columns l
+#pragma unroll
+      for (int c = 0; c < COLS / 32; ++c) {
+        uint32_t u[32];
+        tmem_ld_32x32(tD + lane_off + uint32_t(part * COLS + 32 * c), u);
+        tmem_wait_ld();
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          const int k0 = part * COLS + 32 * c + 8 * ch;
+          uint32_t word = 0;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int k = k0 + j;
+            const float d = __uint_as_float(u[8 * ch + j]);
+            int qv = 0;
+            if (GRAN == FQ_DYNAMIC_ROW) {
+              qv = s_tok != 0.f ? code_scaled(d, f_tok, up, s_tok) : 0;
+            } else if (GRAN == FQ_DYNAMIC_GROUP) {
+              const int g = k * N2 / 128;
+              qv = code_fast(d * up, red[C::R_SG + s * 128 + g], red[C::R_SINV + s * 128 + g]);
+            } else if (k < n1) {
+              qv = code_of(d * up, __ldg(p.sstatic + k * N2 + l));
+            }
+            if (p.xhat && tok_ok && k < n1) p.xhat[size_t(tok) * K + k * N2 + l] = d * up;
+            word = put_nibble(word, qv, 4 * j);
+          }
+          word = transpose_nibbles8(word, lane);
+          const int kr = k0 + (lane & 7);
+          const int l0 = l & ~7;
+          if (tok_ok && kr < n1)
+            *reinterpret_cast<uint32_t*>(p.Q + size_t(tok) * (K / 2) + (kr * N2 + l0) / 2) = word;
+        }
+      }
     }
     tc_fence_before();
-    __syncthreads();
-    phase ^= 1u;
+    bad = named_barrier_or(bar_id, C::TPP, bad);  // D, U^T and the scratch are free again
+    if (bad) break;
   }
+  if (bad && ptid == 0) record_error(p.err, kErrTimeoutMma);
 
   // a copy still in flight after an early exit lands before the CTA leaves
-  if (tid == 0 && inflight && !mbar_wait(barX, inflight_parity)) record_error(p.err, kErrTimeoutDrain);
+  if (!HAS_C && leader && x_pending && !mbar_wait(xfull, ph)) record_error(p.err, kErrTimeoutDrain);
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, C::TMEM_COLS);
+    tmem_dealloc(tmem, 512);
   }
 }
 
-template <int N2, int NP, int GRAN>
-fq_status launch_tc3(const QuantTcParams& p, cudaStream_t stream) {
-  using C = TcCfg<N2, NP>;
-  auto kern = quant_act_tc_kernel<N2, NP, GRAN>;
+template <int N2, int NP, int GRAN, bool HAS_C>
+fq_status launch_tc4(const QuantTcParams& p, cudaStream_t stream) {
+  using C = TcCfg<N2, NP, HAS_C>;
+  CUtensorMap tm;
+  // X viewed as [M * n1 rows][n2] fp16; one box = 64 columns (128 bytes) x n1 rows
+  fq_status st = make_tmap_2d(&tm, p.X, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, uint64_t(p.n2), uint64_t(p.M) * p.n1,
+                              uint64_t(p.n2) * 2, 64u, uint32_t(p.n1), CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != FQ_OK) return st;
+  auto kern = quant_act_tc_kernel<N2, NP, GRAN, HAS_C>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess ||
       cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
     return fail(FQ_ERR_CUDA, "cannot reserve %d bytes of shared memory for the transform kernel", C::SMEM);
-  int per_sm = 1;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kTcThreads, C::SMEM) != cudaSuccess) per_sm = 1;
-  per_sm = std::max(1, std::min(per_sm, 512 / C::TMEM_COLS));
-  const int ntiles = (p.M + C::T - 1) / C::T;
-  const int grid = std::max(1, std::min(ntiles, sm_count() * per_sm));
-  kern<<<grid, kTcThreads, C::SMEM, stream>>>(p);
+  const int ngroups = (p.M + C::G - 1) / C::G;
+  const int grid = std::max(1, std::min((ngroups + C::P - 1) / C::P, sm_count()));
+  kern<<<grid, kTcThreads, C::SMEM, stream>>>(p, tm);
   return check_launch("quant_act_tc_kernel");
+}
+
+template <int N2, int NP, bool HAS_C>
+fq_status launch_tc3(const QuantTcParams& p, cudaStream_t stream) {
+  if (p.gran == FQ_DYNAMIC_ROW) return launch_tc4<N2, NP, FQ_DYNAMIC_ROW, HAS_C>(p, stream);
+  if (p.gran == FQ_DYNAMIC_GROUP) return launch_tc4<N2, NP, FQ_DYNAMIC_GROUP, HAS_C>(p, stream);
+  return launch_tc4<N2, NP, FQ_STATIC_CHANNEL, HAS_C>(p, stream);
 }
 
 template <int N2, int NP>
 fq_status launch_tc(const QuantTcParams& p, cudaStream_t stream) {
-  if (p.gran == FQ_DYNAMIC_ROW) return launch_tc3<N2, NP, FQ_DYNAMIC_ROW>(p, stream);
-  if (p.gran == FQ_DYNAMIC_GROUP) return launch_tc3<N2, NP, FQ_DYNAMIC_GROUP>(p, stream);
-  return launch_tc3<N2, NP, FQ_STATIC_CHANNEL>(p, stream);
+  return p.c ? launch_tc3<N2, NP, true>(p, stream) : launch_tc3<N2, NP, false>(p, stream);
 }
 
 }  // namespace
