@@ -115,30 +115,6 @@ __device__ __noinline__ __half group_scale(float amax, float alpha) {
   return __float2half_rn(__fdiv_rn(__fmul_rn(amax, alpha), 7.0f));
 }
 
-// The same code as code_of(v, s) = clamp(rint(v / s)) with IEEE division,
-// computed with a multiply by inv_s = 1/s (rounded): that quotient is within
-// 1.5 units in the last place of the correctly rounded one, so rounding it
-// to an integer can only differ from rounding the IEEE quotient next to a
-// tie (x.5); there the IEEE division decides.
-__device__ __forceinline__ int code_fast(float v, float s, float inv_s) {
-  if (s == 0.0f) return 0;
-  const float qa = v * inv_s;
-  const float r = rintf(qa);
-  if (0.5f - fabsf(qa - r) <= fabsf(qa) * 9.5367431640625e-07f + 1e-30f)  // 2^-20 relative margin
-    return code_of(v, s);
-  return __float2int_rn(fminf(fmaxf(r, -8.0f), 7.0f));
-}
-
-// The code of v = u * up (up a power of two, exact) for scale s, given
-// f = up * (1/s) (also exact scaling of the rounded reciprocal): the quotient
-// u * f equals v * fl(1/s), so the tie test of code_fast applies unchanged.
-__device__ __forceinline__ int code_scaled(float u, float f, float up, float s) {
-  const float qa = u * f;
-  const float r = rintf(qa);
-  if (0.5f - fabsf(qa - r) <= fabsf(qa) * 9.5367431640625e-07f + 1e-30f) return code_of(u * up, s);
-  return __float2int_rn(fminf(fmaxf(r, -8.0f), 7.0f));
-}
-
 // w with bits [pos, pos + 4) replaced by the low 4 bits of q.
 __device__ __forceinline__ uint32_t put_nibble(uint32_t w, int q, int pos) {
   uint32_t r;
@@ -203,38 +179,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tmem_alloc(tslot, 512);
     tmem_relinquish();
   }
-  // operands and scratch start at zero (padding rows and columns stay zero)
-  for (int c = tid; c < C::OFF_BAR / 16; c += kTcThreads)
-    reinterpret_cast<uint4*>(sm)[c] = make_uint4(0, 0, 0, 0);
-  __syncthreads();
-  // ---- factors -> fp16 hi/lo operands, once per CTA
-  for (int e = tid; e < N2 * N2; e += kTcThreads) {
-    const int j = e / N2, l = e % N2;  // stage-A A operand: row l, K index j, value P2[j][l]
-    const float v = __ldg(p.P2 + e);
-    const __half hi = __float2half_rn(v);
-    const __half lo = __float2half_rn(v - __half2float(hi));
-    const int row = N2 == 64 ? 64 + l : l;
-    const uint32_t off = (N2 == 64 ? 0u : uint32_t(j >> 6) * C::REG) + sw128_offset(row, (j & 63) * 2);
-    *reinterpret_cast<__half*>(sm + C::OFF_SA + off) = hi;
-    *reinterpret_cast<__half*>(sm + C::OFF_SA + C::SA_HALF + off) = lo;
+  // zero what no copy or factor store writes: the zero rows of the
+  // block-diagonal P2^T, and the padding rows/columns beyond n1
+  if (N2 == 64) {
+    constexpr int kZeroChunks = 128 * 128 / 16;  // per half: rows 0..63 and 128..191
+    for (int c = tid; c < 2 * kZeroChunks; c += kTcThreads) {
+      const int half = c / kZeroChunks, r = c % kZeroChunks;
+      const int off = half * C::SA_HALF + (r < kZeroChunks / 2 ? r * 16 : 64 * 128 + r * 16);
+      *reinterpret_cast<uint4*>(sm + C::OFF_SA + off) = make_uint4(0, 0, 0, 0);
+    }
   }
-  for (int e = tid; e < n1 * n1; e += kTcThreads) {
-    const int i = e / n1, k = e % n1;  // stage-B B operand: row k, K index i, value P1[i][k]
-    const float v = __ldg(p.P1 + e);
-    const __half hi = __float2half_rn(v);
-    const __half lo = __float2half_rn(v - __half2float(hi));
-    const uint32_t off = uint32_t(i >> 6) * (NP * 128) + sw128_offset(k, (i & 63) * 2);
-    *reinterpret_cast<__half*>(sm + C::OFF_SL + off) = hi;
-    *reinterpret_cast<__half*>(sm + C::OFF_SL + C::SL_HALF + off) = lo;
+  if (n1 < NP) {
+    for (int c = tid; c < (2 * C::SL_HALF) / 16; c += kTcThreads)
+      *reinterpret_cast<uint4*>(sm + C::OFF_SL + c * 16) = make_uint4(0, 0, 0, 0);
+    for (int c = tid; c < (C::P * C::X_BYTES) / 16; c += kTcThreads)
+      *reinterpret_cast<uint4*>(sm + C::OFF_X + c * 16) = make_uint4(0, 0, 0, 0);
   }
   fence_proxy_async_smem();
-  tc_fence_before();
   __syncthreads();
-  tc_fence_after();
 
-  const uint32_t tmem = *tslot;
-  const uint32_t tD = tmem + uint32_t(pipe * C::TMEM_PIPE);  // D: stage A, then stage B
-  const uint32_t tU = tD + uint32_t(NP);                      // U^T: hi [0, NP/2), lo [NP/2, NP)
   const uint32_t lane_off = uint32_t(q4 * 32) << 16;
   const int bar_id = 1 + pipe;
   const bool leader = pw == 0 && lane == 0;
@@ -259,11 +222,55 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int gstride = gridDim.x * C::P;
   int grp = blockIdx.x * C::P + pipe;
   bool x_pending = false;  // (leader) a TMA into the X tile has not been waited for
-  if (!HAS_C && leader && grp < ngroups) {
+  if (!HAS_C && leader && grp < ngroups) {  // the first rows land while the factors are staged
     prefetch_tensormap(&tmX);
     issue_x(grp);
     x_pending = true;
   }
+
+  // ---- factors -> fp16 hi/lo operands, once per CTA, 8 consecutive K per 16-byte store
+  for (int e = tid; e < N2 * (N2 / 8); e += kTcThreads) {
+    // stage-A A operand: row l, K = j, value P2[j][l]; consecutive threads
+    // take consecutive l, so every load instruction reads whole rows of P2
+    const int l = e % N2, j0 = (e / N2) * 8;
+    uint4 hi, lo;
+    __half* hh = reinterpret_cast<__half*>(&hi);
+    __half* ll = reinterpret_cast<__half*>(&lo);
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj) {
+      const float v = __ldg(p.P2 + (j0 + jj) * N2 + l);
+      hh[jj] = __float2half_rn(v);
+      ll[jj] = __float2half_rn(v - __half2float(hh[jj]));
+    }
+    const int row = N2 == 64 ? 64 + l : l;
+    const uint32_t off = (N2 == 64 ? 0u : uint32_t(j0 >> 6) * C::REG) + sw128_offset(row, (j0 & 63) * 2);
+    *reinterpret_cast<uint4*>(sm + C::OFF_SA + off) = hi;
+    *reinterpret_cast<uint4*>(sm + C::OFF_SA + C::SA_HALF + off) = lo;
+  }
+  const int n1c = (n1 + 7) / 8;
+  for (int e = tid; e < n1 * n1c; e += kTcThreads) {
+    const int k = e % n1, i0 = (e / n1) * 8;  // stage-B B operand: row k, K = i, value P1[i][k]
+    uint4 hi, lo;
+    __half* hh = reinterpret_cast<__half*>(&hi);
+    __half* ll = reinterpret_cast<__half*>(&lo);
+#pragma unroll
+    for (int ii = 0; ii < 8; ++ii) {
+      const float v = i0 + ii < n1 ? __ldg(p.P1 + (i0 + ii) * n1 + k) : 0.f;
+      hh[ii] = __float2half_rn(v);
+      ll[ii] = __float2half_rn(v - __half2float(hh[ii]));
+    }
+    const uint32_t off = uint32_t(i0 >> 6) * (NP * 128) + sw128_offset(k, (i0 & 63) * 2);
+    *reinterpret_cast<uint4*>(sm + C::OFF_SL + off) = hi;
+    *reinterpret_cast<uint4*>(sm + C::OFF_SL + C::SL_HALF + off) = lo;
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+  const uint32_t tD = tmem + uint32_t(pipe * C::TMEM_PIPE);  // D: stage A, then stage B
+  const uint32_t tU = tD + uint32_t(NP);                      // U^T: hi [0, NP/2), lo [NP/2, NP)
+
   uint32_t ph = 0;
   bool bad = false;
   for (; grp < ngroups; grp += gstride, ph ^= 1u) {
@@ -388,18 +395,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tmem_ld_32x32(tD + lane_off + uint32_t(part * COLS + 32 * c), u);
         tmem_wait_ld();
         uint32_t hi[16], lo[16];
+        const float2 sc2 = make_float2(sc, sc), m1 = make_float2(-1.f, -1.f);
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-          float a = __uint_as_float(u[2 * j]), b = __uint_as_float(u[2 * j + 1]);
+          float2 ab = make_float2(__uint_as_float(u[2 * j]), __uint_as_float(u[2 * j + 1]));
           if (HAS_C) {
-            a *= exp2i(xexp[s_of_row * NP + part * COLS + 32 * c + 2 * j]);
-            b *= exp2i(xexp[s_of_row * NP + part * COLS + 32 * c + 2 * j + 1]);
+            ab.x *= exp2i(xexp[s_of_row * NP + part * COLS + 32 * c + 2 * j]);
+            ab.y *= exp2i(xexp[s_of_row * NP + part * COLS + 32 * c + 2 * j + 1]);
           }
-          a *= sc;
-          b *= sc;
-          const __half2 h = __floats2half2_rn(a, b);
-          const float2 hf = __half22float2(h);
-          const __half2 l2 = __floats2half2_rn(a - hf.x, b - hf.y);
+          ab = fmul2(ab, sc2);  // exact: a power of two
+          const __half2 h = __floats2half2_rn(ab.x, ab.y);
+          const float2 r = ffma2(__half22float2(h), m1, ab);  // ab - hi, exact
+          const __half2 l2 = __floats2half2_rn(r.x, r.y);
           hi[j] = *reinterpret_cast<const uint32_t*>(&h);
           lo[j] = *reinterpret_cast<const uint32_t*>(&l2);
         }
@@ -496,7 +503,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         named_barrier(bar_id, C::TPP);
       }
-      // pass 2: codes, 8 columns k per 32-bit word, transposed to 8 columns l
+      // pass 2: codes, 8 columns k per 32-bit word, transposed to 8 columns l.
+      // Two values at a time (f32x2): x = fma(d, f, 1.5 * 2^23) holds the
+      // round-half-even integer of d * f (= v / s up to the rounding of 1/s)
+      // in its low mantissa bits, so its low 4 bits are the two's-complement
+      // nibble; t = d * f - that integer (exact residual) flags the values
+      // next to a tie, where the IEEE quotient decides (code_of).  |v / s|
+      // stays below 7.5 when alpha >= 1, so the clamp to [-8, 7] is needed
+      // only for alpha < 1.
+      constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+      const float2 cc = make_float2(kMagic, kMagic), m1 = make_float2(-1.f, -1.f);
+      const float th = 0.5f - (8.0f / fminf(p.alpha, 1.0f) + 1.0f) * 9.5367431640625e-07f;  // tie band
+      const bool clamp = !(p.alpha >= 1.0f);
 #pragma unroll
       for (int c = 0; c < COLS / 32; ++c) {
         uint32_t u[32];
@@ -505,22 +523,55 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {
           const int k0 = part * COLS + 32 * c + 8 * ch;
+          const uint32_t* uc = u + 8 * ch;
           uint32_t word = 0;
+          if (GRAN == FQ_STATIC_CHANNEL) {
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int k = k0 + j;
-            const float d = __uint_as_float(u[8 * ch + j]);
-            int qv = 0;
-            if (GRAN == FQ_DYNAMIC_ROW) {
-              qv = s_tok != 0.f ? code_scaled(d, f_tok, up, s_tok) : 0;
-            } else if (GRAN == FQ_DYNAMIC_GROUP) {
-              const int g = k * N2 / 128;
-              qv = code_fast(d * up, red[C::R_SG + s * 128 + g], red[C::R_SINV + s * 128 + g]);
-            } else if (k < n1) {
-              qv = code_of(d * up, __ldg(p.sstatic + k * N2 + l));
+            for (int j = 0; j < 8; ++j) {
+              const int k = k0 + j;
+              const int qv = k < n1 ? code_of(__uint_as_float(uc[j]) * up, __ldg(p.sstatic + k * N2 + l)) : 0;
+              word = put_nibble(word, qv, 4 * j);
             }
-            if (p.xhat && tok_ok && k < n1) p.xhat[size_t(tok) * K + k * N2 + l] = d * up;
-            word = put_nibble(word, qv, 4 * j);
+          } else {
+            bool redo = false;  // a value next to a tie, or a zero scale: the IEEE path decides
+#pragma unroll
+            for (int j = 0; j < 8; j += 2) {
+              const int k = k0 + j;
+              const float2 dd = make_float2(__uint_as_float(uc[j]), __uint_as_float(uc[j + 1]));
+              float2 ff;
+              if (GRAN == FQ_DYNAMIC_ROW) {
+                ff = make_float2(f_tok, f_tok);
+              } else {
+                const int g0 = k * N2 / 128, g1 = (k + 1) * N2 / 128;
+                ff = fmul2(make_float2(red[C::R_SINV + s * 128 + g0], red[C::R_SINV + s * 128 + g1]),
+                           make_float2(up, up));
+                redo |= red[C::R_SG + s * 128 + g0] == 0.f || red[C::R_SG + s * 128 + g1] == 0.f;
+              }
+              float2 x = ffma2(dd, ff, cc);                      // 1.5 * 2^23 + rint(d f)
+              const float2 t = ffma2(dd, ff, ffma2(x, m1, cc));  // d f - rint(d f)
+              if (clamp) {
+                x.x = fminf(fmaxf(x.x, kMagic - 8.0f), kMagic + 7.0f);
+                x.y = fminf(fmaxf(x.y, kMagic - 8.0f), kMagic + 7.0f);
+              }
+              redo |= fabsf(t.x) >= th || fabsf(t.y) >= th;
+              word = put_nibble(word, int(__float_as_uint(x.x)), 4 * j);
+              word = put_nibble(word, int(__float_as_uint(x.y)), 4 * j + 4);
+            }
+            if (GRAN == FQ_DYNAMIC_ROW) redo |= s_tok == 0.f;
+            if (redo) {
+              word = 0;
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                const int k = k0 + j;
+                const float sk = GRAN == FQ_DYNAMIC_ROW ? s_tok : red[C::R_SG + s * 128 + k * N2 / 128];
+                word = put_nibble(word, code_of(__uint_as_float(uc[j]) * up, sk), 4 * j);
+              }
+            }
+          }
+          if (p.xhat && tok_ok) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              if (k0 + j < n1) p.xhat[size_t(tok) * K + (k0 + j) * N2 + l] = __uint_as_float(uc[j]) * up;
           }
           word = transpose_nibbles8(word, lane);
           const int kr = k0 + (lane & 7);
