@@ -340,6 +340,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
 
     // ---- 2. stage A: D[row][i] = sum_j P2^T[l][j] Xbar_s[i][j]
+    // The pipelines of a CTA start one stage A apart (pipeline p's first one
+    // waits for pipeline p - 1's), so afterwards one pipeline's tensor-core
+    // work overlaps the others' SIMT work instead of all of them alternating
+    // in lockstep.
+    if (leader && !bad && ph == 0 && grp == int(blockIdx.x) * C::P + pipe && pipe > 0 &&
+        !mbar_wait(mmaA - 3, 0)) {
+      record_error(p.err, kErrTimeoutMma);
+      bad = true;
+    }
     if (leader && !bad) {
       tc_fence_after();
       const uint32_t sa = smem_u32(sm + C::OFF_SA), sx = smem_u32(xt);
