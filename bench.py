@@ -37,6 +37,11 @@ METRIC = "W4A4 linear effective TOPS + quant-kernel GB/s, % of roofline, 1xB200"
 WORKLOAD = ("llama3-8b-like decoder-layer prefill linears qkv/o/gate_up/down, M=2048 tokens, "
             "Kronecker-transformed per-token INT4 activations (64x64 / 112x128), per-channel INT4 weights, fp16 out")
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# DRAM bytes (read + write) of one GEMM launch per layer, from an ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum) of this bench command on the
+# current GEMM kernel; the fp16 outputs that still sit in L2 when a launch
+# ends are not in it.
+GEMM_DRAM_BYTES = {"qkv": 16843776, "o": 12641792, "gate_up": 63073280 + 66820096, "down": 44099584 + 52736}
 INT8_OVER_BF16 = 4.5 / 2.25  # nominal dense ratio (B200: 4.5 POPS int8 vs 2.25 PFLOPS bf16)
 
 
@@ -302,7 +307,10 @@ def run_ours(args, ws, rank, local):
             "unit": "TOPS",
             "frac": round(g_achieved / int8_peak, 4),
             "peak_kind": f"{pk_kind} bf16 sustained x {INT8_OVER_BF16:g} (nominal int8/bf16 dense ratio)",
-            "traffic": None,
+            "traffic": int(statistics.mean(GEMM_DRAM_BYTES[s["d"]["layer"]] for s in state)),
+            "traffic_unit": "bytes per launch (mean over the step's GEMM launches, ncu dram__bytes_read + write)",
+            "algorithmic_bytes": int(statistics.mean(
+                s["m"] * s["k"] // 2 + s["n"] * s["k"] // 2 + 4 * (s["m"] + s["n"]) + 2 * s["m"] * s["n"] for s in state)),
             "note": "achieved = sum of algorithmic 2MNK over the GEMM launches / sum of their CUDA-event durations",
         },
         "e2e": {"value": round(e2e_value, 2), "unit": "TOPS", "h2d_bytes_per_step": int(h2d * ws),
@@ -408,6 +416,8 @@ def run_group(args, dev_index):
     int8_peak = pk["bf16_tflops_sustained"] * INT8_OVER_BF16
     clocks.start()
     for k, n in synth.GROUP_70B_SHAPES:
+        if args.shape and args.shape != f"{k},{n}":
+            continue
         d = synth.prefill_linear(k, n, m=4096, w_kind="t")
         w = torch.from_numpy(d["w"]).to(dev)
         wq, sw = fq.fq_quant_weight(w, qp)
@@ -428,6 +438,8 @@ def run_group(args, dev_index):
         del d, x, xq, sx, y, wq, sw, ws
         torch.cuda.empty_cache()
     clk = clocks.stop()
+    if not rows:
+        raise SystemExit(f"no group shape matches --shape {args.shape}")
     ops = sum(r.pop("ops") for r in rows)
     g_s = sum(r["gemm_us"] for r in rows) * 1e-6
     tops = ops / g_s / 1e12
@@ -455,6 +467,8 @@ def run_decode(args, dev_index):
     pk, pk_kind = peaks()
     clocks.start()
     for k, n in synth.DECODE_70B_SHAPES:
+        if args.shape and not args.shape.endswith(f",{k},{n}"):
+            continue
         d0 = synth.decode_static(synth.DECODE_TOKENS[-1], k, n)
         s_k = torch.from_numpy(d0["static_scale"]).to(dev)
         w = torch.from_numpy(d0["w"]).to(dev)
@@ -462,6 +476,8 @@ def run_decode(args, dev_index):
         del w
         qs = fq.qparams(fq.STATIC)
         for m in synth.DECODE_TOKENS:
+            if args.shape and args.shape != f"{m},{k},{n}":
+                continue
             x = torch.from_numpy(d0["x"][:m].copy()).to(dev)
             xq, _ = fq.fq_quant_act(x, qs, None, s_k)
             y = torch.empty(m, n, dtype=torch.float16, device=dev)
@@ -477,6 +493,8 @@ def run_decode(args, dev_index):
         del wq, sw, s_k, d0
         torch.cuda.empty_cache()
     clk = clocks.stop()
+    if not rows:
+        raise SystemExit(f"no decode shape matches --shape {args.shape}")
     nbytes = sum(r.pop("bytes") for r in rows)
     g_s = sum(r["gemm_us"] for r in rows) * 1e-6
     gbs = nbytes / g_s / 1e9
@@ -588,6 +606,8 @@ def main():
     ap.add_argument("--workload", choices=["prefill", "transform_quant", "group", "decode"], default="prefill",
                     help="prefill (default): the decoder-layer prefill step; the others time one kernel family "
                          "on its own workload (1 GPU)")
+    ap.add_argument("--shape", default=None,
+                    help="one shape of the group (K,N) or decode (M,K,N) workload, e.g. for profiling one launch")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
