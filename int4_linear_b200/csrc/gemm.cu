@@ -5,20 +5,14 @@
 // with s8 x s8 -> s32 MMAs accumulating in tensor memory (FlatQuant notes,
 // 核心思想: Y ~ Q(XP) Q(P^-1 W^T) with integer accumulation).
 //
-// Warp roles inside one CTA (one 128 x BN output tile, a K range):
-//   warp 1      tensor-memory allocation and the single MMA-issuing thread
-//   warps 2-5   epilogue: tcgen05.ld of the accumulator, dequantization, stores
-//               (outside group mode they first unpack with the others)
-//   warps 6-13  unpackers: each lane owns fixed 16-byte packed pieces of the
-//               A/B slices, loads them from global memory several K slices
-//               ahead into registers, and writes them as int8 into a ring of
-//               SU stages in the 128-byte swizzled K-major layout that the
-//               MMA descriptors describe.
-// The packed operands never pass through shared memory: shared-memory
-// bandwidth (unpacked writes plus the tensor core's operand reads) is what
-// bounds this kernel, so the packed round trip a TMA stage would add is left
-// out.  Stages are handed over with mbarriers; every wait is bounded and a
-// wait that gives up records a timeout code in the device error word.
+// Prefill kernel (M > 64): one CTA per 128 x BN output tile and K range.
+// The packed 128-deep K slices of both operands arrive by TMA into a ring in
+// shared memory; A-warps unpack the activation rows into a tensor-memory ring
+// (tcgen05.st), B-warps the weight rows into a 128-byte-swizzled
+// shared-memory ring, and one thread issues the MMAs (A from tensor memory).
+// The warp roles are listed beside gemm_w4a4_kernel.  Stages are handed over
+// with mbarriers; every wait is bounded and a wait that gives up records a
+// timeout code in the device error word.
 //
 // The nibble is unpacked into the high half of its byte (16 q, see
 // unpack8_hi), so the tensor core accumulates 256 * sum(qx qw); the epilogue
@@ -27,8 +21,9 @@
 // Epilogues: per-token x per-output-channel scales, static (migrated) scales,
 // per-group scales summed in float32 (FRM-PTQ group quantization, one group
 // per K slice, double-buffered accumulators), raw int32, or atomic int32
-// partial sums for split-K.  For few tokens (decode) the operands swap roles:
-// the weights fill the 128-row MMA side and the tokens the N side.
+// partial sums for split-K.  For few tokens (decode, gemm_decode_kernel) the
+// operands swap roles: the weights fill the 128-row MMA side and the tokens
+// the N side.
 #include <cuda_fp16.h>
 
 #include <algorithm>
@@ -49,21 +44,36 @@ constexpr int kBK = 128;        // int8 K per stage; equals the quantization gro
 constexpr int kPK = kBK / 2;    // packed bytes per row per stage
 constexpr int kEpiWarps = 4;
 constexpr int kUnpackWarps = 8;
-constexpr int kThreads = 32 * (2 + kEpiWarps + kUnpackWarps);
 
-// Warps that feed a stage: 4 A-warps (one per tensor-memory lane quadrant)
-// write the unpacked A rows into tensor memory; the B-warps write the
-// unpacked B rows into shared memory.  Outside group mode the A-warps are
-// the epilogue warps (the epilogue runs after the main loop); in group mode
-// the epilogue runs alongside, so warps 6..9 take A and 10..13 take B.
+// Warp roles (480 threads):
+//   warp 0      group mode: keeps the per-slice scale ring filled; else idle
+//   warp 1      tensor-memory allocation and the MMA-issuing thread
+//   warps 2-5   epilogue (outside group mode they first unpack A)
+//   warps 6-13  unpack B (outside group mode); group mode: 6-9 A, 10-13 B
+//   warp 14     one thread issues the TMA loads of both packed slices
+// The packed 128-deep K slices of both operands arrive by TMA into a ring of
+// SP stages (A in the 64-byte swizzle, so that the one-row-per-thread reads
+// are free of bank conflicts; B unswizzled, read in consecutive 16-byte
+// pieces); the A-warps unpack their row into a tensor-memory ring and the
+// B-warps into a 128-byte-swizzled shared-memory ring of SU stages.  A
+// packed stage goes back to the producer only after the unpacked data has
+// been stored (its registers consumed), so a refill never overtakes a read.
+constexpr int kWarps = 15;
+constexpr int kThreads = 32 * kWarps;
+constexpr int kProducerWarp = 14;
+
 template <int EPI>
 __host__ __device__ constexpr int b_warps() { return EPI == kEpiGroup ? kUnpackWarps - 4 : kUnpackWarps; }
 template <int EPI>
 __host__ __device__ constexpr int feed_warps() { return 4 + b_warps<EPI>(); }
 
-template <int BN, int EPI, bool SWAP>
+template <int BN, int EPI>
 struct Cfg {
-  static constexpr int SU = 4;                 // unpacked stages (A in tensor memory, B in shared memory)
+  static constexpr int SP = 4;                 // packed stages (TMA ring)
+  static constexpr int SU = BN == 256 ? 3 : 4; // unpacked stages (A in tensor memory, B in shared memory)
+  static constexpr int PA = kBM * kPK;         // packed A slice: 128 rows x 64 bytes
+  static constexpr int PB = BN * kPK;          // packed B slice
+  static constexpr int P_STAGE = PA + PB;
   static constexpr int B_UNP = BN * kBK;
   static constexpr int ACC_COLS = EPI == kEpiGroup ? 3 * BN : BN;
   static constexpr int A_COL0 = ((ACC_COLS + 31) / 32) * 32;   // tensor-memory columns of the A ring
@@ -71,7 +81,8 @@ struct Cfg {
   static constexpr int TMEM_NEED = A_COL0 + SU * A_STAGE_COLS;
   static constexpr int TMEM_COLS = TMEM_NEED <= 64 ? 64 : (TMEM_NEED <= 128 ? 128 : (TMEM_NEED <= 256 ? 256 : 512));
   static constexpr int UNP_STAGE = B_UNP;
-  static constexpr int OFF_UNP = 0;
+  static constexpr int OFF_P = 0;
+  static constexpr int OFF_UNP = OFF_P + SP * P_STAGE;
   static constexpr int OFF_SCALE = OFF_UNP + SU * UNP_STAGE;
   // group mode: a ring of SS per-slice scale stages written by warp 0: the
   // weight scales as {s, s, -1.5*2^23*s, -1.5*2^23*s} pairs for BN columns,
@@ -80,15 +91,16 @@ struct Cfg {
   static constexpr int SC_STAGE = BN * 8 + kBM * 4;
   static constexpr int SCALE_BYTES = EPI == kEpiGroup ? SS * SC_STAGE : 0;
   static constexpr int OFF_BAR = OFF_SCALE + SCALE_BYTES;
-  static constexpr int NBAR = 2 * SU + 5 + (EPI == kEpiGroup ? 2 * SS : 0);
+  static constexpr int NBAR = 2 * SP + 2 * SU + 5 + (EPI == kEpiGroup ? 2 * SS : 0);
   static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
   static constexpr int SMEM = OFF_TMEM + 16 + 1024;  // + slack to align the base to 1024
   // the fp16 output tile is staged in the (then idle) unpacked ring, rows padded by 16 bytes
   static constexpr int OUT_PITCH = 2 * BN + 16;
-  static_assert(UNP_STAGE % 1024 == 0, "unpacked stages must keep 1024-byte alignment");
-  static_assert(SWAP || kBM * OUT_PITCH <= SU * UNP_STAGE, "output tile fits in the ring");
+  static_assert(UNP_STAGE % 1024 == 0 && P_STAGE % 1024 == 0 && PA % 1024 == 0, "1024-byte stage alignment");
+  static_assert(kBM * OUT_PITCH <= SU * UNP_STAGE, "output tile fits in the ring");
   static_assert(TMEM_NEED <= 512, "tensor memory");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
+  static_assert(SMEM <= 227 * 1024, "shared memory");
   static_assert(EPI != kEpiGroup || 3 * BN <= 512, "group epilogue needs 3 x BN tensor-memory columns");
 };
 
@@ -116,14 +128,18 @@ __device__ __forceinline__ void store_half8(__half* dst, const float* v) {
   *reinterpret_cast<uint4*>(dst) = o;
 }
 
-template <int BN, int EPI, bool SWAP>
-__global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(const GemmParams p) {
-  using C = Cfg<BN, EPI, SWAP>;
-  constexpr int SU = C::SU;
+template <int BN, int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_w4a4_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tmA,
+                     const __grid_constant__ CUtensorMap tmB) {
+  using C = Cfg<BN, EPI>;
+  constexpr int SU = C::SU, SP = C::SP;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-  uint64_t* full_u = bars;
+  uint64_t* pfull = bars;
+  uint64_t* pempty = pfull + SP;
+  uint64_t* full_u = pempty + SP;
   uint64_t* empty_u = full_u + SU;
   uint64_t* acc_full = empty_u + SU;
   uint64_t* acc_empty = acc_full + 2;
@@ -138,6 +154,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(const GemmParams
   const int nkb = max(0, min(p.num_kb, kb0 + p.kb_per_split) - kb0);
 
   if (threadIdx.x == 0) {
+    for (int s = 0; s < SP; ++s) {
+      mbar_init(&pfull[s], 1);
+      mbar_init(&pempty[s], feed_warps<EPI>());
+    }
     for (int s = 0; s < SU; ++s) {
       mbar_init(&full_u[s], feed_warps<EPI>());
       mbar_init(&empty_u[s], 1);
@@ -164,7 +184,33 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(const GemmParams
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
+  if (warp == kProducerWarp) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tensormap(&tmA);
+      prefetch_tensormap(&tmB);
+      int issued = 0;
+      for (int i = 0; i < nkb; ++i) {
+        const int sp = i % SP;
+        if (!mbar_wait(&pempty[sp], ((i / SP) & 1) ^ 1)) {
+          record_error(p.err, kErrTimeoutProducer);
+          break;
+        }
+        uint8_t* st = smem + C::OFF_P + sp * C::P_STAGE;
+        mbar_arrive_expect_tx(&pfull[sp], C::P_STAGE);
+        tma_load_2d(st, &tmA, &pfull[sp], (kb0 + i) * kPK, tileA * kBM);
+        tma_load_2d(st + C::PA, &tmB, &pfull[sp], (kb0 + i) * kPK, tileB * BN);
+        ++issued;
+      }
+      // every issued copy has landed before the CTA may leave (normally the
+      // unpacking warps already waited for each of them)
+      for (int i = max(0, issued - SP); i < issued; ++i)
+        if (!mbar_wait(&pfull[i % SP], (i / SP) & 1)) {
+          record_error(p.err, kErrTimeoutDrain);
+          break;
+        }
+    }
+  } else if (warp == 0) {
     if (EPI == kEpiGroup) {
       // ------------------------------------------------------------ group scales -> shared-memory ring
       // Loads run D slices ahead in registers, so their latency is paid once.
@@ -260,66 +306,53 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(const GemmParams
     const bool epi_warp = warp < 2 + kEpiWarps;
     const bool a_warp = EPI == kEpiGroup ? (warp >= 6 && warp < 10) : epi_warp;
     const bool b_warp = EPI == kEpiGroup ? (warp >= 10) : (warp >= 6);
-    const size_t ld = size_t(p.K) / 2;
     if (a_warp) {
-      constexpr int D = SWAP ? 4 : 3;  // K slices of packed A in flight per thread
       // one A row per thread (its tensor-memory lane): 64 packed bytes per slice
       const int q = warp & 3;
       const int row = q * 32 + lane;
-      const int grow = tileA * kBM + row;
-      const bool ok_row = grow < p.rowsA;
-      const uint8_t* src = p.A + (ok_row ? size_t(grow) * ld : 0) + size_t(kb0) * kPK;
+      const int sw = (row >> 1) & 3;  // 64-byte swizzle: chunk c of this row sits at chunk c ^ sw
       const uint32_t ta = tmem + (uint32_t(q * 32) << 16) + uint32_t(C::A_COL0);
-      uint4 w[D][4];
-#pragma unroll
-      for (int d = 0; d < D; ++d)
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          w[d][c] = (d < nkb && ok_row) ? __ldg(reinterpret_cast<const uint4*>(src + d * kPK + c * 16))
-                                        : make_uint4(0, 0, 0, 0);
       bool ok = true;
-      for (int i0 = 0; i0 < nkb && ok; i0 += D) {
+      for (int i = 0; i < nkb; ++i) {
+        const int sp = i % SP, su = i % SU;
+        if (!warp_wait(&pfull[sp], (i / SP) & 1)) {
+          ok = false;
+          break;
+        }
+        const uint8_t* src = smem + C::OFF_P + sp * C::P_STAGE + row * kPK;
+        uint4 w[4];
 #pragma unroll
-        for (int d = 0; d < D; ++d) {
-          const int i = i0 + d;
-          if (i >= nkb) break;
-          const int su = i % SU;
-          if (!warp_wait(&empty_u[su], ((i / SU) & 1) ^ 1)) {
-            if (lane == 0) record_error(p.err, kErrTimeoutUnpack);
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          uint32_t r[32];
+        for (int c = 0; c < 4; ++c) w[c] = *reinterpret_cast<const uint4*>(src + ((c ^ sw) << 4));
+        if (!warp_wait(&empty_u[su], ((i / SU) & 1) ^ 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t r[32];
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            unpack8_hi(w[d][c].x, r[8 * c + 0], r[8 * c + 1]);
-            unpack8_hi(w[d][c].y, r[8 * c + 2], r[8 * c + 3]);
-            unpack8_hi(w[d][c].z, r[8 * c + 4], r[8 * c + 5]);
-            unpack8_hi(w[d][c].w, r[8 * c + 6], r[8 * c + 7]);
-          }
-          tmem_st_32x32(ta + uint32_t(su * C::A_STAGE_COLS), r);
-          tmem_wait_st();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&full_u[su]);
-          if (i + D < nkb) {
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-              w[d][c] = ok_row ? __ldg(reinterpret_cast<const uint4*>(src + (i + D) * kPK + c * 16))
-                               : make_uint4(0, 0, 0, 0);
-          }
+        for (int c = 0; c < 4; ++c) {
+          unpack8_hi(w[c].x, r[8 * c + 0], r[8 * c + 1]);
+          unpack8_hi(w[c].y, r[8 * c + 2], r[8 * c + 3]);
+          unpack8_hi(w[c].z, r[8 * c + 4], r[8 * c + 5]);
+          unpack8_hi(w[c].w, r[8 * c + 6], r[8 * c + 7]);
+        }
+        tmem_st_32x32(ta + uint32_t(su * C::A_STAGE_COLS), r);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&pempty[sp]);
+          mbar_arrive(&full_u[su]);
         }
       }
+      if (!ok && lane == 0) record_error(p.err, kErrTimeoutUnpack);
     } else if (b_warp) {
-      constexpr int D = SWAP ? 6 : 3;  // K slices of packed B in flight per thread
       const int uw = EPI == kEpiGroup ? warp - 10 : warp - 6;
       constexpr int kJobs = BN * 4;  // 16-byte packed pieces of B per stage
       constexpr int JPT = (kJobs + NB * 32 - 1) / (NB * 32);
-      // per-lane pieces, the same in every stage: global source row, two swizzled destinations
-      const uint8_t* gsrc[JPT];
-      uint32_t dst0[JPT], dst1[JPT];
-      bool live[JPT], load_ok[JPT];
+      // per-lane pieces, the same in every stage: packed source offset, two swizzled destinations
+      uint32_t dst0[JPT], dst1[JPT], srcj[JPT];
+      bool live[JPT];
 #pragma unroll
       for (int it = 0; it < JPT; ++it) {
         const int j = (it * NB + uw) * 32 + lane;
@@ -328,54 +361,43 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(const GemmParams
         const uint32_t rb = uint32_t((row >> 3) * 1024 + r7 * 128);
         dst0[it] = rb + uint32_t(((2 * c) ^ r7) << 4);
         dst1[it] = rb + uint32_t(((2 * c + 1) ^ r7) << 4);
-        const int grow = tileB * BN + row;
-        load_ok[it] = live[it] && grow < p.rowsB;
-        gsrc[it] = p.B + (load_ok[it] ? size_t(grow) * ld : 0) + size_t(kb0) * kPK + c * 16;
-      }
-      uint4 w[D][JPT];
-#pragma unroll
-      for (int d = 0; d < D; ++d) {
-#pragma unroll
-        for (int it = 0; it < JPT; ++it)
-          w[d][it] = (d < nkb && load_ok[it]) ? __ldg(reinterpret_cast<const uint4*>(gsrc[it] + d * kPK))
-                                              : make_uint4(0, 0, 0, 0);
+        srcj[it] = uint32_t(live[it] ? j * 16 : 0);
       }
       bool ok = true;
-      for (int i0 = 0; i0 < nkb && ok; i0 += D) {
+      for (int i = 0; i < nkb; ++i) {
+        const int sp = i % SP, su = i % SU;
+        if (!warp_wait(&pfull[sp], (i / SP) & 1)) {
+          ok = false;
+          break;
+        }
+        const uint8_t* pb = smem + C::OFF_P + sp * C::P_STAGE + C::PA;
+        uint4 w[JPT];
 #pragma unroll
-        for (int d = 0; d < D; ++d) {
-          const int i = i0 + d;
-          if (i >= nkb) break;
-          const int su = i % SU;
-          if (!warp_wait(&empty_u[su], ((i / SU) & 1) ^ 1)) {
-            if (lane == 0) record_error(p.err, kErrTimeoutUnpack);
-            ok = false;
-            break;
-          }
-          uint8_t* uk = smem + C::OFF_UNP + su * C::UNP_STAGE;
+        for (int it = 0; it < JPT; ++it) w[it] = *reinterpret_cast<const uint4*>(pb + srcj[it]);
+        if (!warp_wait(&empty_u[su], ((i / SU) & 1) ^ 1)) {
+          ok = false;
+          break;
+        }
+        uint8_t* uk = smem + C::OFF_UNP + su * C::UNP_STAGE;
 #pragma unroll
-          for (int it = 0; it < JPT; ++it) {
-            if (!live[it]) continue;
-            uint4 o0, o1;
-            unpack8_hi(w[d][it].x, o0.x, o0.y);
-            unpack8_hi(w[d][it].y, o0.z, o0.w);
-            unpack8_hi(w[d][it].z, o1.x, o1.y);
-            unpack8_hi(w[d][it].w, o1.z, o1.w);
-            *reinterpret_cast<uint4*>(uk + dst0[it]) = o0;
-            *reinterpret_cast<uint4*>(uk + dst1[it]) = o1;
-          }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&full_u[su]);
-          // refill this register slot with the slice D steps ahead
-          if (i + D < nkb) {
-#pragma unroll
-            for (int it = 0; it < JPT; ++it)
-              w[d][it] = load_ok[it] ? __ldg(reinterpret_cast<const uint4*>(gsrc[it] + (i + D) * kPK))
-                                     : make_uint4(0, 0, 0, 0);
-          }
+        for (int it = 0; it < JPT; ++it) {
+          if (!live[it]) continue;
+          uint4 o0, o1;
+          unpack8_hi(w[it].x, o0.x, o0.y);
+          unpack8_hi(w[it].y, o0.z, o0.w);
+          unpack8_hi(w[it].z, o1.x, o1.y);
+          unpack8_hi(w[it].w, o1.z, o1.w);
+          *reinterpret_cast<uint4*>(uk + dst0[it]) = o0;
+          *reinterpret_cast<uint4*>(uk + dst1[it]) = o1;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&pempty[sp]);
+          mbar_arrive(&full_u[su]);
         }
       }
+      if (!ok && lane == 0) record_error(p.err, kErrTimeoutUnpack);
     }
     if (epi_warp) {
     // ------------------------------------------------------------ epilogue
@@ -395,7 +417,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(const GemmParams
           else
             tmem_ld_32x16(tl + c0, v);
           tmem_wait_ld();
-          if (!SWAP) {
+          {
             // thread owns token row m = arow, columns n = bbase + c0 + j
             const int m = arow;
             if (m < p.M) {
@@ -422,26 +444,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(const GemmParams
                     dst[j] = a;
                   else
                     atomicAdd(dst + j, a);
-                }
-              }
-            }
-          } else {
-            // swapped: thread owns output channel n = arow, columns are tokens m
-            const int n = arow;
-            if (n < p.N) {
-              const float swn = (EPI == kEpiRow || EPI == kEpiStatic) ? __ldg(p.sw + n) : 0.f;
-              for (int j = 0; j < CW; ++j) {
-                const int m = bbase + c0 + j;
-                if (m >= p.M) break;
-                const int32_t ai = int32_t(v[j]) >> 8;
-                if (EPI == kEpiRow) {
-                  p.Y[size_t(m) * p.N + n] = __float2half_rn(__fmul_rn(__fmul_rn(float(ai), __ldg(p.sx + m)), swn));
-                } else if (EPI == kEpiStatic) {
-                  p.Y[size_t(m) * p.N + n] = __float2half_rn(__fmul_rn(float(ai), swn));
-                } else if (EPI == kEpiS32) {
-                  p.acc[size_t(m) * p.N + n] = ai;
-                } else {
-                  atomicAdd(p.acc + size_t(m) * p.N + n, ai);
                 }
               }
             }
@@ -534,7 +536,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(const GemmParams
   }
 
   // fp16 tiles staged in shared memory leave as whole 512-byte row segments
-  constexpr bool kStaged = !SWAP && (EPI == kEpiRow || EPI == kEpiStatic || EPI == kEpiGroup);
+  constexpr bool kStaged = EPI == kEpiRow || EPI == kEpiStatic || EPI == kEpiGroup;
   if (kStaged) {
     __syncthreads();
     const int n0 = tileB * BN;
@@ -906,14 +908,22 @@ Plan make_plan(int M, int N, int K, int epi_final, int sms) {
   return pl;
 }
 
-template <int BN, int EPI, bool SWAP>
+template <int BN, int EPI>
 fq_status launch_gemm(const GemmParams& gp, dim3 grid, cudaStream_t stream) {
-  using C = Cfg<BN, EPI, SWAP>;
-  auto kern = gemm_w4a4_kernel<BN, EPI, SWAP>;
+  using C = Cfg<BN, EPI>;
+  CUtensorMap ta, tb;
+  // packed A: 128 rows x 64 bytes per slice, 64-byte swizzle; packed B: BN rows x 64 bytes
+  fq_status st = make_tmap_2d(&ta, gp.A, CU_TENSOR_MAP_DATA_TYPE_UINT8, uint64_t(gp.K) / 2, uint64_t(gp.rowsA),
+                              uint64_t(gp.K) / 2, uint32_t(kPK), uint32_t(kBM), CU_TENSOR_MAP_SWIZZLE_64B);
+  if (st != FQ_OK) return st;
+  st = make_tmap_2d(&tb, gp.B, CU_TENSOR_MAP_DATA_TYPE_UINT8, uint64_t(gp.K) / 2, uint64_t(gp.rowsB), uint64_t(gp.K) / 2,
+                    uint32_t(kPK), uint32_t(BN));
+  if (st != FQ_OK) return st;
+  auto kern = gemm_w4a4_kernel<BN, EPI>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess ||
       cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
     return fail(FQ_ERR_CUDA, "cannot reserve %d bytes of shared memory for the GEMM", C::SMEM);
-  kern<<<grid, kThreads, C::SMEM, stream>>>(gp);
+  kern<<<grid, kThreads, C::SMEM, stream>>>(gp, ta, tb);
   return check_launch("gemm_w4a4_kernel");
 }
 
@@ -938,10 +948,10 @@ fq_status launch_decode(const GemmParams& gp, dim3 grid, cudaStream_t stream) {
 fq_status dispatch(const Plan& pl, const GemmParams& gp, dim3 grid, cudaStream_t s) {
   if (!pl.swap) {
     switch (pl.epi) {
-      case kEpiRow: return launch_gemm<256, kEpiRow, false>(gp, grid, s);
-      case kEpiStatic: return launch_gemm<256, kEpiStatic, false>(gp, grid, s);
-      case kEpiS32: return launch_gemm<256, kEpiS32, false>(gp, grid, s);
-      case kEpiGroup: return launch_gemm<128, kEpiGroup, false>(gp, grid, s);
+      case kEpiRow: return launch_gemm<256, kEpiRow>(gp, grid, s);
+      case kEpiStatic: return launch_gemm<256, kEpiStatic>(gp, grid, s);
+      case kEpiS32: return launch_gemm<256, kEpiS32>(gp, grid, s);
+      case kEpiGroup: return launch_gemm<128, kEpiGroup>(gp, grid, s);
       default: break;
     }
   } else {
