@@ -89,9 +89,10 @@ struct Cfg {
   // then the activation scales of the 128 rows
   static constexpr int SS = 8;
   static constexpr int SC_STAGE = BN * 8 + kBM * 4;
-  static constexpr int SCALE_BYTES = EPI == kEpiGroup ? SS * SC_STAGE : 0;
+  // row/static: the tile's BN weight scales, staged once by warp 0
+  static constexpr int SCALE_BYTES = EPI == kEpiGroup ? SS * SC_STAGE : ((EPI == kEpiRow || EPI == kEpiStatic) ? BN * 4 : 0);
   static constexpr int OFF_BAR = OFF_SCALE + SCALE_BYTES;
-  static constexpr int NBAR = 2 * SP + 2 * SU + 5 + (EPI == kEpiGroup ? 2 * SS : 0);
+  static constexpr int NBAR = 2 * SP + 2 * SU + 6 + (EPI == kEpiGroup ? 2 * SS : 0);
   static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
   static constexpr int SMEM = OFF_TMEM + 16 + 1024;  // + slack to align the base to 1024
   // the fp16 output tile is staged in the (then idle) unpacked ring, rows padded by 16 bytes
@@ -144,7 +145,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* acc_full = empty_u + SU;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* done_bar = acc_empty + 2;
-  uint64_t* sfull = done_bar + 1;   // group mode: scale stages
+  uint64_t* sw_ready = done_bar + 1;  // row/static: the tile's weight scales are in shared memory
+  uint64_t* sfull = sw_ready + 1;     // group mode: scale stages
   uint64_t* sempty = sfull + C::SS;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM);
 
@@ -167,6 +169,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&acc_empty[b], kEpiWarps);
     }
     mbar_init(done_bar, 1);
+    mbar_init(sw_ready, 1);
     if (EPI == kEpiGroup) {
       for (int s = 0; s < C::SS; ++s) {
         mbar_init(&sfull[s], 1);
@@ -211,6 +214,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
   } else if (warp == 0) {
+    if (EPI == kEpiRow || EPI == kEpiStatic) {
+      float* sws = reinterpret_cast<float*>(smem + C::OFF_SCALE);
+      for (int c = lane; c < BN; c += 32) {
+        const int n = tileB * BN + c;
+        sws[c] = n < p.N ? __ldg(p.sw + n) : 0.f;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sw_ready);
+    }
     if (EPI == kEpiGroup) {
       // ------------------------------------------------------------ group scales -> shared-memory ring
       // Loads run D slices ahead in registers, so their latency is paid once.
@@ -399,7 +411,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok && lane == 0) record_error(p.err, kErrTimeoutUnpack);
     }
-    if (epi_warp) {
+    // outside group mode the first four B-warps (6..9) take the upper half of
+    // the columns in the epilogue, after their last slice
+    const bool epi_hi = EPI != kEpiGroup && warp >= 6 && warp < 10;
+    if (epi_warp || epi_hi) {
     // ------------------------------------------------------------ epilogue
       const int q = warp & 3;  // tensor-memory lane quadrant this warp may access
       const int rloc = q * 32 + lane;
@@ -408,9 +423,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int bbase = tileB * BN;
       if (EPI != kEpiGroup) {
         if (!warp_wait(&acc_full[0], 0) && lane == 0) record_error(p.err, kErrTimeoutEpilogue);
+        if ((EPI == kEpiRow || EPI == kEpiStatic) && !warp_wait(sw_ready, 0) && lane == 0)
+          record_error(p.err, kErrTimeoutEpilogue);
         tc_fence_after();
         constexpr int CW = BN >= 32 ? 32 : 16;
-        for (int c0 = 0; c0 < BN; c0 += CW) {
+        const float* sws = reinterpret_cast<const float*>(smem + C::OFF_SCALE);
+        const int cbeg = epi_hi ? BN / 2 : 0, cend = (EPI == kEpiGroup || epi_hi) ? BN : BN / 2;
+        for (int c0 = cbeg; c0 < cend; c0 += CW) {
           uint32_t v[32];
           if (CW == 32)
             tmem_ld_32x32(tl + c0, v);
@@ -427,9 +446,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float sxm = EPI == kEpiRow ? p.sx[m] : 1.0f;
   #pragma unroll
                 for (int j = 0; j < CW; ++j) {
-                  const int n = min(n0 + j, p.N - 1);
                   const float a = float(int(v[j]) >> 8);
-                  y[j] = EPI == kEpiRow ? __fmul_rn(__fmul_rn(a, sxm), __ldg(p.sw + n)) : __fmul_rn(a, __ldg(p.sw + n));
+                  const float swn = sws[c0 + j];  // the same address in every lane: a broadcast
+                  y[j] = EPI == kEpiRow ? __fmul_rn(__fmul_rn(a, sxm), swn) : __fmul_rn(a, swn);
                 }
                 // staged in shared memory; written out coalesced after the barrier below
                 __half* dst = reinterpret_cast<__half*>(smem + C::OFF_UNP + rloc * C::OUT_PITCH) + c0;
