@@ -578,37 +578,28 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// y = dequant(split-K int32 sums): per-token x per-channel or static scales.
-__global__ void splitk_finalize_kernel(const int32_t* __restrict__ acc, const float* __restrict__ sx,
-                                       const float* __restrict__ sw, __half* __restrict__ Y, int M, int N,
-                                       int row_mode) {
-  const size_t total = size_t(M) * N;
-  for (size_t e = blockIdx.x * size_t(blockDim.x) + threadIdx.x; e < total; e += size_t(gridDim.x) * blockDim.x) {
-    const int m = int(e / N), n = int(e % N);
-    const float a = float(acc[e]);
-    const float y = row_mode ? __fmul_rn(__fmul_rn(a, sx[m]), sw[n]) : __fmul_rn(a, sw[n]);
-    Y[e] = __float2half_rn(y);
-  }
-}
-
 // ---------------------------------------------------------------- decode
 //
 // Few tokens (M <= 64): the GEMM is a stream of the packed weights, so the
-// kernel is built around keeping enough of that stream in flight.  The
-// weights take the 128-row MMA side (one CTA = 128 output channels x a K
-// range), the tokens the N side (BN = 16, 32 or 64).
+// kernel is built around keeping that stream flowing.  The weights take the
+// 128-row MMA side (tiles of 128 output channels), the tokens the N side
+// (BN = 16, 32 or 64).  The launch is one persistent wave (two CTAs per SM);
+// the (tile, K slice) pairs, tile-major, are split into equal contiguous
+// ranges, one per CTA (stream-K), so every CTA streams the same number of
+// weight bytes whatever the tile count.  A range covers whole tiles and at
+// most a partial tile at each end; whole tiles are written directly, the
+// partial ones add their exact int32 sums into the caller's workspace and
+// decode_fixup_kernel dequantizes those tiles afterwards.
 //   warp 0      one thread issues TMA loads of packed 128 x 64-byte weight
-//               slices into a ring of SP stages (64-byte swizzle, so that
-//               the row-per-thread reads below are free of bank conflicts)
-//   warp 1      tensor-memory allocation and the MMA-issuing thread
-//   warps 2-5   read one weight row each from the ring, unpack it and store
-//               it into a tensor-memory A ring (SU stages); afterwards the
-//               epilogue (thread = output channel, columns = tokens)
-//   warps 6-7   unpack the tokens' packed slices (L2-resident) into the
-//               128-byte swizzled shared-memory B ring
-// 256 threads and under 100 KB of shared memory, so two CTAs share an SM
-// and up to 2 x SP x 8 KB of the weight stream are in flight per SM.
-constexpr int kDecThreads = 256;
+//               slices (64-byte swizzle) and the tokens' slices into a ring
+//   warp 1      tensor-memory allocation and the MMA-issuing thread; the
+//               accumulator is double-buffered across tile segments
+//   warps 2-5   read one weight row each from the ring, unpack it into a
+//               tensor-memory A ring
+//   warps 6-7   unpack the tokens into the 128-byte-swizzled B ring
+//   warps 8-11  epilogue of each tile segment, overlapping the next one
+constexpr int kDecWarps = 12;
+constexpr int kDecThreads = 32 * kDecWarps;
 
 template <int BN>
 struct DecCfg {
@@ -621,12 +612,13 @@ struct DecCfg {
   static constexpr int OFF_X = OFF_P + SP * P_STAGE;
   static constexpr int OFF_B = OFF_X + SP * X_STAGE;
   static constexpr int OFF_BAR = OFF_B + SU * B_STAGE;
-  static constexpr int NBAR = 2 * SP + 2 * SU + 2;
+  static constexpr int NBAR = 2 * SP + 2 * SU + 5;
   static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
   // at least 80 KB, so that no more than two CTAs (2 x 256 tensor-memory
   // columns) are resident on one SM
   static constexpr int SMEM = (OFF_TMEM + 16 + 1024) > 80 * 1024 ? (OFF_TMEM + 16 + 1024) : 80 * 1024;
-  static constexpr int A_COL0 = BN < 32 ? 32 : BN;  // accumulator in columns [0, BN)
+  static constexpr int ACC = BN < 32 ? 32 : BN;   // columns of one accumulator buffer
+  static constexpr int A_COL0 = 2 * ACC;          // accumulators in columns [0, 2 ACC)
   static constexpr int A_STAGE_COLS = kBK / 4;
   static constexpr int TMEM_NEED = A_COL0 + SU * A_STAGE_COLS;
   static constexpr int TMEM_COLS = TMEM_NEED <= 128 ? 128 : 256;
@@ -634,6 +626,13 @@ struct DecCfg {
   static_assert(TMEM_NEED <= 256, "two CTAs per SM share the tensor memory");
   static_assert(2 * (SMEM + 1024) <= 228 * 1024, "two CTAs per SM");
 };
+
+// The slice range [b0, b1) of CTA c among g CTAs over t slices, and the CTA
+// that owns slice s (the inverse: b_c = floor(c t / g)).
+__host__ __device__ __forceinline__ long long sk_begin(long long c, long long g, long long t) { return c * t / g; }
+__host__ __device__ __forceinline__ int sk_owner(long long s, long long g, long long t) {
+  return int(((s + 1) * g - 1) / t);
+}
 
 template <int BN, int EPI>
 __global__ void __launch_bounds__(kDecThreads, 2)
@@ -648,14 +647,16 @@ __global__ void __launch_bounds__(kDecThreads, 2)
   uint64_t* pempty = pfull + SP;
   uint64_t* ufull = pempty + SP;
   uint64_t* uempty = ufull + SU;
-  uint64_t* acc_full = uempty + SU;
-  uint64_t* done_bar = acc_full + 1;
+  uint64_t* acc_full = uempty + SU;  // [2]
+  uint64_t* acc_empty = acc_full + 2;  // [2]
+  uint64_t* done_bar = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tileA = blockIdx.x;
-  const int kb0 = blockIdx.z * p.kb_per_split;
-  const int nkb = max(0, min(p.num_kb, kb0 + p.kb_per_split) - kb0);
+  const int nkb = p.num_kb;
+  const long long T = (long long)((p.rowsA + kBM - 1) / kBM) * nkb;
+  const long long b0 = sk_begin(blockIdx.x, gridDim.x, T), b1 = sk_begin(blockIdx.x + 1, gridDim.x, T);
+  const int nsl = int(b1 - b0);  // slices of this CTA
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < SP; ++s) {
@@ -666,7 +667,10 @@ __global__ void __launch_bounds__(kDecThreads, 2)
       mbar_init(&ufull[s], 6);
       mbar_init(&uempty[s], 1);
     }
-    mbar_init(acc_full, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 4);
+    }
     mbar_init(done_bar, 1);
     fence_mbar_init();
   }
@@ -684,18 +688,19 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     if (lane == 0) {
       prefetch_tensormap(&tmA);
       prefetch_tensormap(&tmX);
-      const uint64_t pol = policy_evict_first();  // the weights are read once
+      const uint64_t pol = policy_evict_first();   // the weights are read once
       const uint64_t pol_x = policy_evict_last();  // the tokens are read by every CTA
       int issued = 0;
-      for (int i = 0; i < nkb; ++i) {
+      int tile = int(b0 / nkb), kb = int(b0 - (long long)tile * nkb);  // advanced per slice
+      for (int i = 0; i < nsl; ++i, kb = kb + 1 == nkb ? 0 : kb + 1, tile += kb == 0) {
         const int sp = i % SP;
         if (!mbar_wait(&pempty[sp], ((i / SP) & 1) ^ 1)) {
           record_error(p.err, kErrTimeoutProducer);
           break;
         }
         mbar_arrive_expect_tx(&pfull[sp], C::P_STAGE + C::X_STAGE);
-        tma_load_2d_hint(smem + C::OFF_P + sp * C::P_STAGE, &tmA, &pfull[sp], (kb0 + i) * kPK, tileA * kBM, pol);
-        tma_load_2d_hint(smem + C::OFF_X + sp * C::X_STAGE, &tmX, &pfull[sp], (kb0 + i) * kPK, 0, pol_x);
+        tma_load_2d_hint(smem + C::OFF_P + sp * C::P_STAGE, &tmA, &pfull[sp], kb * kPK, tile * kBM, pol);
+        tma_load_2d_hint(smem + C::OFF_X + sp * C::X_STAGE, &tmX, &pfull[sp], kb * kPK, 0, pol_x);
         ++issued;
       }
       // every issued copy has landed before the CTA may leave (normally the
@@ -710,21 +715,37 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_i8_m128(BN);
-      for (int i = 0; i < nkb; ++i) {
+      int seg = -1;
+      bool ok = true;
+      int kb = int(b0 % nkb);  // advanced per slice
+      for (int i = 0; i < nsl && ok; ++i, kb = kb + 1 == nkb ? 0 : kb + 1) {
         const int su = i % SU;
+        const bool first = i == 0 || kb == 0, last = i == nsl - 1 || kb == nkb - 1;
+        if (first) {
+          ++seg;
+          // the first use of each buffer passes at once (the wait is for the
+          // phase before the first); later uses wait for the epilogue of the
+          // segment two back
+          if (!mbar_wait(&acc_empty[seg & 1], ((seg >> 1) & 1) ^ 1)) {
+            record_error(p.err, kErrTimeoutMma);
+            break;
+          }
+          tc_fence_after();
+        }
         if (!mbar_wait(&ufull[su], (i / SU) & 1)) {
           record_error(p.err, kErrTimeoutMma);
           break;
         }
         tc_fence_after();
+        const uint32_t d = tmem + uint32_t((seg & 1) * C::ACC);
         const uint32_t a0 = tmem + uint32_t(C::A_COL0 + su * C::A_STAGE_COLS);
-        const uint32_t b0 = smem_u32(smem + C::OFF_B + su * C::B_STAGE);
+        const uint32_t bsm = smem_u32(smem + C::OFF_B + su * C::B_STAGE);
 #pragma unroll
         for (int k = 0; k < kBK / 32; ++k)
-          mma_i8_ts(tmem, a0 + uint32_t(8 * k), sdesc_k128_sw128(b0 + 32 * k), idesc, uint32_t(i > 0 || k > 0));
+          mma_i8_ts(d, a0 + uint32_t(8 * k), sdesc_k128_sw128(bsm + 32 * k), idesc, uint32_t(!first || k > 0));
         mma_commit(&uempty[su]);
+        if (last) mma_commit(&acc_full[seg & 1]);
       }
-      mma_commit(acc_full);
       mma_commit(done_bar);
       if (!mbar_wait(done_bar, 0)) record_error(p.err, kErrTimeoutDrain);
     }
@@ -735,7 +756,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     const uint32_t ta = tmem + (uint32_t(q * 32) << 16) + uint32_t(C::A_COL0);
     const int sw = (row >> 1) & 3;  // 64-byte swizzle: chunk c of this row sits at chunk c ^ sw
     bool ok = true;
-    for (int i = 0; i < nkb; ++i) {
+    for (int i = 0; i < nsl; ++i) {
       const int sp = i % SP, su = i % SU;
       if (!warp_wait(&pfull[sp], (i / SP) & 1)) {
         ok = false;
@@ -772,7 +793,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
       }
     }
     if (!ok && lane == 0) record_error(p.err, kErrTimeoutUnpack);
-  } else {
+  } else if (warp < 8) {
     // ------------------------------------------------------------ token rows -> shared memory
     // The packed token slice arrives with the weights in the TMA ring; each
     // lane unpacks fixed 16-byte pieces (consecutive lanes read consecutive
@@ -792,7 +813,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
       dst1[it] = rb + uint32_t(((2 * c + 1) ^ r7) << 4);
     }
     bool ok = true;
-    for (int i = 0; i < nkb; ++i) {
+    for (int i = 0; i < nsl; ++i) {
       const int sp = i % SP, su = i % SU;
       if (!warp_wait(&pfull[sp], (i / SP) & 1)) {
         ok = false;
@@ -828,38 +849,51 @@ __global__ void __launch_bounds__(kDecThreads, 2)
       }
     }
     if (!ok && lane == 0) record_error(p.err, kErrTimeoutUnpack);
-  }
-
-  if (warp >= 2 && warp < 6) {
+  } else {
     // ------------------------------------------------------------ epilogue: thread = output channel n
     const int q = warp & 3;
-    const int n = tileA * kBM + q * 32 + lane;
     const uint32_t tl = tmem + (uint32_t(q * 32) << 16);
-    if (!warp_wait(acc_full, 0) && lane == 0) record_error(p.err, kErrTimeoutEpilogue);
-    tc_fence_after();
-    const float swn = (EPI == kEpiRow || EPI == kEpiStatic) && n < p.N ? __ldg(p.sw + n) : 0.f;
-    constexpr int CW = BN >= 32 ? 32 : 16;
-    for (int c0 = 0; c0 < BN; c0 += CW) {
-      uint32_t v[32];
-      if (CW == 32)
-        tmem_ld_32x32(tl + uint32_t(c0), v);
-      else
-        tmem_ld_32x16(tl + uint32_t(c0), v);
-      tmem_wait_ld();
-      if (n < p.N) {
+    long long s = b0;
+    for (int seg = 0; s < b1; ++seg) {
+      const int tile = int(s / nkb), kb_lo = int(s - (long long)tile * nkb);
+      const int len = int(min((long long)(nkb - kb_lo), b1 - s));
+      const bool whole = kb_lo == 0 && len == nkb;
+      s += len;
+      const int b = seg & 1;
+      if (!warp_wait(&acc_full[b], (seg >> 1) & 1)) {
+        if (lane == 0) record_error(p.err, kErrTimeoutEpilogue);
+        break;
+      }
+      tc_fence_after();
+      const int n = tile * kBM + q * 32 + lane;
+      const float swn = (EPI == kEpiRow || EPI == kEpiStatic) && n < p.N ? __ldg(p.sw + n) : 0.f;
+      constexpr int CW = BN >= 32 ? 32 : 16;
 #pragma unroll
-        for (int j = 0; j < CW; ++j) {
-          const int m = c0 + j;
-          if (m >= p.M) break;
-          const int32_t ai = int32_t(v[j]) >> 8;
-          if (EPI == kEpiRow)
-            p.Y[size_t(m) * p.N + n] = __float2half_rn(__fmul_rn(__fmul_rn(float(ai), __ldg(p.sx + m)), swn));
-          else if (EPI == kEpiStatic)
-            p.Y[size_t(m) * p.N + n] = __float2half_rn(__fmul_rn(float(ai), swn));
-          else
-            atomicAdd(p.acc + size_t(m) * p.N + n, ai);
+      for (int c0 = 0; c0 < BN; c0 += CW) {
+        uint32_t v[32];
+        if (CW == 32)
+          tmem_ld_32x32(tl + uint32_t(b * C::ACC + c0), v);
+        else
+          tmem_ld_32x16(tl + uint32_t(b * C::ACC + c0), v);
+        tmem_wait_ld();
+        if (n < p.N) {
+#pragma unroll
+          for (int j = 0; j < CW; ++j) {
+            const int m = c0 + j;
+            if (m >= p.M) break;
+            const int32_t ai = int32_t(v[j]) >> 8;
+            if (!whole)
+              atomicAdd(p.acc + size_t(m) * p.N + n, ai);
+            else if (EPI == kEpiRow)
+              p.Y[size_t(m) * p.N + n] = __float2half_rn(__fmul_rn(__fmul_rn(float(ai), __ldg(p.sx + m)), swn));
+            else
+              p.Y[size_t(m) * p.N + n] = __float2half_rn(__fmul_rn(float(ai), swn));
+          }
         }
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[b]);
     }
   }
 
@@ -871,12 +905,34 @@ __global__ void __launch_bounds__(kDecThreads, 2)
   }
 }
 
+// y = dequant(int32 sums) for the tiles that the stream-K ranges split
+// between CTAs (the others were written directly by the decode kernel): one
+// CTA of 128 threads per tile of 128 output channels, thread = channel.
+__global__ void __launch_bounds__(128) decode_fixup_kernel(const int32_t* __restrict__ acc,
+                                                           const float* __restrict__ sx,
+                                                           const float* __restrict__ sw, __half* __restrict__ Y,
+                                                           int M, int N, int nkb, int g, int row_mode) {
+  const long long T = (long long)((N + kBM - 1) / kBM) * nkb;
+  const long long t = blockIdx.x;
+  if (sk_owner(t * nkb, g, T) == sk_owner((t + 1) * nkb - 1, g, T)) return;  // one CTA wrote the tile
+  const int n = int(t) * kBM + threadIdx.x;
+  if (n >= N) return;
+  const float swn = sw[n];
+  for (int m = blockIdx.y; m < M; m += gridDim.y) {
+    const float a = float(acc[size_t(m) * N + n]);
+    const float y = row_mode ? __fmul_rn(__fmul_rn(a, sx[m]), swn) : __fmul_rn(a, swn);
+    Y[size_t(m) * N + n] = __float2half_rn(y);
+  }
+}
+
 struct Plan {
-  bool swap;
+  bool swap;          // decode kernel (weights on the 128-row side)
   int bn;
   int epi;
-  int splits;
+  int splits;         // prefill: K splits (always 1)
   int kb_per_split;
+  int ctas;           // decode: persistent CTAs sharing the slice sequence
+  bool partial;       // decode: some tile is split between CTAs (workspace + fixup)
 };
 
 int pick_bn_swap(int M) { return M <= 16 ? 16 : (M <= 32 ? 32 : 64); }
@@ -898,32 +954,24 @@ Plan make_plan(int M, int N, int K, int epi_final, int sms) {
     pl.epi = epi_final;
     return pl;
   }
-  // decode: weights on the 128-row side, tokens on the N side
+  // decode: weights on the 128-row side, tokens on the N side; one wave of
+  // two CTAs per SM, each with at least 8 K slices
   pl.swap = true;
   pl.bn = pick_bn_swap(M);
   pl.epi = epi_final;
-  const int tiles = (N + kBM - 1) / kBM;
-  const int per_sm = 2;  // decode CTAs resident per SM
-  const int slots = sms * per_sm;
-  double best = -1.0;
-  int best_s = 1;
-  for (int s = 1; s <= 16; ++s) {
-    if (nkb / s < 4) break;
-    const int ctas = tiles * s;
-    const int waves = (ctas + slots - 1) / slots;
-    const double eff = double(ctas) / double(waves * slots);
-    // extra traffic of split-K partial sums relative to the weight stream
-    const double extra = s > 1 ? double(M) * N * 4.0 * (s + 1) / (double(N) * K / 2.0) : 0.0;
-    const double score = eff / (1.0 + extra);
-    if (score > best + 1e-3) {
-      best = score;
-      best_s = s;
-    }
-  }
-  pl.splits = best_s;
-  pl.kb_per_split = (nkb + best_s - 1) / best_s;
-  pl.splits = (nkb + pl.kb_per_split - 1) / pl.kb_per_split;
-  if (pl.splits > 1) pl.epi = kEpiAtomic;
+  const long long tiles = (N + kBM - 1) / kBM;
+  const long long T = tiles * nkb;
+  // One CTA per tile when the tiles alone fill the resident slots and the
+  // token count makes the partial-tile path (workspace clear, int32 atomics,
+  // fixup) cost more than the last wave's imbalance; otherwise stream-K over
+  // one wave.
+  const long long slots = 2LL * sms;
+  if (tiles >= slots && M > 16)
+    pl.ctas = int(tiles);
+  else
+    pl.ctas = int(std::max<long long>(1, std::min<long long>(slots, T / 8)));
+  pl.partial = false;
+  for (long long c = 1; c < pl.ctas && !pl.partial; ++c) pl.partial = sk_begin(c, pl.ctas, T) % nkb != 0;
   return pl;
 }
 
@@ -979,7 +1027,6 @@ fq_status dispatch(const Plan& pl, const GemmParams& gp, dim3 grid, cudaStream_t
     switch (pl.epi) {                                                          \
       case kEpiRow: return launch_decode<BNV, kEpiRow>(gp, grid, s);           \
       case kEpiStatic: return launch_decode<BNV, kEpiStatic>(gp, grid, s);     \
-      case kEpiAtomic: return launch_decode<BNV, kEpiAtomic>(gp, grid, s);     \
       default: break;                                                          \
     }                                                                          \
   }
@@ -1015,7 +1062,7 @@ fq_status gemm_impl(const uint8_t* Xq, const void* s_x, const uint8_t* Wq, const
   if (!err) return fail(FQ_ERR_CUDA, "device error word unavailable");
   const int sms = sm_count();
   Plan pl = make_plan(M, N, K, epi_final, sms);
-  const size_t need = pl.splits > 1 ? size_t(M) * N * sizeof(int32_t) : 0;
+  const size_t need = (pl.swap && pl.partial) ? size_t(M) * N * sizeof(int32_t) : 0;
   if (need > 0) FQ_CHECK_ARG(ws && ws_bytes >= need && aligned(ws, 16), "workspace of %zu bytes required", need);
 
   GemmParams gp{};
@@ -1032,25 +1079,24 @@ fq_status gemm_impl(const uint8_t* Xq, const void* s_x, const uint8_t* Wq, const
     gp.gsx = static_cast<const __half*>(s_x);
     gp.gsw = static_cast<const __half*>(s_w);
   }
-  gp.acc = epi_final == kEpiS32 ? acc_out : (pl.splits > 1 ? static_cast<int32_t*>(ws) : nullptr);
+  gp.acc = epi_final == kEpiS32 ? acc_out : (need > 0 ? static_cast<int32_t*>(ws) : nullptr);
 
   gp.A = pl.swap ? Wq : Xq;
   gp.B = pl.swap ? Xq : Wq;
   gp.rowsA = pl.swap ? N : M;
   gp.rowsB = pl.swap ? M : N;
 
-  const dim3 grid((gp.rowsA + kBM - 1) / kBM, (gp.rowsB + pl.bn - 1) / pl.bn, pl.splits);
-  if (pl.splits > 1) {
+  const dim3 grid = pl.swap ? dim3(pl.ctas) : dim3((gp.rowsA + kBM - 1) / kBM, (gp.rowsB + pl.bn - 1) / pl.bn, 1);
+  if (need > 0) {
     if (cudaMemsetAsync(ws, 0, need, stream) != cudaSuccess) return fail(FQ_ERR_CUDA, "workspace clear failed");
   }
   st = dispatch(pl, gp, grid, stream);
   if (st != FQ_OK) return st;
-  if (pl.splits > 1) {
-    const int threads = 256;
-    const int blocks = int(std::min<size_t>((size_t(M) * N + threads - 1) / threads, size_t(sms) * 8));
-    splitk_finalize_kernel<<<blocks, threads, 0, stream>>>(gp.acc, gp.sx, gp.sw, gp.Y, M, N,
-                                                           epi_final == kEpiRow ? 1 : 0);
-    st = check_launch("splitk_finalize_kernel");
+  if (need > 0) {
+    const dim3 fgrid((N + kBM - 1) / kBM, std::min(M, 16));  // tiles x token groups
+    decode_fixup_kernel<<<fgrid, kBM, 0, stream>>>(gp.acc, gp.sx, gp.sw, gp.Y, M, N, gp.num_kb, pl.ctas,
+                                                   epi_final == kEpiRow ? 1 : 0);
+    st = check_launch("decode_fixup_kernel");
   }
   return st;
 }
@@ -1061,7 +1107,7 @@ size_t gemm_workspace_bytes(int M, int N, int K, fq_gran gran) {
   if (M < 1 || N < 8 || K < kBK || K % kBK) return 0;
   const int epi = gran == FQ_DYNAMIC_GROUP ? kEpiGroup : (gran == FQ_STATIC_CHANNEL ? kEpiStatic : kEpiRow);
   const Plan pl = make_plan(M, N, K, epi, sm_count());
-  return pl.splits > 1 ? size_t(M) * N * sizeof(int32_t) : 0;
+  return (pl.swap && pl.partial) ? size_t(M) * N * sizeof(int32_t) : 0;
 }
 
 }  // namespace fq

@@ -41,8 +41,9 @@ def test_noalloc_matches_workspace_gemm_twice(m, n, k, gran):
 
 
 def test_noalloc_rejects_scratch_beyond_its_buffer():
-    """A size whose split-K scratch exceeds the 8 MiB buffer is refused before any launch."""
-    m, n, k = 64, 38016, 65536
+    """A size whose split-K scratch exceeds the 8 MiB buffer is refused before any launch
+    (16 tokens against 139264 output channels: the tiles split between CTAs need M * N int32)."""
+    m, n, k = 16, 139264, 8192
     need = fq.fq_gemm_workspace_size(m, n, k, fq.ROW)
     assert need > 8 << 20
     L = fq.lib()
