@@ -49,8 +49,10 @@ constexpr int kUnpackWarps = 8;
 //   warp 0      group mode: keeps the per-slice scale ring filled; else idle
 //   warp 1      tensor-memory allocation and the MMA-issuing thread
 //   warps 2-5   epilogue (outside group mode they first unpack A)
-//   warps 6-13  unpack B (outside group mode); group mode: 6-9 A, 10-13 B
+//   warps 6-13  unpack B (outside group mode); group mode: 6-9 A,
+//               10-13 a second epilogue set (the upper half of the columns)
 //   warp 14     one thread issues the TMA loads of both packed slices
+//   warps 15-16 group mode only: unpack B
 // The packed 128-deep K slices of both operands arrive by TMA into a ring of
 // SP stages (A in the 64-byte swizzle, so that the one-row-per-thread reads
 // are free of bank conflicts; B unswizzled, read in consecutive 16-byte
@@ -58,12 +60,17 @@ constexpr int kUnpackWarps = 8;
 // B-warps into a 128-byte-swizzled shared-memory ring of SU stages.  A
 // packed stage goes back to the producer only after the unpacked data has
 // been stored (its registers consumed), so a refill never overtakes a read.
-constexpr int kWarps = 15;
-constexpr int kThreads = 32 * kWarps;
 constexpr int kProducerWarp = 14;
 
+// Group mode runs its per-slice epilogue alongside the main loop on eight
+// warps (two per tensor-memory lane quadrant), so it has 17 warps: the weight
+// slice of a 128-column tile is unpacked by warps 15-16.
 template <int EPI>
-__host__ __device__ constexpr int b_warps() { return EPI == kEpiGroup ? kUnpackWarps - 4 : kUnpackWarps; }
+__host__ __device__ constexpr int threads_of() { return 32 * (EPI == kEpiGroup ? 17 : 15); }
+template <int EPI>
+__host__ __device__ constexpr int epi_warps() { return EPI == kEpiGroup ? 2 * kEpiWarps : kEpiWarps; }
+template <int EPI>
+__host__ __device__ constexpr int b_warps() { return EPI == kEpiGroup ? 2 : kUnpackWarps; }
 template <int EPI>
 __host__ __device__ constexpr int feed_warps() { return 4 + b_warps<EPI>(); }
 
@@ -85,10 +92,10 @@ struct Cfg {
   static constexpr int OFF_UNP = OFF_P + SP * P_STAGE;
   static constexpr int OFF_SCALE = OFF_UNP + SU * UNP_STAGE;
   // group mode: a ring of SS per-slice scale stages written by warp 0: the
-  // weight scales as {s, s, -1.5*2^23*s, -1.5*2^23*s} pairs for BN columns,
-  // then the activation scales of the 128 rows
+  // weight scales s_w / 256 of the BN columns, then the activation scales of
+  // the 128 rows
   static constexpr int SS = 8;
-  static constexpr int SC_STAGE = BN * 8 + kBM * 4;
+  static constexpr int SC_STAGE = BN * 4 + kBM * 4;
   // row/static: the tile's BN weight scales, staged once by warp 0
   static constexpr int SCALE_BYTES = EPI == kEpiGroup ? SS * SC_STAGE : ((EPI == kEpiRow || EPI == kEpiStatic) ? BN * 4 : 0);
   static constexpr int OFF_BAR = OFF_SCALE + SCALE_BYTES;
@@ -130,7 +137,7 @@ __device__ __forceinline__ void store_half8(__half* dst, const float* v) {
 }
 
 template <int BN, int EPI>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(threads_of<EPI>(), 1)
     gemm_w4a4_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tmA,
                      const __grid_constant__ CUtensorMap tmB) {
   using C = Cfg<BN, EPI>;
@@ -166,14 +173,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], kEpiWarps);
+      mbar_init(&acc_empty[b], epi_warps<EPI>());
     }
     mbar_init(done_bar, 1);
     mbar_init(sw_ready, 1);
     if (EPI == kEpiGroup) {
       for (int s = 0; s < C::SS; ++s) {
         mbar_init(&sfull[s], 1);
-        mbar_init(&sempty[s], kEpiWarps);
+        mbar_init(&sempty[s], epi_warps<EPI>());
       }
     }
     fence_mbar_init();
@@ -228,7 +235,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       // Loads run D slices ahead in registers, so their latency is paid once.
       constexpr int D = 4;
       constexpr int NP2 = BN / 64;  // column pairs per lane
-      constexpr float kMagicF = 12582912.0f;  // 1.5 * 2^23 (see the group epilogue)
       const int bbase = tileB * BN, abase = tileA * kBM;
       __half2 wv[D][NP2];
       __half xv[D][4];
@@ -263,12 +269,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint8_t* sc = smem + C::OFF_SCALE + st * C::SC_STAGE;
 #pragma unroll
           for (int t = 0; t < NP2; ++t) {
-            const float2 w = __half22float2(wv[d][t]);
-            const float a = w.x * 0.00390625f, b = w.y * 0.00390625f;  // / 256, exact
-            reinterpret_cast<float4*>(sc)[lane + 32 * t] = make_float4(a, b, -kMagicF * a, -kMagicF * b);
+            const float2 w = __half22float2(wv[d][t]);  // / 256 below: exact
+            reinterpret_cast<float2*>(sc)[lane + 32 * t] = make_float2(w.x * 0.00390625f, w.y * 0.00390625f);
           }
 #pragma unroll
-          for (int t = 0; t < 4; ++t) reinterpret_cast<float*>(sc + BN * 8)[lane + 32 * t] = __half2float(xv[d][t]);
+          for (int t = 0; t < 4; ++t) reinterpret_cast<float*>(sc + BN * 4)[lane + 32 * t] = __half2float(xv[d][t]);
           __syncwarp();
           if (lane == 0) mbar_arrive(&sfull[st]);
           load(d, i + D);
@@ -317,7 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int NB = b_warps<EPI>();
     const bool epi_warp = warp < 2 + kEpiWarps;
     const bool a_warp = EPI == kEpiGroup ? (warp >= 6 && warp < 10) : epi_warp;
-    const bool b_warp = EPI == kEpiGroup ? (warp >= 10) : (warp >= 6);
+    const bool b_warp = EPI == kEpiGroup ? (warp >= 15) : (warp >= 6);
     if (a_warp) {
       // one A row per thread (its tensor-memory lane): 64 packed bytes per slice
       const int q = warp & 3;
@@ -359,7 +364,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok && lane == 0) record_error(p.err, kErrTimeoutUnpack);
     } else if (b_warp) {
-      const int uw = EPI == kEpiGroup ? warp - 10 : warp - 6;
+      const int uw = EPI == kEpiGroup ? warp - 15 : warp - 6;
       constexpr int kJobs = BN * 4;  // 16-byte packed pieces of B per stage
       constexpr int JPT = (kJobs + NB * 32 - 1) / (NB * 32);
       // per-lane pieces, the same in every stage: packed source offset, two swizzled destinations
@@ -411,9 +416,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok && lane == 0) record_error(p.err, kErrTimeoutUnpack);
     }
-    // outside group mode the first four B-warps (6..9) take the upper half of
-    // the columns in the epilogue, after their last slice
-    const bool epi_hi = EPI != kEpiGroup && warp >= 6 && warp < 10;
+    // the upper half of the columns: outside group mode the first four
+    // B-warps (6..9) after their last slice, in group mode warps 10..13
+    const bool epi_hi = EPI == kEpiGroup ? (warp >= 10 && warp < 14) : (warp >= 6 && warp < 10);
     if (epi_warp || epi_hi) {
     // ------------------------------------------------------------ epilogue
       const int q = warp & 3;  // tensor-memory lane quadrant this warp may access
@@ -474,21 +479,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Each accumulator buffer is primed with the integer 0x4B400000 (the
         // bits of 1.5 * 2^23) before the MMAs add 256 * sum(qx qw) (|.| <
         // 2^22) to it, so its bits read as the float 1.5 * 2^23 + acc
-        // exactly, with no int-to-float conversion.  Then one fused
-        // multiply-add, fma(f, s', -1.5 * 2^23 * s') with s' = s_w / 256
-        // (both exact in float32), gives fl(sum * s_w) with a single
-        // rounding, and a second one adds it times s_x into the running sum;
-        // both run two columns per instruction (fma.rn.f32x2).  Warp 0 has
-        // the slice's s' and -1.5 * 2^23 * s' pairs and the row scales ready
-        // in a shared-memory ring.
+        // exactly, with no int-to-float conversion: f - 1.5 * 2^23 is the
+        // accumulator, exact; times s' = s_w / 256 (exact) it gives
+        // fl(sum * s_w) with a single rounding, and a fused multiply-add
+        // adds that times s_x into the running sum (zeroed at the start);
+        // two columns per instruction (f32x2).  Warp 0 keeps the slice's s'
+        // and row scales ready in a shared-memory ring; one 16-byte load
+        // gives the scales of four columns.
         constexpr uint32_t kMagic = 0x4B400000u;
         const uint32_t tsum = tl + uint32_t(2 * BN);
+        const int gbeg = epi_hi ? BN / 2 : 0, gend = epi_hi ? BN : BN / 2;  // this warp's columns
         uint32_t mg[32];
 #pragma unroll
         for (int j = 0; j < 32; ++j) mg[j] = kMagic;
 #pragma unroll
         for (int b = 0; b < 2; ++b)
-          for (int c0 = 0; c0 < BN; c0 += 32) tmem_st_32x32(tl + uint32_t(b * BN + c0), mg);
+          for (int c0 = gbeg; c0 < gend; c0 += 32) tmem_st_32x32(tl + uint32_t(b * BN + c0), mg);
+        {
+          uint32_t z[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) z[j] = 0u;
+          for (int c0 = gbeg; c0 < gend; c0 += 32) tmem_st_32x32(tsum + c0, z);
+        }
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -503,28 +515,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           const float4* sbuf = reinterpret_cast<const float4*>(smem + C::OFF_SCALE + st * C::SC_STAGE);
-          const float sxg = reinterpret_cast<const float*>(smem + C::OFF_SCALE + st * C::SC_STAGE + BN * 8)[rloc];
+          const float sxg = reinterpret_cast<const float*>(smem + C::OFF_SCALE + st * C::SC_STAGE + BN * 4)[rloc];
           const float2 sx2 = make_float2(sxg, sxg);
+          const float2 nmag = make_float2(-12582912.0f, -12582912.0f);  // -1.5 * 2^23
           if (!warp_wait(&acc_full[b], (i >> 1) & 1)) {
             if (lane == 0) record_error(p.err, kErrTimeoutEpilogue);
             break;
           }
           tc_fence_after();
-          for (int c0 = 0; c0 < BN; c0 += 32) {
+          for (int c0 = gbeg; c0 < gend; c0 += 32) {
             uint32_t v[32], s[32];
             tmem_ld_32x32(tl + uint32_t(b * BN + c0), v);
-            if (i > 0) tmem_ld_32x32(tsum + c0, s);
+            tmem_ld_32x32(tsum + c0, s);
             tmem_wait_ld();
   #pragma unroll
-            for (int j = 0; j < 32; j += 2) {
-              const float4 q = sbuf[(c0 + j) / 2];
-              const float2 u = ffma2(make_float2(__uint_as_float(v[j]), __uint_as_float(v[j + 1])),
-                                     make_float2(q.x, q.y), make_float2(q.z, q.w));
-              const float2 prev = i > 0 ? make_float2(__uint_as_float(s[j]), __uint_as_float(s[j + 1]))
-                                        : make_float2(0.f, 0.f);
-              const float2 r = ffma2(u, sx2, prev);
-              s[j] = __float_as_uint(r.x);
-              s[j + 1] = __float_as_uint(r.y);
+            for (int j = 0; j < 32; j += 4) {
+              const float4 q = sbuf[(c0 + j) / 4];
+#pragma unroll
+              for (int h = 0; h < 4; h += 2) {
+                const float2 a = fadd2(make_float2(__uint_as_float(v[j + h]), __uint_as_float(v[j + h + 1])), nmag);
+                const float2 u = fmul2(a, h == 0 ? make_float2(q.x, q.y) : make_float2(q.z, q.w));
+                const float2 r = ffma2(u, sx2, make_float2(__uint_as_float(s[j + h]), __uint_as_float(s[j + h + 1])));
+                s[j + h] = __float_as_uint(r.x);
+                s[j + h + 1] = __float_as_uint(r.y);
+              }
             }
             tmem_st_32x32(tsum + c0, s);
             tmem_st_32x32(tl + uint32_t(b * BN + c0), mg);  // re-prime for slice i + 2
@@ -537,7 +551,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive(&sempty[st]);
           }
         }
-        for (int c0 = 0; c0 < BN; c0 += 32) {
+        for (int c0 = gbeg; c0 < gend; c0 += 32) {
           uint32_t s[32];
           tmem_ld_32x32(tsum + c0, s);
           tmem_wait_ld();
@@ -560,7 +574,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     const int n0 = tileB * BN;
     const int chunks = max(0, min(BN, p.N - n0)) / 8;  // 16-byte chunks per row (N % 8 == 0)
-    for (int r = warp; r < kBM; r += kThreads / 32) {
+    for (int r = warp; r < kBM; r += threads_of<EPI>() / 32) {
       const int m = tileA * kBM + r;
       if (m >= p.M) break;
       const uint8_t* src = smem + C::OFF_UNP + r * C::OUT_PITCH;
@@ -990,7 +1004,7 @@ fq_status launch_gemm(const GemmParams& gp, dim3 grid, cudaStream_t stream) {
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess ||
       cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
     return fail(FQ_ERR_CUDA, "cannot reserve %d bytes of shared memory for the GEMM", C::SMEM);
-  kern<<<grid, kThreads, C::SMEM, stream>>>(gp, ta, tb);
+  kern<<<grid, threads_of<EPI>(), C::SMEM, stream>>>(gp, ta, tb);
   return check_launch("gemm_w4a4_kernel");
 }
 
