@@ -36,6 +36,15 @@ __device__ __forceinline__ void record_error(unsigned* err, unsigned code) {
   if (err) atomicCAS(err, 0u, code);
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+
+// Wait until the kernels before this one on the stream have completed and
+// their memory is visible (a no-op when the launch was not programmatic).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Allow the next kernel on the stream to be scheduled (its own pdl_wait still
+// waits for this kernel to complete).
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------------------ mbarrier
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {

@@ -8,6 +8,7 @@
 #include <cstdarg>
 #include <cstddef>
 #include <cstdint>
+#include <utility>
 
 #include "../../include/fq.h"
 
@@ -35,6 +36,27 @@ inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_
 fq_status make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, uint64_t inner,
                        uint64_t rows, uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows,
                        CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_NONE);
+
+// Launch with programmatic stream serialization: the kernel may start while
+// the previous kernel on the stream is still finishing; it must execute
+// pdl_wait() (griddepcontrol.wait) before touching global memory that an
+// earlier kernel may write or read, and it lets its own successor start
+// early with pdl_launch_dependents().
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 constexpr int kGroup = 128;
 constexpr int kMaxK = 65536;

@@ -193,6 +193,10 @@ __global__ void __launch_bounds__(threads_of<EPI>(), 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // the next kernel may be scheduled once every CTA of this one is running;
+  // this one reads its inputs only after the kernels before it completed
+  pdl_launch_dependents();
+  pdl_wait();
 
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ TMA producer
@@ -696,6 +700,8 @@ __global__ void __launch_bounds__(kDecThreads, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_launch_dependents();
+  pdl_wait();
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -1004,7 +1010,11 @@ fq_status launch_gemm(const GemmParams& gp, dim3 grid, cudaStream_t stream) {
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess ||
       cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
     return fail(FQ_ERR_CUDA, "cannot reserve %d bytes of shared memory for the GEMM", C::SMEM);
-  kern<<<grid, threads_of<EPI>(), C::SMEM, stream>>>(gp, ta, tb);
+  const cudaError_t e = launch_pdl(kern, grid, dim3(threads_of<EPI>()), C::SMEM, stream, gp, ta, tb);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(FQ_ERR_CUDA, "gemm_w4a4_kernel: %s", cudaGetErrorString(e));
+  }
   return check_launch("gemm_w4a4_kernel");
 }
 
@@ -1022,7 +1032,11 @@ fq_status launch_decode(const GemmParams& gp, dim3 grid, cudaStream_t stream) {
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess ||
       cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
     return fail(FQ_ERR_CUDA, "cannot reserve %d bytes of shared memory for the decode GEMM", C::SMEM);
-  kern<<<grid, kDecThreads, C::SMEM, stream>>>(gp, tm, tx);
+  const cudaError_t e = launch_pdl(kern, grid, dim3(kDecThreads), C::SMEM, stream, gp, tm, tx);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(FQ_ERR_CUDA, "gemm_decode_kernel: %s", cudaGetErrorString(e));
+  }
   return check_launch("gemm_decode_kernel");
 }
 

@@ -197,6 +197,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
   fence_proxy_async_smem();
   __syncthreads();
+  // the next kernel may be scheduled once every CTA of this one is running;
+  // global memory is touched only after the kernels before this one completed
+  pdl_launch_dependents();
+  pdl_wait();
 
   const uint32_t lane_off = uint32_t(q4 * 32) << 16;
   const int bar_id = 1 + pipe;
@@ -620,7 +624,11 @@ fq_status launch_tc4(const QuantTcParams& p, cudaStream_t stream) {
     return fail(FQ_ERR_CUDA, "cannot reserve %d bytes of shared memory for the transform kernel", C::SMEM);
   const int ngroups = (p.M + C::G - 1) / C::G;
   const int grid = std::max(1, std::min((ngroups + C::P - 1) / C::P, sm_count()));
-  kern<<<grid, kTcThreads, C::SMEM, stream>>>(p, tm);
+  const cudaError_t e = launch_pdl(kern, dim3(grid), dim3(kTcThreads), C::SMEM, stream, p, tm);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(FQ_ERR_CUDA, "quant_act_tc_kernel: %s", cudaGetErrorString(e));
+  }
   return check_launch("quant_act_tc_kernel");
 }
 
