@@ -41,7 +41,7 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # (dram__bytes_read.sum + dram__bytes_write.sum) of this bench command on the
 # current GEMM kernel; the fp16 outputs that still sit in L2 when a launch
 # ends are not in it.
-GEMM_DRAM_BYTES = {"qkv": 16843776, "o": 12641792, "gate_up": 63073280 + 66820096, "down": 44099584 + 52736}
+GEMM_DRAM_BYTES = {"qkv": 16849152, "o": 12634112, "gate_up": 63113216 + 67183616, "down": 44094208 + 187392}
 INT8_OVER_BF16 = 4.5 / 2.25  # nominal dense ratio (B200: 4.5 POPS int8 vs 2.25 PFLOPS bf16)
 
 
@@ -532,12 +532,12 @@ def run_decode(args, dev_index):
     return {
         "metric": METRIC, "workload": "decode", "value": round(gbs, 1), "unit": "GB/s", "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(g_s * 1e3, 4), "higher_is_better": True,
-        "dtype": "int4 (s8 tensor-core MMA, swap-AB, split-K int32), fp16 io", "data": "synthetic",
+        "dtype": "int4 (s8 tensor-core MMA, weights on the 128-row side, stream-K int32 partials), fp16 io", "data": "synthetic",
         "config": {"workload": "decode M in {1, 8, 32, 64} x (K, N) in {(8192, 57344), (28672, 8192)}, static "
                                "per-channel activation scales folded into per-channel INT4 weights",
                    "l2": "256 MiB flush between launches; median of the launches"},
         "rows": rows,
-        "roofline": {"kernel": "gemm_w4a4_kernel swap-AB (+ splitk_finalize_kernel)", "bound": "hbm",
+        "roofline": {"kernel": "gemm_decode_kernel (+ decode_fixup_kernel for split tiles)", "bound": "hbm",
                      "achieved": round(gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
                      "frac": round(gbs / pk["hbm_gbs"], 4), "peak_kind": pk_kind, "traffic": None},
         "clocks": clk,
