@@ -93,6 +93,60 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint64
   return __all_sync(0xffffffffu, ok);
 }
 
+// ------------------------------------------------------------------ CTA pairs (clusters of two)
+
+// Rank of this CTA within its cluster.
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// Every thread of every CTA of the cluster arrives and waits (release /
+// acquire at cluster scope).  Only used where each thread of both CTAs
+// reaches it unconditionally.
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Arrive on the mbarrier at the same shared-memory offset as `bar` in the
+// cluster's CTA `rank`.  Default (CTA-scope release) semantics: what the
+// arrival publishes is made complete beforehand by the caller (tcgen05.wait::st
+// for tensor-memory stores, fence.proxy.async for shared-memory operands the
+// tensor core reads), and a cluster-scope release here costs a memory fence
+// per arrival (it made the CTA-pair GEMM 1.6x slower).
+__device__ __forceinline__ void mbar_arrive_cluster(uint64_t* bar, uint32_t rank) {
+  asm volatile(
+      "{\n\t.reg .b32 ra;\n\t"
+      "mapa.shared::cluster.u32 ra, %0, %1;\n\t"
+      "mbarrier.arrive.shared::cluster.b64 _, [ra];\n\t}" ::"r"(smem_u32(bar)),
+      "r"(rank)
+      : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// mbar_wait with acquire at cluster scope (the phase completes by arrivals
+// of the other CTA of the pair too); false after limit_ns.
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, uint64_t limit_ns = kWaitLimitNs) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if ((i & 63u) == 0 && globaltimer_ns() - t0 > limit_ns) return false;
+  }
+}
+
 // ------------------------------------------------------------------ warps and barriers
 
 // Largest value of v over the 32 lanes (one warp-wide reduction instruction).
@@ -246,6 +300,45 @@ __device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uin
       : "memory");
 }
 
+// ---- CTA-pair forms (.cta_group::2): one warp of each CTA of the pair
+// allocates (the same columns in both tensor memories) and deallocates; the
+// MMA is issued by one thread of the even CTA and reads A and writes D at the
+// same tensor-memory address of both CTAs, B at the same shared-memory
+// offset of both (each CTA holding half of the N rows).
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* slot, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)), "r"(ncols)
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem] over the CTA pair, s8 x s8 -> s32.
+__device__ __forceinline__ void mma_i8_ts_pair(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                               uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrive (once) on the mbarrier at `bar`'s offset in each CTA of `cta_mask`
+// when every tcgen05 operation this thread issued so far completes.
+__device__ __forceinline__ void mma_commit_pair(uint64_t* bar, uint16_t cta_mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"(cta_mask)
+      : "memory");
+}
+
 // Arrive (once) on `bar` when every tcgen05 operation this thread issued so far completes.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
@@ -253,14 +346,16 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
 }
 
 // Instruction descriptor of tcgen05.mma .kind::i8: D = s32, A = B = s8,
-// both K-major, M = 128 rows, N = n (multiple of 16, 16..256).
-__host__ __device__ constexpr uint32_t idesc_i8_m128(int n) {
+// both K-major, M = m rows (128; 256 over a CTA pair), N = n (multiple of
+// 16, 16..256).
+__host__ __device__ constexpr uint32_t idesc_i8(int m, int n) {
   return (2u << 4)      // D format: s32
          | (1u << 7)    // A format: signed 8-bit
          | (1u << 10)   // B format: signed 8-bit
          | (uint32_t(n >> 3) << 17)
-         | (uint32_t(128 >> 4) << 24);
+         | (uint32_t(m >> 4) << 24);
 }
+__host__ __device__ constexpr uint32_t idesc_i8_m128(int n) { return idesc_i8(128, n); }
 
 // Instruction descriptor of tcgen05.mma .kind::f16: D = f32, A = B = f16,
 // both K-major, M = 128 rows, N = n (multiple of 16, 16..256).
