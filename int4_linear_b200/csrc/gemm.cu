@@ -658,6 +658,386 @@ __global__ void __launch_bounds__(threads_of<EPI>(), 1)
   }
 }
 
+// ---------------------------------------------------------------- persistent CTA-pair prefill kernel
+//
+// Per-token / static scales with M > 64.  A persistent grid of CTA pairs
+// (one CTA per SM) walks the 256 x 256 output tiles (pairs of 128-row A
+// tiles x 256 weight rows), so the operand pipeline runs on across tile
+// boundaries and the epilogue of one tile overlaps the main loop of the next:
+//   warp 0        one thread issues the TMA loads of the packed slices
+//   warp 1        tensor-memory allocation; in CTA 0 the thread that issues
+//                 the 256 x 256 pair MMAs (.cta_group::2)
+//   warps 2-5     unpack this CTA's 128 A rows into the tensor-memory ring
+//   warps 6..     unpack this CTA's half of the weight rows (NB warps)
+//   last 8 warps  epilogue: drain the accumulator (two warps per lane
+//                 quadrant, 128 columns each, 32 at a time), scale to fp16
+//                 into a per-warp shared-memory block and TMA-store it; the
+//                 accumulator goes back to the MMA thread as soon as its last
+//                 columns are read
+// The accumulator is single-buffered (256 columns + the A ring); the MMA
+// thread waits for both CTAs' epilogues to have read it, while the feed
+// warps fill the rings ahead of the next tile.
+template <int NB>
+struct PCfg {
+  static constexpr int BN = 256;               // pair tile columns
+  static constexpr int BR = BN / 2;            // weight rows per CTA
+  static constexpr int SP = 6;                 // packed stages (TMA ring)
+  static constexpr int SU = 5;                 // unpacked stages
+  static constexpr int PA = kBM * kPK;
+  static constexpr int PB = BR * kPK;
+  static constexpr int P_STAGE = PA + PB;
+  static constexpr int UNP_STAGE = BR * kBK;
+  static constexpr int A_COL0 = BN;            // A ring after the accumulator
+  static constexpr int A_STAGE_COLS = kBK / 4;
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int OFF_P = 0;
+  static constexpr int OFF_UNP = OFF_P + SP * P_STAGE;
+  static constexpr int OFF_SCALE = OFF_UNP + SU * UNP_STAGE;  // [2][BN] weight scales
+  static constexpr int STG = 32 * 32 * 2;                     // one 32 x 32 fp16 output block
+  static constexpr int OFF_STG = OFF_SCALE + 2 * BN * 4;      // [8 warps][2 blocks]
+  static constexpr int OFF_BAR = OFF_STG + 8 * 2 * STG;
+  static constexpr int NBAR = 2 * SP + 2 * SU + 4;          // + acc_full, acc_empty, done, fin
+  static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM = OFF_TMEM + 16 + 1024;
+  static constexpr int EPI_WARP0 = 6 + NB;
+  static constexpr int THREADS = 32 * (EPI_WARP0 + 8);
+  static constexpr int FEED = 4 + NB;          // feed warps per CTA
+  static_assert(A_COL0 + SU * A_STAGE_COLS <= TMEM_COLS, "tensor memory");
+  static_assert(SMEM <= 227 * 1024, "shared memory");
+  static_assert(P_STAGE % 1024 == 0 && UNP_STAGE % 1024 == 0 && PA % 1024 == 0, "1024-byte stage alignment");
+};
+
+template <int EPI, int NB>
+__global__ void __launch_bounds__(PCfg<NB>::THREADS, 1)
+    gemm_w4a4_persistent_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tmA,
+                                const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmY) {
+  using C = PCfg<NB>;
+  constexpr int SP = C::SP, SU = C::SU, BN = C::BN;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* pfull = bars;
+  uint64_t* pempty = pfull + SP;
+  uint64_t* full_u = pempty + SP;
+  uint64_t* empty_u = full_u + SU;
+  uint64_t* acc_full = empty_u + SU;
+  uint64_t* acc_empty = acc_full + 1;
+  uint64_t* done_bar = acc_empty + 1;
+  uint64_t* fin_bar = done_bar + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM);
+
+  const uint32_t crank = cluster_rank();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int pairs_m = (p.rowsA + 2 * kBM - 1) / (2 * kBM);
+  const int tiles_n = (p.rowsB + BN - 1) / BN;
+  const int ntiles = pairs_m * tiles_n;
+  const int cid = int(blockIdx.x >> 1), ncl = int(gridDim.x >> 1);
+  const int my_tiles = ntiles > cid ? (ntiles - cid + ncl - 1) / ncl : 0;
+  const int nkb = p.num_kb;
+  const uint32_t total = uint32_t(my_tiles) * uint32_t(nkb);  // K slices this CTA streams
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < SP; ++s) {
+      mbar_init(&pfull[s], 1);
+      mbar_init(&pempty[s], C::FEED);
+    }
+    for (int s = 0; s < SU; ++s) {
+      mbar_init(&full_u[s], 2 * C::FEED);
+      mbar_init(&empty_u[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 2 * 8);
+    mbar_init(done_bar, 1);
+    mbar_init(fin_bar, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // the other CTA's barriers are initialized and its tensor memory allocated
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  pdl_launch_dependents();
+  pdl_wait();
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tensormap(&tmA);
+      prefetch_tensormap(&tmB);
+      uint32_t g = 0;
+      int arow = 0, brow = 0;
+      for (int t = cid, i = 0; g < total;) {
+        if (i == 0) {
+          // a pair's second CTA past the last A (or B) rows still feeds its
+          // other operand; it loads in-range rows whose products are never stored
+          const int ta = 2 * (t % pairs_m) + int(crank), tb = t / pairs_m;
+          arow = ta * kBM < p.rowsA ? ta * kBM : 0;
+          const int br = tb * BN + int(crank) * C::BR;
+          brow = br < p.rowsB ? br : 0;
+        }
+        const int sp = int(g % SP);
+        if (!mbar_wait(&pempty[sp], ((g / SP) & 1) ^ 1)) {
+          record_error(p.err, kErrTimeoutProducer);
+          break;
+        }
+        uint8_t* st = smem + C::OFF_P + sp * C::P_STAGE;
+        mbar_arrive_expect_tx(&pfull[sp], C::P_STAGE);
+        tma_load_2d(st, &tmA, &pfull[sp], i * kPK, arow);
+        tma_load_2d(st + C::PA, &tmB, &pfull[sp], i * kPK, brow);
+        ++g;
+        if (++i == nkb) {
+          i = 0;
+          t += ncl;
+        }
+      }
+      for (uint32_t j = g > uint32_t(SP) ? g - SP : 0; j < g; ++j)
+        if (!mbar_wait(&pfull[j % SP], (j / SP) & 1)) {
+          record_error(p.err, kErrTimeoutDrain);
+          break;
+        }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (CTA 0)
+    if (lane == 0 && crank == 0) {
+      constexpr uint32_t idesc = idesc_i8(2 * kBM, BN);
+      uint32_t g = 0;
+      bool ok = true;
+      for (int tl = 0; tl < my_tiles && ok; ++tl) {
+        // both CTAs' epilogues have read the previous tile's accumulator
+        if (!mbar_wait_cluster(acc_empty, (tl & 1) ^ 1)) {
+          record_error(p.err, kErrTimeoutMma);
+          break;
+        }
+        tc_fence_after();
+        for (int i = 0; i < nkb; ++i, ++g) {
+          const int su = int(g % SU);
+          if (!mbar_wait_cluster(&full_u[su], (g / SU) & 1)) {
+            record_error(p.err, kErrTimeoutMma);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = tmem + uint32_t(C::A_COL0 + su * C::A_STAGE_COLS);
+          const uint32_t b0 = smem_u32(smem + C::OFF_UNP + su * C::UNP_STAGE);
+#pragma unroll
+          for (int k = 0; k < kBK / 32; ++k)
+            mma_i8_ts_pair(tmem, a0 + uint32_t(8 * k), sdesc_k128_sw128(b0 + 32 * k), idesc,
+                           uint32_t(i > 0 || k > 0));
+          mma_commit_pair(&empty_u[su], 3);
+        }
+        if (ok) mma_commit_pair(acc_full, 3);
+      }
+      mma_commit_pair(done_bar, 3);
+      if (!mbar_wait(done_bar, 0)) record_error(p.err, kErrTimeoutDrain);
+    } else if (lane == 0) {
+      // CTA 1 stays until CTA 0's MMAs, which read its shared and tensor
+      // memory, have completed
+      if (!mbar_wait(done_bar, 0)) record_error(p.err, kErrTimeoutDrain);
+    }
+  } else if (warp < 6) {
+    // ------------------------------------------------------------ A rows -> tensor-memory ring
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    const int sw = (row >> 1) & 3;  // 64-byte swizzle: chunk c of this row sits at chunk c ^ sw
+    const uint32_t ta = tmem + (uint32_t(q * 32) << 16) + uint32_t(C::A_COL0);
+    bool ok = true;
+    for (uint32_t g = 0; g < total; ++g) {
+      const int sp = int(g % SP), su = int(g % SU);
+      if (!warp_wait(&pfull[sp], (g / SP) & 1)) {
+        ok = false;
+        break;
+      }
+      const uint8_t* src = smem + C::OFF_P + sp * C::P_STAGE + row * kPK;
+      uint4 w[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) w[c] = *reinterpret_cast<const uint4*>(src + ((c ^ sw) << 4));
+      if (!warp_wait(&empty_u[su], ((g / SU) & 1) ^ 1)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t r[32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        unpack8_hi(w[c].x, r[8 * c + 0], r[8 * c + 1]);
+        unpack8_hi(w[c].y, r[8 * c + 2], r[8 * c + 3]);
+        unpack8_hi(w[c].z, r[8 * c + 4], r[8 * c + 5]);
+        unpack8_hi(w[c].w, r[8 * c + 6], r[8 * c + 7]);
+      }
+      tmem_st_32x32(ta + uint32_t(su * C::A_STAGE_COLS), r);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&pempty[sp]);
+        if (crank == 0)
+          mbar_arrive(&full_u[su]);
+        else
+          mbar_arrive_cluster(&full_u[su], 0);
+      }
+    }
+    if (!ok && lane == 0) record_error(p.err, kErrTimeoutUnpack);
+  } else if (warp < C::EPI_WARP0) {
+    // ------------------------------------------------------------ weight rows -> shared-memory ring
+    const int uw = warp - 6;
+    constexpr int kJobs = C::BR * 4;  // 16-byte packed pieces per stage
+    constexpr int JPT = (kJobs + NB * 32 - 1) / (NB * 32);
+    uint32_t dst0[JPT], dst1[JPT], srcj[JPT];
+    bool live[JPT];
+#pragma unroll
+    for (int it = 0; it < JPT; ++it) {
+      const int j = (it * NB + uw) * 32 + lane;
+      live[it] = j < kJobs;
+      const int row = live[it] ? (j >> 2) : 0, c = j & 3, r7 = row & 7;
+      const uint32_t rb = uint32_t((row >> 3) * 1024 + r7 * 128);
+      dst0[it] = rb + uint32_t(((2 * c) ^ r7) << 4);
+      dst1[it] = rb + uint32_t(((2 * c + 1) ^ r7) << 4);
+      srcj[it] = uint32_t(live[it] ? j * 16 : 0);
+    }
+    bool ok = true;
+    for (uint32_t g = 0; g < total; ++g) {
+      const int sp = int(g % SP), su = int(g % SU);
+      if (!warp_wait(&pfull[sp], (g / SP) & 1)) {
+        ok = false;
+        break;
+      }
+      const uint8_t* pb = smem + C::OFF_P + sp * C::P_STAGE + C::PA;
+      uint4 w[JPT];
+#pragma unroll
+      for (int it = 0; it < JPT; ++it) w[it] = *reinterpret_cast<const uint4*>(pb + srcj[it]);
+      if (!warp_wait(&empty_u[su], ((g / SU) & 1) ^ 1)) {
+        ok = false;
+        break;
+      }
+      uint8_t* uk = smem + C::OFF_UNP + su * C::UNP_STAGE;
+#pragma unroll
+      for (int it = 0; it < JPT; ++it) {
+        if (!live[it]) continue;
+        uint4 o0, o1;
+        unpack8_hi(w[it].x, o0.x, o0.y);
+        unpack8_hi(w[it].y, o0.z, o0.w);
+        unpack8_hi(w[it].z, o1.x, o1.y);
+        unpack8_hi(w[it].w, o1.z, o1.w);
+        *reinterpret_cast<uint4*>(uk + dst0[it]) = o0;
+        *reinterpret_cast<uint4*>(uk + dst1[it]) = o1;
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&pempty[sp]);
+        if (crank == 0)
+          mbar_arrive(&full_u[su]);
+        else
+          mbar_arrive_cluster(&full_u[su], 0);
+      }
+    }
+    if (!ok && lane == 0) record_error(p.err, kErrTimeoutUnpack);
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int e = warp - C::EPI_WARP0;  // 0..7
+    const int q = warp & 3;             // tensor-memory lane quadrant this warp may access
+    const int h = e >> 2;               // column half
+    const int et = e * 32 + lane;       // 0..255: loads one weight scale per tile
+    const uint32_t tq = tmem + (uint32_t(q * 32) << 16);
+    float* sws = reinterpret_cast<float*>(smem + C::OFF_SCALE);
+    uint8_t* stg = smem + C::OFF_STG + e * 2 * C::STG;
+    const int swz = (lane >> 1) & 3;  // 64-byte swizzle of the staged block (row = lane)
+    if (lane == 0) prefetch_tensormap(&tmY);
+    int tl = 0, blk = 0;
+    for (int t = cid; t < ntiles; t += ncl, ++tl) {
+      const int ta = 2 * (t % pairs_m) + int(crank), n0 = (t / pairs_m) * BN;
+      float* sb = sws + (tl & 1) * BN;  // double-buffered: the other buffer may still be read
+      sb[et] = n0 + et < p.N ? __ldg(p.sw + n0 + et) : 0.f;
+      const int row0 = ta * kBM + q * 32;
+      const int row = row0 + lane;
+      const float sxm = (EPI == kEpiRow && row < p.M) ? p.sx[row] : 1.0f;
+      const bool got = warp_wait(acc_full, tl & 1);
+      // one decision for all eight warps (they share the barrier below)
+      if (named_barrier_or(1, 256, !got)) {
+        if (lane == 0) record_error(p.err, kErrTimeoutEpilogue);
+        break;
+      }
+      tc_fence_after();
+      // y = fl(fl(sum * s_x) * s_w) with sum = acc / 256 (exact: acc = 256 sum has
+      // at most 23 significant bits, so its conversion is exact too)
+      const float2 k8 = make_float2(0.00390625f, 0.00390625f);
+      const float2 sx2 = make_float2(sxm, sxm);
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c, ++blk) {
+        const int c0 = h * 128 + c * 32;
+        uint8_t* buf = stg + (blk & 1) * C::STG;
+        // the TMA store that last read this block has finished reading it
+        if (lane == 0) bulk_wait_group_read<1>();
+        __syncwarp();
+        uint32_t v[32];
+        tmem_ld_32x32(tq + uint32_t(c0), v);
+        tmem_wait_ld();
+        if (c == 3) {
+          // the accumulator is free for the next tile once every warp of both CTAs has read it
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            if (crank == 0)
+              mbar_arrive(acc_empty);
+            else
+              mbar_arrive_cluster(acc_empty, 0);
+          }
+        }
+        const float4* sb4 = reinterpret_cast<const float4*>(sb + c0);
+#pragma unroll
+        for (int pc = 0; pc < 4; ++pc) {  // 16-byte pieces: 8 columns each
+          uint4 o;
+          uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const float4 w = sb4[2 * pc + hh];  // the same address in every lane: a broadcast
+            float2 a0 = make_float2(__int2float_rn(int(v[8 * pc + 4 * hh])), __int2float_rn(int(v[8 * pc + 4 * hh + 1])));
+            float2 a1 = make_float2(__int2float_rn(int(v[8 * pc + 4 * hh + 2])), __int2float_rn(int(v[8 * pc + 4 * hh + 3])));
+            a0 = fmul2(a0, k8);
+            a1 = fmul2(a1, k8);
+            if (EPI == kEpiRow) {
+              a0 = fmul2(a0, sx2);
+              a1 = fmul2(a1, sx2);
+            }
+            a0 = fmul2(a0, make_float2(w.x, w.y));
+            a1 = fmul2(a1, make_float2(w.z, w.w));
+            const __half2 h0 = __floats2half2_rn(a0.x, a0.y), h1 = __floats2half2_rn(a1.x, a1.y);
+            ow[2 * hh] = *reinterpret_cast<const uint32_t*>(&h0);
+            ow[2 * hh + 1] = *reinterpret_cast<const uint32_t*>(&h1);
+          }
+          *reinterpret_cast<uint4*>(buf + lane * 64 + ((pc ^ swz) << 4)) = o;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          // rows past M and columns past N are clipped by the copy
+          tma_store_2d(&tmY, buf, n0 + c0, row0);
+          bulk_commit_group();
+        }
+      }
+    }
+    // the output is written before the CTA leaves
+    if (lane == 0) bulk_wait_group<0>();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  // neither CTA frees the pair's tensor memory before both are done with it
+  if (threadIdx.x == 0) {
+    mbar_arrive_cluster(fin_bar, crank ^ 1u);
+    if (!mbar_wait_cluster(fin_bar, 0)) record_error(p.err, kErrTimeoutDrain);
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, C::TMEM_COLS);
+  }
+}
+
 // ---------------------------------------------------------------- decode
 //
 // Few tokens (M <= 64): the GEMM is a stream of the packed weights, so the
@@ -1084,6 +1464,38 @@ fq_status launch_gemm(const GemmParams& gp, dim3 grid, cudaStream_t stream) {
   return check_launch("gemm_w4a4_kernel");
 }
 
+constexpr int kPersistNB = 8;  // weight-unpack warps of the persistent kernel
+
+template <int EPI>
+fq_status launch_gemm_persistent(const GemmParams& gp, cudaStream_t stream) {
+  using C = PCfg<kPersistNB>;
+  CUtensorMap ta, tb;
+  fq_status st = make_tmap_2d(&ta, gp.A, CU_TENSOR_MAP_DATA_TYPE_UINT8, uint64_t(gp.K) / 2, uint64_t(gp.rowsA),
+                              uint64_t(gp.K) / 2, uint32_t(kPK), uint32_t(kBM), CU_TENSOR_MAP_SWIZZLE_64B);
+  if (st != FQ_OK) return st;
+  st = make_tmap_2d(&tb, gp.B, CU_TENSOR_MAP_DATA_TYPE_UINT8, uint64_t(gp.K) / 2, uint64_t(gp.rowsB), uint64_t(gp.K) / 2,
+                    uint32_t(kPK), uint32_t(C::BR));
+  if (st != FQ_OK) return st;
+  CUtensorMap ty;  // fp16 output in 32 x 32 blocks, 64-byte swizzle (the staging layout)
+  st = make_tmap_2d(&ty, gp.Y, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, uint64_t(gp.N), uint64_t(gp.M), uint64_t(gp.N) * 2, 32u,
+                    32u, CU_TENSOR_MAP_SWIZZLE_64B);
+  if (st != FQ_OK) return st;
+  auto kern = gemm_w4a4_persistent_kernel<EPI, kPersistNB>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess ||
+      cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
+    return fail(FQ_ERR_CUDA, "cannot reserve %d bytes of shared memory for the GEMM", C::SMEM);
+  const int pairs_m = (gp.rowsA + 2 * kBM - 1) / (2 * kBM);
+  const int tiles_n = (gp.rowsB + C::BN - 1) / C::BN;
+  const int clusters = std::max(1, std::min(pairs_m * tiles_n, sm_count() / 2));
+  const cudaError_t e =
+      launch_pdl_cluster(kern, dim3(2 * clusters), dim3(C::THREADS), C::SMEM, stream, 2, gp, ta, tb, ty);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(FQ_ERR_CUDA, "gemm_w4a4_persistent_kernel: %s", cudaGetErrorString(e));
+  }
+  return check_launch("gemm_w4a4_persistent_kernel");
+}
+
 template <int BN, int EPI>
 fq_status launch_decode(const GemmParams& gp, dim3 grid, cudaStream_t stream) {
   using C = DecCfg<BN>;
@@ -1109,9 +1521,9 @@ fq_status launch_decode(const GemmParams& gp, dim3 grid, cudaStream_t stream) {
 fq_status dispatch(const Plan& pl, const GemmParams& gp, dim3 grid, cudaStream_t s) {
   if (!pl.swap) {
     switch (pl.epi) {
-      case kEpiRow: return pl.pair ? launch_gemm<256, kEpiRow, true>(gp, grid, s) : launch_gemm<256, kEpiRow>(gp, grid, s);
+      case kEpiRow: return pl.pair ? launch_gemm_persistent<kEpiRow>(gp, s) : launch_gemm<256, kEpiRow>(gp, grid, s);
       case kEpiStatic:
-        return pl.pair ? launch_gemm<256, kEpiStatic, true>(gp, grid, s) : launch_gemm<256, kEpiStatic>(gp, grid, s);
+        return pl.pair ? launch_gemm_persistent<kEpiStatic>(gp, s) : launch_gemm<256, kEpiStatic>(gp, grid, s);
       case kEpiS32: return launch_gemm<256, kEpiS32>(gp, grid, s);
       case kEpiGroup: return launch_gemm<128, kEpiGroup>(gp, grid, s);
       default: break;
