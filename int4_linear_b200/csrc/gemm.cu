@@ -5,24 +5,26 @@
 // with s8 x s8 -> s32 MMAs accumulating in tensor memory (FlatQuant notes,
 // 核心思想: Y ~ Q(XP) Q(P^-1 W^T) with integer accumulation).
 //
-// Prefill kernel (M > 64): per-token and static scales run 256 x 256 tiles
-// over CTA pairs (a cluster of two; tcgen05 .cta_group::2): each CTA loads and
-// unpacks its own 128 activation rows and half of the tile's 256 weight rows,
-// and one thread of the even CTA issues 256 x 256 MMAs that read both CTAs'
-// operands, so each SM moves half the weight slice through its shared memory
-// (the unpack traffic through shared memory is what bounds the kernel).  The
-// group-scale epilogue and the raw int32 output run one CTA per 128 x BN tile.
-// The packed 128-deep K slices of both operands arrive by TMA into a ring in
+// Prefill with per-token or static scales (M > 64, gemm_w4a4_persistent_kernel):
+// a persistent grid of CTA pairs (clusters of two; tcgen05 .cta_group::2)
+// walks 256 x 256 output tiles.  Each CTA loads and unpacks its own 128
+// activation rows and half of the tile's 256 weight rows, and one thread of
+// the even CTA issues 256 x 256 MMAs that read both CTAs' operands, so each
+// SM moves half the weight slice through its shared memory; dedicated
+// epilogue warps drain the accumulator and TMA-store fp16 blocks while the
+// next tile's slices are unpacked.  The group-scale epilogue and the raw
+// int32 output run gemm_w4a4_kernel, one CTA per 128 x BN tile.  In both, the
+// packed 128-deep K slices of both operands arrive by TMA into a ring in
 // shared memory; A-warps unpack the activation rows into a tensor-memory ring
 // (tcgen05.st), B-warps the weight rows into a 128-byte-swizzled
 // shared-memory ring, and one thread issues the MMAs (A from tensor memory).
-// The warp roles are listed beside gemm_w4a4_kernel.  Stages are handed over
+// The warp roles are listed beside each kernel.  Stages are handed over
 // with mbarriers; every wait is bounded and a wait that gives up records a
 // timeout code in the device error word.
 //
 // The nibble is unpacked into the high half of its byte (16 q, see
-// unpack8_hi), so the tensor core accumulates 256 * sum(qx qw); the epilogue
-// removes the factor with an exact arithmetic shift.
+// unpack8_hi), so the tensor core accumulates 256 * sum(qx qw); the epilogues
+// remove the factor exactly (an arithmetic shift, or a multiply by 2^-8).
 //
 // Epilogues: per-token x per-output-channel scales, static (migrated) scales,
 // per-group scales summed in float32 (FRM-PTQ group quantization, one group
@@ -80,17 +82,14 @@ __host__ __device__ constexpr int b_warps() { return EPI == kEpiGroup ? 2 : kUnp
 template <int EPI>
 __host__ __device__ constexpr int feed_warps() { return 4 + b_warps<EPI>(); }
 
-template <int BN, int EPI, bool PAIR = false>
+template <int BN, int EPI>
 struct Cfg {
-  // PAIR: the tile is 256 x BN over a CTA pair; each CTA holds its 128 A rows
-  // and half of the BN B rows
-  static constexpr int BR = PAIR ? BN / 2 : BN;           // B rows held by this CTA
-  static constexpr int SP = PAIR ? 8 : 4;                 // packed stages (TMA ring)
-  static constexpr int SU = PAIR ? 4 : (BN == 256 ? 3 : 4); // unpacked stages (A in tensor memory, B in shared memory)
+  static constexpr int SP = 4;                 // packed stages (TMA ring)
+  static constexpr int SU = BN == 256 ? 3 : 4; // unpacked stages (A in tensor memory, B in shared memory)
   static constexpr int PA = kBM * kPK;         // packed A slice: 128 rows x 64 bytes
-  static constexpr int PB = BR * kPK;          // packed B slice
+  static constexpr int PB = BN * kPK;          // packed B slice
   static constexpr int P_STAGE = PA + PB;
-  static constexpr int B_UNP = BR * kBK;
+  static constexpr int B_UNP = BN * kBK;
   static constexpr int ACC_COLS = EPI == kEpiGroup ? 3 * BN : BN;
   static constexpr int A_COL0 = ((ACC_COLS + 31) / 32) * 32;   // tensor-memory columns of the A ring
   static constexpr int A_STAGE_COLS = kBK / 4;                 // 4 int8 per 32-bit column
@@ -108,17 +107,14 @@ struct Cfg {
   // row/static: the tile's BN weight scales, staged once by warp 0
   static constexpr int SCALE_BYTES = EPI == kEpiGroup ? SS * SC_STAGE : ((EPI == kEpiRow || EPI == kEpiStatic) ? BN * 4 : 0);
   static constexpr int OFF_BAR = OFF_SCALE + SCALE_BYTES;
-  static constexpr int NBAR = 2 * SP + 2 * SU + 6 + (EPI == kEpiGroup ? 2 * SS : 0) + (PAIR ? 1 : 0);
+  static constexpr int NBAR = 2 * SP + 2 * SU + 6 + (EPI == kEpiGroup ? 2 * SS : 0);
   static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
   static constexpr int SMEM = OFF_TMEM + 16 + 1024;  // + slack to align the base to 1024
-  // the fp16 output tile is staged in the (then idle) unpacked ring (PAIR:
-  // both rings), rows padded by 16 bytes
+  // the fp16 output tile is staged in the (then idle) unpacked ring, rows padded by 16 bytes
   static constexpr int OUT_PITCH = 2 * BN + 16;
-  static constexpr int OFF_OUT = PAIR ? OFF_P : OFF_UNP;
-  static constexpr int OUT_AREA = PAIR ? SP * P_STAGE + SU * UNP_STAGE : SU * UNP_STAGE;
+  static constexpr int OFF_OUT = OFF_UNP;
   static_assert(UNP_STAGE % 1024 == 0 && P_STAGE % 1024 == 0 && PA % 1024 == 0, "1024-byte stage alignment");
-  static_assert(kBM * OUT_PITCH <= OUT_AREA, "output tile fits in the ring");
-  static_assert(!PAIR || (EPI != kEpiGroup && BN == 256), "CTA pairs: per-token / static / int32 epilogues, BN = 256");
+  static_assert(kBM * OUT_PITCH <= SU * UNP_STAGE, "output tile fits in the ring");
   static_assert(TMEM_NEED <= 512, "tensor memory");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
   static_assert(SMEM <= 227 * 1024, "shared memory");
@@ -149,11 +145,11 @@ __device__ __forceinline__ void store_half8(__half* dst, const float* v) {
   *reinterpret_cast<uint4*>(dst) = o;
 }
 
-template <int BN, int EPI, bool PAIR>
+template <int BN, int EPI>
 __global__ void __launch_bounds__(threads_of<EPI>(), 1)
     gemm_w4a4_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tmA,
                      const __grid_constant__ CUtensorMap tmB) {
-  using C = Cfg<BN, EPI, PAIR>;
+  using C = Cfg<BN, EPI>;
   constexpr int SU = C::SU, SP = C::SP;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -168,11 +164,7 @@ __global__ void __launch_bounds__(threads_of<EPI>(), 1)
   uint64_t* sw_ready = done_bar + 1;  // row/static: the tile's weight scales are in shared memory
   uint64_t* sfull = sw_ready + 1;     // group mode: scale stages
   uint64_t* sempty = sfull + C::SS;
-  uint64_t* fin_bar = bars + C::NBAR - 1;  // PAIR: the other CTA has finished with the tensor memory
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM);
-  // PAIR: CTA 0 of the pair issues the MMAs; CTA 1's feed warps signal CTA 0's barriers
-  const uint32_t crank = PAIR ? cluster_rank() : 0u;
-  const bool mma_cta = !PAIR || crank == 0;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tileA = blockIdx.x, tileB = blockIdx.y;
@@ -185,10 +177,9 @@ __global__ void __launch_bounds__(threads_of<EPI>(), 1)
       mbar_init(&pempty[s], feed_warps<EPI>());
     }
     for (int s = 0; s < SU; ++s) {
-      mbar_init(&full_u[s], feed_warps<EPI>() * (PAIR ? 2 : 1));
+      mbar_init(&full_u[s], feed_warps<EPI>());
       mbar_init(&empty_u[s], 1);
     }
-    if (PAIR) mbar_init(fin_bar, 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], epi_warps<EPI>());
@@ -204,26 +195,13 @@ __global__ void __launch_bounds__(threads_of<EPI>(), 1)
     fence_mbar_init();
   }
   if (warp == 1) {
-    if (PAIR) {
-      tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
-      tmem_relinquish_pair();
-    } else {
-      tmem_alloc(tmem_slot, C::TMEM_COLS);
-      tmem_relinquish();
-    }
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
-  if (PAIR) cluster_sync();  // the other CTA's barriers are initialized and its tensor memory allocated
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // arrival on a full_u stage (PAIR: on CTA 0's barrier)
-  auto arrive_full = [&](uint64_t* bar) {
-    if (PAIR && crank != 0)
-      mbar_arrive_cluster(bar, 0);
-    else
-      mbar_arrive(bar);
-  };
   // the next kernel may be scheduled once every CTA of this one is running;
   // this one reads its inputs only after the kernels before it completed
   pdl_launch_dependents();
@@ -234,11 +212,6 @@ __global__ void __launch_bounds__(threads_of<EPI>(), 1)
     if (lane == 0) {
       prefetch_tensormap(&tmA);
       prefetch_tensormap(&tmB);
-      // a pair's second CTA past the last A (or B) rows still feeds its other
-      // operand; it loads in-range rows whose products are never stored
-      const int arow0 = tileA * kBM < p.rowsA ? tileA * kBM : 0;
-      const int brow = tileB * BN + int(crank) * C::BR;
-      const int brow0 = brow < p.rowsB ? brow : 0;
       int issued = 0;
       for (int i = 0; i < nkb; ++i) {
         const int sp = i % SP;
@@ -248,8 +221,8 @@ __global__ void __launch_bounds__(threads_of<EPI>(), 1)
         }
         uint8_t* st = smem + C::OFF_P + sp * C::P_STAGE;
         mbar_arrive_expect_tx(&pfull[sp], C::P_STAGE);
-        tma_load_2d(st, &tmA, &pfull[sp], (kb0 + i) * kPK, arow0);
-        tma_load_2d(st + C::PA, &tmB, &pfull[sp], (kb0 + i) * kPK, brow0);
+        tma_load_2d(st, &tmA, &pfull[sp], (kb0 + i) * kPK, tileA * kBM);
+        tma_load_2d(st + C::PA, &tmB, &pfull[sp], (kb0 + i) * kPK, tileB * BN);
         ++issued;
       }
       // every issued copy has landed before the CTA may leave (normally the
@@ -322,8 +295,8 @@ __global__ void __launch_bounds__(threads_of<EPI>(), 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && mma_cta) {
-      constexpr uint32_t idesc = idesc_i8(PAIR ? 2 * kBM : kBM, BN);
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_i8(kBM, BN);
       for (int i = 0; i < nkb; ++i) {
         const int su = i % SU;
         uint32_t d = tmem;
@@ -337,7 +310,7 @@ __global__ void __launch_bounds__(threads_of<EPI>(), 1)
           tc_fence_after();
           d = tmem + uint32_t(b * BN);
         }
-        if (!(PAIR ? mbar_wait_cluster(&full_u[su], (i / SU) & 1) : mbar_wait(&full_u[su], (i / SU) & 1))) {
+        if (!mbar_wait(&full_u[su], (i / SU) & 1)) {
           record_error(p.err, kErrTimeoutMma);
           break;
         }
@@ -348,28 +321,13 @@ __global__ void __launch_bounds__(threads_of<EPI>(), 1)
         for (int k = 0; k < kBK / 32; ++k) {
           // group mode accumulates onto the primed offset (see the group epilogue)
           const uint32_t accum = EPI == kEpiGroup ? 1u : uint32_t(i > 0 || k > 0);
-          if (PAIR)
-            mma_i8_ts_pair(d, a0 + uint32_t(8 * k), sdesc_k128_sw128(b0 + 32 * k), idesc, accum);
-          else
-            mma_i8_ts(d, a0 + uint32_t(8 * k), sdesc_k128_sw128(b0 + 32 * k), idesc, accum);
+          mma_i8_ts(d, a0 + uint32_t(8 * k), sdesc_k128_sw128(b0 + 32 * k), idesc, accum);
         }
-        if (PAIR)
-          mma_commit_pair(&empty_u[su], 3);
-        else
-          mma_commit(&empty_u[su]);
+        mma_commit(&empty_u[su]);
         if (EPI == kEpiGroup) mma_commit(&acc_full[i & 1]);
       }
-      if (PAIR) {
-        mma_commit_pair(&acc_full[0], 3);
-        mma_commit_pair(done_bar, 3);
-      } else {
-        if (EPI != kEpiGroup) mma_commit(&acc_full[0]);
-        mma_commit(done_bar);
-      }
-      if (!mbar_wait(done_bar, 0)) record_error(p.err, kErrTimeoutDrain);
-    } else if (PAIR && lane == 0) {
-      // CTA 1 stays until CTA 0's MMAs, which read its shared and tensor
-      // memory, have completed
+      if (EPI != kEpiGroup) mma_commit(&acc_full[0]);
+      mma_commit(done_bar);
       if (!mbar_wait(done_bar, 0)) record_error(p.err, kErrTimeoutDrain);
     }
   } else {
@@ -414,13 +372,13 @@ __global__ void __launch_bounds__(threads_of<EPI>(), 1)
         __syncwarp();
         if (lane == 0) {
           mbar_arrive(&pempty[sp]);
-          arrive_full(&full_u[su]);
+          mbar_arrive(&full_u[su]);
         }
       }
       if (!ok && lane == 0) record_error(p.err, kErrTimeoutUnpack);
     } else if (b_warp) {
       const int uw = EPI == kEpiGroup ? warp - 15 : warp - 6;
-      constexpr int kJobs = C::BR * 4;  // 16-byte packed pieces of B per stage
+      constexpr int kJobs = BN * 4;  // 16-byte packed pieces of B per stage
       constexpr int JPT = (kJobs + NB * 32 - 1) / (NB * 32);
       // per-lane pieces, the same in every stage: packed source offset, two swizzled destinations
       uint32_t dst0[JPT], dst1[JPT], srcj[JPT];
@@ -466,7 +424,7 @@ __global__ void __launch_bounds__(threads_of<EPI>(), 1)
         __syncwarp();
         if (lane == 0) {
           mbar_arrive(&pempty[sp]);
-          arrive_full(&full_u[su]);
+          mbar_arrive(&full_u[su]);
         }
       }
       if (!ok && lane == 0) record_error(p.err, kErrTimeoutUnpack);
@@ -641,20 +599,9 @@ __global__ void __launch_bounds__(threads_of<EPI>(), 1)
 
   tc_fence_before();
   __syncthreads();
-  if (PAIR) {
-    // neither CTA frees the pair's tensor memory before both are done with it
-    if (threadIdx.x == 0) {
-      mbar_arrive_cluster(fin_bar, crank ^ 1u);
-      if (!mbar_wait_cluster(fin_bar, 0)) record_error(p.err, kErrTimeoutDrain);
-    }
-    __syncthreads();
-  }
   if (warp == 1) {
     tc_fence_after();
-    if (PAIR)
-      tmem_dealloc_pair(tmem, C::TMEM_COLS);
-    else
-      tmem_dealloc(tmem, C::TMEM_COLS);
+    tmem_dealloc(tmem, C::TMEM_COLS);
   }
 }
 
@@ -1439,24 +1386,22 @@ Plan make_plan(int M, int N, int K, int epi_final, int sms) {
   return pl;
 }
 
-template <int BN, int EPI, bool PAIR = false>
+template <int BN, int EPI>
 fq_status launch_gemm(const GemmParams& gp, dim3 grid, cudaStream_t stream) {
-  using C = Cfg<BN, EPI, PAIR>;
+  using C = Cfg<BN, EPI>;
   CUtensorMap ta, tb;
-  // packed A: 128 rows x 64 bytes per slice, 64-byte swizzle; packed B: BR rows x 64 bytes
+  // packed A: 128 rows x 64 bytes per slice, 64-byte swizzle; packed B: BN rows x 64 bytes
   fq_status st = make_tmap_2d(&ta, gp.A, CU_TENSOR_MAP_DATA_TYPE_UINT8, uint64_t(gp.K) / 2, uint64_t(gp.rowsA),
                               uint64_t(gp.K) / 2, uint32_t(kPK), uint32_t(kBM), CU_TENSOR_MAP_SWIZZLE_64B);
   if (st != FQ_OK) return st;
   st = make_tmap_2d(&tb, gp.B, CU_TENSOR_MAP_DATA_TYPE_UINT8, uint64_t(gp.K) / 2, uint64_t(gp.rowsB), uint64_t(gp.K) / 2,
-                    uint32_t(kPK), uint32_t(C::BR));
+                    uint32_t(kPK), uint32_t(BN));
   if (st != FQ_OK) return st;
-  auto kern = gemm_w4a4_kernel<BN, EPI, PAIR>;
+  auto kern = gemm_w4a4_kernel<BN, EPI>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess ||
       cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
     return fail(FQ_ERR_CUDA, "cannot reserve %d bytes of shared memory for the GEMM", C::SMEM);
-  if (PAIR) grid.x = (grid.x + 1) & ~1u;  // whole pairs
-  const cudaError_t e = PAIR ? launch_pdl_cluster(kern, grid, dim3(threads_of<EPI>()), C::SMEM, stream, 2, gp, ta, tb)
-                             : launch_pdl(kern, grid, dim3(threads_of<EPI>()), C::SMEM, stream, gp, ta, tb);
+  const cudaError_t e = launch_pdl(kern, grid, dim3(threads_of<EPI>()), C::SMEM, stream, gp, ta, tb);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return fail(FQ_ERR_CUDA, "gemm_w4a4_kernel: %s", cudaGetErrorString(e));
