@@ -614,8 +614,10 @@ __global__ void __launch_bounds__(threads_of<EPI>(), 1)
 //   warp 0        one thread issues the TMA loads of the packed slices
 //   warp 1        tensor-memory allocation; in CTA 0 the thread that issues
 //                 the 256 x 256 pair MMAs (.cta_group::2)
-//   warps 2-5     unpack this CTA's 128 A rows into the tensor-memory ring
-//   warps 6..     unpack this CTA's half of the weight rows (NB warps)
+//   warps 2-9     unpack this CTA's 128 A rows into the tensor-memory ring
+//                 (two warps per lane quadrant, alternate K slices)
+//   warps 10..    unpack this CTA's half of the weight rows, NB warps taking
+//                 whole K slices in turn
 //   last 8 warps  epilogue: drain the accumulator (two warps per lane
 //                 quadrant, 128 columns each, 32 at a time), scale to fp16
 //                 into a per-warp shared-memory block and TMA-store it; the
@@ -646,12 +648,16 @@ struct PCfg {
   static constexpr int NBAR = 2 * SP + 2 * SU + 4;          // + acc_full, acc_empty, done, fin
   static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
   static constexpr int SMEM = OFF_TMEM + 16 + 1024;
-  static constexpr int EPI_WARP0 = 6 + NB;
+  static constexpr int B_WARP0 = 10;           // A: warps 2-9, two per lane quadrant
+  static constexpr int EPI_WARP0 = B_WARP0 + NB;
   static constexpr int THREADS = 32 * (EPI_WARP0 + 8);
-  static constexpr int FEED = 4 + NB;          // feed warps per CTA
+  static constexpr int FEED = 4 + 1;           // arrivals per slice and CTA: 4 A-warps, 1 B-warp
   static_assert(A_COL0 + SU * A_STAGE_COLS <= TMEM_COLS, "tensor memory");
   static_assert(SMEM <= 227 * 1024, "shared memory");
   static_assert(P_STAGE % 1024 == 0 && UNP_STAGE % 1024 == 0 && PA % 1024 == 0, "1024-byte stage alignment");
+  // a warp that takes every NB-th (A: every 2nd) slice must never wait on a
+  // stage more than one phase ahead of its barrier (parity waits alias)
+  static_assert(NB < SU && NB < SP && 2 < SU, "slices per feed warp");
 };
 
 template <int EPI, int NB>
@@ -785,14 +791,16 @@ __global__ void __launch_bounds__(PCfg<NB>::THREADS, 1)
       // memory, have completed
       if (!mbar_wait(done_bar, 0)) record_error(p.err, kErrTimeoutDrain);
     }
-  } else if (warp < 6) {
+  } else if (warp < C::B_WARP0) {
     // ------------------------------------------------------------ A rows -> tensor-memory ring
-    const int q = warp & 3;
+    // two warps per lane quadrant take alternate slices, so each has two
+    // slice periods for its load - unpack - store - arrive chain
+    const int q = warp & 3, par = (warp - 2) >> 2;
     const int row = q * 32 + lane;
     const int sw = (row >> 1) & 3;  // 64-byte swizzle: chunk c of this row sits at chunk c ^ sw
     const uint32_t ta = tmem + (uint32_t(q * 32) << 16) + uint32_t(C::A_COL0);
     bool ok = true;
-    for (uint32_t g = 0; g < total; ++g) {
+    for (uint32_t g = uint32_t(par); g < total; g += 2) {
       const int sp = int(g % SP), su = int(g % SU);
       if (!warp_wait(&pfull[sp], (g / SP) & 1)) {
         ok = false;
@@ -830,48 +838,43 @@ __global__ void __launch_bounds__(PCfg<NB>::THREADS, 1)
     if (!ok && lane == 0) record_error(p.err, kErrTimeoutUnpack);
   } else if (warp < C::EPI_WARP0) {
     // ------------------------------------------------------------ weight rows -> shared-memory ring
-    const int uw = warp - 6;
-    constexpr int kJobs = C::BR * 4;  // 16-byte packed pieces per stage
-    constexpr int JPT = (kJobs + NB * 32 - 1) / (NB * 32);
-    uint32_t dst0[JPT], dst1[JPT], srcj[JPT];
-    bool live[JPT];
-#pragma unroll
-    for (int it = 0; it < JPT; ++it) {
-      const int j = (it * NB + uw) * 32 + lane;
-      live[it] = j < kJobs;
-      const int row = live[it] ? (j >> 2) : 0, c = j & 3, r7 = row & 7;
-      const uint32_t rb = uint32_t((row >> 3) * 1024 + r7 * 128);
-      dst0[it] = rb + uint32_t(((2 * c) ^ r7) << 4);
-      dst1[it] = rb + uint32_t(((2 * c + 1) ^ r7) << 4);
-      srcj[it] = uint32_t(live[it] ? j * 16 : 0);
-    }
+    // B-warp b unpacks whole half-slices g = b, b + NB, ...: lane l takes the
+    // 16-byte pieces it * 32 + l (row it * 8 + l / 4, piece l % 4 of the row)
+    const int bw = warp - C::B_WARP0;
+    const int r7 = lane >> 2, c = lane & 3;
+    const uint32_t dst0 = uint32_t(r7 * 128 + (((2 * c) ^ r7) << 4));
+    const uint32_t dst1 = uint32_t(r7 * 128 + (((2 * c + 1) ^ r7) << 4));
     bool ok = true;
-    for (uint32_t g = 0; g < total; ++g) {
+    for (uint32_t g = uint32_t(bw); g < total; g += NB) {
       const int sp = int(g % SP), su = int(g % SU);
       if (!warp_wait(&pfull[sp], (g / SP) & 1)) {
         ok = false;
         break;
       }
-      const uint8_t* pb = smem + C::OFF_P + sp * C::P_STAGE + C::PA;
-      uint4 w[JPT];
-#pragma unroll
-      for (int it = 0; it < JPT; ++it) w[it] = *reinterpret_cast<const uint4*>(pb + srcj[it]);
-      if (!warp_wait(&empty_u[su], ((g / SU) & 1) ^ 1)) {
-        ok = false;
-        break;
-      }
+      const uint8_t* pb = smem + C::OFF_P + sp * C::P_STAGE + C::PA + lane * 16;
       uint8_t* uk = smem + C::OFF_UNP + su * C::UNP_STAGE;
+      constexpr int kIt = C::BR / 8;  // 8 rows (32 pieces) per step
 #pragma unroll
-      for (int it = 0; it < JPT; ++it) {
-        if (!live[it]) continue;
-        uint4 o0, o1;
-        unpack8_hi(w[it].x, o0.x, o0.y);
-        unpack8_hi(w[it].y, o0.z, o0.w);
-        unpack8_hi(w[it].z, o1.x, o1.y);
-        unpack8_hi(w[it].w, o1.z, o1.w);
-        *reinterpret_cast<uint4*>(uk + dst0[it]) = o0;
-        *reinterpret_cast<uint4*>(uk + dst1[it]) = o1;
+      for (int it0 = 0; it0 < kIt; it0 += 4) {
+        uint4 w[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) w[u] = *reinterpret_cast<const uint4*>(pb + (it0 + u) * 512);
+        if (it0 == 0 && !warp_wait(&empty_u[su], ((g / SU) & 1) ^ 1)) {
+          ok = false;
+          break;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          uint4 o0, o1;
+          unpack8_hi(w[u].x, o0.x, o0.y);
+          unpack8_hi(w[u].y, o0.z, o0.w);
+          unpack8_hi(w[u].z, o1.x, o1.y);
+          unpack8_hi(w[u].w, o1.z, o1.w);
+          *reinterpret_cast<uint4*>(uk + (it0 + u) * 1024 + dst0) = o0;
+          *reinterpret_cast<uint4*>(uk + (it0 + u) * 1024 + dst1) = o1;
+        }
       }
+      if (!ok) break;
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
@@ -1409,7 +1412,7 @@ fq_status launch_gemm(const GemmParams& gp, dim3 grid, cudaStream_t stream) {
   return check_launch("gemm_w4a4_kernel");
 }
 
-constexpr int kPersistNB = 8;  // weight-unpack warps of the persistent kernel
+constexpr int kPersistNB = 3;  // weight-unpack warps of the persistent kernel
 
 template <int EPI>
 fq_status launch_gemm_persistent(const GemmParams& gp, cudaStream_t stream) {
