@@ -114,7 +114,12 @@ fq_status fq_quant_weight(const uint16_t* W, int N, int K, const fq_qparams* qp,
  * qp     FQ_DYNAMIC_ROW: s_x float32 [M];  FQ_DYNAMIC_GROUP: s_x fp16 [K/128][M];
  *        FQ_STATIC_CHANNEL: static_scale float32 [K] is used and s_x is not written
  *        (may be NULL); alpha = alpha_a.
- * t      NULL or the transform (P1, P2, c).
+ * t      NULL or the transform (P1, P2, c).  P1 and P2 are parameters: the
+ *        kernel may read them while the kernels enqueued just before it on
+ *        the stream are still finishing (programmatic dependent launch), so
+ *        they must not be written by such work (no call of this library
+ *        writes them).  X, c and the scales are read only after the earlier
+ *        work on the stream has completed.
  * Xq     uint8 [M, K/2] packed codes (out). */
 fq_status fq_quant_act(const uint16_t* X, int M, int K, const fq_qparams* qp,
                        const fq_transform* t, const float* static_scale,

@@ -197,10 +197,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
   fence_proxy_async_smem();
   __syncthreads();
-  // the next kernel may be scheduled once every CTA of this one is running;
-  // global memory is touched only after the kernels before this one completed
+  // The next kernel may be scheduled once every CTA of this one is running.
+  // The transform factors (parameters: no kernel of this library writes them)
+  // are staged below while the kernels ahead on the stream may still run;
+  // the activations, scales and outputs are touched only after pdl_wait().
   pdl_launch_dependents();
-  pdl_wait();
 
   const uint32_t lane_off = uint32_t(q4 * 32) << 16;
   const int bar_id = 1 + pipe;
@@ -226,52 +227,84 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int gstride = gridDim.x * C::P;
   int grp = blockIdx.x * C::P + pipe;
   bool x_pending = false;  // (leader) a TMA into the X tile has not been waited for
-  if (!HAS_C && leader && grp < ngroups) {  // the first rows land while the factors are staged
-    prefetch_tensormap(&tmX);
-    issue_x(grp);
-    x_pending = true;
-  }
+  if (!HAS_C && leader) prefetch_tensormap(&tmX);
 
-  // ---- factors -> fp16 hi/lo operands, once per CTA, 8 consecutive K per 16-byte store
-  for (int e = tid; e < N2 * (N2 / 8); e += kTcThreads) {
+  // ---- factors -> fp16 hi/lo operands, once per CTA, 8 consecutive K per 16-byte store.
+  // Each thread first issues the loads of all its items, so their latencies
+  // overlap, then converts and stores.
+  {
     // stage-A A operand: row l, K = j, value P2[j][l]; consecutive threads
     // take consecutive l, so every load instruction reads whole rows of P2
-    const int l = e % N2, j0 = (e / N2) * 8;
-    uint4 hi, lo;
-    __half* hh = reinterpret_cast<__half*>(&hi);
-    __half* ll = reinterpret_cast<__half*>(&lo);
+    constexpr int kItems = N2 * (N2 / 8);
+    constexpr int kPer = (kItems + kTcThreads - 1) / kTcThreads;
+    float v[kPer][8];
 #pragma unroll
-    for (int jj = 0; jj < 8; ++jj) {
-      const float v = __ldg(p.P2 + (j0 + jj) * N2 + l);
-      hh[jj] = __float2half_rn(v);
-      ll[jj] = __float2half_rn(v - __half2float(hh[jj]));
+    for (int it = 0; it < kPer; ++it) {
+      const int e = tid + it * kTcThreads;
+      const int l = e % N2, j0 = (e / N2) * 8;
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj) v[it][jj] = e < kItems ? __ldg(p.P2 + (j0 + jj) * N2 + l) : 0.f;
     }
-    const int row = N2 == 64 ? 64 + l : l;
-    const uint32_t off = (N2 == 64 ? 0u : uint32_t(j0 >> 6) * C::REG) + sw128_offset(row, (j0 & 63) * 2);
-    *reinterpret_cast<uint4*>(sm + C::OFF_SA + off) = hi;
-    *reinterpret_cast<uint4*>(sm + C::OFF_SA + C::SA_HALF + off) = lo;
+#pragma unroll
+    for (int it = 0; it < kPer; ++it) {
+      const int e = tid + it * kTcThreads;
+      if (e >= kItems) break;
+      const int l = e % N2, j0 = (e / N2) * 8;
+      uint4 hi, lo;
+      __half* hh = reinterpret_cast<__half*>(&hi);
+      __half* ll = reinterpret_cast<__half*>(&lo);
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj) {
+        hh[jj] = __float2half_rn(v[it][jj]);
+        ll[jj] = __float2half_rn(v[it][jj] - __half2float(hh[jj]));
+      }
+      const int row = N2 == 64 ? 64 + l : l;
+      const uint32_t off = (N2 == 64 ? 0u : uint32_t(j0 >> 6) * C::REG) + sw128_offset(row, (j0 & 63) * 2);
+      *reinterpret_cast<uint4*>(sm + C::OFF_SA + off) = hi;
+      *reinterpret_cast<uint4*>(sm + C::OFF_SA + C::SA_HALF + off) = lo;
+    }
   }
-  const int n1c = (n1 + 7) / 8;
-  for (int e = tid; e < n1 * n1c; e += kTcThreads) {
-    const int k = e % n1, i0 = (e / n1) * 8;  // stage-B B operand: row k, K = i, value P1[i][k]
-    uint4 hi, lo;
-    __half* hh = reinterpret_cast<__half*>(&hi);
-    __half* ll = reinterpret_cast<__half*>(&lo);
+  {
+    // stage-B B operand: row k, K = i, value P1[i][k]
+    const int n1c = (n1 + 7) / 8;
+    constexpr int kPer = (NP * (NP / 8) + kTcThreads - 1) / kTcThreads;
+    const int items = n1 * n1c;
+    float v[kPer][8];
 #pragma unroll
-    for (int ii = 0; ii < 8; ++ii) {
-      const float v = i0 + ii < n1 ? __ldg(p.P1 + (i0 + ii) * n1 + k) : 0.f;
-      hh[ii] = __float2half_rn(v);
-      ll[ii] = __float2half_rn(v - __half2float(hh[ii]));
+    for (int it = 0; it < kPer; ++it) {
+      const int e = tid + it * kTcThreads;
+      const int k = e % n1, i0 = (e / n1) * 8;
+#pragma unroll
+      for (int ii = 0; ii < 8; ++ii) v[it][ii] = (e < items && i0 + ii < n1) ? __ldg(p.P1 + (i0 + ii) * n1 + k) : 0.f;
     }
-    const uint32_t off = uint32_t(i0 >> 6) * (NP * 128) + sw128_offset(k, (i0 & 63) * 2);
-    *reinterpret_cast<uint4*>(sm + C::OFF_SL + off) = hi;
-    *reinterpret_cast<uint4*>(sm + C::OFF_SL + C::SL_HALF + off) = lo;
+#pragma unroll
+    for (int it = 0; it < kPer; ++it) {
+      const int e = tid + it * kTcThreads;
+      if (e >= items) break;
+      const int k = e % n1, i0 = (e / n1) * 8;
+      uint4 hi, lo;
+      __half* hh = reinterpret_cast<__half*>(&hi);
+      __half* ll = reinterpret_cast<__half*>(&lo);
+#pragma unroll
+      for (int ii = 0; ii < 8; ++ii) {
+        hh[ii] = __float2half_rn(v[it][ii]);
+        ll[ii] = __float2half_rn(v[it][ii] - __half2float(hh[ii]));
+      }
+      const uint32_t off = uint32_t(i0 >> 6) * (NP * 128) + sw128_offset(k, (i0 & 63) * 2);
+      *reinterpret_cast<uint4*>(sm + C::OFF_SL + off) = hi;
+      *reinterpret_cast<uint4*>(sm + C::OFF_SL + C::SL_HALF + off) = lo;
+    }
   }
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tslot;
+  pdl_wait();  // the kernels ahead on the stream have completed: X may be read
+  if (!HAS_C && leader && grp < ngroups) {
+    issue_x(grp);
+    x_pending = true;
+  }
   const uint32_t tD = tmem + uint32_t(pipe * C::TMEM_PIPE);  // D: stage A, then stage B
   const uint32_t tU = tD + uint32_t(NP);                      // U^T: hi [0, NP/2), lo [NP/2, NP)
 
