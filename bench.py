@@ -164,7 +164,9 @@ def run_ours(args, ws, rank, local):
         sx = torch.empty(m, dtype=torch.float32, device=dev)
         y = torch.empty(m, n, dtype=torch.float16, device=dev)
         lws = torch.empty(max(fq.fq_linear_workspace_size(m, n, k, fq.ROW), 256), dtype=torch.uint8, device=dev)
-        state.append(dict(d=d, x=x, wq=wq, sw=sw, t=t, xq=xq, sx=sx, y=y, lws=lws, m=m, k=k, n=n))
+        # GEMM scratch (stream-K partial sums), allocated once like every other buffer
+        gws = torch.empty(max(fq.fq_gemm_workspace_size(m, n, k, fq.ROW), 256), dtype=torch.uint8, device=dev)
+        state.append(dict(d=d, x=x, wq=wq, sw=sw, t=t, xq=xq, sx=sx, y=y, lws=lws, gws=gws, m=m, k=k, n=n))
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream(dev)
     L = len(state)
@@ -176,7 +178,7 @@ def run_ours(args, ws, rank, local):
             fq.fq_quant_act(s["x"], qp, s["t"], None, s["xq"], s["sx"], stream=stream)
             if evs is not None:
                 evs[i][1].record(stream)
-            fq.fq_w4a4_gemm(s["xq"], s["sx"], s["wq"], s["sw"], fq.ROW, Y=s["y"], stream=stream)
+            fq.fq_w4a4_gemm(s["xq"], s["sx"], s["wq"], s["sw"], fq.ROW, Y=s["y"], workspace=s["gws"], stream=stream)
             if evs is not None:
                 evs[i][2].record(stream)
 

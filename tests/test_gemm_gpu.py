@@ -105,3 +105,31 @@ def test_gemm_workspace_is_reused_correctly():
     C.check_fp16_exact(y1, ref)
     C.check_fp16_exact(y2, ref)
     fq.fq_check_device_error()
+
+
+# Prefill shapes for the persistent CTA-pair kernel: tile counts below, at and
+# above the 74 pairs, ragged A pairs and weight tiles, repeated launches on a
+# garbage workspace, and the entry point without a workspace.
+PERSISTENT_SHAPES = [
+    (1024, 4096, 2048),   # 64 tiles: fewer tiles than pairs
+    (2048, 10240, 1024),  # 320 tiles: four rounds, the last one partial
+    (384, 1024, 8192),    # 8 tiles, the second A pair half out of range
+    (640, 776, 8192),     # ragged M and N tiles
+]
+
+
+@pytest.mark.parametrize("m,n,k", PERSISTENT_SHAPES)
+def test_gemm_persistent_exact(m, n, k):
+    a, b = _operands(13 * m + n + k, m, n, k)
+    g = synth.generator(m + 6)
+    sx, sw = synth.random_scales(g, m), synth.random_scales(g, n)
+    acc = O.gemm_int(C.unpack(a), C.unpack(b))
+    A, B = C.dev(a), C.dev(b)
+    ws = torch.full((max(fq.fq_gemm_workspace_size(m, n, k, fq.ROW), 256),), 0xA5, dtype=torch.uint8, device="cuda")
+    ref = O.dequant_row(acc, sx, sw)
+    for _ in range(3):
+        C.check_fp16_exact(C.host(fq.fq_w4a4_gemm(A, C.dev(sx), B, C.dev(sw), fq.ROW, workspace=ws)), ref)
+    refs = O.dequant_static(acc, sw)
+    C.check_fp16_exact(C.host(fq.fq_w4a4_gemm(A, None, B, C.dev(sw), fq.STATIC, workspace=ws)), refs)
+    C.check_fp16_exact(C.host(fq.fq_w4a4_gemm_noalloc(A, C.dev(sx), B, C.dev(sw), fq.ROW)), ref)
+    fq.fq_check_device_error()
