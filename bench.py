@@ -41,7 +41,7 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # (dram__bytes_read.sum + dram__bytes_write.sum) of this bench command on the
 # current GEMM kernel; the fp16 outputs that still sit in L2 when a launch
 # ends are not in it.
-GEMM_DRAM_BYTES = {"qkv": 16849152, "o": 12634112, "gate_up": 63113216 + 67183616, "down": 44094208 + 187392}
+GEMM_DRAM_BYTES = {"qkv": 16842240, "o": 12640000, "gate_up": 63101696 + 69518336, "down": 44100096 + 29440}
 INT8_OVER_BF16 = 4.5 / 2.25  # nominal dense ratio (B200: 4.5 POPS int8 vs 2.25 PFLOPS bf16)
 
 
@@ -332,7 +332,7 @@ def run_ours(args, ws, rank, local):
                          "bytes_per_step": int(sum(q_bytes))},
         "breakdown": breakdown,
         "roofline": {
-            "kernel": "gemm_w4a4_kernel",
+            "kernel": "gemm_w4a4_persistent_kernel",
             "bound": "tensor",
             "achieved": round(g_achieved, 1),
             "peak": round(int8_peak, 1),
