@@ -28,10 +28,9 @@
 //
 // Epilogues: per-token x per-output-channel scales, static (migrated) scales,
 // per-group scales summed in float32 (FRM-PTQ group quantization, one group
-// per K slice, double-buffered accumulators), raw int32, or atomic int32
-// partial sums for split-K.  For few tokens (decode, gemm_decode_kernel) the
-// operands swap roles: the weights fill the 128-row MMA side and the tokens
-// the N side.
+// per K slice, double-buffered accumulators) or raw int32.  For few tokens
+// (decode, gemm_decode_kernel) the operands swap roles: the weights fill the
+// 128-row MMA side and the tokens the N side.
 #include <cuda_fp16.h>
 
 #include <algorithm>
@@ -45,7 +44,7 @@ namespace fq {
 
 namespace {
 
-enum Epi { kEpiRow = 0, kEpiStatic = 1, kEpiGroup = 2, kEpiS32 = 3, kEpiAtomic = 4 };
+enum Epi { kEpiRow = 0, kEpiStatic = 1, kEpiGroup = 2, kEpiS32 = 3 };
 
 constexpr int kBM = 128;        // rows of the A operand per tile (MMA M)
 constexpr int kBK = 128;        // int8 K per stage; equals the quantization group
@@ -127,13 +126,12 @@ struct GemmParams {
   int M, N, K;        // Y is [M][N]
   int rowsA, rowsB;   // rows of the A (128-row tiles) and B (BN-row tiles) operands
   int num_kb;         // K / 128
-  int kb_per_split;   // K slices per CTA along gridDim.z
   const float* sx;    // [M]           per-token scales
   const float* sw;    // [N]           per-channel (or migrated static) scales
   const __half* gsx;  // [K/128][M]    group scales of the activations
   const __half* gsw;  // [K/128][N]    group scales of the weights
   __half* Y;          // [M][N]
-  int32_t* acc;       // [M][N]        int32 output / split-K partial sums
+  int32_t* acc;       // [M][N]        int32 output / decode stream-K partial sums
   unsigned* err;
 };
 
@@ -168,8 +166,8 @@ __global__ void __launch_bounds__(threads_of<EPI>(), 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tileA = blockIdx.x, tileB = blockIdx.y;
-  const int kb0 = blockIdx.z * p.kb_per_split;
-  const int nkb = max(0, min(p.num_kb, kb0 + p.kb_per_split) - kb0);
+  const int kb0 = 0;  // every CTA covers the whole K
+  const int nkb = p.num_kb;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < SP; ++s) {
@@ -476,11 +474,7 @@ __global__ void __launch_bounds__(threads_of<EPI>(), 1)
                 int32_t* dst = p.acc + size_t(m) * p.N + n0;
                 for (int j = 0; j < CW; ++j) {
                   if (n0 + j >= p.N) break;
-                  const int32_t a = int32_t(v[j]) >> 8;
-                  if (EPI == kEpiS32)
-                    dst[j] = a;
-                  else
-                    atomicAdd(dst + j, a);
+                  dst[j] = int32_t(v[j]) >> 8;
                 }
               }
             }
@@ -1342,8 +1336,6 @@ struct Plan {
   bool pair;          // prefill: 256 x BN tiles over CTA pairs
   int bn;
   int epi;
-  int splits;         // prefill: K splits (always 1)
-  int kb_per_split;
   int ctas;           // decode: persistent CTAs sharing the slice sequence
   bool partial;       // decode: some tile is split between CTAs (workspace + fixup)
 };
@@ -1353,8 +1345,6 @@ int pick_bn_swap(int M) { return M <= 16 ? 16 : (M <= 32 ? 32 : 64); }
 Plan make_plan(int M, int N, int K, int epi_final, int sms) {
   Plan pl{};
   const int nkb = K / kBK;
-  pl.splits = 1;
-  pl.kb_per_split = nkb;
   if (epi_final == kEpiGroup) {
     pl.swap = false;
     pl.bn = 128;
@@ -1525,7 +1515,6 @@ fq_status gemm_impl(const uint8_t* Xq, const void* s_x, const uint8_t* Wq, const
   gp.N = N;
   gp.K = K;
   gp.num_kb = K / kBK;
-  gp.kb_per_split = pl.kb_per_split;
   gp.err = err;
   gp.Y = reinterpret_cast<__half*>(Y);
   if (epi_final == kEpiRow) gp.sx = static_cast<const float*>(s_x);
