@@ -110,6 +110,66 @@ def unpack_int4(p: np.ndarray) -> np.ndarray:
     return out
 
 
+# ------------------------------------------------------------------ general quantizer
+#
+# Q(W) = clamp(round(W/s) + z, 0, 2^b - 1) for any bit width b and zero point
+# z (FRM-PTQ page, 初步介绍), with the asymmetric (min-max) choice of s and z.
+# Not on the hot path yet: the CUDA library answers FQ_ERR_UNSUPPORTED for
+# z != 2^(b-1) or b != 4; these functions are the oracle that path will be
+# held to.
+
+def minmax_params(v32: np.ndarray, bits: int, alpha: float = 1.0):
+    """Per-row asymmetric scale and zero point.
+
+    The row's range is widened to contain 0 (so that 0 is exactly a code):
+    lo = min(0, min v), hi = max(0, max v); s = ((hi - lo) * alpha) / (2^b - 1)
+    in float32; z = clamp(round(-lo / s), 0, 2^b - 1) with an IEEE float32
+    division and round half to even; a row of zeros has s = 0 and z = 0.
+    Returns (s float32 [rows], z int32 [rows]).
+    Parity pinned by: tests/golden/rtn_asym_worked.txt, the bound
+    |v - s (u - z)| <= s/2 on unclipped values, 0 mapping to z.
+    """
+    v32 = np.asarray(v32, dtype=np.float32)
+    qmax = np.float32((1 << bits) - 1)
+    lo = np.minimum(v32.min(axis=-1), np.float32(0))
+    hi = np.maximum(v32.max(axis=-1), np.float32(0))
+    s = ((hi - lo) * np.float32(alpha)) / qmax        # float32 throughout
+    with np.errstate(divide="ignore", invalid="ignore"):
+        zf = np.rint(-lo / s)
+    z = np.where(s == 0, 0, np.clip(zf, 0, qmax)).astype(np.int32)
+    return s.astype(np.float32), z
+
+
+def quantize_u(v32: np.ndarray, s32: np.ndarray, z: np.ndarray, bits: int) -> np.ndarray:
+    """Unsigned codes u = clamp(round(v/s) + z, 0, 2^b - 1), one (s, z) per row.
+
+    FRM-PTQ page, 初步介绍; IEEE float32 division, round half to even; s = 0
+    gives u = z (the code of 0).
+    Parity pinned by: tests/golden/rtn_asym_worked.txt; with b = 4, z = 8 and
+    the symmetric scale it equals quantize() + 8.
+    """
+    v32 = np.asarray(v32, dtype=np.float32)
+    s32 = np.asarray(s32, dtype=np.float32).reshape(-1, 1)
+    z = np.asarray(z, dtype=np.int64).reshape(-1, 1)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        ratio = v32 / s32
+    u = np.clip(np.rint(ratio) + z, 0, (1 << bits) - 1)
+    u = np.where(s32 == 0, z, u)
+    return u.astype(np.uint8)
+
+
+def gemm_asym(ux: np.ndarray, zx: np.ndarray, uw: np.ndarray, zw: np.ndarray) -> np.ndarray:
+    """acc[m, n] = sum_k (ux[m, k] - zx[m]) (uw[n, k] - zw[n]), exact, int64:
+    the integer product of the dequantized-up-to-scale codes, so that
+    y = fl(fl(acc * s_x[m]) * s_w[n]) as in dequant_row.
+    Parity pinned by: brute force on tiny shapes, and its expansion
+    sum ux uw - zw sum ux - zx sum uw + K zx zw (the form a kernel computes).
+    """
+    cx = np.asarray(ux, np.float64) - np.asarray(zx, np.float64).reshape(-1, 1)
+    cw = np.asarray(uw, np.float64) - np.asarray(zw, np.float64).reshape(-1, 1)
+    return (cx @ cw.T).astype(np.int64)
+
+
 # ------------------------------------------------------------------ transform
 
 def kron_apply(v64: np.ndarray, left: np.ndarray, right: np.ndarray) -> np.ndarray:

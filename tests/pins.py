@@ -295,7 +295,81 @@ def check_qsm_fold(o):
     assert np.all(np.abs(y - ref) <= bound)
 
 
+def check_asym_golden(o):
+    """Hand-worked rows of the general quantizer in tests/golden/rtn_asym_worked.txt
+    (Q(W) with a zero point and any bit width; FRM-PTQ page, 初步介绍)."""
+    for ln in _lines("rtn_asym_worked.txt"):
+        head, xs, ss, zs, us = [p.strip() for p in ln.split("|")]
+        bits, alpha = head.split()
+        x = np.array([[float(v) for v in xs.split()]], dtype=np.float16).astype(np.float32)
+        s, z = o.minmax_params(x, int(bits), float(alpha))
+        assert np.float32(s[0]) == np.float32(float(ss)), (ln, s[0])
+        assert int(z[0]) == int(zs), (ln, z[0])
+        u = o.quantize_u(x, s, z, int(bits))
+        assert np.array_equal(u[0], np.array([int(v) for v in us.split()])), (ln, u[0])
+
+
+def check_asym_bounds(o):
+    """Codes lie in [0, 2^b - 1]; 0 quantizes to z exactly; every unclipped value
+    satisfies |v - s (u - z)| <= s/2; with alpha = 1 nothing clips, and each
+    row's extremes land within one code of the ends of the range."""
+    g = np.random.Generator(np.random.PCG64(17))
+    x = (g.standard_normal((48, 200)) * g.uniform(0.01, 20, (48, 1)) + g.uniform(-3, 3, (48, 1)))
+    x = x.astype(np.float16).astype(np.float32)
+    x[5] = np.abs(x[5])       # all non-negative: lo = 0, z = 0
+    x[6] = -np.abs(x[6])      # all non-positive: hi = 0
+    for bits in (2, 3, 4, 8):
+        qmax = (1 << bits) - 1
+        for alpha in (1.0, 0.9):
+            s, z = o.minmax_params(x, bits, alpha)
+            u = o.quantize_u(x, s, z, bits).astype(np.int64)
+            assert u.min() >= 0 and u.max() <= qmax
+            assert np.all((z >= 0) & (z <= qmax))
+            zero_code = o.quantize_u(np.zeros_like(x[:, :1]), s, z, bits)[:, 0]
+            assert np.array_equal(zero_code.astype(np.int64), z.astype(np.int64))
+            deq = (u - z[:, None]).astype(np.float64) * s[:, None].astype(np.float64)
+            r32 = (x / s[:, None]).astype(np.float32)   # the float32 quotient the codes come from
+            unclipped = (np.rint(r32) + z[:, None] >= 0) & (np.rint(r32) + z[:, None] <= qmax)
+            # s/2, plus the float32 rounding of the quotient (at most 2^b ulps of 1)
+            bound = s[:, None].astype(np.float64) * (0.5 + (1 << bits) * 2.0 ** -23) * np.ones_like(x, dtype=np.float64)
+            assert np.all(np.abs(deq - x)[unclipped] <= bound[unclipped])
+            if alpha == 1.0:
+                assert unclipped.all()
+                assert np.all(u.max(axis=1) >= qmax - 1) or np.all(u.min(axis=1) <= 1)
+    assert x[5].min() >= 0 and o.minmax_params(x[5:6], 4)[1][0] == 0
+
+
+def check_asym_symmetric_case(o):
+    """b = 4 with z = 8 and the symmetric absmax scale is the symmetric quantizer."""
+    g = np.random.Generator(np.random.PCG64(19))
+    x = (g.standard_normal((32, 256)) * 3).astype(np.float16).astype(np.float32)
+    s = o.scale_row(x, 1.0)
+    u = o.quantize_u(x, s, np.full(32, 8), 4).astype(np.int64)
+    assert np.array_equal(u - 8, o.quantize(x, s[:, None]).astype(np.int64))
+
+
+def check_asym_gemm(o):
+    """gemm_asym equals the brute-force centred sum on tiny shapes and the
+    expansion sum ux uw - zw sum ux - zx sum uw + K zx zw (no cross term dropped)."""
+    g = np.random.Generator(np.random.PCG64(23))
+    for (m, n, k) in ((1, 1, 1), (3, 5, 7), (4, 6, 256)):
+        ux = g.integers(0, 16, (m, k))
+        uw = g.integers(0, 16, (n, k))
+        zx = g.integers(0, 16, m)
+        zw = g.integers(0, 16, n)
+        acc = o.gemm_asym(ux, zx, uw, zw)
+        for i in range(m):
+            for j in range(n):
+                assert acc[i, j] == sum((int(ux[i, t]) - int(zx[i])) * (int(uw[j, t]) - int(zw[j])) for t in range(k))
+        expand = (ux @ uw.T) - zw[None, :] * ux.sum(1)[:, None] - zx[:, None] * uw.sum(1)[None, :] + k * np.outer(zx, zw)
+        assert np.array_equal(acc, expand)
+
+
 ALL_CHECKS = [
+    check_asym_golden,
+    check_asym_bounds,
+    check_asym_symmetric_case,
+    check_asym_gemm,
     check_rtn_golden, check_rtn_bounds, check_pack, check_kron_golden,
     check_kron_explicit, check_function_preservation, check_identity_transform,
     check_flop_count, check_gemm_bruteforce, check_linear_golden,

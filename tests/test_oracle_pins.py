@@ -113,7 +113,40 @@ def _quant_weight_qsm_rows(w, gran=0, alpha=1.0, p1_inv=None, p2_inv=None, c=Non
     return quantize(v32, s[:, None]), s, v32  # noqa: F821
 
 
+def _minmax_no_zero(v32, bits, alpha=1.0):
+    # range not widened to contain 0
+    v32 = np.asarray(v32, dtype=np.float32)
+    qmax = np.float32((1 << bits) - 1)
+    lo, hi = v32.min(axis=-1), v32.max(axis=-1)
+    s = ((hi - lo) * np.float32(alpha)) / qmax
+    with np.errstate(divide="ignore", invalid="ignore"):
+        z = np.where(s == 0, 0, np.clip(np.rint(-lo / s), 0, qmax)).astype(np.int32)
+    return s.astype(np.float32), z
+
+
+def _minmax_zero_sign(v32, bits, alpha=1.0):
+    # zero point from +lo instead of -lo
+    v32 = np.asarray(v32, dtype=np.float32)
+    qmax = np.float32((1 << bits) - 1)
+    lo = np.minimum(v32.min(axis=-1), np.float32(0))
+    hi = np.maximum(v32.max(axis=-1), np.float32(0))
+    s = ((hi - lo) * np.float32(alpha)) / qmax
+    with np.errstate(divide="ignore", invalid="ignore"):
+        z = np.where(s == 0, 0, np.clip(np.rint(lo / s), 0, qmax)).astype(np.int32)
+    return s.astype(np.float32), z
+
+
+def _gemm_asym_no_cross(ux, zx, uw, zw):
+    # the K zx zw term dropped
+    ux, uw = np.asarray(ux, np.int64), np.asarray(uw, np.int64)
+    zx, zw = np.asarray(zx, np.int64), np.asarray(zw, np.int64)
+    return ux @ uw.T - zw[None, :] * ux.sum(1)[:, None] - zx[:, None] * uw.sum(1)[None, :]
+
+
 MUTANTS = {
+    "asym_range_without_zero": dict(minmax_params=_minmax_no_zero),
+    "asym_zero_point_sign": dict(minmax_params=_minmax_zero_sign),
+    "asym_gemm_drops_cross_term": dict(gemm_asym=_gemm_asym_no_cross),
     "act_P1_not_transposed": dict(act_transform=_act_transform_untransposed),
     "weight_P2inv_not_transposed": dict(weight_transform=_weight_transform_untransposed),
     "weight_c_multiplied": dict(weight_transform=_weight_transform_c_times),
