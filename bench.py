@@ -60,6 +60,24 @@ def dist_env():
     return ws, rank, local
 
 
+def max_over_ranks(ms: float, ws: int, device) -> float:
+    """The largest of every rank's time (one all-reduce, taken by every rank in
+    the same order); a single process returns its own."""
+    if ws <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tops(ops_per_rank_step: float, ws: int, ms_per_step: float) -> float:
+    """Whole-job throughput: the operations all ranks did in one step over the
+    (max-over-ranks) step time; every rank runs the same step (replicas)."""
+    return ops_per_rank_step * ws / (ms_per_step * 1e-3) / 1e12
+
+
 def workload(seed=0, only=None):
     out = []
     for name, k, n in SHAPES:
@@ -222,10 +240,7 @@ def run_ours(args, ws, rank, local):
     q_ms = [v / nb for v in q_ms]
     g_ms = [v / nb for v in g_ms]
 
-    if ws > 1:
-        tt = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(total_ms, ws, dev)
 
     # ------------------------------------------------ end to end through fq_linear with host buffers
     xh = [torch.from_numpy(s["d"]["x"]).pin_memory() for s in state]
@@ -275,11 +290,8 @@ def run_ours(args, ws, rank, local):
         stream.wait_event(ev)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, ws, dev)
     if ws > 1:
-        tt = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
         dist.barrier()
         dist.destroy_process_group()
 
@@ -288,7 +300,7 @@ def run_ours(args, ws, rank, local):
 
     ops_step = sum(2.0 * s["m"] * s["n"] * s["k"] for s in state)
     ms_step = total_ms / args.steps
-    value = ops_step * ws / (ms_step * 1e-3) / 1e12
+    value = job_tops(ops_step, ws, ms_step)
     pk, pk_kind = peaks()
     int8_peak = pk["bf16_tflops_sustained"] * INT8_OVER_BF16
     g_ops = sum(2.0 * s["m"] * s["n"] * s["k"] for s in state)
@@ -306,7 +318,7 @@ def run_ours(args, ws, rank, local):
             "quant_gbs": round(q_bytes[i] / (q_ms[i] * 1e-3) / 1e9, 1),
             "kron": [s["d"]["n1"], s["d"]["n2"]],
         }
-    e2e_value = ops_step * ws / (e2e_ms * 1e-3) / 1e12
+    e2e_value = job_tops(ops_step, ws, e2e_ms)
     out = {
         "metric": METRIC,
         "value": round(value, 2),
