@@ -649,9 +649,13 @@ struct PCfg {
   static_assert(A_COL0 + SU * A_STAGE_COLS <= TMEM_COLS, "tensor memory");
   static_assert(SMEM <= 227 * 1024, "shared memory");
   static_assert(P_STAGE % 1024 == 0 && UNP_STAGE % 1024 == 0 && PA % 1024 == 0, "1024-byte stage alignment");
-  // a warp that takes every NB-th (A: every 2nd) slice must never wait on a
-  // stage more than one phase ahead of its barrier (parity waits alias)
-  static_assert(NB < SU && NB < SP && 2 < SU, "slices per feed warp");
+  // A warp that takes every n-th slice (A: n = 2, B: n = NB) must never wait
+  // on a stage more than one phase ahead of its barrier (parity waits alias).
+  // For the unpacked ring the MMA has consumed slice h - n - SU when the warp
+  // reaches slice h, so n <= SU suffices; for the packed ring the TMA copies
+  // may land out of order, so the warp must itself have waited for the
+  // stage's previous fill (slice h - SP): SP a multiple of n.
+  static_assert(NB <= SU && 2 <= SU && SP % NB == 0 && SP % 2 == 0, "slices per feed warp");
 };
 
 template <int EPI, int NB>
