@@ -67,6 +67,11 @@ struct QuantParams {
   float* s_row;          // [R]
   __half* s_grp;         // [K/128][R]
   float* xhat;           // [R][K] or null
+  // general quantizer (per-row min-max zero point, b = 3 or 4): per row the
+  // offset o = 2^(b-1) - z and the sum of the stored signed codes
+  int asym, bits;
+  int32_t* zoff;         // [R]
+  int32_t* zsum;         // [R]
 };
 
 // Left factor as used by the column pass: Lc(k, i) multiplies U[i][l] into
@@ -107,10 +112,15 @@ __global__ void __launch_bounds__(kThreads) quant_rows_kernel(QuantParams p) {
   const int pad = xf ? 1 : 0;
   const int row_floats = xf ? n1 * (n2 + 1) : K;
   float* xs = smem;                       // row buffer
-  float* sL = xs + row_floats;            // [i][k] = Lc(k, i)   (PSMEM)
+  // activations with a transform: the fp16 input row, tile rows padded to
+  // n2 + 2 halves (an odd word stride: lane-per-row reads are conflict-free)
+  __half* xin = reinterpret_cast<__half*>(xs + row_floats);
+  const int xstride = n2 + 2;
+  const int xin_floats = (SIDE == kAct && xf) ? (n1 * xstride + 1) / 2 : 0;
+  float* sL = xs + row_floats + xin_floats;  // [i][k] = Lc(k, i)   (PSMEM)
   float* sR = sL + (PSMEM ? n1 * n1 : 0); // [j][l] = Rr(j, l)   (PSMEM)
-  float* red = sR + (PSMEM ? n2 * n2 : 0);  // [kWarps]
-  float* gsc = red + kWarps;                // [K/128] group scales
+  float* red = sR + (PSMEM ? n2 * n2 : 0);  // [2][kWarps]
+  float* gsc = red + 2 * kWarps;            // [K/128] group scales
 
   if (PSMEM && xf) {
     for (int e = tid; e < n1 * n1; e += kThreads) {
@@ -126,9 +136,18 @@ __global__ void __launch_bounds__(kThreads) quant_rows_kernel(QuantParams p) {
 
   const int ngroups = K / kGroup;
   for (int r = blockIdx.x; r < p.R; r += gridDim.x) {
-    // 1. load + channel scale
+    // 1. load + channel scale (activations with a transform: the fp16 row as
+    // is; c is applied in float64 inside the transform)
     const __half* xrow = p.X + size_t(r) * K;
-    for (int e0 = tid * 8; e0 < K; e0 += kThreads * 8) {
+    if (SIDE == kAct && xf) {
+      for (int e0 = tid * 8; e0 < K; e0 += kThreads * 8) {
+        const uint4 raw = *reinterpret_cast<const uint4*>(xrow + e0);
+        const __half* h = reinterpret_cast<const __half*>(&raw);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) xin[((e0 + j) / n2) * xstride + (e0 + j) % n2] = h[j];
+      }
+    }
+    for (int e0 = tid * 8; e0 < K && !(SIDE == kAct && xf); e0 += kThreads * 8) {
       const uint4 raw = *reinterpret_cast<const uint4*>(xrow + e0);
       const __half2* h2 = reinterpret_cast<const __half2*>(&raw);
 #pragma unroll
@@ -151,7 +170,74 @@ __global__ void __launch_bounds__(kThreads) quant_rows_kernel(QuantParams p) {
     __syncthreads();
 
     // 2. transform
-    if (xf) {
+    if (SIDE == kAct && xf) {
+      // Activations: every product and sum in float64 (the fp16 inputs, c
+      // and the float32 factors are exact in it), one rounding to float32
+      // per element.  A warp takes 4 columns l at a time: lane owns the
+      // tile rows i = lane + 32 q for U[i][l] = sum_j Xbar[i][j] P2[j][l],
+      // then the outputs k = lane + 32 q of Xhat[k][l] = sum_i P1[i][k] U[i][l],
+      // each U[i][l] broadcast from its owner lane.
+      constexpr int CB = 4, NQ = 8;  // n1 <= 256
+      const int nq = (n1 + 31) / 32;
+      for (int l0 = warp * CB; l0 < n2; l0 += kWarps * CB) {
+        double acc[NQ][CB];
+#pragma unroll
+        for (int q = 0; q < NQ; ++q)
+#pragma unroll
+          for (int c = 0; c < CB; ++c) acc[q][c] = 0.0;
+        for (int j = 0; j < n2; ++j) {
+          double pv[CB];
+#pragma unroll
+          for (int c = 0; c < CB; ++c)
+            pv[c] = l0 + c < n2 ? double(PSMEM ? sR[j * n2 + l0 + c] : right_at<SIDE>(p.Rt, n2, j, l0 + c)) : 0.0;
+#pragma unroll
+          for (int q = 0; q < NQ; ++q) {
+            const int i = lane + 32 * q;
+            if (q < nq) {
+              double x = i < n1 ? double(__half2float(xin[i * xstride + j])) : 0.0;
+              if (p.c && i < n1) x *= double(__ldg(p.c + i * n2 + j));
+#pragma unroll
+              for (int c = 0; c < CB; ++c) acc[q][c] = fma(x, pv[c], acc[q][c]);
+            }
+          }
+        }
+        double out[NQ][CB];
+#pragma unroll
+        for (int q = 0; q < NQ; ++q)
+#pragma unroll
+          for (int c = 0; c < CB; ++c) out[q][c] = 0.0;
+#pragma unroll
+        for (int qi = 0; qi < NQ; ++qi) {
+          if (qi >= nq) break;
+          for (int ii = 0; ii < 32; ++ii) {
+            const int i = 32 * qi + ii;
+            if (i >= n1) break;
+            double u[CB];
+#pragma unroll
+            for (int c = 0; c < CB; ++c) u[c] = __shfl_sync(0xffffffffu, acc[qi][c], ii);
+#pragma unroll
+            for (int q = 0; q < NQ; ++q) {
+              const int k = lane + 32 * q;
+              if (q < nq) {
+                const double lv = k < n1 ? double(PSMEM ? sL[i * n1 + k] : left_at<SIDE>(p.L, n1, k, i)) : 0.0;
+#pragma unroll
+                for (int c = 0; c < CB; ++c) out[q][c] = fma(lv, u[c], out[q][c]);
+              }
+            }
+          }
+        }
+#pragma unroll
+        for (int q = 0; q < NQ; ++q) {
+          const int k = lane + 32 * q;
+          if (q < nq && k < n1) {
+#pragma unroll
+            for (int c = 0; c < CB; ++c)
+              if (l0 + c < n2) xs[k * (n2 + 1) + l0 + c] = float(out[q][c]);
+          }
+        }
+      }
+      __syncthreads();
+    } else if (xf) {
       // row pass: U[i][l] = sum_j Xbar[i][j] Rr(j, l), rows split over warps
       for (int i = warp; i < n1; i += kWarps) {
         float acc[8];
@@ -216,7 +302,41 @@ __global__ void __launch_bounds__(kThreads) quant_rows_kernel(QuantParams p) {
 
     // 4. scales
     float s_row = 0.f;
-    if (p.gran == FQ_DYNAMIC_ROW) {
+    int z_row = 0;
+    if (p.asym) {
+      // Q(W) = clamp(round(W/s) + z, 0, 2^b - 1) with the row's range widened
+      // to contain 0: lo = min(0, min v), hi = max(0, max v),
+      // s = ((hi - lo) alpha) / (2^b - 1), z = clamp(round(-lo / s), 0, 2^b - 1)
+      float mn = 0.f, mx = 0.f;
+      for (int e = tid; e < K; e += kThreads) {
+        const float v = xs[slot(e, n2, pad)];
+        mn = fminf(mn, v);
+        mx = fmaxf(mx, v);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      }
+      if (lane == 0) {
+        red[warp] = mn;
+        red[kWarps + warp] = mx;
+      }
+      __syncthreads();
+      float lo = red[0], hi = red[kWarps];
+#pragma unroll
+      for (int w = 1; w < kWarps; ++w) {
+        lo = fminf(lo, red[w]);
+        hi = fmaxf(hi, red[kWarps + w]);
+      }
+      const float qmax = float((1 << p.bits) - 1);
+      s_row = __fdiv_rn(__fmul_rn(__fsub_rn(hi, lo), p.alpha), qmax);
+      z_row = s_row == 0.f ? 0 : int(fminf(fmaxf(rintf(__fdiv_rn(-lo, s_row)), 0.f), qmax));
+      if (tid == 0) {
+        p.s_row[r] = s_row;
+        p.zoff[r] = (1 << (p.bits - 1)) - z_row;
+      }
+    } else if (p.gran == FQ_DYNAMIC_ROW) {
       float m = 0.f;
       for (int e = tid; e < K; e += kThreads) m = fmaxf(m, fabsf(xs[slot(e, n2, pad)]));
       m = warp_max(m);
@@ -244,6 +364,37 @@ __global__ void __launch_bounds__(kThreads) quant_rows_kernel(QuantParams p) {
 
     // 5. codes, packed 8 per thread-iteration (one 32-bit store)
     uint32_t* qrow = reinterpret_cast<uint32_t*>(p.Q + size_t(r) * (K / 2));
+    if (p.asym) {
+      // u = clamp(round(v / s) + z, 0, 2^b - 1) (u = z when s = 0), stored as
+      // the signed nibble q = u - 2^(b-1); the row's sum of q goes with it
+      const int qmax = (1 << p.bits) - 1, half = 1 << (p.bits - 1);
+      int sum = 0;
+      for (int e0 = tid * 8; e0 < K; e0 += kThreads * 8) {
+        uint32_t word = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float v = xs[slot(e0 + j, n2, pad)];
+          int u = z_row;
+          if (s_row != 0.f) u = min(max(int(rintf(__fdiv_rn(v, s_row))) + z_row, 0), qmax);
+          const int q = u - half;
+          sum += q;
+          word |= (uint32_t(q) & 0xFu) << (4 * j);
+        }
+        qrow[e0 / 8] = word;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+      __syncthreads();  // red is free again
+      if (lane == 0) reinterpret_cast<int*>(red)[warp] = sum;
+      __syncthreads();
+      if (tid == 0) {
+        int tot = 0;
+        for (int w = 0; w < kWarps; ++w) tot += reinterpret_cast<int*>(red)[w];
+        p.zsum[r] = tot;
+      }
+      __syncthreads();
+      continue;
+    }
     for (int e0 = tid * 8; e0 < K; e0 += kThreads * 8) {
       uint32_t word = 0;
 #pragma unroll
@@ -313,15 +464,15 @@ fq_status launch_quant_static(const QuantParams& qp, cudaStream_t stream) {
   return check_launch("quant_static_kernel");
 }
 
-size_t smem_bytes(int K, int n1, int n2, bool psmem) {
-  const size_t row = n1 > 0 ? size_t(n1) * (n2 + 1) : size_t(K);
+size_t smem_bytes(int K, int n1, int n2, bool psmem, bool act) {
+  const size_t row = n1 > 0 ? size_t(n1) * (n2 + 1) + (act ? (size_t(n1) * (n2 + 2) + 1) / 2 : 0) : size_t(K);
   const size_t pm = (psmem && n1 > 0) ? size_t(n1) * n1 + size_t(n2) * n2 : 0;
-  return (row + pm + kWarps + K / kGroup) * sizeof(float);
+  return (row + pm + 2 * kWarps + K / kGroup) * sizeof(float);
 }
 
 template <int SIDE, bool PSMEM>
 fq_status launch_quant(const QuantParams& qp, cudaStream_t stream) {
-  const size_t smem = smem_bytes(qp.K, qp.n1, qp.n2, PSMEM);
+  const size_t smem = smem_bytes(qp.K, qp.n1, qp.n2, PSMEM, SIDE == kAct);
   auto kern = quant_rows_kernel<SIDE, PSMEM>;
   if (smem > 48 * 1024) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
@@ -338,10 +489,19 @@ fq_status launch_quant(const QuantParams& qp, cudaStream_t stream) {
 
 fq_status check_qparams(const fq_qparams* qp, bool act) {
   FQ_CHECK_ARG(qp != nullptr, "qparams is NULL");
-  if (qp->bits != 4) return fail(FQ_ERR_UNSUPPORTED, "bits = %d: only b = 4 is provided", qp->bits);
-  if (qp->zero_point != 8)
-    return fail(FQ_ERR_UNSUPPORTED, "zero_point = %d: only the symmetric z = 2^(b-1) = 8 is provided",
-                qp->zero_point);
+  if (qp->zero_point == FQ_ZERO_POINT_MINMAX) {
+    // the general quantizer: b = 3 or 4, per-row scale and zero point
+    if (qp->bits != 3 && qp->bits != 4)
+      return fail(FQ_ERR_UNSUPPORTED, "bits = %d: the min-max quantizer provides b = 3 and 4", qp->bits);
+    if (qp->gran != FQ_DYNAMIC_ROW)
+      return fail(FQ_ERR_UNSUPPORTED, "the min-max quantizer is per row (FQ_DYNAMIC_ROW) only");
+  } else {
+    if (qp->bits != 4) return fail(FQ_ERR_UNSUPPORTED, "bits = %d: the symmetric quantizer provides b = 4", qp->bits);
+    if (qp->zero_point != 8)
+      return fail(FQ_ERR_UNSUPPORTED,
+                  "zero_point = %d: provided are the symmetric z = 2^(b-1) = 8 and FQ_ZERO_POINT_MINMAX",
+                  qp->zero_point);
+  }
   if (qp->gran == FQ_DYNAMIC_GROUP && qp->group_size != kGroup)
     return fail(FQ_ERR_UNSUPPORTED, "group_size = %d: only 128 is provided", qp->group_size);
   if (qp->gran != FQ_DYNAMIC_ROW && qp->gran != FQ_DYNAMIC_GROUP && !(act && qp->gran == FQ_STATIC_CHANNEL))
@@ -374,6 +534,13 @@ fq_status quant_common(int side, const uint16_t* X, int R, int K, const fq_qpara
   p.Q = Q;
   p.xhat = xhat;
   if (qp->gran == FQ_DYNAMIC_ROW) p.s_row = static_cast<float*>(s_out);
+  if (qp->zero_point == FQ_ZERO_POINT_MINMAX) {
+    // scale block: float32 s[R], int32 o[R] = 2^(b-1) - z, int32 code sums[R]
+    p.asym = 1;
+    p.bits = qp->bits;
+    p.zoff = reinterpret_cast<int32_t*>(static_cast<float*>(s_out) + R);
+    p.zsum = reinterpret_cast<int32_t*>(static_cast<float*>(s_out) + 2 * size_t(R));
+  }
   if (qp->gran == FQ_DYNAMIC_GROUP) p.s_grp = static_cast<__half*>(s_out);
   if (side == kAct && qp->gran == FQ_STATIC_CHANNEL) p.sstatic = extra;
   if (side == kWeight) p.qsm = extra;
@@ -392,7 +559,7 @@ fq_status quant_common(int side, const uint16_t* X, int R, int K, const fq_qpara
     }
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (side == kAct && p.n1 > 0 && quant_act_tc_supported(K, p.n1, p.n2)) {
+  if (side == kAct && p.n1 > 0 && !p.asym && quant_act_tc_supported(K, p.n1, p.n2)) {
     // activations with the transform: tensor-core kernel
     unsigned* err = device_error_word();
     if (!err) return fail(FQ_ERR_CUDA, "device error word unavailable");
@@ -420,8 +587,9 @@ fq_status quant_common(int side, const uint16_t* X, int R, int K, const fq_qpara
   if (side == kAct && qp->gran == FQ_STATIC_CHANNEL && p.n1 == 0 && aligned(extra, 16) &&
       (!p.c || aligned(p.c, 16)))
     return launch_quant_static(p, s);
-  const bool psmem = smem_bytes(K, p.n1, p.n2, true) <= size_t(kSmemBudget);
-  if (smem_bytes(K, p.n1, p.n2, false) > size_t(kSmemBudget))
+  const bool act = side == kAct;
+  const bool psmem = smem_bytes(K, p.n1, p.n2, true, act) <= size_t(kSmemBudget);
+  if (smem_bytes(K, p.n1, p.n2, false, act) > size_t(kSmemBudget))
     return fail(FQ_ERR_UNSUPPORTED, "row of K = %d does not fit in shared memory", K);
   if (side == kAct) return psmem ? launch_quant<kAct, true>(p, s) : launch_quant<kAct, false>(p, s);
   return psmem ? launch_quant<kWeight, true>(p, s) : launch_quant<kWeight, false>(p, s);

@@ -77,21 +77,29 @@ def test_quant_act_tiny_workload():
 
 
 def _transform_case(d, gname, m=None):
+    """Transformed values, scales and codes against the oracle (see gpu_checks)."""
     gf, go = GRAN[gname]
     x = d["x"] if m is None else d["x"][:m]
     alpha = d.get("alpha_a", 1.0)
     t = fq.Transform(C.dev(d["p1"]), C.dev(d["p2"]), C.dev(d["c"]) if d.get("c") is not None else None)
     xq, sx, xhat = fq.fq_quant_act_debug(C.dev(x), fq.qparams(gf, alpha), t)
+    xq2, sx2 = fq.fq_quant_act(C.dev(x), fq.qparams(gf, alpha), t)
+    assert torch.equal(xq, xq2) and torch.equal(sx, sx2), "the debug kernel quantized differently"
     q_ref, s_ref, v_ref = O.quant_act(x, go, alpha, d["p1"], d["p2"], d.get("c"))
-    worst = C.check_values(C.host(xhat), v_ref, go)
+    vg = C.host(xhat)
+    qg = C.unpack(C.host(xq))
+    worst = C.check_values(vg, v_ref)
     s_gpu = _gpu_scales(sx, gf)
+    C.check_own_scales(s_gpu, vg, go, alpha)
+    C.check_own_codes(qg, vg, s_gpu, go)
     if gname == "row":
         C.check_scales_row(s_gpu, s_ref)
     else:
         C.check_scales_group(s_gpu, s_ref, v_ref, alpha)
     ex = C.exempt_mask(v_ref, s_ref, s_gpu, go)
-    n_ex, n_diff = C.check_codes(C.unpack(C.host(xq)), q_ref, ex)
-    print(f"{d['name']} {gname}: max |dv|/amax {worst:.2e}, boundary-exempt {n_ex}, differing codes {n_diff}")
+    n_ex, n_diff = C.check_codes(qg, q_ref, ex)
+    print(f"{d['name']} {gname}: max |dv|/max(|v|, 2^-10 amax) {worst:.2e}, boundary-exempt {n_ex}, "
+          f"differing codes {n_diff}")
     return n_ex, n_diff
 
 
