@@ -55,7 +55,7 @@ extern "C" {
 typedef enum {
   FQ_OK = 0,
   FQ_ERR_INVALID = 1,      /* a NULL/misaligned pointer or a size outside the ranges above */
-  FQ_ERR_UNSUPPORTED = 2,  /* b != 4, z != 2^(b-1), group size != 128, or a mode/argument combination not provided */
+  FQ_ERR_UNSUPPORTED = 2,  /* b, z, group size or a mode/argument combination not provided */
   FQ_ERR_CUDA = 3,         /* the CUDA runtime or driver reported an error (launch, tensor-map encode) */
   FQ_ERR_TIMEOUT = 4       /* a kernel's bounded wait gave up (reported by fq_check_device_error) */
 } fq_status;
@@ -64,15 +64,31 @@ typedef enum {
 typedef enum {
   FQ_DYNAMIC_ROW = 0,    /* one scale per token (activations) / per output channel (weights) */
   FQ_DYNAMIC_GROUP = 1,  /* one scale per row and group of 128 along K */
-  FQ_STATIC_CHANNEL = 2  /* activations only: caller-given float32 scale per input channel */
+  FQ_STATIC_CHANNEL = 2, /* activations only: caller-given float32 scale per input channel */
+  FQ_DYNAMIC_ROW_ZP = 3  /* GEMM / linear only: both operands from the min-max quantizer
+                            (FQ_ZERO_POINT_MINMAX): per-row scale and zero point */
 } fq_gran;
+
+/* fq_qparams.zero_point value that selects the general (asymmetric) form of
+ * Q(W) = clamp(round(W/s) + z, 0, 2^b - 1) (FRM-PTQ page, 初步介绍) with the
+ * min-max choice of s and z, per row (gran FQ_DYNAMIC_ROW), b = 3 or 4:
+ *   lo = min(0, min v), hi = max(0, max v)   (the range always contains 0)
+ *   s  = ((hi - lo) * alpha) / (2^b - 1)      float32, each step rounded
+ *   z  = clamp(round(-lo / s), 0, 2^b - 1)    IEEE division, half to even; z = 0 when s = 0
+ *   u  = clamp(round(v / s) + z, 0, 2^b - 1)  u = z when s = 0
+ * Codes are stored as the signed nibble q = u - 2^(b-1) (in [-4, 3] for
+ * b = 3), two per byte as usual.  The scale output is then a block of
+ * 3 R 32-bit words: float32 s[R], int32 o[R] = 2^(b-1) - z, int32 S[R] =
+ * sum over k of q[r][k]; the GEMM needs o and S to form
+ * sum_k (u_x - z_x)(u_w - z_w) = sum q_x q_w + o_w S_x + o_x S_w + K o_x o_w. */
+#define FQ_ZERO_POINT_MINMAX (-1)
 
 /* Parameters of Q(W) = clamp(round(W/s) + z, 0, 2^b - 1) (FRM-PTQ page, 初步介绍)
  * and the clip ratio alpha of s = max|v| * alpha / 7 (FlatQuant notes,
  * 可学习裁剪阈值).  Host memory, read during the call only. */
 typedef struct {
-  int bits;         /* b: only 4 */
-  int zero_point;   /* z: only 2^(b-1) = 8 (the symmetric quantizer) */
+  int bits;         /* b: 4 (symmetric), or 3 and 4 with FQ_ZERO_POINT_MINMAX */
+  int zero_point;   /* z: 2^(b-1) = 8 (the symmetric quantizer) or FQ_ZERO_POINT_MINMAX */
   fq_gran gran;     /* scale extent */
   int group_size;   /* 128 when gran == FQ_DYNAMIC_GROUP, ignored otherwise */
   float alpha;      /* clip ratio in (0, 1]; unused for FQ_STATIC_CHANNEL */
@@ -96,8 +112,8 @@ typedef struct {
 /* Offline weight quantization (FlatQuant notes, Kronecker 分解: Q(P1^-1 W P2^-T);
  * MergeQuant 核心思路: quantization step migration).
  * W      fp16 [N, K]: weights, one row per output channel.
- * qp     gran FQ_DYNAMIC_ROW (s_w float32 [N]) or FQ_DYNAMIC_GROUP (s_w fp16 [K/128][N]);
- *        alpha = alpha_w.
+ * qp     gran FQ_DYNAMIC_ROW (s_w float32 [N]; with FQ_ZERO_POINT_MINMAX the 3 N-word
+ *        scale block) or FQ_DYNAMIC_GROUP (s_w fp16 [K/128][N]); alpha = alpha_w.
  * inv    NULL or the inverse transform (P1^-1, P2^-1, c): see fq_transform.
  * qsm_scale NULL or float32 [K]: static activation scales s_k folded into the
  *        weights, w'[n,k] = v[n,k] * s_k in float32 after the transform, so
@@ -111,7 +127,8 @@ fq_status fq_quant_weight(const uint16_t* W, int N, int K, const fq_qparams* qp,
 /* Online activation quantization (FlatQuant notes, 高效 Kernel 设计: the
  * transform and the quantization fused, intermediates kept on chip).
  * X      fp16 [M, K] token rows.
- * qp     FQ_DYNAMIC_ROW: s_x float32 [M];  FQ_DYNAMIC_GROUP: s_x fp16 [K/128][M];
+ * qp     FQ_DYNAMIC_ROW: s_x float32 [M] (FQ_ZERO_POINT_MINMAX: the 3 M-word scale
+ *        block);  FQ_DYNAMIC_GROUP: s_x fp16 [K/128][M];
  *        FQ_STATIC_CHANNEL: static_scale float32 [K] is used and s_x is not written
  *        (may be NULL); alpha = alpha_a.
  * t      NULL or the transform (P1, P2, c).  P1 and P2 are parameters: the
@@ -139,6 +156,10 @@ fq_status fq_quant_act_debug(const uint16_t* X, int M, int K, const fq_qparams* 
  *   FQ_DYNAMIC_GROUP:  y = fp16(sum_g float(acc_g) * s_x[g][m] * s_w[g][n]), the sum in
  *                      float32, acc_g the exact product over k in [128g, 128g+128);
  *                      s_x fp16 [K/128][M], s_w fp16 [K/128][N].
+ *   FQ_DYNAMIC_ROW_ZP: y = fp16((float(a) * s_x[m]) * s_w[n]) with the exact
+ *                      a = sum_k (u_x - z_x)(u_w - z_w); s_x, s_w the 3 M- and 3 N-word
+ *                      scale blocks of FQ_ZERO_POINT_MINMAX.  Runs as the exact int32
+ *                      product into the workspace, then a zero-point epilogue.
  * workspace / ws_bytes: device scratch of at least fq_gemm_workspace_size()
  *   bytes (may be NULL when that size is 0); contents on entry are ignored. */
 fq_status fq_w4a4_gemm(const uint8_t* Xq, const void* s_x, const uint8_t* Wq, const void* s_w,
@@ -173,9 +194,10 @@ fq_status fq_w4a4_gemm_s32(const uint8_t* Xq, const uint8_t* Wq, int M, int N, i
 /* The linear layer: fq_quant_act into the workspace, then fq_w4a4_gemm, on
  * one stream.  Arguments as in those two calls; Wq/s_w come from
  * fq_quant_weight with the matching inverse transform (and, for
- * FQ_STATIC_CHANNEL, the same static scales folded in).  workspace must hold
- * fq_linear_workspace_size() bytes (packed activations, their scales and the
- * GEMM's scratch). */
+ * FQ_STATIC_CHANNEL, the same static scales folded in; for
+ * FQ_ZERO_POINT_MINMAX, the weights' min-max scale block).  workspace must
+ * hold fq_linear_workspace_size() bytes (packed activations, their scales and
+ * the GEMM's scratch; pass FQ_DYNAMIC_ROW_ZP there for the min-max quantizer). */
 fq_status fq_linear(const uint16_t* X, int M, int K, const fq_qparams* act_qp,
                     const fq_transform* t, const float* static_scale,
                     const uint8_t* Wq, const void* s_w, int N, uint16_t* Y,

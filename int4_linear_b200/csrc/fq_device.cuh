@@ -110,16 +110,16 @@ __device__ __forceinline__ void cluster_sync() {
 }
 
 // Arrive on the mbarrier at the same shared-memory offset as `bar` in the
-// cluster's CTA `rank`.  Default (CTA-scope release) semantics: what the
-// arrival publishes is made complete beforehand by the caller (tcgen05.wait::st
-// for tensor-memory stores, fence.proxy.async for shared-memory operands the
-// tensor core reads), and a cluster-scope release here costs a memory fence
-// per arrival (it made the CTA-pair GEMM 1.6x slower).
+// cluster's CTA `rank`, with release semantics at cluster scope: the writes
+// this thread made (or that its warp made and ordered before it with
+// __syncwarp, tcgen05.wait::st / fence.proxy.async for what the tensor core
+// reads) are visible to a thread of the other CTA that acquires the
+// barrier's phase at cluster scope (mbar_wait_cluster).
 __device__ __forceinline__ void mbar_arrive_cluster(uint64_t* bar, uint32_t rank) {
   asm volatile(
       "{\n\t.reg .b32 ra;\n\t"
       "mapa.shared::cluster.u32 ra, %0, %1;\n\t"
-      "mbarrier.arrive.shared::cluster.b64 _, [ra];\n\t}" ::"r"(smem_u32(bar)),
+      "mbarrier.arrive.release.cluster.shared::cluster.b64 _, [ra];\n\t}" ::"r"(smem_u32(bar)),
       "r"(rank)
       : "memory");
 }

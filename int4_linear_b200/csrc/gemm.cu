@@ -608,9 +608,9 @@ __global__ void __launch_bounds__(threads_of<EPI>(), 1)
 //   warp 0        one thread issues the TMA loads of the packed slices
 //   warp 1        tensor-memory allocation; in CTA 0 the thread that issues
 //                 the 256 x 256 pair MMAs (.cta_group::2)
-//   warps 2-9     unpack this CTA's 128 A rows into the tensor-memory ring
-//                 (two warps per lane quadrant, alternate K slices)
-//   warps 10..    unpack this CTA's half of the weight rows, NB warps taking
+//   warps 2-13    unpack this CTA's 128 A rows into the tensor-memory ring
+//                 (three warps per lane quadrant, K slices in turn)
+//   warps 14..    unpack this CTA's half of the weight rows, NB warps taking
 //                 whole K slices in turn
 //   last 8 warps  epilogue: drain the accumulator (two warps per lane
 //                 quadrant, 128 columns each, 32 at a time), scale to fp16
@@ -642,7 +642,8 @@ struct PCfg {
   static constexpr int NBAR = 2 * SP + 2 * SU + 4;          // + acc_full, acc_empty, done, fin
   static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
   static constexpr int SMEM = OFF_TMEM + 16 + 1024;
-  static constexpr int B_WARP0 = 10;           // A: warps 2-9, two per lane quadrant
+  static constexpr int NA = 3;                 // A-warps per lane quadrant (slices in turn)
+  static constexpr int B_WARP0 = 2 + 4 * NA;   // A: warps 2 .. 2 + 4 NA - 1
   static constexpr int EPI_WARP0 = B_WARP0 + NB;
   static constexpr int THREADS = 32 * (EPI_WARP0 + 8);
   static constexpr int FEED = 4 + 1;           // arrivals per slice and CTA: 4 A-warps, 1 B-warp
@@ -655,7 +656,7 @@ struct PCfg {
   // reaches slice h, so n <= SU suffices; for the packed ring the TMA copies
   // may land out of order, so the warp must itself have waited for the
   // stage's previous fill (slice h - SP): SP a multiple of n.
-  static_assert(NB <= SU && 2 <= SU && SP % NB == 0 && SP % 2 == 0, "slices per feed warp");
+  static_assert(NB <= SU && NA <= SU && SP % NB == 0 && SP % NA == 0, "slices per feed warp");
 };
 
 template <int EPI, int NB>
@@ -791,14 +792,15 @@ __global__ void __launch_bounds__(PCfg<NB>::THREADS, 1)
     }
   } else if (warp < C::B_WARP0) {
     // ------------------------------------------------------------ A rows -> tensor-memory ring
-    // two warps per lane quadrant take alternate slices, so each has two
-    // slice periods for its load - unpack - store - arrive chain
-    const int q = warp & 3, par = (warp - 2) >> 2;
+    // NA warps per lane quadrant take the slices in turn, so each has NA
+    // slice periods for its load - unpack - store - fence - arrive chain (in
+    // CTA 1 the arrival is a cluster-scope release, a memory fence)
+    const int q = warp & 3, par = (warp - 2) >> 2;  // quadrant, turn (0 .. NA - 1)
     const int row = q * 32 + lane;
     const int sw = (row >> 1) & 3;  // 64-byte swizzle: chunk c of this row sits at chunk c ^ sw
     const uint32_t ta = tmem + (uint32_t(q * 32) << 16) + uint32_t(C::A_COL0);
     bool ok = true;
-    for (uint32_t g = uint32_t(par); g < total; g += 2) {
+    for (uint32_t g = uint32_t(par); g < total; g += C::NA) {
       const int sp = int(g % SP), su = int(g % SU);
       if (!warp_wait(&pfull[sp], (g / SP) & 1)) {
         ok = false;
@@ -830,7 +832,7 @@ __global__ void __launch_bounds__(PCfg<NB>::THREADS, 1)
         if (crank == 0)
           mbar_arrive(&full_u[su]);
         else
-          mbar_arrive_cluster(&full_u[su], 0);
+          mbar_arrive_cluster(&full_u[su], 0);  // cluster-scope release of this warp's operands
       }
     }
     if (!ok && lane == 0) record_error(p.err, kErrTimeoutUnpack);
@@ -880,7 +882,7 @@ __global__ void __launch_bounds__(PCfg<NB>::THREADS, 1)
         if (crank == 0)
           mbar_arrive(&full_u[su]);
         else
-          mbar_arrive_cluster(&full_u[su], 0);
+          mbar_arrive_cluster(&full_u[su], 0);  // cluster-scope release of this warp's operands
       }
     }
     if (!ok && lane == 0) record_error(p.err, kErrTimeoutUnpack);
@@ -1335,6 +1337,41 @@ __global__ void __launch_bounds__(128) decode_fixup_kernel(const int32_t* __rest
   }
 }
 
+// Zero-point epilogue of the general (min-max) quantizer: with the exact
+// int32 products acc = sum_k q_x q_w of the stored signed codes
+// (q = u - 2^(b-1)), the product of the dequantized-up-to-scale codes is
+// a = acc + o_w S_x + o_x S_w + K o_x o_w (o = 2^(b-1) - z, S = sum_k q per
+// row: sum_k (u_x - z_x)(u_w - z_w) expanded), and y = fp16((a * s_x) * s_w).
+// |a| <= 15 * 15 * K < 2^24, so its float32 conversion is exact.
+// One thread: 8 consecutive outputs of one row (a 16-byte store).
+__global__ void __launch_bounds__(256) zp_epilogue_kernel(const int32_t* __restrict__ acc,
+                                                          const float* __restrict__ bx,
+                                                          const float* __restrict__ bw, __half* __restrict__ Y,
+                                                          int M, int N, int K) {
+  const int32_t* ox = reinterpret_cast<const int32_t*>(bx + M);
+  const int32_t* Sx = reinterpret_cast<const int32_t*>(bx + 2 * size_t(M));
+  const int32_t* ow = reinterpret_cast<const int32_t*>(bw + N);
+  const int32_t* Sw = reinterpret_cast<const int32_t*>(bw + 2 * size_t(N));
+  const size_t pieces = size_t(M) * (N / 8);
+  for (size_t pc = blockIdx.x * size_t(blockDim.x) + threadIdx.x; pc < pieces; pc += size_t(gridDim.x) * blockDim.x) {
+    const int m = int(pc / (N / 8)), n0 = int(pc % (N / 8)) * 8;
+    const int4 a0 = *reinterpret_cast<const int4*>(acc + size_t(m) * N + n0);
+    const int4 a1 = *reinterpret_cast<const int4*>(acc + size_t(m) * N + n0 + 4);
+    const int av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+    const float sxm = __ldg(bx + m);
+    const int oxm = __ldg(ox + m), Sxm = __ldg(Sx + m);
+    float y[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int n = n0 + j;
+      const int own = __ldg(ow + n);
+      const int a = av[j] + own * Sxm + oxm * __ldg(Sw + n) + K * oxm * own;
+      y[j] = __fmul_rn(__fmul_rn(__int2float_rn(a), sxm), __ldg(bw + n));
+    }
+    store_half8(Y + size_t(m) * N + n0, y);
+  }
+}
+
 struct Plan {
   bool swap;          // decode kernel (weights on the 128-row side)
   bool pair;          // prefill: 256 x BN tiles over CTA pairs
@@ -1549,10 +1586,32 @@ fq_status gemm_impl(const uint8_t* Xq, const void* s_x, const uint8_t* Wq, const
   return st;
 }
 
+// The general quantizer's GEMM: the exact int32 products of the stored codes
+// into the workspace, then the zero-point epilogue.
+fq_status gemm_zp(const uint8_t* Xq, const void* s_x, const uint8_t* Wq, const void* s_w, int M, int N, int K,
+                  uint16_t* Y, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  fq_status st = check_sizes(M, N, K);
+  if (st != FQ_OK) return st;
+  FQ_CHECK_ARG(Y && aligned(Y, 16), "Y must be non-NULL and 16-byte aligned");
+  FQ_CHECK_ARG(s_x && s_w && aligned(s_x, 4) && aligned(s_w, 4), "the scale blocks must be non-NULL and aligned");
+  const size_t need = size_t(M) * N * sizeof(int32_t);
+  FQ_CHECK_ARG(ws && ws_bytes >= need && aligned(ws, 16), "workspace of %zu bytes required", need);
+  st = gemm_impl(Xq, nullptr, Wq, nullptr, M, N, K, kEpiS32, nullptr, static_cast<int32_t*>(ws), nullptr, 0,
+                 stream);
+  if (st != FQ_OK) return st;
+  const size_t pieces = size_t(M) * (N / 8);
+  const int grid = int(std::max<size_t>(1, std::min<size_t>((pieces + 255) / 256, size_t(sm_count()) * 8)));
+  zp_epilogue_kernel<<<grid, 256, 0, stream>>>(static_cast<const int32_t*>(ws), static_cast<const float*>(s_x),
+                                               static_cast<const float*>(s_w), reinterpret_cast<__half*>(Y), M, N,
+                                               K);
+  return check_launch("zp_epilogue_kernel");
+}
+
 }  // namespace
 
 size_t gemm_workspace_bytes(int M, int N, int K, fq_gran gran) {
   if (M < 1 || N < 8 || K < kBK || K % kBK) return 0;
+  if (gran == FQ_DYNAMIC_ROW_ZP) return size_t(M) * N * sizeof(int32_t);  // the exact int32 products
   const int epi = gran == FQ_DYNAMIC_GROUP ? kEpiGroup : (gran == FQ_STATIC_CHANNEL ? kEpiStatic : kEpiRow);
   const Plan pl = make_plan(M, N, K, epi, sm_count());
   return (pl.swap && pl.partial) ? size_t(M) * N * sizeof(int32_t) : 0;
@@ -1570,6 +1629,8 @@ fq_status fq_w4a4_gemm(const uint8_t* Xq, const void* s_x, const uint8_t* Wq, co
     case FQ_DYNAMIC_ROW: epi = fq::kEpiRow; break;
     case FQ_STATIC_CHANNEL: epi = fq::kEpiStatic; break;
     case FQ_DYNAMIC_GROUP: epi = fq::kEpiGroup; break;
+    case FQ_DYNAMIC_ROW_ZP: return fq::gemm_zp(Xq, s_x, Wq, s_w, M, N, K, Y, workspace, ws_bytes,
+                                               static_cast<cudaStream_t>(stream));
     default: return fq::fail(FQ_ERR_UNSUPPORTED, "granularity %d is not provided", int(gran));
   }
   return fq::gemm_impl(Xq, s_x, Wq, s_w, M, N, K, epi, Y, nullptr, workspace, ws_bytes,

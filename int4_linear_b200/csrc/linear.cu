@@ -12,6 +12,7 @@ size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 size_t act_scale_bytes(int M, int K, fq_gran gran) {
   if (gran == FQ_DYNAMIC_ROW) return size_t(M) * sizeof(float);
+  if (gran == FQ_DYNAMIC_ROW_ZP) return 3 * size_t(M) * sizeof(float);  // s, o = 2^(b-1) - z, code sums
   if (gran == FQ_DYNAMIC_GROUP) return size_t(K / kGroup) * M * 2;
   return 0;
 }
@@ -37,19 +38,21 @@ fq_status fq_linear(const uint16_t* X, int M, int K, const fq_qparams* act_qp, c
   if (!act_qp) return fq::fail(FQ_ERR_INVALID, "act_qp is NULL");
   if (M < 1 || K < fq::kGroup || K % fq::kGroup || N < 8 || N % 8)
     return fq::fail(FQ_ERR_INVALID, "sizes M = %d, N = %d, K = %d out of range", M, N, K);
-  const size_t need = fq::linear_workspace_bytes(M, N, K, act_qp->gran);
+  // the min-max quantizer's activations go with the zero-point GEMM
+  const fq_gran gran = act_qp->zero_point == FQ_ZERO_POINT_MINMAX ? FQ_DYNAMIC_ROW_ZP : act_qp->gran;
+  const size_t need = fq::linear_workspace_bytes(M, N, K, gran);
   if (!workspace || ws_bytes < need || !fq::aligned(workspace, 256))
     return fq::fail(FQ_ERR_INVALID, "workspace of %zu bytes (256-byte aligned) required, got %zu", need, ws_bytes);
   uint8_t* base = static_cast<uint8_t*>(workspace);
   uint8_t* xq = base;
   size_t off = fq::up(size_t(M) * (K / 2));
   void* sx = act_qp->gran == FQ_STATIC_CHANNEL ? nullptr : static_cast<void*>(base + off);
-  off += fq::up(fq::act_scale_bytes(M, K, act_qp->gran));
+  off += fq::up(fq::act_scale_bytes(M, K, gran));
   void* gws = base + off;
   const size_t gws_bytes = ws_bytes - off;
   fq_status st = fq_quant_act(X, M, K, act_qp, t, static_scale, xq, sx, stream);
   if (st != FQ_OK) return st;
-  return fq_w4a4_gemm(xq, sx, Wq, s_w, M, N, K, act_qp->gran, Y, gws, gws_bytes, stream);
+  return fq_w4a4_gemm(xq, sx, Wq, s_w, M, N, K, gran, Y, gws, gws_bytes, stream);
 }
 
 }  // extern "C"

@@ -13,8 +13,9 @@ from dataclasses import dataclass
 
 import torch
 
-ROW, GROUP, STATIC = 0, 1, 2          # fq_gran
+ROW, GROUP, STATIC, ROW_ZP = 0, 1, 2, 3  # fq_gran
 GROUP_SIZE = 128
+ZERO_POINT_MINMAX = -1                   # fq_qparams.zero_point: per-row min-max (asymmetric) quantizer
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libfq.so")
@@ -131,7 +132,10 @@ def _s(stream):
     return stream.cuda_stream if hasattr(stream, "cuda_stream") else stream
 
 
-def _scales_out(gran, rows, k, dev):
+def _scales_out(gran, rows, k, dev, zero_point=8):
+    if gran == ROW and zero_point == ZERO_POINT_MINMAX:
+        # float32 s[rows], int32 o[rows] = 2^(b-1) - z, int32 code sums[rows]
+        return torch.empty(3, rows, dtype=torch.float32, device=dev)
     if gran == ROW:
         return torch.empty(rows, dtype=torch.float32, device=dev)
     if gran == GROUP:
@@ -146,7 +150,7 @@ def fq_quant_weight(W, qp: QParams, inv: Transform | None = None, qsm_scale=None
     _check(qsm_scale, torch.float32, "qsm_scale")
     n, k = W.shape
     Wq = torch.empty(n, k // 2, dtype=torch.uint8, device=W.device) if Wq is None else Wq
-    s_w = _scales_out(qp.gran, n, k, W.device) if s_w is None else s_w
+    s_w = _scales_out(qp.gran, n, k, W.device, qp.zero_point) if s_w is None else s_w
     t = inv.as_c() if inv is not None else None
     st = lib().fq_quant_weight(W.data_ptr(), n, k, ctypes.byref(qp), ctypes.byref(t) if t else None,
                                _p(qsm_scale), Wq.data_ptr(), _p(s_w), _s(stream))
@@ -161,7 +165,7 @@ def fq_quant_act(X, qp: QParams, t: Transform | None = None, static_scale=None,
     _check(static_scale, torch.float32, "static_scale")
     m, k = X.shape
     Xq = torch.empty(m, k // 2, dtype=torch.uint8, device=X.device) if Xq is None else Xq
-    s_x = _scales_out(qp.gran, m, k, X.device) if s_x is None else s_x
+    s_x = _scales_out(qp.gran, m, k, X.device, qp.zero_point) if s_x is None else s_x
     tc = t.as_c() if t is not None else None
     st = lib().fq_quant_act(X.data_ptr(), m, k, ctypes.byref(qp), ctypes.byref(tc) if tc else None,
                             _p(static_scale), Xq.data_ptr(), _p(s_x), _s(stream))
@@ -175,13 +179,20 @@ def fq_quant_act_debug(X, qp: QParams, t: Transform | None = None, static_scale=
     _check(static_scale, torch.float32, "static_scale")
     m, k = X.shape
     Xq = torch.empty(m, k // 2, dtype=torch.uint8, device=X.device)
-    s_x = _scales_out(qp.gran, m, k, X.device)
+    s_x = _scales_out(qp.gran, m, k, X.device, qp.zero_point)
     xhat = torch.empty(m, k, dtype=torch.float32, device=X.device)
     tc = t.as_c() if t is not None else None
     st = lib().fq_quant_act_debug(X.data_ptr(), m, k, ctypes.byref(qp), ctypes.byref(tc) if tc else None,
                                   _p(static_scale), Xq.data_ptr(), _p(s_x), xhat.data_ptr(), _s(stream))
     _raise(st)
     return Xq, s_x, xhat
+
+
+def split_zero_point_block(block):
+    """The min-max quantizer's scale block -> (s float32 [R], o int32 [R] =
+    2^(b-1) - z, S int32 [R] = the rows' sums of the stored codes)."""
+    b = block.reshape(3, -1)
+    return b[0], b[1].view(torch.int32), b[2].view(torch.int32)
 
 
 def fq_gemm_workspace_size(m, n, k, gran) -> int:
@@ -258,7 +269,8 @@ def fq_linear(X, qp: QParams, Wq, s_w, t: Transform | None = None, static_scale=
     n = Wq.shape[0]
     Y = torch.empty(m, n, dtype=torch.float16, device=X.device) if Y is None else Y
     _check(Y, torch.float16, "Y")
-    ws, wsb = _workspace(fq_linear_workspace_size(m, n, k, qp.gran), X.device, workspace)
+    gran = ROW_ZP if qp.zero_point == ZERO_POINT_MINMAX else qp.gran
+    ws, wsb = _workspace(fq_linear_workspace_size(m, n, k, gran), X.device, workspace)
     tc = t.as_c() if t is not None else None
     st = lib().fq_linear(X.data_ptr(), m, k, ctypes.byref(qp), ctypes.byref(tc) if tc else None,
                          _p(static_scale), Wq.data_ptr(), _p(s_w), n, Y.data_ptr(), _p(ws), wsb,

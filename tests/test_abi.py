@@ -54,8 +54,12 @@ A = 1 << 20
 
 
 @pytest.mark.parametrize("kw,status", [
-    (dict(bits=3), fq.FQ_ERR_UNSUPPORTED),
+    (dict(bits=3), fq.FQ_ERR_UNSUPPORTED),            # symmetric b = 3: not provided
     (dict(zero_point=0), fq.FQ_ERR_UNSUPPORTED),
+    (dict(bits=5, zero_point=fq.ZERO_POINT_MINMAX), fq.FQ_ERR_UNSUPPORTED),
+    (dict(bits=2, zero_point=fq.ZERO_POINT_MINMAX), fq.FQ_ERR_UNSUPPORTED),
+    (dict(gran=fq.GROUP, zero_point=fq.ZERO_POINT_MINMAX), fq.FQ_ERR_UNSUPPORTED),
+    (dict(gran=fq.STATIC, zero_point=fq.ZERO_POINT_MINMAX), fq.FQ_ERR_UNSUPPORTED),
     (dict(gran=fq.GROUP, group_size=64), fq.FQ_ERR_UNSUPPORTED),
     (dict(alpha=0.0), fq.FQ_ERR_INVALID),
     (dict(alpha=1.5), fq.FQ_ERR_INVALID),
@@ -129,3 +133,13 @@ def test_workspace_sizes(L):
 def test_debug_timeout_rejects_limits(L):
     assert L.fq_debug_wait_timeout(0, None) == fq.FQ_ERR_INVALID
     assert L.fq_debug_wait_timeout(1000000, None) == fq.FQ_ERR_INVALID
+
+
+def test_zero_point_gemm_needs_its_workspace(L):
+    """The min-max quantizer's GEMM keeps the exact int32 products in the
+    caller's workspace: M * N * 4 bytes, and refuses to run without them."""
+    assert L.fq_gemm_workspace_size(8, 256, 256, fq.ROW_ZP) == 8 * 256 * 4
+    st = L.fq_w4a4_gemm(A, A, A, A, 8, 256, 256, fq.ROW_ZP, A, None, 0, None)
+    assert st == fq.FQ_ERR_INVALID and b"workspace" in L.fq_last_error()
+    ws = L.fq_linear_workspace_size(8, 256, 256, fq.ROW_ZP)
+    assert ws >= 8 * 128 + 3 * 8 * 4 + 8 * 256 * 4

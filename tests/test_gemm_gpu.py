@@ -133,3 +133,23 @@ def test_gemm_persistent_exact(m, n, k):
     C.check_fp16_exact(C.host(fq.fq_w4a4_gemm(A, None, B, C.dev(sw), fq.STATIC, workspace=ws)), refs)
     C.check_fp16_exact(C.host(fq.fq_w4a4_gemm_noalloc(A, C.dev(sx), B, C.dev(sw), fq.ROW)), ref)
     fq.fq_check_device_error()
+
+
+def test_gemm_persistent_stress_repeated():
+    """The CTA-pair GEMM 50 times, interleaving tile counts from 1 to 512 (so the
+    pairs' share of tiles and the cross-CTA barrier phases differ from launch
+    to launch): every launch bit-exact, no bounded wait giving up."""
+    shapes = [(256, 256, 512), (1024, 2048, 512), (2048, 10240, 256), (640, 776, 1024), (4096, 8192, 256)]
+    cases = []
+    for i, (m, n, k) in enumerate(shapes):
+        a, b = _operands(17 * i + 1, m, n, k)
+        g = synth.generator(i + 40)
+        sx, sw = synth.random_scales(g, m), synth.random_scales(g, n)
+        ref = O.dequant_row(O.gemm_int(C.unpack(a), C.unpack(b)), sx, sw)
+        ws = torch.empty(max(fq.fq_gemm_workspace_size(m, n, k, fq.ROW), 256), dtype=torch.uint8, device="cuda")
+        cases.append((C.dev(a), C.dev(sx), C.dev(b), C.dev(sw), ws, C.dev(ref.view(np.uint16).astype(np.int16))))
+    for it in range(50):
+        A, SX, B, SW, ws, ref = cases[(it * 3) % len(cases)]
+        y = fq.fq_w4a4_gemm(A, SX, B, SW, fq.ROW, workspace=ws)
+        assert torch.equal(y.view(torch.int16), ref), f"launch {it} differs"
+    fq.fq_check_device_error()

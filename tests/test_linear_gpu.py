@@ -1,7 +1,22 @@
-"""fq_linear end to end at the workloads' full sizes, in the launch
-configuration the benchmark times, against the CPU oracle on sampled outputs."""
+"""The linear layer at the workloads' full sizes, in the launch configuration
+the benchmark times, against the CPU oracle.
+
+Each full-size case runs the layer three ways on the same device inputs:
+fq_linear (the product call), and its two halves as the benchmark calls them
+(fq_quant_act, then fq_w4a4_gemm with a preallocated workspace), plus the
+debug quantization that also returns the transformed values.  The halves must
+reproduce fq_linear bit for bit.  Then, on rows and columns sampled so that
+every 256 x 256 output tile is hit:
+* the quantization is checked against the oracle (transformed values, scales,
+  codes; see gpu_checks), and
+* the GEMM is checked DECOUPLED from it: the GPU's own codes and scales go
+  through the oracle's integer GEMM and dequantization, and the fp16 outputs
+  must match bit-exactly (per token, static) or within 1 fp16 ulp / the
+  float32 cancellation bound (group).
+"""
 import numpy as np
 import pytest
+import torch
 
 import gpu_checks as C
 from int4_linear_b200 import fq, synth
@@ -21,46 +36,47 @@ def test_linear_tiny_exact():
     fq.fq_check_device_error()
 
 
-def _samples(seed, m, n, nm=24, nn=384):
-    g = synth.generator(seed)
-    ms = np.unique(np.concatenate([[0, m - 1], g.integers(0, m, nm)]))
-    ns = np.unique(np.concatenate([[0, n - 1], g.integers(0, n, nn)]))
-    return ms, ns
+def _bits(y):
+    return np.asarray(y).view(np.uint16)
 
 
-def _check_sampled(y_gpu, d, ms, ns, gran_o, wgran_o):
-    """Oracle on the sampled token rows and output channels (rows are independent)."""
-    x = d["x"][ms]
-    alpha = d.get("alpha_a", 1.0)
-    qw, sw, _ = O.quant_weight(d["w"][ns], wgran_o, d.get("alpha_w", 1.0))
-    qx, sx, vx = O.quant_act(x, gran_o, alpha, d.get("p1"), d.get("p2"), d.get("c"))
-    yg = y_gpu[np.ix_(ms, ns)].astype(np.float64)
+def _run_three_ways(d, qp, gran, wq, sw, t=None, static_scale=None):
+    """fq_linear, then quant + GEMM (bench's calls), then the debug quantization.
+    Returns (Y, Xq, s_x, xhat) as host arrays (xhat None without a transform)."""
+    X = C.dev(d["x"])
+    m, k = d["x"].shape
+    n = wq.shape[0]
+    y_lin = C.host(fq.fq_linear(X, qp, wq, sw, t, static_scale=static_scale))
+    xq, sx = fq.fq_quant_act(X, qp, t, static_scale)
+    ws = torch.empty(max(fq.fq_gemm_workspace_size(m, n, k, gran), 256), dtype=torch.uint8, device="cuda")
+    y = C.host(fq.fq_w4a4_gemm(xq, sx, wq, sw, gran, workspace=ws))
+    assert np.array_equal(_bits(y), _bits(y_lin)), "fq_linear differs from quantization + GEMM"
+    xhat = None
+    if t is not None:
+        xq_d, sx_d, xhat_d = fq.fq_quant_act_debug(X, qp, t)
+        assert torch.equal(xq_d, xq) and torch.equal(sx_d, sx), "the debug kernel quantized differently"
+        xhat = C.host(xhat_d)
+    fq.fq_check_device_error()
+    return y, C.host(xq), (None if sx is None else C.host(sx)), xhat
+
+
+def _quant_checks(d, rows, gran_o, alpha, xq, sx_rows, xhat):
+    """Transformed values, scales and codes of the sampled rows against the oracle."""
+    q_ref, s_ref, v_ref = O.quant_act(d["x"][rows], gran_o, alpha, d.get("p1"), d.get("p2"), d.get("c"))
+    vg = xhat[rows]
+    qg = C.unpack(xq[rows])
+    worst = C.check_values(vg, v_ref)
+    C.check_own_scales(sx_rows, vg, gran_o, alpha)
+    C.check_own_codes(qg, vg, sx_rows, gran_o)
     if gran_o == O.ROW:
-        ref = O.dequant_row(O.gemm_int(qx, qw), sx, sw).astype(np.float64)
-        ex = C.exempt_mask(vx, sx, sx * (1 + C.TOL_REL), O.ROW) if "p1" in d else np.zeros(qx.shape, bool)
-        wsum = (ex.astype(np.float64) @ np.abs(qw).T.astype(np.float64)) * sx[:, None] * sw[None, :]
-        bound = C.ulp16(ref) + np.abs(ref) * 1.01 * C.TOL_REL + wsum
-        err = np.abs(yg - ref)
-        assert np.all(err <= bound), f"{(err > bound).sum()} outputs beyond the bound (max {err.max()})"
-        exact = (err == 0).mean()
+        C.check_scales_row(sx_rows, s_ref)
     else:
-        ref = O.dequant_group(qx, qw, sx, sw).astype(np.float64)
-        ex = C.exempt_mask(vx, sx, sx * (1 + 2 ** -10), O.GROUPED) if "p1" in d else np.zeros(qx.shape, bool)
-        absum = np.zeros_like(ref)
-        wsum = np.zeros_like(ref)
-        for g in range(qx.shape[1] // O.GROUP):
-            sl = slice(g * O.GROUP, (g + 1) * O.GROUP)
-            s2 = sx[:, g:g + 1].astype(np.float64) * sw[None, :, g].astype(np.float64)
-            absum += np.abs(O.gemm_int(qx[:, sl], qw[:, sl]).astype(np.float64) * s2)
-            wsum += (ex[:, sl].astype(np.float64) @ np.abs(qw[:, sl]).T.astype(np.float64)) * s2
-        ng = qx.shape[1] // O.GROUP
-        slack = 2.0 ** -10 if "p1" in d else 0.0
-        bound = C.ulp16(ref) + (ng * 2.0 ** -23 + slack) * absum + wsum
-        err = np.abs(yg - ref)
-        assert np.all(err <= bound), f"{(err > bound).sum()} outputs beyond the bound (max {err.max()})"
-        exact = (err <= C.ulp16(ref)).mean()
-    print(f"{d['name']}: {len(ms)}x{len(ns)} sampled outputs, exempt act codes {int(ex.sum())}, "
-          f"fraction within 1 ulp/exact {exact:.4f}")
+        C.check_scales_group(sx_rows, s_ref, v_ref, alpha)
+    ex = C.exempt_mask(v_ref, s_ref, sx_rows, gran_o)
+    n_ex, n_diff = C.check_codes(qg, q_ref, ex)
+    print(f"{d['name']}: {len(rows)} rows, max |dv|/max(|v|, 2^-10 amax) {worst:.2e}, "
+          f"boundary-exempt {n_ex}, differing codes {n_diff}")
+    return qg
 
 
 @pytest.mark.parametrize("k,n", synth.PREFILL_8B_SHAPES)
@@ -68,11 +84,16 @@ def test_linear_prefill_8b(k, n):
     """M = 2048 tokens, Kronecker-transformed per-token activations, per-channel weights."""
     d = synth.prefill_linear(k, n, m=2048)
     t = fq.Transform(C.dev(d["p1"]), C.dev(d["p2"]))
-    wq, sw = fq.fq_quant_weight(C.dev(d["w"]), fq.qparams(fq.ROW, 1.0))
-    y = C.host(fq.fq_linear(C.dev(d["x"]), fq.qparams(fq.ROW, 1.0), wq, sw, t))
-    fq.fq_check_device_error()
-    ms, ns = _samples(k + n, 2048, n)
-    _check_sampled(y, d, ms, ns, O.ROW, O.ROW)
+    qp = fq.qparams(fq.ROW, 1.0)
+    wq, sw = fq.fq_quant_weight(C.dev(d["w"]), qp)
+    y, xq, sx, xhat = _run_three_ways(d, qp, fq.ROW, wq, sw, t)
+    rows = C.tile_samples(k + n, d["m"])
+    cols = C.tile_samples(k + n + 1, n)
+    qx = _quant_checks(d, rows, O.ROW, 1.0, xq, sx[rows], xhat)
+    qw, sw_ref, _ = O.quant_weight(d["w"][cols], O.ROW, 1.0)
+    assert np.array_equal(C.host(wq)[cols], O.pack_int4(qw))
+    assert np.array_equal(C.host(sw)[cols], sw_ref)
+    C.check_gemm_decoupled(y[np.ix_(rows, cols)], qx, sx[rows], qw, sw_ref, O.ROW)
 
 
 @pytest.mark.parametrize("k,n", synth.GROUP_70B_SHAPES)
@@ -80,23 +101,33 @@ def test_linear_group_70b(k, n):
     """M = 4096, group-128 scales on both sides, Student-t weights."""
     d = synth.prefill_linear(k, n, m=4096, w_kind="t")
     t = fq.Transform(C.dev(d["p1"]), C.dev(d["p2"]))
-    wq, sw = fq.fq_quant_weight(C.dev(d["w"]), fq.qparams(fq.GROUP, 1.0))
-    y = C.host(fq.fq_linear(C.dev(d["x"]), fq.qparams(fq.GROUP, 1.0), wq, sw, t))
-    fq.fq_check_device_error()
-    ms, ns = _samples(k + n + 1, 4096, n, nm=12, nn=256)
-    _check_sampled(y, d, ms, ns, O.GROUPED, O.GROUPED)
+    qp = fq.qparams(fq.GROUP, 1.0)
+    wq, sw = fq.fq_quant_weight(C.dev(d["w"]), qp)
+    y, xq, sx, xhat = _run_three_ways(d, qp, fq.GROUP, wq, sw, t)
+    rows = C.tile_samples(k + n, d["m"])
+    cols = C.tile_samples(k + n + 1, n)
+    sx_rows = sx.T[rows].astype(np.float32)      # group-major [K/128][M] -> [rows, K/128]
+    qx = _quant_checks(d, rows, O.GROUPED, 1.0, xq, sx_rows, xhat)
+    qw, sw_ref, _ = O.quant_weight(d["w"][cols], O.GROUPED, 1.0)
+    assert np.array_equal(C.host(wq)[cols], O.pack_int4(qw))
+    assert np.array_equal(C.host(sw).T[cols].astype(np.float32), sw_ref)
+    n_canc = C.check_gemm_decoupled(y[np.ix_(rows, cols)], qx, sx_rows, qw, sw_ref, O.GROUPED)
+    print(f"{d['name']}: {len(rows)}x{len(cols)} outputs, {n_canc} within the cancellation bound only")
 
 
 @pytest.mark.parametrize("m", synth.DECODE_TOKENS)
 @pytest.mark.parametrize("k,n", synth.DECODE_70B_SHAPES)
 def test_linear_decode_static(m, k, n):
-    """Static per-channel activation scales migrated into the weights: bit-exact."""
+    """Static per-channel activation scales migrated into the weights: bit-exact
+    (no transform, so the oracle's codes are the GPU's)."""
     d = synth.decode_static(m, k, n)
     s_k = d["static_scale"]
+    qp = fq.qparams(fq.STATIC)
     wq, sw = fq.fq_quant_weight(C.dev(d["w"]), fq.qparams(fq.ROW, 1.0), None, C.dev(s_k))
-    y = C.host(fq.fq_linear(C.dev(d["x"]), fq.qparams(fq.STATIC), wq, sw, static_scale=C.dev(s_k)))
-    fq.fq_check_device_error()
-    ns = _samples(m + k, m, n, nn=1024)[1]
-    qw, sw_ref, _ = O.quant_weight(d["w"][ns], O.ROW, 1.0, qsm_scale=s_k)
-    ref = O.linear(d["x"], qw, sw_ref, O.STATIC, static_scale=s_k)
-    C.check_fp16_exact(y[:, ns], ref)
+    y, xq, _, _ = _run_three_ways(d, qp, fq.STATIC, wq, sw, static_scale=C.dev(s_k))
+    cols = C.tile_samples(m + k, n)
+    q_ref, _, _ = O.quant_act(d["x"], O.STATIC, static_scale=s_k)
+    assert np.array_equal(xq, O.pack_int4(q_ref))
+    qw, sw_ref, _ = O.quant_weight(d["w"][cols], O.ROW, 1.0, qsm_scale=s_k)
+    assert np.array_equal(C.host(wq)[cols], O.pack_int4(qw))
+    C.check_gemm_decoupled(y[:, cols], q_ref, None, qw, sw_ref, O.STATIC)
