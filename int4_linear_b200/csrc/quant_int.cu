@@ -62,7 +62,7 @@ struct QuantTcParams {
 
 namespace {
 
-constexpr int kIntThreads = 128;
+constexpr int kIntThreads = 256;
 constexpr float kMagic = 12582912.0f;       // 1.5 * 2^23
 constexpr uint32_t kMagicBits = 0x4B400000u;
 
@@ -84,16 +84,25 @@ struct IC {
   // so both can share the bytes
   static constexpr int XU = (XL * X_PL > BG * 4 * U_PL) ? XL * X_PL : BG * 4 * U_PL;
   static constexpr int OFF_U = OFF_X;
-  static constexpr int OFF_RED = OFF_X + XU;
-  // reduction scratch (32-bit words): [4] warp maxima, [2][128] group maxima
-  // (uint bits), [2][128] group scales, [2][128] their inverses
+  // the item's packed codes (G tokens of up to NP * N2 / 2 bytes), written to
+  // global memory by one bulk copy
+  static constexpr int CODE = G * NP * N2 / 2;
+  static constexpr int OFF_CODE = OFF_X + XU;
+  static constexpr int OFF_RED = OFF_CODE + CODE;
+  // tensor memory: stage A's four level blocks (256 columns), stage B's five
+  // blocks reuse them; with four stage-B chunks (NP = 128) the float values
+  // of the row wait in columns 256..383 for the token's scale
+  static constexpr int TMEM_COLS = NP == 128 ? 512 : 256;
+  static constexpr int STASH = 256;
+  // reduction scratch (32-bit words): [8] warp maxima, [2][128] halves of
+  // the tile rows' maxima, [8][64] group maxima (uint bits), [2][64] group scales
   static constexpr int R_WARP = 0;
-  static constexpr int R_GMAX = 4;
-  static constexpr int R_SG = R_GMAX + 2 * 128;
-  static constexpr int R_SINV = R_SG + 2 * 128;
-  static constexpr int R_WORDS = R_SINV + 2 * 128;
-  static constexpr int OFF_BAR = OFF_RED + R_WORDS * 4;
-  static constexpr int OFF_CONST = OFF_BAR + 8;  // ints: [0] f2, [1] f1, [4] tensor memory, [8 + 2 s + c] t
+  static constexpr int R_XM = 8;
+  static constexpr int R_GMAX = R_XM + 2 * 128;
+  static constexpr int R_SG = R_GMAX + 8 * 64;
+  static constexpr int R_WORDS = R_SG + 2 * 64;
+  static constexpr int OFF_BAR = OFF_RED + R_WORDS * 4;  // [0] MMA completion, [1] factor loads
+  static constexpr int OFF_CONST = OFF_BAR + 16;  // ints: [0] f2, [1] f1, [4] tensor memory, [8 + 2 s + c] t
   static constexpr int SMEM = OFF_CONST + 64 + 1024;
   static_assert(N2 == 64 || N2 == 128, "n2");
   static_assert(NP == 64 || NP == 128, "padded n1");
@@ -251,67 +260,79 @@ struct RowB {
 };
 
 template <int N2, int NP, int GRAN, bool HAS_C>
-__global__ void __launch_bounds__(kIntThreads) quant_act_int_kernel(const QuantTcParams p) {
+__global__ void __launch_bounds__(kIntThreads, (N2 == 64 ? 2 : 1)) quant_act_int_kernel(const QuantTcParams p) {
   using C = IC<N2, NP, HAS_C>;
   constexpr int G = C::G, XL = C::XL;
+  constexpr int H2 = N2 / 2;  // tile columns (l, or j) per thread: a row's two halves
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const int r = t & 127, h = t >> 7;  // the row (tensor-memory lane) and the half of it this thread owns
   const int n1 = p.n1, K = p.K, M = p.M;
   const int nitems = (M + G - 1) / G;
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + C::OFF_BAR);
   int* cst = reinterpret_cast<int*>(sm + C::OFF_CONST);  // [0] f2 [1] f1 [4] tmem [8 + 2 s + c] t of V
   uint32_t* red = reinterpret_cast<uint32_t*>(sm + C::OFF_RED);
   float* sg = reinterpret_cast<float*>(red + C::R_SG);
-  float* sinv = reinterpret_cast<float*>(red + C::R_SINV);
+  float* xm = reinterpret_cast<float*>(red + C::R_XM);
   uint32_t* gmax = red + C::R_GMAX;
   const uint32_t sbase = smem_u32(sm);
-  (void)sinv;
 
+  uint64_t* lbar = bar + 1;
   if (t == 0) {
     mbar_init(bar, 1);
+    mbar_init(lbar, 1);
     fence_mbar_init();
   }
   if (warp == 0) {
-    tmem_alloc(reinterpret_cast<uint32_t*>(cst + 4), 256);
+    tmem_alloc(reinterpret_cast<uint32_t*>(cst + 4), C::TMEM_COLS);
     tmem_relinquish();
   }
+  __syncthreads();
   // The next kernel may be scheduled once every CTA of this one runs.  The
   // factors are parameters (no kernel of this library writes them) and are
   // prepared below while the kernels ahead on the stream may still run; the
   // activations, c and the outputs are touched only after pdl_wait().
   pdl_launch_dependents();
 
-  // ---- factors: fixed-point exponents and stacked limbs
+  // ---- factors: staged as float32 in the operand bytes (one bulk copy each
+  // when aligned), then fixed-point exponents and stacked limbs
   {
-    float m2 = 0.f, m1 = 0.f;
-    for (int e = t; e < N2 * N2; e += kIntThreads) m2 = fmaxf(m2, fabsf(__ldg(p.P2 + e)));
-    for (int e = t; e < n1 * n1; e += kIntThreads) m1 = fmaxf(m1, fabsf(__ldg(p.P1 + e)));
-    m2 = __uint_as_float(warp_max_u32(__float_as_uint(m2)));
-    m1 = __uint_as_float(warp_max_u32(__float_as_uint(m1)));
-    if (lane == 0) {
-      red[2 * warp + 0] = __float_as_uint(m2);
-      red[2 * warp + 1] = __float_as_uint(m1);
-    }
-    __syncthreads();
-    if (t == 0) {
-      float a = 0.f, b = 0.f;
-      for (int w = 0; w < 4; ++w) {
-        a = fmaxf(a, __uint_as_float(red[2 * w]));
-        b = fmaxf(b, __uint_as_float(red[2 * w + 1]));
+    float* sf = reinterpret_cast<float*>(sm + C::OFF_X);
+    auto stage = [&](const float* src, int count, uint32_t parity) {
+      const uint32_t bytes = uint32_t(count) * 4u;
+      const bool bulk = (reinterpret_cast<uintptr_t>(src) & 15u) == 0 && (bytes & 15u) == 0;
+      if (bulk) {
+        if (t == 0) {
+          mbar_arrive_expect_tx(lbar, bytes);
+          bulk_load(sf, src, bytes, lbar);
+        }
+        if (!mbar_wait(lbar, parity)) record_error(p.err, kErrTimeoutProducer);
+      } else {
+        for (int e = t; e < count; e += kIntThreads) sf[e] = __ldg(src + e);
+        __syncthreads();
       }
-      cst[0] = a > 0.f ? ilog2f(a) - 29 : 0;  // |P2| * 2^-f2 < 2^30
-      cst[1] = b > 0.f ? ilog2f(b) - 29 : 0;
-    }
-    __syncthreads();
-    const int f2 = cst[0], f1 = cst[1];
-    const float s2 = pow2f(-f2), s1 = pow2f(-f1);
+    };
+    auto maxabs = [&](int count) {
+      float m = 0.f;
+      for (int e = t; e < count; e += kIntThreads) m = fmaxf(m, fabsf(sf[e]));
+      m = __uint_as_float(warp_max_u32(__float_as_uint(m)));
+      if (lane == 0) red[C::R_WARP + warp] = __float_as_uint(m);
+      __syncthreads();
+      float a = 0.f;
+#pragma unroll
+      for (int w = 0; w < kIntThreads / 32; ++w) a = fmaxf(a, __uint_as_float(red[C::R_WARP + w]));
+      return a > 0.f ? ilog2f(a) - 29 : 0;  // |P| * 2^-f < 2^30
+    };
     // P2 stacks: chunk c, row (3 - b) * 64 + l', byte j = limb b of P2[j][64 c + l']
+    stage(p.P2, N2 * N2, 0);
+    const int f2 = maxabs(N2 * N2);
+    const float s2 = pow2f(-f2);
     for (int e = t; e < N2 * (N2 / 4); e += kIntThreads) {
       const int l = e % N2, j0 = (e / N2) * 4;
       uint32_t y[4];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) y[q] = uint32_t(__float2int_rn(__ldg(p.P2 + (j0 + q) * N2 + l) * s2)) + 0x80808080u;
+      for (int q = 0; q < 4; ++q) y[q] = uint32_t(__float2int_rn(sf[(j0 + q) * N2 + l] * s2)) + 0x80808080u;
       uint32_t w[4];
       planes4(y[0], y[1], y[2], y[3], w);
       uint8_t* stk = sm + C::OFF_P2 + (l >> 6) * C::P2_CH;
@@ -319,15 +340,20 @@ __global__ void __launch_bounds__(kIntThreads) quant_act_int_kernel(const QuantT
       for (int b = 0; b < 4; ++b)
         *reinterpret_cast<uint32_t*>(stk + krow_offset<N2>(uint32_t((3 - b) * 64 + (l & 63)), uint32_t(j0))) = w[b];
     }
+    fence_proxy_async_smem();
+    __syncthreads();  // P2 read: the staging bytes take P1
     // P1 stacks: chunk kc (32 columns k), row (3 - b) * 32 + k', byte i = limb b
     // of P1[i][32 kc + k'] (0 past n1); rows 128..159 of a chunk are zero
+    stage(p.P1, n1 * n1, 1);
+    const int f1 = maxabs(n1 * n1);
+    const float s1 = pow2f(-f1);
     for (int e = t; e < NP * (NP / 4); e += kIntThreads) {
       const int k = e % NP, i0 = (e / NP) * 4;
       uint32_t y[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const int i = i0 + q;
-        const int v = (i < n1 && k < n1) ? __float2int_rn(__ldg(p.P1 + i * n1 + k) * s1) : 0;
+        const int v = (i < n1 && k < n1) ? __float2int_rn(sf[i * n1 + k] * s1) : 0;
         y[q] = uint32_t(v) + 0x80808080u;
       }
       uint32_t w[4];
@@ -338,9 +364,13 @@ __global__ void __launch_bounds__(kIntThreads) quant_act_int_kernel(const QuantT
         *reinterpret_cast<uint32_t*>(stk + krow_offset<NP>(uint32_t((3 - b) * 32 + (k & 31)), uint32_t(i0))) = w[b];
     }
     for (int e = t; e < C::KCB * 32 * (NP / 16); e += kIntThreads) {
-      const int kc = e / (32 * (NP / 16)), r = (e / (NP / 16)) % 32, c16 = e % (NP / 16);
-      *reinterpret_cast<uint4*>(sm + C::OFF_P1 + kc * C::P1_CH + krow_offset<NP>(uint32_t(128 + r), uint32_t(16 * c16))) =
+      const int kc = e / (32 * (NP / 16)), rr = (e / (NP / 16)) % 32, c16 = e % (NP / 16);
+      *reinterpret_cast<uint4*>(sm + C::OFF_P1 + kc * C::P1_CH + krow_offset<NP>(uint32_t(128 + rr), uint32_t(16 * c16))) =
           make_uint4(0, 0, 0, 0);
+    }
+    if (t == 0) {
+      cst[0] = f2;
+      cst[1] = f1;
     }
   }
   fence_proxy_async_smem();
@@ -349,70 +379,94 @@ __global__ void __launch_bounds__(kIntThreads) quant_act_int_kernel(const QuantT
   tc_fence_after();
   const uint32_t tmem = uint32_t(cst[4]);
   const int f2 = cst[0], f1 = cst[1];
-  const uint32_t lane_off = uint32_t(warp * 32) << 16;
+  const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
   const uint32_t xbase = sbase + C::OFF_X, ubase = sbase + C::OFF_U;
   const uint32_t p2base = sbase + C::OFF_P2, p1base = sbase + C::OFF_P1;
   pdl_wait();  // X, c and the outputs may be touched from here on
 
   uint32_t ph = 0;
   bool bad = false;
+  // this thread's tile row of an item: (token s, tile row i), columns [h H2, h H2 + H2)
+  const int s = G == 2 ? (r >> 6) : 0, i = G == 2 ? (r & 63) : r;
+  auto load_row = [&](int item, uint4 (&raw)[H2 / 8]) {
+    const int tok = item * G + s;
+    const bool ok = item < nitems && i < n1 && tok < M;
+    const __half* xrow = p.X + size_t(tok) * K + size_t(i) * N2 + h * H2;
+#pragma unroll
+    for (int q = 0; q < H2 / 8; ++q) raw[q] = ok ? *reinterpret_cast<const uint4*>(xrow + 8 * q) : make_uint4(0, 0, 0, 0);
+  };
+  uint4 raw[H2 / 8];
+  load_row(blockIdx.x, raw);
   for (int item = blockIdx.x; item < nitems && !bad; item += gridDim.x) {
     const int tok0 = item * G;
+    // the previous item's code tile has been read by its bulk copy before
+    // any thread writes this item's codes (several barriers lie between)
+    if (t == 0) bulk_wait_group_read<0>();
     // ---------------------------------------------------------------- 1. tile row -> limbs
-    const int s = G == 2 ? (t >> 6) : 0, i = G == 2 ? (t & 63) : t;
     const int tok = tok0 + s;
     const bool rv = i < n1 && tok < M;
-    uint4 raw[N2 / 8];
-    const __half* xrow = p.X + size_t(tok) * K + size_t(i) * N2;
+    const float4* crow = HAS_C ? reinterpret_cast<const float4*>(p.c + size_t(i) * N2 + h * H2) : nullptr;
+    float mh = 0.f;
 #pragma unroll
-    for (int q = 0; q < N2 / 8; ++q) raw[q] = rv ? *reinterpret_cast<const uint4*>(xrow + 8 * q) : make_uint4(0, 0, 0, 0);
-    const float* crow = HAS_C ? p.c + size_t(i) * N2 : nullptr;
-    float mx = 0.f;
-#pragma unroll
-    for (int q = 0; q < N2 / 8; ++q) {
+    for (int q = 0; q < H2 / 8; ++q) {
       const __half2* h2 = reinterpret_cast<const __half2*>(&raw[q]);
+      float4 c0 = make_float4(1.f, 1.f, 1.f, 1.f), c1 = c0;
+      if (HAS_C && rv) {
+        c0 = __ldg(crow + 2 * q);
+        c1 = __ldg(crow + 2 * q + 1);
+      }
+      const float cv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         float2 v = __half22float2(h2[u]);
-        if (HAS_C && rv) {
-          v.x = __fmul_rn(v.x, __ldg(crow + 8 * q + 2 * u));
-          v.y = __fmul_rn(v.y, __ldg(crow + 8 * q + 2 * u + 1));
+        if (HAS_C) {
+          v.x = __fmul_rn(v.x, cv[2 * u]);
+          v.y = __fmul_rn(v.y, cv[2 * u + 1]);
         }
-        mx = fmaxf(mx, fmaxf(fabsf(v.x), fabsf(v.y)));
+        mh = fmaxf(mh, fmaxf(fabsf(v.x), fabsf(v.y)));
       }
     }
+    // the row's largest |x c| from its two halves
+    xm[h * 128 + r] = mh;
+    __syncthreads();
+    const float mx = fmaxf(xm[r], xm[128 + r]);
     const int ei = mx > 0.f ? ilog2f(mx) - 29 : 0;  // |x c| 2^-e < 2^30
     {
       const float sc = pow2f(-ei);
       uint8_t* xs = sm + C::OFF_X;
 #pragma unroll
-      for (int q0 = 0; q0 < N2 / 16; ++q0) {  // 16 values: raw[2 q0], raw[2 q0 + 1]
+      for (int q0 = 0; q0 < H2 / 16; ++q0) {  // 16 values: raw[2 q0], raw[2 q0 + 1]
         uint32_t y[16];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const __half2* h2 = reinterpret_cast<const __half2*>(&raw[2 * q0 + h]);
+        for (int hh = 0; hh < 2; ++hh) {
+          const __half2* h2 = reinterpret_cast<const __half2*>(&raw[2 * q0 + hh]);
+          float4 c0 = make_float4(0.f, 0.f, 0.f, 0.f), c1 = c0;
+          if (HAS_C && rv) {
+            c0 = __ldg(crow + 2 * (2 * q0 + hh));
+            c1 = __ldg(crow + 2 * (2 * q0 + hh) + 1);
+          }
+          const float cv8[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             const float2 v = __half22float2(h2[u]);
 #pragma unroll
             for (int z = 0; z < 2; ++z) {
               const float x = z ? v.y : v.x;
-              const int jj = 16 * q0 + 8 * h + 2 * u + z;
               // x (times c) exactly as hi + lo, then round(x c 2^-e) as A * 256 + B
               // with both parts in the range where adding 1.5 * 2^23 rounds to an
               // integer (|A| <= 2^22, |B| <= 2^7 + 1)
               float hi = x, lo = 0.f;
               if (HAS_C) {
-                const float cv = rv ? __ldg(crow + jj) : 0.f;
+                const float cv = cv8[2 * u + z];
                 hi = __fmul_rn(x, cv);
                 lo = __fmaf_rn(x, cv, -hi);
               }
               const float af = __fmaf_rn(hi, sc * (1.0f / 256.0f), kMagic);
               const float Af = __fsub_rn(af, kMagic);
-              const float r = __fmaf_rn(Af, -256.0f * pow2f(ei), hi);
-              const float bf = __fmaf_rn(HAS_C ? __fadd_rn(r, lo) : r, sc, kMagic);
+              const float rr = __fmaf_rn(Af, -256.0f * pow2f(ei), hi);
+              const float bf = __fmaf_rn(HAS_C ? __fadd_rn(rr, lo) : rr, sc, kMagic);
               const int Ai = int(__float_as_uint(af) - kMagicBits), Bi = int(__float_as_uint(bf) - kMagicBits);
-              y[8 * h + 2 * u + z] = uint32_t(Ai * 256 + Bi) + 0x80808080u;
+              y[8 * hh + 2 * u + z] = uint32_t(Ai * 256 + Bi) + 0x80808080u;
             }
           }
         }
@@ -421,10 +475,12 @@ __global__ void __launch_bounds__(kIntThreads) quant_act_int_kernel(const QuantT
         for (int g4 = 0; g4 < 4; ++g4) planes4(y[4 * g4], y[4 * g4 + 1], y[4 * g4 + 2], y[4 * g4 + 3], w[g4]);
 #pragma unroll
         for (int a = 0; a < XL; ++a)
-          *reinterpret_cast<uint4*>(xs + a * C::X_PL + krow_offset<N2>(uint32_t(t), uint32_t(16 * q0))) =
+          *reinterpret_cast<uint4*>(xs + a * C::X_PL + krow_offset<N2>(uint32_t(r), uint32_t(h * H2 + 16 * q0))) =
               make_uint4(w[0][a], w[1][a], w[2][a], w[3][a]);
       }
     }
+    // the next item's rows load while this item runs
+    load_row(item + gridDim.x, raw);
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -433,8 +489,9 @@ __global__ void __launch_bounds__(kIntThreads) quant_act_int_kernel(const QuantT
     // V = U 2^-t per (token, 64-column chunk of l): t from the chunk's
     // largest |U| (its scale only has to be common along the contraction
     // index i of stage B).  Row (s, i) holds U = W 2^(8 (XL - 1) + e_i + f2)
-    // with W = hi 2^16 + lo; |lo| < 2^31 bounds the low part.
-    int vv[C::LCH][64];
+    // with W = hi 2^16 + lo; |lo| < 2^31 bounds the low part.  This thread
+    // takes columns l in [32 h, 32 h + 32) of each chunk.
+    int vv[C::LCH][32];
 #pragma unroll
     for (int ch = 0; ch < C::LCH; ++ch) {
       if (t == 0) {
@@ -445,33 +502,36 @@ __global__ void __launch_bounds__(kIntThreads) quant_act_int_kernel(const QuantT
       if (!warp_wait(bar, ph)) bad = true;
       ph ^= 1u;
       tc_fence_after();
-      // pass 1: this row's largest |hi|, in units common to the token's rows
-      uint32_t mh = 0;
+      // pass 1: the largest |hi| of this row half, in units common to the token's rows
+      uint32_t mhi = 0;
 #pragma unroll
-      for (int sl = 0; sl < 4; ++sl) {
+      for (int sl = 0; sl < 2; ++sl) {
         uint32_t d0[16], d1[16];
-        tmem_ld_32x16(tmem + lane_off + uint32_t(16 * sl), *reinterpret_cast<uint32_t(*)[32]>(d0));
-        tmem_ld_32x16(tmem + lane_off + uint32_t(16 * sl + 64), *reinterpret_cast<uint32_t(*)[32]>(d1));
+        const uint32_t col = uint32_t(32 * h + 16 * sl);
+        tmem_ld_32x16(tmem + lane_off + col, *reinterpret_cast<uint32_t(*)[32]>(d0));
+        tmem_ld_32x16(tmem + lane_off + col + 64u, *reinterpret_cast<uint32_t(*)[32]>(d1));
         tmem_wait_ld();
 #pragma unroll
-        for (int q = 0; q < 16; ++q) mh = max(mh, uint32_t(abs(int(d0[q]) * 256 + int(d1[q]))));
+        for (int q = 0; q < 16; ++q) mhi = max(mhi, uint32_t(abs(int(d0[q]) * 256 + int(d1[q]))));
       }
-      const float rowmax = mx > 0.f ? (float(mh) + 32768.0f) * pow2f(16 + ei) : 0.f;
+      const float rowmax = mx > 0.f ? (float(mhi) + 32768.0f) * pow2f(16 + ei) : 0.f;
       const uint32_t wmx = warp_max_u32(__float_as_uint(rowmax));
       if (lane == 0) red[C::R_WARP + warp] = wmx;
       bad = __syncthreads_or(bad);
       if (t < G) {
+        // token t: rows [64 t, 64 t + 64) (G = 2: warps 2t, 2t + 1 and their second halves), else all
         float tm = 0.f;
-        for (int w = (G == 2 ? 2 * t : 0); w < (G == 2 ? 2 * t + 2 : 4); ++w) tm = fmaxf(tm, __uint_as_float(red[C::R_WARP + w]));
+        for (int w = 0; w < kIntThreads / 32; ++w)
+          if (G == 1 || ((w & 3) >> 1) == t) tm = fmaxf(tm, __uint_as_float(red[C::R_WARP + w]));
         // |V| = |U| 2^-t < 2^29
         cst[8 + 2 * t + ch] = tm > 0.f ? ilog2f(tm) + 1 + 8 * (XL - 1) + f2 - 29 : 0;
       }
       __syncthreads();
       const int n = min(63, max(0, cst[8 + 2 * s + ch] - ei - f2 - 8 * (XL - 1)));
 #pragma unroll
-      for (int sl = 0; sl < 4; ++sl) {
+      for (int sl = 0; sl < 2; ++sl) {
         uint32_t d[4][16];
-        load_levels16(tmem + lane_off + uint32_t(16 * sl), d);
+        load_levels16(tmem + lane_off + uint32_t(32 * h + 16 * sl), d);
         tmem_wait_ld();
 #pragma unroll
         for (int q = 0; q < 16; ++q) vv[ch][16 * sl + q] = int(combine_levels(d[0][q], d[1][q], d[2][q], d[3][q]) >> n);
@@ -488,7 +548,7 @@ __global__ void __launch_bounds__(kIntThreads) quant_act_int_kernel(const QuantT
 #pragma unroll
       for (int ch = 0; ch < C::LCH; ++ch) {
 #pragma unroll
-        for (int q0 = 0; q0 < 4; ++q0) {
+        for (int q0 = 0; q0 < 2; ++q0) {
           uint32_t w[4][4];
 #pragma unroll
           for (int g4 = 0; g4 < 4; ++g4) {
@@ -496,7 +556,7 @@ __global__ void __launch_bounds__(kIntThreads) quant_act_int_kernel(const QuantT
             planes4(uint32_t(vv[ch][l]) + 0x80808080u, uint32_t(vv[ch][l + 1]) + 0x80808080u,
                     uint32_t(vv[ch][l + 2]) + 0x80808080u, uint32_t(vv[ch][l + 3]) + 0x80808080u, w[g4]);
           }
-          const int m0 = (N2 == 64 ? s * 64 : ch * 64) + 16 * q0;
+          const int m0 = (N2 == 64 ? s * 64 : ch * 64) + 32 * h + 16 * q0;
 #pragma unroll
           for (int b = 0; b < 4; ++b)
             *reinterpret_cast<uint4*>(ub + b * C::U_PL + sw128_offset(uint32_t(i), uint32_t(m0))) =
@@ -511,20 +571,35 @@ __global__ void __launch_bounds__(kIntThreads) quant_act_int_kernel(const QuantT
     // Per 32-column chunk of k: five level blocks of 32 columns (weights
     // 256^6 .. 256^2 of V's limbs times P1's), so that the rows of V far
     // below its largest one (an outlier row sets the token's scale) keep
-    // their full precision.
+    // their full precision.  This thread takes k in [16 h, 16 h + 16) of each
+    // chunk.  The packed codes of the item go to a shared-memory tile and
+    // leave in one bulk copy.
+    uint8_t* ctile = sm + C::OFF_CODE;
     for (int g = 0; g < C::BG && !bad; ++g) {
-      const int sb = RowB<N2, G>::token(t, g);
-      const int l = RowB<N2, G>::col(t);
+      const int sb = RowB<N2, G>::token(r, g);
+      const int l = RowB<N2, G>::col(r);
       const int tk = tok0 + sb;
       const bool tok_ok = tk < M;
+      uint8_t* crow_t = ctile + sb * (K / 2);  // this row's token in the tile
       // X̂ = W' 2^(16 + t + f1), W' = D0 2^32 + D1 2^24 + D2 2^16 + D3 2^8 + D4,
       // t of this row's (token, l-chunk)
       const int Es = 16 + cst[8 + 2 * sb + (N2 == 128 ? (l >> 6) : 0)] + f1;
       const float up = pow2f(Es);
-      float fv[NP];
+      constexpr bool kStash = C::TMEM_COLS == 512;  // four chunks: the values wait in tensor memory
+      float fv[kStash ? 16 : NP / 2];
       float tmax = 0.f;
+      // 8 codes (k = kbase .. kbase + 7 of this row's column l) into the tile
+      auto put_codes = [&](int kbase, uint32_t word) {
+        word = transpose_nibbles8(word, lane);
+        const int kr = kbase + (lane & 7);
+        if (tok_ok && kr < n1)
+          *reinterpret_cast<uint32_t*>(crow_t + (size_t(kr) * N2 + (l & ~7)) / 2) = word;
+      };
+      // the 4 warps (n2 = 128) or 2 warps (n2 = 64, token sb) that hold half hh of the chunk
+      auto half_warp = [&](int tt, int hh, int q) { return N2 == 128 ? 4 * hh + q : 4 * hh + 2 * tt + q; };
 #pragma unroll
       for (int kc = 0; kc < C::KCB; ++kc) {
+        float* fc = fv + (kStash ? 0 : 16 * kc);
         if (t == 0) {
           tc_fence_after();
           issue_stage<4, 5, 32, NP / 32, true, 0, C::U_PL, NP>(tmem, ubase + uint32_t(g * 4 * C::U_PL),
@@ -534,12 +609,11 @@ __global__ void __launch_bounds__(kIntThreads) quant_act_int_kernel(const QuantT
         if (!warp_wait(bar, ph)) bad = true;
         ph ^= 1u;
         tc_fence_after();
-#pragma unroll
-        for (int sl = 0; sl < 2; ++sl) {
+        {
           uint32_t d[5][16];
 #pragma unroll
           for (int bk = 0; bk < 5; ++bk)
-            tmem_ld_32x16(tmem + lane_off + uint32_t(32 * bk + 16 * sl), *reinterpret_cast<uint32_t(*)[32]>(d[bk]));
+            tmem_ld_32x16(tmem + lane_off + uint32_t(32 * bk + 16 * h), *reinterpret_cast<uint32_t(*)[32]>(d[bk]));
           tmem_wait_ld();
 #pragma unroll
           for (int q = 0; q < 16; ++q) {
@@ -551,9 +625,16 @@ __global__ void __launch_bounds__(kIntThreads) quant_act_int_kernel(const QuantT
             const int mid = int(d[2][q]) * 256 + int(d[3][q]);
             const float f = __fmaf_rn(__int2float_rn(hi), 16777216.0f,
                                       __fmaf_rn(__int2float_rn(mid), 256.0f, __int2float_rn(int(d[4][q]))));
-            fv[32 * kc + 16 * sl + q] = f;
+            fc[q] = f;
             tmax = fmaxf(tmax, fabsf(f));
           }
+        }
+        if (kStash && GRAN == FQ_DYNAMIC_ROW) {
+          uint32_t u[16];
+#pragma unroll
+          for (int q = 0; q < 16; ++q) u[q] = __float_as_uint(fc[q]);
+          tmem_st_32x16(tmem + lane_off + uint32_t(C::STASH + 32 * kc + 16 * h), u);
+          tmem_wait_st();
         }
         tc_fence_before();
         bad = __syncthreads_or(bad);  // D read by every thread: free for the next MMA
@@ -561,20 +642,22 @@ __global__ void __launch_bounds__(kIntThreads) quant_act_int_kernel(const QuantT
           // groups: n2 = 128 -> row k (all 128 rows of D); n2 = 64 -> rows k, k + 1 of token sb (64 rows)
           constexpr int KPG = 128 / N2;
 #pragma unroll
-          for (int k = 0; k < 32; k += KPG) {
-            float a = fabsf(fv[32 * kc + k]);
-            if (KPG == 2) a = fmaxf(a, fabsf(fv[32 * kc + k + 1]));
-            const uint32_t r = warp_max_u32(__float_as_uint(a * up));  // exact: a power of two
-            if (lane == 0) gmax[warp * 64 + k / KPG] = r;
+          for (int k = 0; k < 16; k += KPG) {
+            float a = fabsf(fc[k]);
+            if (KPG == 2) a = fmaxf(a, fabsf(fc[k + 1]));
+            const uint32_t rx = warp_max_u32(__float_as_uint(a * up));  // exact: a power of two
+            if (lane == 0) gmax[warp * 64 + k / KPG] = rx;
           }
           __syncthreads();
-          // group scales of this chunk: n2 = 128: 32 groups, over 4 warps;
-          // n2 = 64: 16 groups per token, over the token's 2 warps
+          // group scales of this chunk: n2 = 128: 32 groups (k), over the 4 warps of
+          // the k's half; n2 = 64: 16 groups (k pairs) per token, over 2 warps
           if (t < 32) {
             const int tt = N2 == 128 ? 0 : (t >> 4), gi = N2 == 128 ? t : (t & 15);
-            const int w0 = N2 == 128 ? 0 : 2 * tt, nw = N2 == 128 ? 4 : 2;
+            const int per_half = N2 == 128 ? 16 : 8;  // groups per half of the chunk
+            const int hh = gi / per_half, gl = gi % per_half;
+            const int nw = N2 == 128 ? 4 : 2;
             float am = 0.f;
-            for (int w = w0; w < w0 + nw; ++w) am = fmaxf(am, __uint_as_float(gmax[w * 64 + gi]));
+            for (int q = 0; q < nw; ++q) am = fmaxf(am, __uint_as_float(gmax[half_warp(tt, hh, q) * 64 + gl]));
             const __half sh = group_scale_h(am, p.alpha);
             sg[tt * 64 + gi] = __half2float(sh);
             const int tkk = tok0 + (N2 == 128 ? g : tt);
@@ -584,95 +667,114 @@ __global__ void __launch_bounds__(kIntThreads) quant_act_int_kernel(const QuantT
           __syncthreads();
         }
         if (GRAN != FQ_DYNAMIC_ROW) {
-          // codes of this chunk
+          // codes of this chunk half
           const int sidx = N2 == 128 ? 0 : sb;
 #pragma unroll
-          for (int k0 = 0; k0 < 32; k0 += 8) {
+          for (int k0 = 0; k0 < 16; k0 += 8) {
             uint32_t word = 0;
 #pragma unroll
             for (int b = 0; b < 8; ++b) {
-              const int k = kc * 32 + k0 + b;
-              const float v = fv[k] * up;
+              const int kl = 16 * h + k0 + b;  // within the chunk
+              const int k = kc * 32 + kl;
+              const float v = fc[k0 + b] * up;
               int qv;
               if (GRAN == FQ_STATIC_CHANNEL) {
                 qv = (k < n1 && tok_ok) ? code_ieee(v, __ldg(p.sstatic + k * N2 + l)) : 0;
               } else {
-                qv = code_ieee(v, sg[sidx * 64 + (k0 + b) / (128 / N2)]);
+                qv = code_ieee(v, sg[sidx * 64 + kl / (128 / N2)]);
               }
               word = put_nibble(word, qv, 4 * b);
             }
             if (p.xhat && tok_ok) {
 #pragma unroll
-              for (int b = 0; b < 8; ++b)
-                if (kc * 32 + k0 + b < n1) p.xhat[size_t(tk) * K + size_t(kc * 32 + k0 + b) * N2 + l] = fv[kc * 32 + k0 + b] * up;
+              for (int b = 0; b < 8; ++b) {
+                const int k = kc * 32 + 16 * h + k0 + b;
+                if (k < n1) p.xhat[size_t(tk) * K + size_t(k) * N2 + l] = fc[k0 + b] * up;
+              }
             }
-            word = transpose_nibbles8(word, lane);
-            const int kr = kc * 32 + k0 + (lane & 7);
-            if (tok_ok && kr < n1)
-              *reinterpret_cast<uint32_t*>(p.Q + size_t(tk) * (K / 2) + (size_t(kr) * N2 + (l & ~7)) / 2) = word;
+            put_codes(kc * 32 + 16 * h + k0, word);
           }
           if (GRAN == FQ_DYNAMIC_GROUP) __syncthreads();  // sg is rewritten by the next chunk
         }
       }
       if (GRAN == FQ_DYNAMIC_ROW) {
-        // token maximum: n2 = 64 -> warps 2 sb, 2 sb + 1; n2 = 128 -> all four
-        const uint32_t r = warp_max_u32(__float_as_uint(tmax * up));  // exact: a power of two
-        if (lane == 0) red[C::R_WARP + warp] = r;
+        // token maximum: n2 = 64 -> the 4 warps of token sb; n2 = 128 -> all 8
+        const uint32_t rx = warp_max_u32(__float_as_uint(tmax * up));  // exact: a power of two
+        if (lane == 0) red[C::R_WARP + warp] = rx;
         __syncthreads();
         float amax = 0.f;
-        for (int w = (N2 == 64 ? 2 * sb : 0); w < (N2 == 64 ? 2 * sb + 2 : 4); ++w)
-          amax = fmaxf(amax, __uint_as_float(red[C::R_WARP + w]));
+        for (int w = 0; w < kIntThreads / 32; ++w)
+          if (N2 == 128 || ((w & 3) >> 1) == sb) amax = fmaxf(amax, __uint_as_float(red[C::R_WARP + w]));
         const float s_tok = __fdiv_rn(__fmul_rn(amax, p.alpha), 7.0f);
-        if (tok_ok && l == 0) p.s_row[tk] = s_tok;
+        if (tok_ok && l == 0 && h == 0) p.s_row[tk] = s_tok;
         const float ftok = s_tok != 0.f ? (1.0f / s_tok) * up : 0.f;
         // x = fma(f, ftok, 1.5 * 2^23) holds rint(f * ftok) in its low bits;
         // next to a tie (or for s = 0) the IEEE quotient decides
         const float th = 0.5f - (8.0f / fminf(p.alpha, 1.0f) + 1.0f) * 9.5367431640625e-07f;
         const bool clampq = !(p.alpha >= 1.0f);
 #pragma unroll
-        for (int k0 = 0; k0 < NP; k0 += 8) {
-          uint32_t word = 0;
-          bool redo = s_tok == 0.f;
+        for (int kc = 0; kc < C::KCB; ++kc) {
+          float* fc = fv + (kStash ? 0 : 16 * kc);
+          if (kStash) {
+            uint32_t u[16];
+            tmem_ld_32x16(tmem + lane_off + uint32_t(C::STASH + 32 * kc + 16 * h), *reinterpret_cast<uint32_t(*)[32]>(u));
+            tmem_wait_ld();
 #pragma unroll
-          for (int b = 0; b < 8; b += 2) {
-            const float2 dd = make_float2(fv[k0 + b], fv[k0 + b + 1]);
-            float2 x = ffma2(dd, make_float2(ftok, ftok), make_float2(kMagic, kMagic));
-            const float2 rr =
-                ffma2(dd, make_float2(ftok, ftok), ffma2(x, make_float2(-1.f, -1.f), make_float2(kMagic, kMagic)));
-            if (clampq) {
-              x.x = fminf(fmaxf(x.x, kMagic - 8.0f), kMagic + 7.0f);
-              x.y = fminf(fmaxf(x.y, kMagic - 8.0f), kMagic + 7.0f);
+            for (int q = 0; q < 16; ++q) fc[q] = __uint_as_float(u[q]);
+          }
+#pragma unroll
+          for (int k0 = 0; k0 < 16; k0 += 8) {
+            uint32_t word = 0;
+            bool redo = s_tok == 0.f;
+#pragma unroll
+            for (int b = 0; b < 8; b += 2) {
+              const float2 dd = make_float2(fc[k0 + b], fc[k0 + b + 1]);
+              float2 x = ffma2(dd, make_float2(ftok, ftok), make_float2(kMagic, kMagic));
+              const float2 rr =
+                  ffma2(dd, make_float2(ftok, ftok), ffma2(x, make_float2(-1.f, -1.f), make_float2(kMagic, kMagic)));
+              if (clampq) {
+                x.x = fminf(fmaxf(x.x, kMagic - 8.0f), kMagic + 7.0f);
+                x.y = fminf(fmaxf(x.y, kMagic - 8.0f), kMagic + 7.0f);
+              }
+              redo |= fabsf(rr.x) >= th || fabsf(rr.y) >= th;
+              word = put_nibble(word, int(__float_as_uint(x.x)), 4 * b);
+              word = put_nibble(word, int(__float_as_uint(x.y)), 4 * b + 4);
             }
-            redo |= fabsf(rr.x) >= th || fabsf(rr.y) >= th;
-            word = put_nibble(word, int(__float_as_uint(x.x)), 4 * b);
-            word = put_nibble(word, int(__float_as_uint(x.y)), 4 * b + 4);
-          }
-          if (redo) {
-            word = 0;
+            if (redo) {
+              word = 0;
 #pragma unroll
-            for (int b = 0; b < 8; ++b) word = put_nibble(word, code_ieee(fv[k0 + b] * up, s_tok), 4 * b);
-          }
-          if (p.xhat && tok_ok) {
+              for (int b = 0; b < 8; ++b) word = put_nibble(word, code_ieee(fc[k0 + b] * up, s_tok), 4 * b);
+            }
+            if (p.xhat && tok_ok) {
 #pragma unroll
-            for (int b = 0; b < 8; ++b)
-              if (k0 + b < n1) p.xhat[size_t(tk) * K + size_t(k0 + b) * N2 + l] = fv[k0 + b] * up;
+              for (int b = 0; b < 8; ++b) {
+                const int k = kc * 32 + 16 * h + k0 + b;
+                if (k < n1) p.xhat[size_t(tk) * K + size_t(k) * N2 + l] = fc[k0 + b] * up;
+              }
+            }
+            put_codes(kc * 32 + 16 * h + k0, word);
           }
-          word = transpose_nibbles8(word, lane);
-          const int kr = k0 + (lane & 7);
-          if (tok_ok && kr < n1)
-            *reinterpret_cast<uint32_t*>(p.Q + size_t(tk) * (K / 2) + (size_t(kr) * N2 + (l & ~7)) / 2) = word;
         }
         __syncthreads();  // red is reused by the next group / item
       }
     }
+    // the item's codes: one bulk copy of the valid tokens' rows
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (t == 0 && !bad) {
+      const int ntok = min(G, M - tok0);
+      bulk_store(p.Q + size_t(tok0) * (K / 2), ctile, uint32_t(ntok * (K / 2)));
+      bulk_commit_group();
+    }
     if (__syncthreads_or(bad)) break;
   }
   if (bad && t == 0) record_error(p.err, kErrTimeoutMma);
+  if (t == 0) bulk_wait_group<0>();  // the codes are written before the CTA leaves
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, C::TMEM_COLS);
   }
 }
 
@@ -683,9 +785,9 @@ fq_status launch_int4(const QuantTcParams& p, cudaStream_t stream) {
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess ||
       cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
     return fail(FQ_ERR_CUDA, "cannot reserve %d bytes of shared memory for the transform kernel", C::SMEM);
-  int per_sm = 1;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kIntThreads, C::SMEM) != cudaSuccess) per_sm = 1;
-  per_sm = std::max(1, std::min(per_sm, 2));  // 256 tensor-memory columns each
+  // CTAs per SM: 256 tensor-memory columns each (at most 2), and what fits in
+  // the SM's 228 KB of shared memory (1 KB of it reserved per CTA)
+  const int per_sm = (2 * (C::SMEM + 1024) <= 228 * 1024) ? 2 : 1;
   const int nitems = (p.M + C::G - 1) / C::G;
   const int grid = std::max(1, std::min(nitems, sm_count() * per_sm));
   const cudaError_t e = launch_pdl(kern, dim3(grid), dim3(kIntThreads), C::SMEM, stream, p);
