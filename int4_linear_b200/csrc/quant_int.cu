@@ -91,9 +91,13 @@ struct IC {
   static constexpr int OFF_RED = OFF_CODE + CODE;
   // tensor memory: stage A's four level blocks (256 columns), stage B's five
   // blocks reuse them; with four stage-B chunks (NP = 128) the float values
-  // of the row wait in columns 256..383 for the token's scale
-  static constexpr int TMEM_COLS = NP == 128 ? 512 : 256;
-  static constexpr int STASH = 256;
+  // of the row wait in columns 320..447 for the token's scale
+  // With 512 columns (n2 = 128: one CTA per SM) stage A's two chunks get
+  // their own blocks and stage B's chunks alternate between two 160-column
+  // buffers, so the next chunk's MMAs run while this one is read.
+  static constexpr int TMEM_COLS = N2 == 128 ? 512 : 256;
+  static constexpr bool DB = TMEM_COLS == 512;
+  static constexpr int STASH = 320;
   // reduction scratch (32-bit words): [8] warp maxima, [2][128] halves of
   // the tile rows' maxima, [8][64] group maxima (uint bits), [2][64] group scales
   static constexpr int R_WARP = 0;
@@ -101,8 +105,11 @@ struct IC {
   static constexpr int R_GMAX = R_XM + 2 * 128;
   static constexpr int R_SG = R_GMAX + 8 * 64;
   static constexpr int R_WORDS = R_SG + 2 * 64;
-  static constexpr int OFF_BAR = OFF_RED + R_WORDS * 4;  // [0] MMA completion, [1] factor loads
-  static constexpr int OFF_CONST = OFF_BAR + 16;  // ints: [0] f2, [1] f1, [4] tensor memory, [8 + 2 s + c] t
+  // mbarriers: [0] factor loads, [1 + c] MMAs of stage-A chunk buffer c,
+  // [3 + b] MMAs of stage-B buffer b (one barrier per buffer, so that none
+  // runs more than one phase ahead of its waiters)
+  static constexpr int OFF_BAR = OFF_RED + R_WORDS * 4;
+  static constexpr int OFF_CONST = OFF_BAR + 40;  // ints: [0] f2, [1] f1, [4] tensor memory, [8 + 2 s + c] t
   static constexpr int SMEM = OFF_CONST + 64 + 1024;
   static_assert(N2 == 64 || N2 == 128, "n2");
   static_assert(NP == 64 || NP == 128, "padded n1");
@@ -278,10 +285,11 @@ __global__ void __launch_bounds__(kIntThreads, (N2 == 64 ? 2 : 1)) quant_act_int
   uint32_t* gmax = red + C::R_GMAX;
   const uint32_t sbase = smem_u32(sm);
 
-  uint64_t* lbar = bar + 1;
+  uint64_t* lbar = bar;
+  uint64_t* mA = bar + 1;  // [2]
+  uint64_t* mB = bar + 3;  // [2]
   if (t == 0) {
-    mbar_init(bar, 1);
-    mbar_init(lbar, 1);
+    for (int b = 0; b < 5; ++b) mbar_init(bar + b, 1);
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -384,7 +392,7 @@ __global__ void __launch_bounds__(kIntThreads, (N2 == 64 ? 2 : 1)) quant_act_int
   const uint32_t p2base = sbase + C::OFF_P2, p1base = sbase + C::OFF_P1;
   pdl_wait();  // X, c and the outputs may be touched from here on
 
-  uint32_t ph = 0;
+  uint32_t phA[2] = {0, 0}, phB[2] = {0, 0};
   bool bad = false;
   // this thread's tile row of an item: (token s, tile row i), columns [h H2, h H2 + H2)
   const int s = G == 2 ? (r >> 6) : 0, i = G == 2 ? (r & 63) : r;
@@ -492,15 +500,27 @@ __global__ void __launch_bounds__(kIntThreads, (N2 == 64 ? 2 : 1)) quant_act_int
     // with W = hi 2^16 + lo; |lo| < 2^31 bounds the low part.  This thread
     // takes columns l in [32 h, 32 h + 32) of each chunk.
     int vv[C::LCH][32];
+    if (t == 0) {
+      tc_fence_after();
+      // both chunks up front when each has its own columns
+#pragma unroll
+      for (int ch = 0; ch < (C::DB ? C::LCH : 1); ++ch) {
+        issue_stage<XL, 4, 64, N2 / 32, false, N2, C::X_PL, N2>(tmem + uint32_t(C::DB ? 256 * ch : 0), xbase,
+                                                                 p2base + uint32_t(ch * C::P2_CH));
+        mma_commit(&mA[ch]);
+      }
+    }
 #pragma unroll
     for (int ch = 0; ch < C::LCH; ++ch) {
-      if (t == 0) {
+      const uint32_t dA = tmem + uint32_t(C::DB ? 256 * ch : 0);
+      const int ba = C::DB ? ch : 0;
+      if (!C::DB && ch > 0 && t == 0) {
         tc_fence_after();
         issue_stage<XL, 4, 64, N2 / 32, false, N2, C::X_PL, N2>(tmem, xbase, p2base + uint32_t(ch * C::P2_CH));
-        mma_commit(bar);
+        mma_commit(&mA[0]);
       }
-      if (!warp_wait(bar, ph)) bad = true;
-      ph ^= 1u;
+      if (!warp_wait(&mA[ba], phA[ba])) bad = true;
+      phA[ba] ^= 1u;
       tc_fence_after();
       // pass 1: the largest |hi| of this row half, in units common to the token's rows
       uint32_t mhi = 0;
@@ -508,8 +528,8 @@ __global__ void __launch_bounds__(kIntThreads, (N2 == 64 ? 2 : 1)) quant_act_int
       for (int sl = 0; sl < 2; ++sl) {
         uint32_t d0[16], d1[16];
         const uint32_t col = uint32_t(32 * h + 16 * sl);
-        tmem_ld_32x16(tmem + lane_off + col, *reinterpret_cast<uint32_t(*)[32]>(d0));
-        tmem_ld_32x16(tmem + lane_off + col + 64u, *reinterpret_cast<uint32_t(*)[32]>(d1));
+        tmem_ld_32x16(dA + lane_off + col, *reinterpret_cast<uint32_t(*)[32]>(d0));
+        tmem_ld_32x16(dA + lane_off + col + 64u, *reinterpret_cast<uint32_t(*)[32]>(d1));
         tmem_wait_ld();
 #pragma unroll
         for (int q = 0; q < 16; ++q) mhi = max(mhi, uint32_t(abs(int(d0[q]) * 256 + int(d1[q]))));
@@ -531,7 +551,7 @@ __global__ void __launch_bounds__(kIntThreads, (N2 == 64 ? 2 : 1)) quant_act_int
 #pragma unroll
       for (int sl = 0; sl < 2; ++sl) {
         uint32_t d[4][16];
-        load_levels16(tmem + lane_off + uint32_t(32 * h + 16 * sl), d);
+        load_levels16(dA + lane_off + uint32_t(32 * h + 16 * sl), d);
         tmem_wait_ld();
 #pragma unroll
         for (int q = 0; q < 16; ++q) vv[ch][16 * sl + q] = int(combine_levels(d[0][q], d[1][q], d[2][q], d[3][q]) >> n);
@@ -585,7 +605,7 @@ __global__ void __launch_bounds__(kIntThreads, (N2 == 64 ? 2 : 1)) quant_act_int
       // t of this row's (token, l-chunk)
       const int Es = 16 + cst[8 + 2 * sb + (N2 == 128 ? (l >> 6) : 0)] + f1;
       const float up = pow2f(Es);
-      constexpr bool kStash = C::TMEM_COLS == 512;  // four chunks: the values wait in tensor memory
+      constexpr bool kStash = NP == 128;  // four chunks: the values wait in tensor memory
       float fv[kStash ? 16 : NP / 2];
       float tmax = 0.f;
       // 8 codes (k = kbase .. kbase + 7 of this row's column l) into the tile
@@ -597,23 +617,32 @@ __global__ void __launch_bounds__(kIntThreads, (N2 == 64 ? 2 : 1)) quant_act_int
       };
       // the 4 warps (n2 = 128) or 2 warps (n2 = 64, token sb) that hold half hh of the chunk
       auto half_warp = [&](int tt, int hh, int q) { return N2 == 128 ? 4 * hh + q : 4 * hh + 2 * tt + q; };
+      auto issue_b = [&](int kc) {
+        tc_fence_after();
+        issue_stage<4, 5, 32, NP / 32, true, 0, C::U_PL, NP>(tmem + uint32_t(C::DB ? 160 * (kc & 1) : 0),
+                                                              ubase + uint32_t(g * 4 * C::U_PL),
+                                                              p1base + uint32_t(kc * C::P1_CH));
+        mma_commit(&mB[C::DB ? (kc & 1) : 0]);
+      };
+      if (t == 0) issue_b(0);
 #pragma unroll
       for (int kc = 0; kc < C::KCB; ++kc) {
         float* fc = fv + (kStash ? 0 : 16 * kc);
-        if (t == 0) {
-          tc_fence_after();
-          issue_stage<4, 5, 32, NP / 32, true, 0, C::U_PL, NP>(tmem, ubase + uint32_t(g * 4 * C::U_PL),
-                                                                p1base + uint32_t(kc * C::P1_CH));
-          mma_commit(bar);
+        // the next chunk's MMAs run while this one is read (its buffer was
+        // last read before the barrier that closed the previous chunk)
+        if (t == 0 && kc + 1 < C::KCB && C::DB) issue_b(kc + 1);
+        {
+          const int bb = C::DB ? (kc & 1) : 0;
+          if (!warp_wait(&mB[bb], phB[bb])) bad = true;
+          phB[bb] ^= 1u;
         }
-        if (!warp_wait(bar, ph)) bad = true;
-        ph ^= 1u;
         tc_fence_after();
         {
+          const uint32_t dB = tmem + uint32_t(C::DB ? 160 * (kc & 1) : 0);
           uint32_t d[5][16];
 #pragma unroll
           for (int bk = 0; bk < 5; ++bk)
-            tmem_ld_32x16(tmem + lane_off + uint32_t(32 * bk + 16 * h), *reinterpret_cast<uint32_t(*)[32]>(d[bk]));
+            tmem_ld_32x16(dB + lane_off + uint32_t(32 * bk + 16 * h), *reinterpret_cast<uint32_t(*)[32]>(d[bk]));
           tmem_wait_ld();
 #pragma unroll
           for (int q = 0; q < 16; ++q) {
@@ -638,6 +667,7 @@ __global__ void __launch_bounds__(kIntThreads, (N2 == 64 ? 2 : 1)) quant_act_int
         }
         tc_fence_before();
         bad = __syncthreads_or(bad);  // D read by every thread: free for the next MMA
+        if (t == 0 && kc + 1 < C::KCB && !C::DB) issue_b(kc + 1);
         if (GRAN == FQ_DYNAMIC_GROUP) {
           // groups: n2 = 128 -> row k (all 128 rows of D); n2 = 64 -> rows k, k + 1 of token sb (64 rows)
           constexpr int KPG = 128 / N2;
