@@ -18,7 +18,10 @@ It restates, step by step and in plain numpy, what the pages define:
 * group-wise quantization in groups of 128 along K (FRM-PTQ abstract,
   multi-granularity group quantization);
 * the INT4 x INT4 product with integer accumulation and the dequantization
-  y = acc * s_x * s_w (FlatQuant notes, 核心思想: Y ~ Q(XP) Q(P^-1 W^T)).
+  y = acc * s_x * s_w (FlatQuant notes, 核心思想: Y ~ Q(XP) Q(P^-1 W^T));
+* the general quantizer (any b, min-max zero point; FRM-PTQ page) and the
+  per-token residual scaling S_n ahead of static quantization (FPTQuant
+  explainer, 伪动态残差缩放).
 
 Precision: the transform is evaluated in float64 and rounded once to float32
 (the "transformed value"); scales, the division and round-half-to-even are
@@ -114,9 +117,6 @@ def unpack_int4(p: np.ndarray) -> np.ndarray:
 #
 # Q(W) = clamp(round(W/s) + z, 0, 2^b - 1) for any bit width b and zero point
 # z (FRM-PTQ page, 初步介绍), with the asymmetric (min-max) choice of s and z.
-# Not on the hot path yet: the CUDA library answers FQ_ERR_UNSUPPORTED for
-# z != 2^(b-1) or b != 4; these functions are the oracle that path will be
-# held to.
 
 def minmax_params(v32: np.ndarray, bits: int, alpha: float = 1.0):
     """Per-row asymmetric scale and zero point.
@@ -264,6 +264,42 @@ def quant_weight(w, gran=ROW, alpha=1.0, p1_inv=None, p2_inv=None, c=None,
     else:
         raise ValueError(gran)
     return q, s, v32
+
+
+# ------------------------------------------------------------------ residual scaling
+
+def residual_rms(x) -> np.ndarray:
+    """S_n = sqrt(sum_k x_k^2 / K) per token, in float64, rounded once to float32.
+
+    FPTQuant explainer, 伪动态残差缩放 (S_n): a per-token factor from the
+    root-mean-square of the residual stream (RMSNorm applied to the
+    residual; the page gives no epsilon, so none is added).
+    Parity pinned by: tests/golden/residual_worked.txt, scaling a token by a
+    power of two scaling S_n by the same power.
+    """
+    x64 = np.asarray(x, np.float64)
+    return np.sqrt((x64 * x64).sum(axis=1) / x64.shape[1]).astype(np.float32)
+
+
+def quant_act_residual(x, static_scale):
+    """Static per-channel INT4 codes of the token divided by its S_n.
+
+    v = fl32(x / S_n) (IEEE float32 division; a token of zeros gives v = 0),
+    then the static quantizer of quant_act with the caller's s_k.  The
+    per-token factor leaves through the GEMM: a bias-free linear layer
+    commutes with per-token scaling, so y = (acc * S_n) * s_w' with the
+    static scales migrated into s_w' (MergeQuant quantization step
+    migration) restores the unscaled output.
+    Returns (codes int8 [M, K], S_n float32 [M], v float32 [M, K]).
+    Parity pinned by: tests/golden/residual_worked.txt, invariance of the
+    codes under power-of-two token scaling, |x / S_n - s q| <= s/2.
+    """
+    s_n = residual_rms(x)
+    x32 = np.asarray(x, np.float32)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        v = np.where(s_n[:, None] > 0, x32 / s_n[:, None], np.float32(0)).astype(np.float32)
+    q = quantize(v, np.asarray(static_scale, np.float32)[None, :])
+    return q, s_n, v
 
 
 # ------------------------------------------------------------------ GEMM + dequant

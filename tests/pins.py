@@ -392,3 +392,47 @@ def mutant(o, **overrides):
         if isinstance(f, types.FunctionType):
             m.__dict__[name] = types.FunctionType(f.__code__, m.__dict__, f.__name__, f.__defaults__, f.__closure__)
     return m
+
+
+# ------------------------------------------------------------------ residual scaling (S_n)
+
+RES_SCALES = (0.4, 0.4, 1.0, 0.25)
+
+
+def check_residual_golden(o):
+    """Hand-worked tokens in tests/golden/residual_worked.txt (FPTQuant, 伪动态残差缩放)."""
+    s = np.array(RES_SCALES, dtype=np.float32)
+    for ln in _lines("residual_worked.txt"):
+        xs, ss, qs = [p.strip() for p in ln.split("|")]
+        x = np.array([float(v) for v in xs.split()], dtype=np.float16)[None, :]
+        q, s_n, _ = o.quant_act_residual(x, s)
+        assert np.float32(s_n[0]) == np.float32(float(ss)), (ln, s_n[0])
+        assert np.array_equal(q[0], np.array([int(v) for v in qs.split()], dtype=np.int8)), (ln, q[0])
+
+
+def check_residual_invariants(o):
+    """S_n is the root-mean-square (mean of x^2 over K, then a square root):
+    a token times 2^p has S_n times 2^p and the same codes; the codes
+    reconstruct x / S_n within s/2 where unclipped; and the residual-scaled
+    codes of a token whose RMS is 1 equal the plain static codes."""
+    g = np.random.Generator(np.random.PCG64(21))
+    k = 256
+    x = (g.standard_normal((32, k)) * g.uniform(0.05, 20, (32, 1))).astype(np.float16)
+    s = (g.uniform(0.05, 0.6, k)).astype(np.float32)
+    q, s_n, v = o.quant_act_residual(x, s)
+    ref = np.sqrt((x.astype(np.float64) ** 2).mean(axis=1))
+    assert np.allclose(s_n, ref, rtol=1e-6), "S_n is not the root-mean-square"
+    for p in (-3, 2, 5):
+        q2, s2, _ = o.quant_act_residual((x.astype(np.float32) * np.float32(2.0 ** p)).astype(np.float16), s)
+        assert np.array_equal(q2, q) and np.array_equal(s2, (s_n * np.float32(2.0 ** p)).astype(np.float32))
+    un = (q > -8) & (q < 7)
+    err = np.abs(v.astype(np.float64) - q.astype(np.float64) * s[None, :].astype(np.float64))
+    assert np.all(err[un] <= s[None, :].repeat(32, 0)[un] / 2 * (1 + 1e-6))
+    # a token with RMS exactly 1 (entries +-1): the codes are the static codes of x itself
+    ones = np.where(g.standard_normal((4, k)) > 0, 1.0, -1.0).astype(np.float16)
+    q1, s1, _ = o.quant_act_residual(ones, s)
+    assert np.all(s1 == 1.0)
+    assert np.array_equal(q1, o.quant_act(ones, o.STATIC, static_scale=s)[0])
+
+
+ALL_CHECKS += [check_residual_golden, check_residual_invariants]

@@ -143,7 +143,29 @@ def _gemm_asym_no_cross(ux, zx, uw, zw):
     return ux @ uw.T - zw[None, :] * ux.sum(1)[:, None] - zx[:, None] * uw.sum(1)[None, :]
 
 
+def _residual_rms_no_mean(x):
+    # sum of squares without the division by K
+    x64 = np.asarray(x, np.float64)
+    return np.sqrt((x64 * x64).sum(axis=1)).astype(np.float32)
+
+
+def _residual_rms_no_sqrt(x):
+    # mean square instead of its root
+    x64 = np.asarray(x, np.float64)
+    return ((x64 * x64).sum(axis=1) / x64.shape[1]).astype(np.float32)
+
+
+def _quant_act_residual_times(x, static_scale):
+    # the token multiplied by S_n instead of divided
+    s_n = residual_rms(x)  # noqa: F821
+    v = (np.asarray(x, np.float32) * s_n[:, None]).astype(np.float32)
+    return quantize(v, np.asarray(static_scale, np.float32)[None, :]), s_n, v  # noqa: F821
+
+
 MUTANTS = {
+    "residual_rms_without_mean": dict(residual_rms=_residual_rms_no_mean),
+    "residual_rms_without_sqrt": dict(residual_rms=_residual_rms_no_sqrt),
+    "residual_multiplied": dict(quant_act_residual=_quant_act_residual_times),
     "asym_range_without_zero": dict(minmax_params=_minmax_no_zero),
     "asym_zero_point_sign": dict(minmax_params=_minmax_zero_sign),
     "asym_gemm_drops_cross_term": dict(gemm_asym=_gemm_asym_no_cross),
