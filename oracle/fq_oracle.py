@@ -32,6 +32,8 @@ check it against something other than itself.
 """
 from __future__ import annotations
 
+import math
+
 import numpy as np
 
 BITS = 4                      # b in Q(W)
@@ -269,16 +271,30 @@ def quant_weight(w, gran=ROW, alpha=1.0, p1_inv=None, p2_inv=None, c=None,
 # ------------------------------------------------------------------ residual scaling
 
 def residual_rms(x) -> np.ndarray:
-    """S_n = sqrt(sum_k x_k^2 / K) per token, in float64, rounded once to float32.
+    """S_n = sqrt(sum_k x_k^2 / K) per token, rounded once to float32.
 
     FPTQuant explainer, 伪动态残差缩放 (S_n): a per-token factor from the
     root-mean-square of the residual stream (RMSNorm applied to the
-    residual; the page gives no epsilon, so none is added).
+    residual; the page gives no epsilon, so none is added).  The page fixes
+    no summation order, so the sum of squares is taken exactly and rounded
+    once to float64 (math.fsum; every square of a float32 value is exact in
+    float64), then divided by K and square-rooted in float64 and rounded to
+    float32: a result that does not depend on any order of additions.
     Parity pinned by: tests/golden/residual_worked.txt, scaling a token by a
-    power of two scaling S_n by the same power.
+    power of two scaling S_n by the same power, and an exact rational
+    evaluation of tokens whose float64 partial sums round.
+    """
+    return np.sqrt(residual_sumsq(x) / np.asarray(x).shape[1]).astype(np.float32)
+
+
+def residual_sumsq(x) -> np.ndarray:
+    """sum_k x_k^2 per token, exact, rounded once to float64 (the sum inside S_n).
+
+    Parity pinned by: an exact rational evaluation (fractions) of tokens
+    whose float64 partial sums round in any order of additions.
     """
     x64 = np.asarray(x, np.float64)
-    return np.sqrt((x64 * x64).sum(axis=1) / x64.shape[1]).astype(np.float32)
+    return np.array([math.fsum(row * row) for row in x64], np.float64)
 
 
 def quant_act_residual(x, static_scale):

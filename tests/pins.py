@@ -435,4 +435,22 @@ def check_residual_invariants(o):
     assert np.array_equal(q1, o.quant_act(ones, o.STATIC, static_scale=s)[0])
 
 
-ALL_CHECKS += [check_residual_golden, check_residual_invariants]
+def check_residual_exact_sum(o):
+    """The sum of squares inside S_n is the exact sum rounded once: checked by
+    rational arithmetic on tokens mixing one large entry with many small ones
+    (2^30 + 255 * 2^-24 needs 55 bits), where a float64 running or pairwise
+    sum drops the small squares."""
+    from fractions import Fraction
+    g = np.random.Generator(np.random.PCG64(23))
+    rows = [np.array([32768.0] + [2.0 ** -12] * 255, np.float16),
+            np.array([2.0 ** -12] * 200 + [-32768.0] + [2.0 ** -12] * 55, np.float16),
+            (g.standard_normal(256) * np.where(g.uniform(size=256) < 0.02, 4000.0, 0.01)).astype(np.float16)]
+    x = np.stack(rows)
+    got = o.residual_sumsq(x)
+    for i, row in enumerate(x):
+        exact = sum(Fraction(float(v)) ** 2 for v in row)
+        assert got[i] == float(exact), (i, got[i], float(exact))
+    assert np.array_equal(o.residual_rms(x), np.sqrt(got / 256).astype(np.float32))
+
+
+ALL_CHECKS += [check_residual_golden, check_residual_invariants, check_residual_exact_sum]

@@ -155,6 +155,12 @@ def _residual_rms_no_sqrt(x):
     return ((x64 * x64).sum(axis=1) / x64.shape[1]).astype(np.float32)
 
 
+def _residual_sumsq_pairwise(x):
+    # float64 numpy sum (order-dependent rounding) instead of the exact sum
+    x64 = np.asarray(x, np.float64)
+    return (x64 * x64).sum(axis=1)
+
+
 def _quant_act_residual_times(x, static_scale):
     # the token multiplied by S_n instead of divided
     s_n = residual_rms(x)  # noqa: F821
@@ -166,6 +172,7 @@ MUTANTS = {
     "residual_rms_without_mean": dict(residual_rms=_residual_rms_no_mean),
     "residual_rms_without_sqrt": dict(residual_rms=_residual_rms_no_sqrt),
     "residual_multiplied": dict(quant_act_residual=_quant_act_residual_times),
+    "residual_sum_rounded_per_add": dict(residual_sumsq=_residual_sumsq_pairwise),
     "asym_range_without_zero": dict(minmax_params=_minmax_no_zero),
     "asym_zero_point_sign": dict(minmax_params=_minmax_zero_sign),
     "asym_gemm_drops_cross_term": dict(gemm_asym=_gemm_asym_no_cross),
