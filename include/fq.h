@@ -65,8 +65,13 @@ typedef enum {
   FQ_DYNAMIC_ROW = 0,    /* one scale per token (activations) / per output channel (weights) */
   FQ_DYNAMIC_GROUP = 1,  /* one scale per row and group of 128 along K */
   FQ_STATIC_CHANNEL = 2, /* activations only: caller-given float32 scale per input channel */
-  FQ_DYNAMIC_ROW_ZP = 3  /* GEMM / linear only: both operands from the min-max quantizer
+  FQ_DYNAMIC_ROW_ZP = 3, /* GEMM / linear only: both operands from the min-max quantizer
                             (FQ_ZERO_POINT_MINMAX): per-row scale and zero point */
+  FQ_STATIC_RESIDUAL = 4 /* activations only (no transform, no c): each token divided by its
+                            root-mean-square S_n = sqrt(sum x^2 / K), then the static
+                            per-channel scales (FPTQuant explainer, 伪动态残差缩放); s_x
+                            receives S_n float32 [M], and the GEMM runs FQ_DYNAMIC_ROW
+                            with s_x = S_n and weights whose s_w carries the static scales */
 } fq_gran;
 
 /* fq_qparams.zero_point value that selects the general (asymmetric) form of
@@ -130,7 +135,9 @@ fq_status fq_quant_weight(const uint16_t* W, int N, int K, const fq_qparams* qp,
  * qp     FQ_DYNAMIC_ROW: s_x float32 [M] (FQ_ZERO_POINT_MINMAX: the 3 M-word scale
  *        block);  FQ_DYNAMIC_GROUP: s_x fp16 [K/128][M];
  *        FQ_STATIC_CHANNEL: static_scale float32 [K] is used and s_x is not written
- *        (may be NULL); alpha = alpha_a.
+ *        (may be NULL); FQ_STATIC_RESIDUAL: static_scale float32 [K] is used on
+ *        x / S_n and s_x receives S_n float32 [M] (S_n = 0, codes 0 for a token of
+ *        zeros); alpha = alpha_a.
  * t      NULL or the transform (P1, P2, c).  P1 and P2 are parameters: the
  *        kernel may read them while the kernels enqueued just before it on
  *        the stream are still finishing (programmatic dependent launch), so

@@ -11,7 +11,7 @@ constexpr size_t kAlign = 256;
 size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 size_t act_scale_bytes(int M, int K, fq_gran gran) {
-  if (gran == FQ_DYNAMIC_ROW) return size_t(M) * sizeof(float);
+  if (gran == FQ_DYNAMIC_ROW || gran == FQ_STATIC_RESIDUAL) return size_t(M) * sizeof(float);
   if (gran == FQ_DYNAMIC_ROW_ZP) return 3 * size_t(M) * sizeof(float);  // s, o = 2^(b-1) - z, code sums
   if (gran == FQ_DYNAMIC_GROUP) return size_t(K / kGroup) * M * 2;
   return 0;
@@ -52,7 +52,9 @@ fq_status fq_linear(const uint16_t* X, int M, int K, const fq_qparams* act_qp, c
   const size_t gws_bytes = ws_bytes - off;
   fq_status st = fq_quant_act(X, M, K, act_qp, t, static_scale, xq, sx, stream);
   if (st != FQ_OK) return st;
-  return fq_w4a4_gemm(xq, sx, Wq, s_w, M, N, K, gran, Y, gws, gws_bytes, stream);
+  // the residual scaling leaves through the per-token epilogue: s_x = S_n
+  const fq_gran ggran = gran == FQ_STATIC_RESIDUAL ? FQ_DYNAMIC_ROW : gran;
+  return fq_w4a4_gemm(xq, sx, Wq, s_w, M, N, K, ggran, Y, gws, gws_bytes, stream);
 }
 
 }  // extern "C"

@@ -103,6 +103,18 @@ __device__ __forceinline__ int rtn_code(float v, float s) {
 // when a transform is applied, so that the column pass is free of bank conflicts.
 __device__ __forceinline__ int slot(int e, int n2, int pad) { return pad ? (e / n2) * (n2 + 1) + (e % n2) : e; }
 
+// An unsigned 128-bit integer (hi, lo) rounded once to the nearest float64:
+// the top 64 significant bits, with every bit below them folded into a
+// sticky bit 0, are rounded by the 64-bit conversion (its rounding position
+// lies 11 bits above bit 0), then scaled by the exact power of two.
+__device__ __forceinline__ double u128_to_double_rn(unsigned long long hi, unsigned long long lo) {
+  if (hi == 0) return __ull2double_rn(lo);
+  const int lz = __clzll(static_cast<long long>(hi));
+  const unsigned long long top = lz ? (hi << lz) | (lo >> (64 - lz)) : hi;
+  const unsigned long long rest = lz ? (lo << lz) : lo;
+  return ldexp(__ull2double_rn(top | (rest ? 1ull : 0ull)), 64 - lz);
+}
+
 template <int SIDE, bool PSMEM>
 __global__ void __launch_bounds__(kThreads) quant_rows_kernel(QuantParams p) {
   extern __shared__ __align__(16) float smem[];
@@ -119,8 +131,8 @@ __global__ void __launch_bounds__(kThreads) quant_rows_kernel(QuantParams p) {
   const int xin_floats = (SIDE == kAct && xf) ? (n1 * xstride + 1) / 2 : 0;
   float* sL = xs + row_floats + xin_floats;  // [i][k] = Lc(k, i)   (PSMEM)
   float* sR = sL + (PSMEM ? n1 * n1 : 0); // [j][l] = Rr(j, l)   (PSMEM)
-  float* red = sR + (PSMEM ? n2 * n2 : 0);  // [2][kWarps]
-  float* gsc = red + 2 * kWarps;            // [K/128] group scales
+  float* red = sR + (PSMEM ? n2 * n2 : 0);  // [4][kWarps] (8-byte aligned when there is no transform)
+  float* gsc = red + 4 * kWarps;            // [K/128] group scales
 
   if (PSMEM && xf) {
     for (int e = tid; e < n1 * n1; e += kThreads) {
@@ -168,6 +180,66 @@ __global__ void __launch_bounds__(kThreads) quant_rows_kernel(QuantParams p) {
       }
     }
     __syncthreads();
+
+    // 1b. per-token residual scaling (FPTQuant S_n): the token's sum of
+    // squares taken exactly -- every fp16 square is an integer multiple of
+    // 2^-48 below 2^82, so a 128-bit integer sum of K <= 2^16 of them cannot
+    // overflow -- rounded once to float64, then /K, sqrt and float32; then
+    // v = fl32(x / S_n) in place (v = 0 unless S_n > 0).  Non-finite
+    // entries give S_n = +inf (an infinity) or NaN (a NaN), as the float64
+    // sum would.
+    if (SIDE == kAct && p.gran == FQ_STATIC_RESIDUAL) {
+      unsigned long long lo = 0, hi = 0;
+      unsigned nonfin = 0;
+      for (int e = tid; e < K; e += kThreads) {
+        const unsigned h = __half_as_ushort(__float2half_rn(xs[e]));  // exact: xs holds fp16 values
+        const unsigned E = (h >> 10) & 31u, F = h & 1023u;
+        if (E == 31u) {
+          nonfin |= F ? 2u : 1u;
+          continue;
+        }
+        const unsigned long long m = E ? (F | 1024u) : F;
+        const unsigned long long m2 = m * m;  // x^2 = m2 * 2^(2E-50), or m2 * 2^-48 when E = 0
+        const int sh = E ? int(2 * E) - 2 : 0;  // in units of 2^-48, at most 58
+        const unsigned long long alo = m2 << sh, ahi = sh ? m2 >> (64 - sh) : 0ull;
+        lo += alo;
+        hi += ahi + (lo < alo ? 1ull : 0ull);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const unsigned long long olo = __shfl_xor_sync(0xffffffffu, lo, o);
+        const unsigned long long ohi = __shfl_xor_sync(0xffffffffu, hi, o);
+        lo += olo;
+        hi += ohi + (lo < olo ? 1ull : 0ull);
+      }
+      nonfin = __reduce_or_sync(0xffffffffu, nonfin);
+      unsigned long long* red64 = reinterpret_cast<unsigned long long*>(red);  // [kWarps][2]
+      if (lane == 0) {
+        red64[2 * warp] = lo;
+        red64[2 * warp + 1] = hi | (static_cast<unsigned long long>(nonfin) << 62);  // hi < 2^32
+      }
+      __syncthreads();
+      unsigned long long tlo = 0, thi = 0;
+      unsigned tnf = 0;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) {
+        const unsigned long long wlo = red64[2 * w], whi = red64[2 * w + 1];
+        tlo += wlo;
+        thi += (whi & ((1ull << 62) - 1)) + (tlo < wlo ? 1ull : 0ull);
+        tnf |= unsigned(whi >> 62);
+      }
+      float s_n;
+      if (tnf & 2u)
+        s_n = __int_as_float(0x7fc00000);
+      else if (tnf)
+        s_n = __int_as_float(0x7f800000);
+      else
+        s_n = __double2float_rn(sqrt(u128_to_double_rn(thi, tlo) * 0x1p-48 / double(K)));
+      __syncthreads();  // every thread has read red64
+      if (tid == 0) p.s_row[r] = s_n;
+      for (int e = tid; e < K; e += kThreads) xs[e] = s_n > 0.f ? __fdiv_rn(xs[e], s_n) : 0.f;
+      __syncthreads();
+    }
 
     // 2. transform
     if (SIDE == kAct && xf) {
@@ -407,7 +479,7 @@ __global__ void __launch_bounds__(kThreads) quant_rows_kernel(QuantParams p) {
         else if (p.gran == FQ_DYNAMIC_GROUP)
           s = gsc[e / kGroup];
         else
-          s = p.sstatic[e];
+          s = p.sstatic[e];  // static, and static after the residual scaling
         word |= (uint32_t(rtn_code(v, s)) & 0xFu) << (4 * j);
       }
       qrow[e0 / 8] = word;
@@ -467,7 +539,7 @@ fq_status launch_quant_static(const QuantParams& qp, cudaStream_t stream) {
 size_t smem_bytes(int K, int n1, int n2, bool psmem, bool act) {
   const size_t row = n1 > 0 ? size_t(n1) * (n2 + 1) + (act ? (size_t(n1) * (n2 + 2) + 1) / 2 : 0) : size_t(K);
   const size_t pm = (psmem && n1 > 0) ? size_t(n1) * n1 + size_t(n2) * n2 : 0;
-  return (row + pm + 2 * kWarps + K / kGroup) * sizeof(float);
+  return (row + pm + 4 * kWarps + K / kGroup) * sizeof(float);
 }
 
 template <int SIDE, bool PSMEM>
@@ -504,9 +576,10 @@ fq_status check_qparams(const fq_qparams* qp, bool act) {
   }
   if (qp->gran == FQ_DYNAMIC_GROUP && qp->group_size != kGroup)
     return fail(FQ_ERR_UNSUPPORTED, "group_size = %d: only 128 is provided", qp->group_size);
-  if (qp->gran != FQ_DYNAMIC_ROW && qp->gran != FQ_DYNAMIC_GROUP && !(act && qp->gran == FQ_STATIC_CHANNEL))
+  if (qp->gran != FQ_DYNAMIC_ROW && qp->gran != FQ_DYNAMIC_GROUP &&
+      !(act && (qp->gran == FQ_STATIC_CHANNEL || qp->gran == FQ_STATIC_RESIDUAL)))
     return fail(FQ_ERR_UNSUPPORTED, "granularity %d is not provided here", int(qp->gran));
-  if (qp->gran != FQ_STATIC_CHANNEL)
+  if (qp->gran != FQ_STATIC_CHANNEL && qp->gran != FQ_STATIC_RESIDUAL)
     FQ_CHECK_ARG(qp->alpha > 0.f && qp->alpha <= 1.f, "alpha = %g must lie in (0, 1]", double(qp->alpha));
   return FQ_OK;
 }
@@ -521,10 +594,12 @@ fq_status quant_common(int side, const uint16_t* X, int R, int K, const fq_qpara
   FQ_CHECK_ARG(K >= kGroup && K <= kMaxQuantK && K % kGroup == 0, "K = %d must be a multiple of 128 in [128, %d]",
                K, kMaxQuantK);
   FQ_CHECK_ARG(aligned(X, 16) && aligned(Q, 16), "X and the packed output must be 16-byte aligned");
-  if (qp->gran == FQ_STATIC_CHANNEL)
-    FQ_CHECK_ARG(extra && aligned(extra, 4), "static scales [K] are required for FQ_STATIC_CHANNEL");
-  else
+  if (qp->gran == FQ_STATIC_CHANNEL || qp->gran == FQ_STATIC_RESIDUAL)
+    FQ_CHECK_ARG(extra && aligned(extra, 4), "static scales [K] are required for the static granularities");
+  if (qp->gran != FQ_STATIC_CHANNEL)
     FQ_CHECK_ARG(s_out && aligned(s_out, 4), "the scale output must be non-NULL and aligned");
+  if (qp->gran == FQ_STATIC_RESIDUAL && t && (t->P1 || t->c))
+    return fail(FQ_ERR_UNSUPPORTED, "FQ_STATIC_RESIDUAL takes no transform and no c");
   QuantParams p{};
   p.X = reinterpret_cast<const __half*>(X);
   p.R = R;
@@ -533,7 +608,7 @@ fq_status quant_common(int side, const uint16_t* X, int R, int K, const fq_qpara
   p.alpha = qp->alpha;
   p.Q = Q;
   p.xhat = xhat;
-  if (qp->gran == FQ_DYNAMIC_ROW) p.s_row = static_cast<float*>(s_out);
+  if (qp->gran == FQ_DYNAMIC_ROW || qp->gran == FQ_STATIC_RESIDUAL) p.s_row = static_cast<float*>(s_out);
   if (qp->zero_point == FQ_ZERO_POINT_MINMAX) {
     // scale block: float32 s[R], int32 o[R] = 2^(b-1) - z, int32 code sums[R]
     p.asym = 1;
@@ -542,7 +617,7 @@ fq_status quant_common(int side, const uint16_t* X, int R, int K, const fq_qpara
     p.zsum = reinterpret_cast<int32_t*>(static_cast<float*>(s_out) + 2 * size_t(R));
   }
   if (qp->gran == FQ_DYNAMIC_GROUP) p.s_grp = static_cast<__half*>(s_out);
-  if (side == kAct && qp->gran == FQ_STATIC_CHANNEL) p.sstatic = extra;
+  if (side == kAct && (qp->gran == FQ_STATIC_CHANNEL || qp->gran == FQ_STATIC_RESIDUAL)) p.sstatic = extra;
   if (side == kWeight) p.qsm = extra;
   if (t) {
     p.c = t->c;

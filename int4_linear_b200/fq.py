@@ -13,7 +13,7 @@ from dataclasses import dataclass
 
 import torch
 
-ROW, GROUP, STATIC, ROW_ZP = 0, 1, 2, 3  # fq_gran
+ROW, GROUP, STATIC, ROW_ZP, STATIC_RESIDUAL = 0, 1, 2, 3, 4  # fq_gran
 GROUP_SIZE = 128
 ZERO_POINT_MINMAX = -1                   # fq_qparams.zero_point: per-row min-max (asymmetric) quantizer
 
@@ -136,7 +136,7 @@ def _scales_out(gran, rows, k, dev, zero_point=8):
     if gran == ROW and zero_point == ZERO_POINT_MINMAX:
         # float32 s[rows], int32 o[rows] = 2^(b-1) - z, int32 code sums[rows]
         return torch.empty(3, rows, dtype=torch.float32, device=dev)
-    if gran == ROW:
+    if gran in (ROW, STATIC_RESIDUAL):
         return torch.empty(rows, dtype=torch.float32, device=dev)
     if gran == GROUP:
         return torch.empty(k // GROUP_SIZE, rows, dtype=torch.float16, device=dev)

@@ -188,6 +188,38 @@ def decode_static(m: int, k: int, n: int, seed: int = 0, calib_seed: int = 1,
                 static_scale=s_k, alpha_a=1.0, alpha_w=1.0, outlier_cols=cols)
 
 
+def residual_static(m: int, k: int, n: int, seed: int = 0, calib_seed: int = 1,
+                    calib_tokens: int = 512) -> dict:
+    """Residual-stream tokens for the static quantizer with per-token S_n
+    (FPTQuant explainer, 伪动态残差缩放): token magnitudes that vary by orders.
+
+    X fp16 [m, k] = r_t * z_t with z ~ N(0, 1) and 1% outlier channels x30 and
+    r_t = 2^u, u ~ U(-4, 6) per token (the residual stream's norm grows and
+    spikes across tokens); W fp16 [n, k] ~ N(0, 0.02).  The stand-in static
+    scale comes from a calibration draw Z_cal [calib_tokens, k] of z alone
+    (the unit-magnitude tokens the scaling is meant to produce):
+    s_k = float32(max_t |Z_cal[t, k]|) / (7 * rms_cs), rms_cs = the root of
+    the mean square of the column scales (the expected RMS of z) -- a property
+    of this generator, not S_n itself.  Draw order: r, z, W; calibration
+    stream: Z_cal.
+    """
+    h = generator(seed + 1_000_003)
+    cols = outlier_channels(h, k)
+    cs = np.ones(k)
+    cs[cols] = 30.0
+    g = generator(seed)
+    r = 2.0 ** g.uniform(-4.0, 6.0, m)
+    x = _draw(g, (m, k), "normal", 1.0, col_scale=cs, row_scale=r)
+    w = _draw(g, (n, k), "normal", 0.02)
+    gc = generator(calib_seed)
+    zc = _draw(gc, (calib_tokens, k), "normal", 1.0, col_scale=cs)
+    amax = np.abs(zc.astype(np.float32)).max(axis=0)
+    rms_cs = np.float32(np.sqrt(np.mean(cs * cs)))
+    s_k = (amax / (np.float32(7.0) * rms_cs)).astype(np.float32)
+    return dict(name=f"residual_static_{m}x{k}x{n}", x=x, w=w, m=m, k=k, n=n,
+                static_scale=s_k, token_scale=r, outlier_cols=cols)
+
+
 # The LLaMA-3-8B-like decoder-layer linears at prefill, M = 2048 tokens:
 # (K, N) for qkv, o, gate+up, down.
 PREFILL_8B_SHAPES = [(4096, 6144), (4096, 4096), (4096, 28672), (14336, 4096)]

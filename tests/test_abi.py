@@ -100,6 +100,23 @@ def test_static_needs_scales(L):
     assert st == fq.FQ_ERR_UNSUPPORTED  # weights have no static granularity
 
 
+def test_residual_scaling_arguments(L):
+    """FQ_STATIC_RESIDUAL needs the static scales and the S_n output, takes no
+    transform and no c, and is an activation granularity only (the GEMM runs
+    per token with s_x = S_n)."""
+    qp = _qp(gran=fq.STATIC_RESIDUAL)
+    assert L.fq_quant_act(A, 4, 256, ctypes.byref(qp), None, None, A, A, None) == fq.FQ_ERR_INVALID
+    assert L.fq_quant_act(A, 4, 256, ctypes.byref(qp), None, A, A, None, None) == fq.FQ_ERR_INVALID
+    t = fq._Transform(16, 16, A, A, None)
+    st = L.fq_quant_act(A, 4, 256, ctypes.byref(qp), ctypes.byref(t), A, A, A, None)
+    assert st == fq.FQ_ERR_UNSUPPORTED and b"RESIDUAL" in L.fq_last_error()
+    t = fq._Transform(0, 0, None, None, A)
+    assert L.fq_quant_act(A, 4, 256, ctypes.byref(qp), ctypes.byref(t), A, A, A, None) == fq.FQ_ERR_UNSUPPORTED
+    assert L.fq_quant_weight(A, 4, 256, ctypes.byref(qp), None, None, A, A, None) == fq.FQ_ERR_UNSUPPORTED
+    assert L.fq_w4a4_gemm(A, A, A, A, 4, 256, 256, fq.STATIC_RESIDUAL, A, None, 0, None) == fq.FQ_ERR_UNSUPPORTED
+    assert L.fq_linear_workspace_size(16, 256, 256, fq.STATIC_RESIDUAL) == L.fq_linear_workspace_size(16, 256, 256, fq.ROW)
+
+
 @pytest.mark.parametrize("m,n,k", [(0, 256, 256), (4, 12, 256), (4, 256, 200), (4, 256, 131072)])
 def test_gemm_rejects_sizes(L, m, n, k):
     st = L.fq_w4a4_gemm(A, A, A, A, m, n, k, fq.ROW, A, None, 0, None)
