@@ -155,6 +155,10 @@ fq_status fq_quant_act_debug(const uint16_t* X, int M, int K, const fq_qparams* 
                              const fq_transform* t, const float* static_scale,
                              uint8_t* Xq, void* s_x, float* xhat, void* stream);
 
+/* Leading bytes of every workspace that the library reserves for counters
+ * (see fq_w4a4_gemm and fq_linear). */
+#define FQ_WORKSPACE_SYNC_BYTES 16384
+
 /* INT4 x INT4 GEMM with exact integer accumulation and fp16 dequantization
  * (FlatQuant notes, 核心思想: Y ~ Q(XP) Q(P^-1 W^T)).
  * Xq uint8 [M, K/2], Wq uint8 [N, K/2] packed codes; Y fp16 [M, N] (out):
@@ -168,7 +172,14 @@ fq_status fq_quant_act_debug(const uint16_t* X, int M, int K, const fq_qparams* 
  *                      scale blocks of FQ_ZERO_POINT_MINMAX.  Runs as the exact int32
  *                      product into the workspace, then a zero-point epilogue.
  * workspace / ws_bytes: device scratch of at least fq_gemm_workspace_size()
- *   bytes (may be NULL when that size is 0); contents on entry are ignored. */
+ *   bytes, 256-byte aligned (may be NULL when that size is 0).  Its first
+ *   FQ_WORKSPACE_SYNC_BYTES (when the size is nonzero) hold the decode
+ *   kernels' counters: they must be zero before the first call on a
+ *   workspace, and every call that returns FQ_OK leaves them as the next
+ *   call needs them (all zero but for the 32-bit word at byte 4, a barrier
+ *   generation number that may hold any value); after a call whose kernels
+ *   recorded FQ_ERR_TIMEOUT, zero them again.  The rest of the workspace may
+ *   hold anything on entry. */
 fq_status fq_w4a4_gemm(const uint8_t* Xq, const void* s_x, const uint8_t* Wq, const void* s_w,
                        int M, int N, int K, fq_gran gran, uint16_t* Y,
                        void* workspace, size_t ws_bytes, void* stream);
@@ -178,17 +189,20 @@ fq_status fq_w4a4_gemm(const uint8_t* Xq, const void* s_x, const uint8_t* Wq, co
  * loop that forbids allocation after start-up).  The pages have no
  * counterpart of this call; it exists for those callers only.
  * Same arguments and results as fq_w4a4_gemm without the workspace: the
- * split-K partial sums use a static 8 MiB device buffer inside libfq.so,
+ * split-K partial sums use a static 32 MiB device buffer inside libfq.so,
  * which every GPU that loads the library holds until the process exits.
- * - Sizes whose split-K scratch (fq_gemm_workspace_size) exceeds 8 MiB are
- *   rejected with FQ_ERR_INVALID; the call enqueues nothing then.
+ * - Sizes whose split-K scratch (fq_gemm_workspace_size) exceeds 32 MiB are
+ *   rejected with FQ_ERR_INVALID; the call enqueues nothing then (on a
+ *   148-SM B200 no size needs more than 20 MiB: the scratch grows with M and
+ *   the number of CTAs, not with N).
  * - The first call on a device that needs the buffer looks up its device
  *   address (cudaGetSymbolAddress) with that device current; make that
  *   first call before any stream capture.
  * - All calls share the one buffer: calls that may overlap on the GPU (on
  *   different streams, or from several threads) race and give wrong
- *   results; serialize them on one stream.  Each call clears the part it
- *   uses before use, so the previous call's contents do no harm.
+ *   results; serialize them on one stream.  The buffer's counters start
+ *   at zero and every call leaves them zero; its partial sums are written
+ *   before they are read, so the previous call's contents do no harm.
  * - Calls no allocating routine (no cudaMalloc/cudaFree). */
 fq_status fq_w4a4_gemm_noalloc(const uint8_t* Xq, const void* s_x, const uint8_t* Wq, const void* s_w,
                                int M, int N, int K, fq_gran gran, uint16_t* Y, void* stream);
@@ -201,10 +215,17 @@ fq_status fq_w4a4_gemm_s32(const uint8_t* Xq, const uint8_t* Wq, int M, int N, i
 /* The linear layer: fq_quant_act into the workspace, then fq_w4a4_gemm, on
  * one stream.  Arguments as in those two calls; Wq/s_w come from
  * fq_quant_weight with the matching inverse transform (and, for
- * FQ_STATIC_CHANNEL, the same static scales folded in; for
- * FQ_ZERO_POINT_MINMAX, the weights' min-max scale block).  workspace must
- * hold fq_linear_workspace_size() bytes (packed activations, their scales and
- * the GEMM's scratch; pass FQ_DYNAMIC_ROW_ZP there for the min-max quantizer). */
+ * FQ_STATIC_CHANNEL and FQ_STATIC_RESIDUAL, the same static scales folded
+ * in; for FQ_ZERO_POINT_MINMAX, the weights' min-max scale block).
+ * Decode (M <= 64) with FQ_STATIC_CHANNEL, no Kronecker factors and 16-byte
+ * aligned static_scale (and c) runs as ONE cooperative launch: the decode
+ * GEMM quantizes the tokens itself (same codes as fq_quant_act) before a
+ * grid-wide barrier; where a cooperative launch is not available it falls
+ * back to the two launches.  workspace: fq_linear_workspace_size() bytes,
+ * 256-byte aligned (the GEMM's scratch with its counter block first, then the
+ * packed activations and their scales; pass FQ_DYNAMIC_ROW_ZP there for the
+ * min-max quantizer); its first FQ_WORKSPACE_SYNC_BYTES follow the rule of
+ * fq_w4a4_gemm's workspace. */
 fq_status fq_linear(const uint16_t* X, int M, int K, const fq_qparams* act_qp,
                     const fq_transform* t, const float* static_scale,
                     const uint8_t* Wq, const void* s_w, int N, uint16_t* Y,

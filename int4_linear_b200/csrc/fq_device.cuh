@@ -184,6 +184,94 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Order this thread's generic-proxy global-memory accesses with its later
+// (or, after an acquire, with other threads' earlier) async-proxy accesses:
+// a TMA load of data that generic stores wrote in the same kernel.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// ------------------------------------------------------------------ grid-wide synchronization
+
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Barrier over the G CTAs of a cooperative launch, on two words of global
+// memory: arrive[0] counts arrivals (atomicInc wraps it back to 0 at the G-th,
+// so it is 0 again after every completed barrier and must be 0 before the
+// first), arrive[1] is a generation number that the last arrival advances.
+// Called by one thread per CTA after a __syncthreads that follows the CTA's
+// writes; the writes of every CTA are visible to the generic and the async
+// proxy of every CTA once grid_barrier_wait returns true.
+__device__ __forceinline__ unsigned grid_barrier_arrive(unsigned* arrive, unsigned G) {
+  const unsigned gen = ld_acquire_gpu(arrive + 1);
+  fence_proxy_async_global();
+  __threadfence();
+  if (atomicInc(arrive, G - 1) == G - 1) {
+    __threadfence();
+    atomicAdd(arrive + 1, 1u);
+  }
+  return gen;
+}
+// false after limit_ns (the error is the caller's to record)
+__device__ __forceinline__ bool grid_barrier_wait(const unsigned* arrive, unsigned gen,
+                                                  uint64_t limit_ns = kWaitLimitNs) {
+  const uint64_t t0 = globaltimer_ns();
+  while (ld_acquire_gpu(arrive + 1) == gen) {
+    if (globaltimer_ns() - t0 > limit_ns) return false;
+    __nanosleep(100);
+  }
+  fence_proxy_async_global();
+  return true;
+}
+
+// ------------------------------------------------------------------ static INT4 codes
+
+// Symmetric INT4 code of v with scale s: clamp(rint(v / s), -8, 7) after an
+// IEEE division (rint rounds half to even); 0 when s = 0.
+__device__ __forceinline__ int rtn_code(float v, float s) {
+  if (s == 0.0f) return 0;
+  const float r = rintf(__fdiv_rn(v, s));
+  return static_cast<int>(fminf(fmaxf(r, -8.0f), 7.0f));
+}
+
+// Eight packed static codes (low nibble first) of the fp16 values in `raw`
+// with the per-channel scales s[0..7] and, when c is non-NULL, the channel
+// factors c[0..7] applied first (v = fl32(x c)).  s and c 16-byte aligned.
+// When v_out is non-NULL the eight values v are written there.
+__device__ __forceinline__ uint32_t static_codes8(uint4 raw, const float* __restrict__ s,
+                                                  const float* __restrict__ c, float* v_out = nullptr) {
+  const __half2* h2 = reinterpret_cast<const __half2*>(&raw);
+  const float4 s0 = __ldg(reinterpret_cast<const float4*>(s));
+  const float4 s1 = __ldg(reinterpret_cast<const float4*>(s + 4));
+  const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+  float v[8];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float2 f = __half22float2(h2[j]);
+    v[2 * j] = f.x;
+    v[2 * j + 1] = f.y;
+  }
+  if (c) {
+    const float4 c0 = __ldg(reinterpret_cast<const float4*>(c));
+    const float4 c1 = __ldg(reinterpret_cast<const float4*>(c + 4));
+    const float cv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = __fmul_rn(v[j], cv[j]);
+  }
+  uint32_t word = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) word |= (uint32_t(rtn_code(v[j], sv[j])) & 0xFu) << (4 * j);
+  if (v_out) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v_out[j] = v[j];
+  }
+  return word;
+}
+
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }

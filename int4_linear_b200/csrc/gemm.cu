@@ -131,9 +131,26 @@ struct GemmParams {
   const __half* gsx;  // [K/128][M]    group scales of the activations
   const __half* gsw;  // [K/128][N]    group scales of the weights
   __half* Y;          // [M][N]
-  int32_t* acc;       // [M][N]        int32 output / decode stream-K partial sums
+  int32_t* acc;       // [M][N]        int32 output
   unsigned* err;
+  // decode
+  unsigned* sync;     // the workspace's synchronization block (all zero between calls)
+  int32_t* slots;     // [2 G][M][128]  int32 partial sums of the tiles split between CTAs
+  // fused decode linear: the tokens are quantized inside the GEMM launch
+  const __half* X;    // [M][K]        fp16 tokens
+  const float* sst;   // [K]           static scales
+  const float* cst;   // [K] or null   channel factors
+  uint8_t* Xq;        // [M][K/2]      their packed codes (the B operand)
 };
+
+// The first kSyncBytes of a decode workspace: word 0 counts the CTAs at the
+// fused kernel's grid barrier, word 1 is that barrier's generation number,
+// words kSyncTile0 + t count the CTAs that have stored their share of split
+// tile t.  Every counter returns to 0 by the end of a call (the generation
+// number only changes).
+constexpr size_t kSyncBytes = FQ_WORKSPACE_SYNC_BYTES;
+constexpr int kSyncTile0 = 16;
+constexpr int kMaxSyncTiles = int(kSyncBytes / 4) - kSyncTile0;
 
 __device__ __forceinline__ void store_half8(__half* dst, const float* v) {
   uint4 o;
@@ -997,24 +1014,54 @@ __global__ void __launch_bounds__(PCfg<NB>::THREADS, 1)
 // the (tile, K slice) pairs, tile-major, are split into equal contiguous
 // ranges, one per CTA (stream-K), so every CTA streams the same number of
 // weight bytes whatever the tile count.  A range covers whole tiles and at
-// most a partial tile at each end; whole tiles are written directly, the
-// partial ones add their exact int32 sums into the caller's workspace and
-// decode_fixup_kernel dequantizes those tiles afterwards.
+// most a partial tile at each end; whole tiles are written directly.  For a
+// split tile each CTA stores its exact int32 sums into its own slot of the
+// workspace and counts itself in on the tile's counter; the CTA that arrives
+// last adds the slots of all the tile's CTAs (integer sums: the order does
+// not matter), dequantizes and writes the tile, and its arrival has already
+// wrapped the counter back to 0.
+// Fused decode linear (FUSED): the tokens arrive as fp16 and each CTA first
+// quantizes an equal share of them with the static per-channel scales (the
+// same static_codes8 as fq_quant_act) into the workspace; a grid barrier
+// (the launch is cooperative, so every CTA is resident) orders those codes
+// before the first token tile is loaded.  The first weight stages are issued
+// before the quantization, so the weight stream starts at once.
 //   warp 0      one thread issues TMA loads of packed 128 x 64-byte weight
 //               slices (64-byte swizzle) and the tokens' slices into a ring
 //   warp 1      tensor-memory allocation and the MMA-issuing thread; the
 //               accumulator is double-buffered across tile segments
-//   warps 2-5   read one weight row each from the ring, unpack it into a
-//               tensor-memory A ring
-//   warps 6-7   unpack the tokens into the 128-byte-swizzled B ring
-//   warps 8-11  epilogue of each tile segment, overlapping the next one
-constexpr int kDecWarps = 12;
-constexpr int kDecThreads = 32 * kDecWarps;
+//   UG groups of 4 warps read one weight row each from the ring and unpack it
+//               into a tensor-memory A ring (group g takes the slices
+//               i = g mod UG, so UG slices are unpacked at once)
+//   UG groups of 2 warps unpack the tokens into the 128-byte-swizzled B ring
+//   4 warps     epilogue of each tile segment, overlapping the next one
+// Two CTAs per SM run one unpacking group each; the fused kernel's single
+// CTA per SM runs two.
 
-template <int BN>
+// ONE: one CTA per SM (the fused kernel's cooperative launch: the occupancy
+// calculation counts one resident CTA per SM for kernels that allocate
+// tensor memory), with a deeper ring to keep as many weight bytes in flight
+// as two CTAs do.
+template <int BN, bool ONE = false>
 struct DecCfg {
-  static constexpr int SP = BN == 64 ? 6 : 8;     // packed stages (TMA ring: weights + tokens)
-  static constexpr int SU = 4;                    // unpacked stages
+  static constexpr int SP = ONE ? (BN == 64 ? 12 : 16) : (BN == 64 ? 6 : 8);  // packed stages (weights + tokens)
+  static constexpr int UG = ONE ? 2 : 1;          // unpacking groups
+  static constexpr int ACC = BN < 32 ? 32 : BN;   // columns of one accumulator
+  // MMA-issuing threads (warp 1, then warps I_WARP0...): a tcgen05.mma of
+  // N = BN <= 64 holds its issuing thread for about as long as the tensor
+  // core needs for it, so one issuer caps a CTA at about one K slice per four
+  // MMA issue times.  Issuer j issues k-steps j, j + NI, ... of every slice
+  // into its own accumulator; the epilogue adds the NI accumulators.
+  static constexpr int NI = ONE ? (BN == 64 ? 2 : 4) : 2;
+  // accumulator buffers per issuer (2: the epilogue of one tile segment
+  // overlaps the MMAs of the next)
+  static constexpr int NACC = (!ONE && BN == 64) ? 1 : 2;
+  static constexpr int W_WARP0 = 2;               // first weight-unpacking warp
+  static constexpr int T_WARP0 = W_WARP0 + 4 * UG;  // first token-unpacking warp
+  static constexpr int E_WARP0 = T_WARP0 + 2 * UG;  // first epilogue warp
+  static constexpr int I_WARP0 = E_WARP0 + 4;     // issuers 1 .. NI - 1
+  static constexpr int THREADS = 32 * (I_WARP0 + NI - 1);
+  static constexpr int SU = ONE ? 8 : 4;          // unpacked stages (each a full MMA round trip deep)
   static constexpr int P_STAGE = kBM * kPK;       // weights: 128 rows x 64 bytes
   static constexpr int X_STAGE = BN * kPK;        // tokens: BN rows x 64 bytes
   static constexpr int B_STAGE = BN * kBK;        // BN rows x 128 int8, 128-byte swizzle
@@ -1023,18 +1070,21 @@ struct DecCfg {
   static constexpr int OFF_B = OFF_X + SP * X_STAGE;
   static constexpr int OFF_BAR = OFF_B + SU * B_STAGE;
   static constexpr int NBAR = 2 * SP + 2 * SU + 5;
-  static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
-  // at least 80 KB, so that no more than two CTAs (2 x 256 tensor-memory
-  // columns) are resident on one SM
-  static constexpr int SMEM = (OFF_TMEM + 16 + 1024) > 80 * 1024 ? (OFF_TMEM + 16 + 1024) : 80 * 1024;
-  static constexpr int ACC = BN < 32 ? 32 : BN;   // columns of one accumulator buffer
-  static constexpr int A_COL0 = 2 * ACC;          // accumulators in columns [0, 2 ACC)
+  static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;  // tmem address, count of tiles to finish, those tiles
+  // two per SM: at least 80 KB, so that no more than two CTAs (2 x 256
+  // tensor-memory columns) are resident on one SM
+  static constexpr int SMEM_MIN = ONE ? 0 : 80 * 1024;
+  static constexpr int SMEM = (OFF_TMEM + 16 + 1024) > SMEM_MIN ? (OFF_TMEM + 16 + 1024) : SMEM_MIN;
+  static constexpr int A_COL0 = NACC * NI * ACC;  // accumulators: [buffer][issuer][ACC]
   static constexpr int A_STAGE_COLS = kBK / 4;
   static constexpr int TMEM_NEED = A_COL0 + SU * A_STAGE_COLS;
-  static constexpr int TMEM_COLS = TMEM_NEED <= 128 ? 128 : 256;
+  static constexpr int TMEM_COLS = TMEM_NEED <= 128 ? 128 : (TMEM_NEED <= 256 ? 256 : 512);
   static_assert(B_STAGE % 1024 == 0 && P_STAGE % 1024 == 0 && X_STAGE % 1024 == 0, "stage alignment");
-  static_assert(TMEM_NEED <= 256, "two CTAs per SM share the tensor memory");
-  static_assert(2 * (SMEM + 1024) <= 228 * 1024, "two CTAs per SM");
+  static_assert(TMEM_NEED <= (ONE ? 512 : 256), "tensor memory of the CTAs resident on one SM");
+  static_assert(ONE ? SMEM <= 227 * 1024 : 2 * (SMEM + 1024) <= 228 * 1024, "resident CTAs per SM");
+  static_assert(SP * P_STAGE >= 512, "the finishing pass keeps its slot table in the weight ring");
+  static_assert(SP % UG == 0 && SU % UG == 0, "each stage is used by one unpacking group");
+  static_assert((kBK / 32) % NI == 0, "every issuer issues the same k-steps of each slice");
 };
 
 // The slice range [b0, b1) of CTA c among g CTAs over t slices, and the CTA
@@ -1044,11 +1094,11 @@ __host__ __device__ __forceinline__ int sk_owner(long long s, long long g, long 
   return int(((s + 1) * g - 1) / t);
 }
 
-template <int BN, int EPI>
-__global__ void __launch_bounds__(kDecThreads, 2)
+template <int BN, int EPI, bool FUSED>
+__global__ void __launch_bounds__(DecCfg<BN, FUSED>::THREADS, FUSED ? 1 : 2)
     gemm_decode_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tmA,
                        const __grid_constant__ CUtensorMap tmX) {
-  using C = DecCfg<BN>;
+  using C = DecCfg<BN, FUSED>;
   constexpr int SP = C::SP, SU = C::SU;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -1061,27 +1111,31 @@ __global__ void __launch_bounds__(kDecThreads, 2)
   uint64_t* acc_empty = acc_full + 2;  // [2]
   uint64_t* done_bar = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM);
+  int* fin = reinterpret_cast<int*>(smem + C::OFF_TMEM + 4);  // [0] count, [1..2] split tiles this CTA finishes
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nkb = p.num_kb;
   const long long T = (long long)((p.rowsA + kBM - 1) / kBM) * nkb;
   const long long b0 = sk_begin(blockIdx.x, gridDim.x, T), b1 = sk_begin(blockIdx.x + 1, gridDim.x, T);
   const int nsl = int(b1 - b0);  // slices of this CTA
+  // fused: stages whose weight tiles are issued before the token quantization
+  const int pre = FUSED ? min(nsl, SP) : 0;
 
   if (threadIdx.x == 0) {
+    fin[0] = 0;
     for (int s = 0; s < SP; ++s) {
       mbar_init(&pfull[s], 1);
       mbar_init(&pempty[s], 6);  // 4 weight-row warps + 2 token warps
     }
     for (int s = 0; s < SU; ++s) {
       mbar_init(&ufull[s], 6);
-      mbar_init(&uempty[s], 1);
+      mbar_init(&uempty[s], C::NI);
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_full[b], C::NI);
       mbar_init(&acc_empty[b], 4);
     }
-    mbar_init(done_bar, 1);
+    mbar_init(done_bar, C::NI);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -1095,6 +1149,32 @@ __global__ void __launch_bounds__(kDecThreads, 2)
   pdl_launch_dependents();
   pdl_wait();
 
+  unsigned gen = 0;
+  if (FUSED) {
+    // the first weight stages (their barriers expect the token bytes too)
+    if (threadIdx.x == 0) {
+      prefetch_tensormap(&tmA);
+      const uint64_t pol = policy_evict_first();
+      int tile = int(b0 / nkb), kb = int(b0 - (long long)tile * nkb);
+      for (int i = 0; i < pre; ++i, kb = kb + 1 == nkb ? 0 : kb + 1, tile += kb == 0) {
+        mbar_arrive_expect_tx(&pfull[i], C::P_STAGE + C::X_STAGE);
+        tma_load_2d_hint(smem + C::OFF_P + i * C::P_STAGE, &tmA, &pfull[i], kb * kPK, tile * kBM, pol);
+      }
+    }
+    // this CTA's share of the token codes, 8 per thread-iteration
+    const int kp = p.K / 8;
+    const long long pieces = (long long)p.M * kp;
+    const long long lo = pieces * blockIdx.x / gridDim.x, hi = pieces * (blockIdx.x + 1) / gridDim.x;
+    for (long long pc = lo + threadIdx.x; pc < hi; pc += C::THREADS) {
+      const int r = int(pc / kp), e0 = int(pc - (long long)r * kp) * 8;
+      const uint4 raw = *reinterpret_cast<const uint4*>(p.X + size_t(r) * p.K + e0);
+      const uint32_t word = static_codes8(raw, p.sst + e0, p.cst ? p.cst + e0 : nullptr);
+      reinterpret_cast<uint32_t*>(p.Xq + size_t(r) * (p.K / 2))[e0 / 8] = word;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) gen = grid_barrier_arrive(p.sync, gridDim.x);
+  }
+
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
@@ -1104,7 +1184,16 @@ __global__ void __launch_bounds__(kDecThreads, 2)
       const uint64_t pol_x = policy_evict_last();  // the tokens are read by every CTA
       int issued = 0;
       int tile = int(b0 / nkb), kb = int(b0 - (long long)tile * nkb);  // advanced per slice
-      for (int i = 0; i < nsl; ++i, kb = kb + 1 == nkb ? 0 : kb + 1, tile += kb == 0) {
+      if (FUSED) {
+        // the token codes of every CTA are in memory; on a timeout the error
+        // is recorded and the pipeline still runs to its end (every copy
+        // lands, the results are not to be used)
+        if (!grid_barrier_wait(p.sync, gen)) record_error(p.err, kErrTimeoutProducer);
+        for (int i = 0; i < pre; ++i, kb = kb + 1 == nkb ? 0 : kb + 1, tile += kb == 0)
+          tma_load_2d_hint(smem + C::OFF_X + i * C::X_STAGE, &tmX, &pfull[i], kb * kPK, 0, pol_x);
+        issued = pre;
+      }
+      for (int i = pre; i < nsl; ++i, kb = kb + 1 == nkb ? 0 : kb + 1, tile += kb == 0) {
         const int sp = i % SP;
         if (!mbar_wait(&pempty[sp], ((i / SP) & 1) ^ 1)) {
           record_error(p.err, kErrTimeoutProducer);
@@ -1123,9 +1212,10 @@ __global__ void __launch_bounds__(kDecThreads, 2)
           break;
         }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 || warp >= C::I_WARP0) {
+    // ------------------------------------------------------------ MMA issuers
     if (lane == 0) {
+      const int iss = warp == 1 ? 0 : warp - C::I_WARP0 + 1;
       constexpr uint32_t idesc = idesc_i8_m128(BN);
       int seg = -1;
       bool ok = true;
@@ -1138,7 +1228,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
           // the first use of each buffer passes at once (the wait is for the
           // phase before the first); later uses wait for the epilogue of the
           // segment two back
-          if (!mbar_wait(&acc_empty[seg & 1], ((seg >> 1) & 1) ^ 1)) {
+          if (!mbar_wait(&acc_empty[seg % C::NACC], ((seg / C::NACC) & 1) ^ 1)) {
             record_error(p.err, kErrTimeoutMma);
             break;
           }
@@ -1149,26 +1239,27 @@ __global__ void __launch_bounds__(kDecThreads, 2)
           break;
         }
         tc_fence_after();
-        const uint32_t d = tmem + uint32_t((seg & 1) * C::ACC);
+        const uint32_t d = tmem + uint32_t(((seg % C::NACC) * C::NI + iss) * C::ACC);
         const uint32_t a0 = tmem + uint32_t(C::A_COL0 + su * C::A_STAGE_COLS);
         const uint32_t bsm = smem_u32(smem + C::OFF_B + su * C::B_STAGE);
 #pragma unroll
-        for (int k = 0; k < kBK / 32; ++k)
-          mma_i8_ts(d, a0 + uint32_t(8 * k), sdesc_k128_sw128(bsm + 32 * k), idesc, uint32_t(!first || k > 0));
+        for (int k = iss; k < kBK / 32; k += C::NI)
+          mma_i8_ts(d, a0 + uint32_t(8 * k), sdesc_k128_sw128(bsm + 32 * k), idesc, uint32_t(!first || k >= C::NI));
         mma_commit(&uempty[su]);
-        if (last) mma_commit(&acc_full[seg & 1]);
+        if (last) mma_commit(&acc_full[seg % C::NACC]);
       }
       mma_commit(done_bar);
       if (!mbar_wait(done_bar, 0)) record_error(p.err, kErrTimeoutDrain);
     }
-  } else if (warp < 6) {
+  } else if (warp < C::T_WARP0) {
     // ------------------------------------------------------------ weight rows -> tensor memory
-    const int q = warp & 3;
+    const int q = warp & 3;  // tensor-memory lane quadrant this warp may access
+    const int grp = (warp - C::W_WARP0) >> 2;
     const int row = q * 32 + lane;
     const uint32_t ta = tmem + (uint32_t(q * 32) << 16) + uint32_t(C::A_COL0);
     const int sw = (row >> 1) & 3;  // 64-byte swizzle: chunk c of this row sits at chunk c ^ sw
     bool ok = true;
-    for (int i = 0; i < nsl; ++i) {
+    for (int i = grp; i < nsl; i += C::UG) {
       const int sp = i % SP, su = i % SU;
       if (!warp_wait(&pfull[sp], (i / SP) & 1)) {
         ok = false;
@@ -1205,14 +1296,15 @@ __global__ void __launch_bounds__(kDecThreads, 2)
       }
     }
     if (!ok && lane == 0) record_error(p.err, kErrTimeoutUnpack);
-  } else if (warp < 8) {
+  } else if (warp < C::E_WARP0) {
     // ------------------------------------------------------------ token rows -> shared memory
     // The packed token slice arrives with the weights in the TMA ring; each
     // lane unpacks fixed 16-byte pieces (consecutive lanes read consecutive
     // pieces, so the reads are free of bank conflicts).
     constexpr int kJobs = BN * 4;                  // 16-byte packed pieces per stage
     constexpr int JPT = (kJobs + 63) / 64;         // per thread (two warps)
-    const int t = (warp - 6) * 32 + lane;
+    const int grp = (warp - C::T_WARP0) >> 1;
+    const int t = ((warp - C::T_WARP0) & 1) * 32 + lane;
     uint32_t dst0[JPT], dst1[JPT];
     bool live[JPT];
 #pragma unroll
@@ -1225,7 +1317,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
       dst1[it] = rb + uint32_t(((2 * c + 1) ^ r7) << 4);
     }
     bool ok = true;
-    for (int i = 0; i < nsl; ++i) {
+    for (int i = grp; i < nsl; i += C::UG) {
       const int sp = i % SP, su = i % SU;
       if (!warp_wait(&pfull[sp], (i / SP) & 1)) {
         ok = false;
@@ -1264,48 +1356,80 @@ __global__ void __launch_bounds__(kDecThreads, 2)
   } else {
     // ------------------------------------------------------------ epilogue: thread = output channel n
     const int q = warp & 3;
+    const int nl = q * 32 + lane;  // channel within the tile
     const uint32_t tl = tmem + (uint32_t(q * 32) << 16);
+    const int tile0 = int(b0 / nkb);
     long long s = b0;
     for (int seg = 0; s < b1; ++seg) {
       const int tile = int(s / nkb), kb_lo = int(s - (long long)tile * nkb);
       const int len = int(min((long long)(nkb - kb_lo), b1 - s));
       const bool whole = kb_lo == 0 && len == nkb;
       s += len;
-      const int b = seg & 1;
-      if (!warp_wait(&acc_full[b], (seg >> 1) & 1)) {
+      const int b = seg % C::NACC;
+      // the four epilogue warps agree on the outcome (they meet at named barriers below)
+      const bool ok = warp_wait(&acc_full[b], (seg / C::NACC) & 1);
+      if (named_barrier_or(1, 128, !ok)) {
         if (lane == 0) record_error(p.err, kErrTimeoutEpilogue);
         break;
       }
       tc_fence_after();
-      const int n = tile * kBM + q * 32 + lane;
+      const int n = tile * kBM + nl;
       const float swn = (EPI == kEpiRow || EPI == kEpiStatic) && n < p.N ? __ldg(p.sw + n) : 0.f;
+      // this CTA's slot for a split tile: 2c for its first tile, 2c + 1 for its last
+      int32_t* slot = whole ? nullptr : p.slots + (size_t(2 * blockIdx.x + (tile == tile0 ? 0 : 1)) * p.M) * kBM + nl;
       constexpr int CW = BN >= 32 ? 32 : 16;
 #pragma unroll
       for (int c0 = 0; c0 < BN; c0 += CW) {
         uint32_t v[32];
+        const uint32_t col = tl + uint32_t(b * C::NI * C::ACC + c0);
         if (CW == 32)
-          tmem_ld_32x32(tl + uint32_t(b * C::ACC + c0), v);
+          tmem_ld_32x32(col, v);
         else
-          tmem_ld_32x16(tl + uint32_t(b * C::ACC + c0), v);
+          tmem_ld_32x16(col, v);
         tmem_wait_ld();
-        if (n < p.N) {
 #pragma unroll
-          for (int j = 0; j < CW; ++j) {
-            const int m = c0 + j;
-            if (m >= p.M) break;
-            const int32_t ai = int32_t(v[j]) >> 8;
-            if (!whole)
-              atomicAdd(p.acc + size_t(m) * p.N + n, ai);
-            else if (EPI == kEpiRow)
-              p.Y[size_t(m) * p.N + n] = __float2half_rn(__fmul_rn(__fmul_rn(float(ai), __ldg(p.sx + m)), swn));
-            else
-              p.Y[size_t(m) * p.N + n] = __float2half_rn(__fmul_rn(float(ai), swn));
-          }
+        for (int ch = 1; ch < C::NI; ++ch) {
+          uint32_t w[32];
+          if (CW == 32)
+            tmem_ld_32x32(col + uint32_t(ch * C::ACC), w);
+          else
+            tmem_ld_32x16(col + uint32_t(ch * C::ACC), w);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < CW; ++j) v[j] += w[j];  // exact int32 sums (two's complement)
+        }
+#pragma unroll
+        for (int j = 0; j < CW; ++j) {
+          const int m = c0 + j;
+          if (m >= p.M) break;
+          const int32_t ai = int32_t(v[j]) >> 8;
+          if (!whole)
+            slot[size_t(m) * kBM] = ai;
+          else if (n >= p.N)
+            continue;
+          else if (EPI == kEpiRow)
+            p.Y[size_t(m) * p.N + n] = __float2half_rn(__fmul_rn(__fmul_rn(float(ai), __ldg(p.sx + m)), swn));
+          else
+            p.Y[size_t(m) * p.N + n] = __float2half_rn(__fmul_rn(float(ai), swn));
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[b]);
+      if (whole) continue;
+      // split tile: count in; the last of its CTAs finishes it at the end
+      named_barrier(1, 128);  // every slot row of this CTA is stored
+      if (warp == C::E_WARP0 && lane == 0) {
+        __threadfence();
+        const int cf = sk_owner((long long)tile * nkb, gridDim.x, T);
+        const int cl = sk_owner((long long)(tile + 1) * nkb - 1, gridDim.x, T);
+        const unsigned nc = unsigned(cl - cf + 1);
+        if (atomicInc(p.sync + kSyncTile0 + tile, nc - 1) == nc - 1) {
+          __threadfence();
+          fin[1 + fin[0]] = tile;
+          fin[0] += 1;
+        }
+      }
     }
   }
 
@@ -1315,25 +1439,56 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
-}
 
-// y = dequant(int32 sums) for the tiles that the stream-K ranges split
-// between CTAs (the others were written directly by the decode kernel): one
-// CTA of 128 threads per tile of 128 output channels, thread = channel.
-__global__ void __launch_bounds__(128) decode_fixup_kernel(const int32_t* __restrict__ acc,
-                                                           const float* __restrict__ sx,
-                                                           const float* __restrict__ sw, __half* __restrict__ Y,
-                                                           int M, int N, int nkb, int g, int row_mode) {
-  const long long T = (long long)((N + kBM - 1) / kBM) * nkb;
-  const long long t = blockIdx.x;
-  if (sk_owner(t * nkb, g, T) == sk_owner((t + 1) * nkb - 1, g, T)) return;  // one CTA wrote the tile
-  const int n = int(t) * kBM + threadIdx.x;
-  if (n >= N) return;
-  const float swn = sw[n];
-  for (int m = blockIdx.y; m < M; m += gridDim.y) {
-    const float a = float(acc[size_t(m) * N + n]);
-    const float y = row_mode ? __fmul_rn(__fmul_rn(a, sx[m]), swn) : __fmul_rn(a, swn);
-    Y[size_t(m) * N + n] = __float2half_rn(y);
+  // The split tiles this CTA arrived last at (at most its first and its
+  // last): every thread adds the CTAs' slots, 4 channels per 16-byte load,
+  // and writes the fp16 outputs.  The weight ring is idle now; it holds the
+  // slot index of each contributing CTA.
+  const int nfin = fin[0];
+  int* sidx = reinterpret_cast<int*>(smem + C::OFF_P);
+  for (int f = 0; f < nfin; ++f) {
+    const int tile = fin[1 + f];
+    const int cf = sk_owner((long long)tile * nkb, gridDim.x, T);
+    const int cl = sk_owner((long long)(tile + 1) * nkb - 1, gridDim.x, T);
+    const int nc = cl - cf + 1;
+    const long long t_lo = (long long)tile * nkb;
+    __syncthreads();  // the previous tile's readers are done with sidx
+    for (int j = threadIdx.x; j < nc; j += C::THREADS)
+      sidx[j] = 2 * (cf + j) + (sk_begin(cf + j, gridDim.x, T) >= t_lo ? 0 : 1);
+    __syncthreads();
+    for (int it = threadIdx.x; it < p.M * (kBM / 4); it += C::THREADS) {
+      const int m = it / (kBM / 4), nl = (it % (kBM / 4)) * 4;
+      const int n = tile * kBM + nl;
+      if (n >= p.N) continue;  // N % 8 == 0: four channels are all in range or all out
+      int4 a = make_int4(0, 0, 0, 0);
+#pragma unroll 8
+      for (int j = 0; j < nc; ++j) {
+        const int4 v = __ldcg(reinterpret_cast<const int4*>(p.slots + (size_t(sidx[j]) * p.M + m) * kBM + nl));
+        a.x += v.x;
+        a.y += v.y;
+        a.z += v.z;
+        a.w += v.w;
+      }
+      const float4 w = make_float4(__ldg(p.sw + n), __ldg(p.sw + n + 1), __ldg(p.sw + n + 2), __ldg(p.sw + n + 3));
+      float y[4];
+      if (EPI == kEpiRow) {
+        const float sxm = __ldg(p.sx + m);
+        y[0] = __fmul_rn(__fmul_rn(float(a.x), sxm), w.x);
+        y[1] = __fmul_rn(__fmul_rn(float(a.y), sxm), w.y);
+        y[2] = __fmul_rn(__fmul_rn(float(a.z), sxm), w.z);
+        y[3] = __fmul_rn(__fmul_rn(float(a.w), sxm), w.w);
+      } else {
+        y[0] = __fmul_rn(float(a.x), w.x);
+        y[1] = __fmul_rn(float(a.y), w.y);
+        y[2] = __fmul_rn(float(a.z), w.z);
+        y[3] = __fmul_rn(float(a.w), w.w);
+      }
+      uint2 o;
+      __half2* h = reinterpret_cast<__half2*>(&o);
+      h[0] = __floats2half2_rn(y[0], y[1]);
+      h[1] = __floats2half2_rn(y[2], y[3]);
+      *reinterpret_cast<uint2*>(p.Y + size_t(m) * p.N + n) = o;
+    }
   }
 }
 
@@ -1378,12 +1533,14 @@ struct Plan {
   int bn;
   int epi;
   int ctas;           // decode: persistent CTAs sharing the slice sequence
-  bool partial;       // decode: some tile is split between CTAs (workspace + fixup)
+  bool partial;       // decode: some tile is split between CTAs (workspace slots + counters)
 };
 
 int pick_bn_swap(int M) { return M <= 16 ? 16 : (M <= 32 ? 32 : 64); }
 
-Plan make_plan(int M, int N, int K, int epi_final, int sms) {
+// fused: the decode kernel that quantizes the tokens itself waits at a grid
+// barrier, so all its CTAs must be resident: one wave at most.
+Plan make_plan(int M, int N, int K, int epi_final, int sms, bool fused = false) {
   Plan pl{};
   const int nkb = K / kBK;
   if (epi_final == kEpiGroup) {
@@ -1407,11 +1564,11 @@ Plan make_plan(int M, int N, int K, int epi_final, int sms) {
   const long long tiles = (N + kBM - 1) / kBM;
   const long long T = tiles * nkb;
   // One CTA per tile when the tiles alone fill the resident slots and the
-  // token count makes the partial-tile path (workspace clear, int32 atomics,
-  // fixup) cost more than the last wave's imbalance; otherwise stream-K over
+  // token count makes the split-tile path (slot stores, the finishing CTA's
+  // reads) cost more than the last wave's imbalance; otherwise stream-K over
   // one wave.
-  const long long slots = 2LL * sms;
-  if (tiles >= slots && M > 16)
+  const long long slots = (fused ? 1LL : 2LL) * sms;
+  if (tiles >= slots && M > 16 && !fused)
     pl.ctas = int(tiles);
   else
     pl.ctas = int(std::max<long long>(1, std::min<long long>(slots, T / 8)));
@@ -1475,9 +1632,9 @@ fq_status launch_gemm_persistent(const GemmParams& gp, cudaStream_t stream) {
   return check_launch("gemm_w4a4_persistent_kernel");
 }
 
-template <int BN, int EPI>
+template <int BN, int EPI, bool FUSED>
 fq_status launch_decode(const GemmParams& gp, dim3 grid, cudaStream_t stream) {
-  using C = DecCfg<BN>;
+  using C = DecCfg<BN, FUSED>;
   CUtensorMap tm, tx;
   fq_status st = make_tmap_2d(&tm, gp.A, CU_TENSOR_MAP_DATA_TYPE_UINT8, uint64_t(gp.K) / 2, uint64_t(gp.rowsA),
                               uint64_t(gp.K) / 2, uint32_t(kPK), uint32_t(kBM), CU_TENSOR_MAP_SWIZZLE_64B);
@@ -1485,14 +1642,29 @@ fq_status launch_decode(const GemmParams& gp, dim3 grid, cudaStream_t stream) {
   st = make_tmap_2d(&tx, gp.B, CU_TENSOR_MAP_DATA_TYPE_UINT8, uint64_t(gp.K) / 2, uint64_t(gp.rowsB), uint64_t(gp.K) / 2,
                     uint32_t(kPK), uint32_t(BN));
   if (st != FQ_OK) return st;
-  auto kern = gemm_decode_kernel<BN, EPI>;
+  auto kern = gemm_decode_kernel<BN, EPI, FUSED>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess ||
       cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
     return fail(FQ_ERR_CUDA, "cannot reserve %d bytes of shared memory for the decode GEMM", C::SMEM);
-  const cudaError_t e = launch_pdl(kern, grid, dim3(kDecThreads), C::SMEM, stream, gp, tm, tx);
-  if (e != cudaSuccess) {
-    cudaGetLastError();
-    return fail(FQ_ERR_CUDA, "gemm_decode_kernel: %s", cudaGetErrorString(e));
+  if (FUSED) {
+    // every CTA must be resident at once for the grid barrier
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, C::THREADS, C::SMEM) != cudaSuccess ||
+        static_cast<long long>(per_sm) * sm_count() < static_cast<long long>(grid.x)) {
+      cudaGetLastError();
+      return FQ_ERR_UNSUPPORTED;  // the caller quantizes separately
+    }
+    const cudaError_t e = launch_coop_pdl(kern, grid, dim3(C::THREADS), C::SMEM, stream, gp, tm, tx);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return FQ_ERR_UNSUPPORTED;
+    }
+  } else {
+    const cudaError_t e = launch_pdl(kern, grid, dim3(C::THREADS), C::SMEM, stream, gp, tm, tx);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return fail(FQ_ERR_CUDA, "gemm_decode_kernel: %s", cudaGetErrorString(e));
+    }
   }
   return check_launch("gemm_decode_kernel");
 }
@@ -1511,8 +1683,10 @@ fq_status dispatch(const Plan& pl, const GemmParams& gp, dim3 grid, cudaStream_t
 #define FQ_SWAP_CASES(BNV)                                                     \
   if (pl.bn == BNV) {                                                          \
     switch (pl.epi) {                                                          \
-      case kEpiRow: return launch_decode<BNV, kEpiRow>(gp, grid, s);           \
-      case kEpiStatic: return launch_decode<BNV, kEpiStatic>(gp, grid, s);     \
+      case kEpiRow: return launch_decode<BNV, kEpiRow, false>(gp, grid, s);    \
+      case kEpiStatic:                                                         \
+        return gp.X ? launch_decode<BNV, kEpiStatic, true>(gp, grid, s)        \
+                    : launch_decode<BNV, kEpiStatic, false>(gp, grid, s);      \
       default: break;                                                          \
     }                                                                          \
   }
@@ -1524,6 +1698,22 @@ fq_status dispatch(const Plan& pl, const GemmParams& gp, dim3 grid, cudaStream_t
   return fail(FQ_ERR_UNSUPPORTED, "no GEMM variant for this plan");
 }
 
+// Tokens that the fused decode kernel quantizes itself (static scales).
+struct FusedTokens {
+  const __half* X;
+  const float* sst;
+  const float* cst;
+};
+
+// Decode workspace: the synchronization block, then the split tiles' slots
+// (two per CTA).  The fused kernel always needs the block (its grid barrier).
+size_t decode_ws_bytes(const Plan& pl, int M, int N, bool fused) {
+  (void)N;
+  if (!pl.swap) return 0;
+  if (!pl.partial) return fused ? kSyncBytes : 0;
+  return kSyncBytes + size_t(2) * pl.ctas * M * kBM * sizeof(int32_t);
+}
+
 fq_status check_sizes(int M, int N, int K) {
   FQ_CHECK_ARG(M >= 1, "M = %d must be >= 1", M);
   FQ_CHECK_ARG(N >= 8 && N % 8 == 0, "N = %d must be a positive multiple of 8", N);
@@ -1532,7 +1722,8 @@ fq_status check_sizes(int M, int N, int K) {
 }
 
 fq_status gemm_impl(const uint8_t* Xq, const void* s_x, const uint8_t* Wq, const void* s_w, int M, int N, int K,
-                    int epi_final, uint16_t* Y, int32_t* acc_out, void* ws, size_t ws_bytes, cudaStream_t stream) {
+                    int epi_final, uint16_t* Y, int32_t* acc_out, void* ws, size_t ws_bytes, cudaStream_t stream,
+                    const FusedTokens* fused = nullptr) {
   fq_status st = check_sizes(M, N, K);
   if (st != FQ_OK) return st;
   FQ_CHECK_ARG(Xq && Wq, "Xq and Wq must be non-NULL");
@@ -1547,9 +1738,11 @@ fq_status gemm_impl(const uint8_t* Xq, const void* s_x, const uint8_t* Wq, const
   unsigned* err = device_error_word();
   if (!err) return fail(FQ_ERR_CUDA, "device error word unavailable");
   const int sms = sm_count();
-  Plan pl = make_plan(M, N, K, epi_final, sms);
-  const size_t need = (pl.swap && pl.partial) ? size_t(M) * N * sizeof(int32_t) : 0;
-  if (need > 0) FQ_CHECK_ARG(ws && ws_bytes >= need && aligned(ws, 16), "workspace of %zu bytes required", need);
+  Plan pl = make_plan(M, N, K, epi_final, sms, fused != nullptr);
+  const size_t need = decode_ws_bytes(pl, M, N, fused != nullptr);
+  if (need > 0) FQ_CHECK_ARG(ws && ws_bytes >= need && aligned(ws, 256), "workspace of %zu bytes required", need);
+  if (pl.swap && pl.partial)
+    FQ_CHECK_ARG((N + kBM - 1) / kBM <= kMaxSyncTiles, "N = %d has more than %d tiles of 128", N, kMaxSyncTiles);
 
   GemmParams gp{};
   gp.M = M;
@@ -1564,7 +1757,17 @@ fq_status gemm_impl(const uint8_t* Xq, const void* s_x, const uint8_t* Wq, const
     gp.gsx = static_cast<const __half*>(s_x);
     gp.gsw = static_cast<const __half*>(s_w);
   }
-  gp.acc = epi_final == kEpiS32 ? acc_out : (need > 0 ? static_cast<int32_t*>(ws) : nullptr);
+  gp.acc = epi_final == kEpiS32 ? acc_out : nullptr;
+  if (need > 0) {
+    gp.sync = static_cast<unsigned*>(ws);
+    gp.slots = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + kSyncBytes);
+  }
+  if (fused) {
+    gp.X = fused->X;
+    gp.sst = fused->sst;
+    gp.cst = fused->cst;
+    gp.Xq = const_cast<uint8_t*>(Xq);
+  }
 
   gp.A = pl.swap ? Wq : Xq;
   gp.B = pl.swap ? Xq : Wq;
@@ -1572,18 +1775,7 @@ fq_status gemm_impl(const uint8_t* Xq, const void* s_x, const uint8_t* Wq, const
   gp.rowsB = pl.swap ? M : N;
 
   const dim3 grid = pl.swap ? dim3(pl.ctas) : dim3((gp.rowsA + kBM - 1) / kBM, (gp.rowsB + pl.bn - 1) / pl.bn, 1);
-  if (need > 0) {
-    if (cudaMemsetAsync(ws, 0, need, stream) != cudaSuccess) return fail(FQ_ERR_CUDA, "workspace clear failed");
-  }
-  st = dispatch(pl, gp, grid, stream);
-  if (st != FQ_OK) return st;
-  if (need > 0) {
-    const dim3 fgrid((N + kBM - 1) / kBM, std::min(M, 16));  // tiles x token groups
-    decode_fixup_kernel<<<fgrid, kBM, 0, stream>>>(gp.acc, gp.sx, gp.sw, gp.Y, M, N, gp.num_kb, pl.ctas,
-                                                   epi_final == kEpiRow ? 1 : 0);
-    st = check_launch("decode_fixup_kernel");
-  }
-  return st;
+  return dispatch(pl, gp, grid, stream);
 }
 
 // The general quantizer's GEMM: the exact int32 products of the stored codes
@@ -1594,14 +1786,15 @@ fq_status gemm_zp(const uint8_t* Xq, const void* s_x, const uint8_t* Wq, const v
   if (st != FQ_OK) return st;
   FQ_CHECK_ARG(Y && aligned(Y, 16), "Y must be non-NULL and 16-byte aligned");
   FQ_CHECK_ARG(s_x && s_w && aligned(s_x, 4) && aligned(s_w, 4), "the scale blocks must be non-NULL and aligned");
-  const size_t need = size_t(M) * N * sizeof(int32_t);
-  FQ_CHECK_ARG(ws && ws_bytes >= need && aligned(ws, 16), "workspace of %zu bytes required", need);
-  st = gemm_impl(Xq, nullptr, Wq, nullptr, M, N, K, kEpiS32, nullptr, static_cast<int32_t*>(ws), nullptr, 0,
-                 stream);
+  // the products go after the synchronization block, which stays untouched
+  const size_t need = kSyncBytes + size_t(M) * N * sizeof(int32_t);
+  FQ_CHECK_ARG(ws && ws_bytes >= need && aligned(ws, 256), "workspace of %zu bytes required", need);
+  int32_t* acc = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + kSyncBytes);
+  st = gemm_impl(Xq, nullptr, Wq, nullptr, M, N, K, kEpiS32, nullptr, acc, nullptr, 0, stream);
   if (st != FQ_OK) return st;
   const size_t pieces = size_t(M) * (N / 8);
   const int grid = int(std::max<size_t>(1, std::min<size_t>((pieces + 255) / 256, size_t(sm_count()) * 8)));
-  zp_epilogue_kernel<<<grid, 256, 0, stream>>>(static_cast<const int32_t*>(ws), static_cast<const float*>(s_x),
+  zp_epilogue_kernel<<<grid, 256, 0, stream>>>(acc, static_cast<const float*>(s_x),
                                                static_cast<const float*>(s_w), reinterpret_cast<__half*>(Y), M, N,
                                                K);
   return check_launch("zp_epilogue_kernel");
@@ -1611,10 +1804,28 @@ fq_status gemm_zp(const uint8_t* Xq, const void* s_x, const uint8_t* Wq, const v
 
 size_t gemm_workspace_bytes(int M, int N, int K, fq_gran gran) {
   if (M < 1 || N < 8 || K < kBK || K % kBK) return 0;
-  if (gran == FQ_DYNAMIC_ROW_ZP) return size_t(M) * N * sizeof(int32_t);  // the exact int32 products
+  if (gran == FQ_DYNAMIC_ROW_ZP) return kSyncBytes + size_t(M) * N * sizeof(int32_t);  // the exact int32 products
   const int epi = gran == FQ_DYNAMIC_GROUP ? kEpiGroup : (gran == FQ_STATIC_CHANNEL ? kEpiStatic : kEpiRow);
   const Plan pl = make_plan(M, N, K, epi, sm_count());
-  return (pl.swap && pl.partial) ? size_t(M) * N * sizeof(int32_t) : 0;
+  size_t need = decode_ws_bytes(pl, M, N, false);
+  if (gran == FQ_STATIC_CHANNEL)  // room for the fused decode linear's plan too
+    need = std::max(need, decode_ws_bytes(make_plan(M, N, K, epi, sm_count(), true), M, N, true));
+  return need;
+}
+
+size_t sync_block_bytes() { return kSyncBytes; }
+
+// The fused decode linear: static per-channel quantization of the tokens
+// inside the decode GEMM launch.  FQ_ERR_UNSUPPORTED (with no error text and
+// nothing launched) when the shape is not a decode shape or the cooperative
+// launch is not available; the caller then quantizes in a launch of its own.
+fq_status decode_linear_fused(const uint16_t* X, const float* sst, const float* cst, uint8_t* Xq, const uint8_t* Wq,
+                              const void* s_w, int M, int N, int K, uint16_t* Y, void* ws, size_t ws_bytes,
+                              cudaStream_t stream) {
+  const Plan pl = make_plan(M, N, K, kEpiStatic, sm_count(), true);
+  if (!pl.swap) return FQ_ERR_UNSUPPORTED;
+  const FusedTokens ft{reinterpret_cast<const __half*>(X), sst, cst};
+  return gemm_impl(Xq, nullptr, Wq, s_w, M, N, K, kEpiStatic, Y, nullptr, ws, ws_bytes, stream, &ft);
 }
 
 }  // namespace fq
@@ -1659,7 +1870,7 @@ size_t fq_gemm_workspace_size(int M, int N, int K, fq_gran gran) { return fq::ge
 // the library keeps this buffer for the life of the process.
 namespace fq {
 namespace {
-constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB: M * N int32 partial sums
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB: counters + split tiles' partial sums
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 constexpr int kNoAllocMaxDevices = 64;

@@ -1,10 +1,20 @@
 // The W4A4 linear layer: online activation quantization into the caller's
 // workspace, then the INT4 x INT4 GEMM, on one stream (FlatQuant notes,
-// 核心思想: Y ~ Q(XP) Q(P^-1 W^T)).
+// 核心思想: Y ~ Q(XP) Q(P^-1 W^T)).  Decode with static per-channel scales
+// and no Kronecker transform (MergeQuant's setting) runs as one launch: the
+// decode GEMM quantizes the tokens itself.
+#include <algorithm>
+
 #include "fq_host.h"
 
 namespace fq {
 size_t gemm_workspace_bytes(int M, int N, int K, fq_gran gran);
+size_t sync_block_bytes();
+fq_status check_act_args(const uint16_t* X, int M, int K, const fq_qparams* qp, const fq_transform* t,
+                         const float* static_scale, uint8_t* Xq, void* s_x);
+fq_status decode_linear_fused(const uint16_t* X, const float* sst, const float* cst, uint8_t* Xq, const uint8_t* Wq,
+                              const void* s_w, int M, int N, int K, uint16_t* Y, void* ws, size_t ws_bytes,
+                              cudaStream_t stream);
 
 namespace {
 constexpr size_t kAlign = 256;
@@ -18,9 +28,16 @@ size_t act_scale_bytes(int M, int K, fq_gran gran) {
 }
 }  // namespace
 
+// Workspace layout: the GEMM's part first (its synchronization block at
+// offset 0 for every shape, so that no call writes there but to leave it
+// zero), then the packed activations, then their scales.
+size_t linear_gemm_part(int M, int N, int K, fq_gran gran) {
+  return up(std::max(sync_block_bytes(), gemm_workspace_bytes(M, N, K, gran)));
+}
+
 size_t linear_workspace_bytes(int M, int N, int K, fq_gran gran) {
   if (M < 1 || K < kGroup || K % kGroup) return 0;
-  return up(size_t(M) * (K / 2)) + up(act_scale_bytes(M, K, gran)) + up(gemm_workspace_bytes(M, N, K, gran));
+  return linear_gemm_part(M, N, K, gran) + up(size_t(M) * (K / 2)) + up(act_scale_bytes(M, K, gran));
 }
 
 }  // namespace fq
@@ -44,13 +61,23 @@ fq_status fq_linear(const uint16_t* X, int M, int K, const fq_qparams* act_qp, c
   if (!workspace || ws_bytes < need || !fq::aligned(workspace, 256))
     return fq::fail(FQ_ERR_INVALID, "workspace of %zu bytes (256-byte aligned) required, got %zu", need, ws_bytes);
   uint8_t* base = static_cast<uint8_t*>(workspace);
-  uint8_t* xq = base;
-  size_t off = fq::up(size_t(M) * (K / 2));
+  void* gws = base;
+  const size_t gws_bytes = fq::linear_gemm_part(M, N, K, gran);
+  size_t off = gws_bytes;
+  uint8_t* xq = base + off;
+  off += fq::up(size_t(M) * (K / 2));
   void* sx = act_qp->gran == FQ_STATIC_CHANNEL ? nullptr : static_cast<void*>(base + off);
-  off += fq::up(fq::act_scale_bytes(M, K, gran));
-  void* gws = base + off;
-  const size_t gws_bytes = ws_bytes - off;
-  fq_status st = fq_quant_act(X, M, K, act_qp, t, static_scale, xq, sx, stream);
+  fq_status st;
+  if (gran == FQ_STATIC_CHANNEL && act_qp->zero_point == 8 && (!t || !t->P1) && fq::aligned(static_scale, 16) &&
+      (!t || !t->c || fq::aligned(t->c, 16))) {
+    st = fq::check_act_args(X, M, K, act_qp, t, static_scale, xq, sx);
+    if (st != FQ_OK) return st;
+    st = fq::decode_linear_fused(X, static_scale, t ? t->c : nullptr, xq, Wq, s_w, M, N, K, Y, gws, gws_bytes,
+                                 static_cast<cudaStream_t>(stream));
+    if (st != FQ_ERR_UNSUPPORTED) return st;
+    fq::clear_error();  // not a decode shape: quantize in a launch of its own
+  }
+  st = fq_quant_act(X, M, K, act_qp, t, static_scale, xq, sx, stream);
   if (st != FQ_OK) return st;
   // the residual scaling leaves through the per-token epilogue: s_x = S_n
   const fq_gran ggran = gran == FQ_STATIC_RESIDUAL ? FQ_DYNAMIC_ROW : gran;

@@ -93,12 +93,6 @@ __device__ __forceinline__ float warp_max(float v) {
   return v;
 }
 
-__device__ __forceinline__ int rtn_code(float v, float s) {
-  if (s == 0.0f) return 0;
-  const float r = rintf(__fdiv_rn(v, s));
-  return static_cast<int>(fminf(fmaxf(r, -8.0f), 7.0f));
-}
-
 // Index of flat element e in the row buffer: padded by one float per tile row
 // when a transform is applied, so that the column pass is free of bank conflicts.
 __device__ __forceinline__ int slot(int e, int n2, int pad) { return pad ? (e / n2) * (n2 + 1) + (e % n2) : e; }
@@ -498,27 +492,8 @@ __global__ void __launch_bounds__(kThreads) quant_static_kernel(QuantParams p) {
   for (size_t pc = blockIdx.x * size_t(kThreads) + threadIdx.x; pc < pieces; pc += size_t(gridDim.x) * kThreads) {
     const int r = int(pc / kp), e0 = int(pc % kp) * 8;
     const uint4 raw = *reinterpret_cast<const uint4*>(p.X + size_t(r) * p.K + e0);
-    const __half2* h2 = reinterpret_cast<const __half2*>(&raw);
-    const float4 s0 = __ldg(reinterpret_cast<const float4*>(p.sstatic + e0));
-    const float4 s1 = __ldg(reinterpret_cast<const float4*>(p.sstatic + e0 + 4));
-    const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
     float v[8];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float2 f = __half22float2(h2[j]);
-      v[2 * j] = f.x;
-      v[2 * j + 1] = f.y;
-    }
-    if (p.c) {
-      const float4 c0 = __ldg(reinterpret_cast<const float4*>(p.c + e0));
-      const float4 c1 = __ldg(reinterpret_cast<const float4*>(p.c + e0 + 4));
-      const float cv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-#pragma unroll
-      for (int j = 0; j < 8; ++j) v[j] = __fmul_rn(v[j], cv[j]);
-    }
-    uint32_t word = 0;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) word |= (uint32_t(rtn_code(v[j], sv[j])) & 0xFu) << (4 * j);
+    const uint32_t word = static_codes8(raw, p.sstatic + e0, p.c ? p.c + e0 : nullptr, v);
     reinterpret_cast<uint32_t*>(p.Q + size_t(r) * (p.K / 2))[e0 / 8] = word;
     if (p.xhat) {
       float4* xo = reinterpret_cast<float4*>(p.xhat + size_t(r) * p.K + e0);
@@ -584,8 +559,9 @@ fq_status check_qparams(const fq_qparams* qp, bool act) {
   return FQ_OK;
 }
 
+// dry: validate every argument as for a launch, launch nothing
 fq_status quant_common(int side, const uint16_t* X, int R, int K, const fq_qparams* qp, const fq_transform* t,
-                       const float* extra, uint8_t* Q, void* s_out, float* xhat, void* stream) {
+                       const float* extra, uint8_t* Q, void* s_out, float* xhat, void* stream, bool dry = false) {
   clear_error();
   fq_status st = check_qparams(qp, side == kAct);
   if (st != FQ_OK) return st;
@@ -633,6 +609,7 @@ fq_status quant_common(int side, const uint16_t* X, int R, int K, const fq_qpara
       p.Rt = t->P2;
     }
   }
+  if (dry) return FQ_OK;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (side == kAct && p.n1 > 0 && !p.asym && quant_act_tc_supported(K, p.n1, p.n2)) {
     // activations with the transform: tensor-core kernel
@@ -671,6 +648,14 @@ fq_status quant_common(int side, const uint16_t* X, int R, int K, const fq_qpara
 }
 
 }  // namespace
+
+// The checks of fq_quant_act, with nothing launched (the fused decode linear
+// quantizes inside the GEMM launch).
+fq_status check_act_args(const uint16_t* X, int M, int K, const fq_qparams* qp, const fq_transform* t,
+                         const float* static_scale, uint8_t* Xq, void* s_x) {
+  return quant_common(kAct, X, M, K, qp, t, static_scale, Xq, s_x, nullptr, nullptr, true);
+}
+
 }  // namespace fq
 
 extern "C" {

@@ -14,6 +14,7 @@ from dataclasses import dataclass
 import torch
 
 ROW, GROUP, STATIC, ROW_ZP, STATIC_RESIDUAL = 0, 1, 2, 3, 4  # fq_gran
+SYNC_BYTES = 16384  # FQ_WORKSPACE_SYNC_BYTES: leading workspace bytes kept zero between calls
 GROUP_SIZE = 128
 ZERO_POINT_MINMAX = -1                   # fq_qparams.zero_point: per-row min-max (asymmetric) quantizer
 
@@ -207,7 +208,8 @@ def _workspace(nbytes, dev, ws):
     if nbytes == 0:
         return None, 0
     if ws is None:
-        ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+        # zeroed: the library's counters at the start of a workspace must be 0 on first use
+        ws = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
     if ws.numel() < nbytes:
         raise ValueError(f"workspace needs {nbytes} bytes")
     return ws, ws.numel()
@@ -231,7 +233,7 @@ def fq_w4a4_gemm(Xq, s_x, Wq, s_w, gran: int, Y=None, workspace=None, stream=Non
 
 def fq_w4a4_gemm_noalloc(Xq, s_x, Wq, s_w, gran: int, Y=None, stream=None):
     """fq_w4a4_gemm without a workspace, for callers that cannot allocate device
-    memory: the library's static 8 MiB scratch holds the split-K partial sums.
+    memory: the library's static 32 MiB scratch holds the split-K partial sums.
     Calls that overlap on the GPU share that scratch and race; keep them on one
     stream.  (Y is allocated here only when the caller passes none.)"""
     _check(Xq, torch.uint8, "Xq")

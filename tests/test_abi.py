@@ -139,12 +139,21 @@ def test_linear_needs_workspace(L):
 
 
 def test_workspace_sizes(L):
-    # prefill needs no GEMM scratch; decode with few output tiles splits K
+    """Prefill needs no GEMM scratch.  Decode with few output tiles splits K
+    over one wave of 2 x 148 CTAs (the SM count assumed without a GPU): the
+    counter block plus two slots of M x 128 int32 per CTA, whatever N is.
+    The fused static decode needs the counter block even without split tiles,
+    and the linear layer always reserves it first."""
     assert L.fq_gemm_workspace_size(2048, 4096, 4096, fq.ROW) == 0
     assert L.fq_gemm_workspace_size(4096, 8192, 8192, fq.GROUP) == 0
-    assert L.fq_gemm_workspace_size(8, 8192, 28672, fq.ROW) == 8 * 8192 * 4
+    slots = 2 * 296 * 8 * 128 * 4
+    assert L.fq_gemm_workspace_size(8, 8192, 28672, fq.ROW) == fq.SYNC_BYTES + slots
+    assert L.fq_gemm_workspace_size(8, 139264, 8192, fq.ROW) == fq.SYNC_BYTES + slots
     ws = L.fq_linear_workspace_size(8, 8192, 28672, fq.STATIC)
-    assert ws >= 8 * 28672 // 2 + 8 * 8192 * 4
+    assert ws >= fq.SYNC_BYTES + slots + 8 * 28672 // 2
+    assert L.fq_linear_workspace_size(2048, 4096, 4096, fq.ROW) >= fq.SYNC_BYTES + 2048 * 2048 + 2048 * 4
+    # 64 tokens: the largest decode scratch stays within the no-alloc entry's 32 MiB
+    assert L.fq_gemm_workspace_size(64, 8192, 28672, fq.ROW) <= 32 << 20
 
 
 def test_debug_timeout_rejects_limits(L):
@@ -155,7 +164,7 @@ def test_debug_timeout_rejects_limits(L):
 def test_zero_point_gemm_needs_its_workspace(L):
     """The min-max quantizer's GEMM keeps the exact int32 products in the
     caller's workspace: M * N * 4 bytes, and refuses to run without them."""
-    assert L.fq_gemm_workspace_size(8, 256, 256, fq.ROW_ZP) == 8 * 256 * 4
+    assert L.fq_gemm_workspace_size(8, 256, 256, fq.ROW_ZP) == fq.SYNC_BYTES + 8 * 256 * 4
     st = L.fq_w4a4_gemm(A, A, A, A, 8, 256, 256, fq.ROW_ZP, A, None, 0, None)
     assert st == fq.FQ_ERR_INVALID and b"workspace" in L.fq_last_error()
     ws = L.fq_linear_workspace_size(8, 256, 256, fq.ROW_ZP)

@@ -93,18 +93,22 @@ def test_gemm_decode_split_k_repeatable(m):
 
 
 def test_gemm_workspace_is_reused_correctly():
-    """Two split-K calls in a row on one workspace give the same exact result."""
+    """Two split-K calls in a row on one workspace give the same exact result:
+    garbage beyond the counter block does not leak into the sums, and the
+    counters are back at zero after each call."""
     m, n, k = 8, 8192, 28672
     a, b = _operands(99, m, n, k)
     g = synth.generator(4)
     sx, sw = synth.random_scales(g, m), synth.random_scales(g, n)
     ws = torch.full((fq.fq_gemm_workspace_size(m, n, k, fq.ROW),), 0x5A, dtype=torch.uint8, device="cuda")
+    ws[: fq.SYNC_BYTES].zero_()
     y1 = C.host(fq.fq_w4a4_gemm(C.dev(a), C.dev(sx), C.dev(b), C.dev(sw), fq.ROW, workspace=ws))
     y2 = C.host(fq.fq_w4a4_gemm(C.dev(a), C.dev(sx), C.dev(b), C.dev(sw), fq.ROW, workspace=ws))
     ref = O.dequant_row(O.gemm_int(C.unpack(a), C.unpack(b)), sx, sw)
     C.check_fp16_exact(y1, ref)
     C.check_fp16_exact(y2, ref)
     fq.fq_check_device_error()
+    assert not ws[: fq.SYNC_BYTES].any(), "the counter block is not back at zero"
 
 
 # Prefill shapes for the persistent CTA-pair kernel: tile counts below, at and
@@ -146,7 +150,7 @@ def test_gemm_persistent_stress_repeated():
         g = synth.generator(i + 40)
         sx, sw = synth.random_scales(g, m), synth.random_scales(g, n)
         ref = O.dequant_row(O.gemm_int(C.unpack(a), C.unpack(b)), sx, sw)
-        ws = torch.empty(max(fq.fq_gemm_workspace_size(m, n, k, fq.ROW), 256), dtype=torch.uint8, device="cuda")
+        ws = torch.zeros(max(fq.fq_gemm_workspace_size(m, n, k, fq.ROW), 256), dtype=torch.uint8, device="cuda")
         cases.append((C.dev(a), C.dev(sx), C.dev(b), C.dev(sw), ws, C.dev(ref.view(np.uint16).astype(np.int16))))
     for it in range(50):
         A, SX, B, SW, ws, ref = cases[(it * 3) % len(cases)]

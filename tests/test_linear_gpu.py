@@ -48,7 +48,7 @@ def _run_three_ways(d, qp, gran, wq, sw, t=None, static_scale=None):
     n = wq.shape[0]
     y_lin = C.host(fq.fq_linear(X, qp, wq, sw, t, static_scale=static_scale))
     xq, sx = fq.fq_quant_act(X, qp, t, static_scale)
-    ws = torch.empty(max(fq.fq_gemm_workspace_size(m, n, k, gran), 256), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(max(fq.fq_gemm_workspace_size(m, n, k, gran), 256), dtype=torch.uint8, device="cuda")
     y = C.host(fq.fq_w4a4_gemm(xq, sx, wq, sw, gran, workspace=ws))
     assert np.array_equal(_bits(y), _bits(y_lin)), "fq_linear differs from quantization + GEMM"
     xhat = None
@@ -131,3 +131,47 @@ def test_linear_decode_static(m, k, n):
     qw, sw_ref, _ = O.quant_weight(d["w"][cols], O.ROW, 1.0, qsm_scale=s_k)
     assert np.array_equal(C.host(wq)[cols], O.pack_int4(qw))
     C.check_gemm_decoupled(y[:, cols], q_ref, None, qw, sw_ref, O.STATIC)
+
+
+def _kernel_names(fn):
+    """Names of the kernels that fn launches (CUDA activity from the profiler)."""
+    from torch.profiler import ProfilerActivity, profile
+    torch.cuda.synchronize()
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        fn()
+        torch.cuda.synchronize()
+    return [e.name for e in prof.events() if e.device_type.name == "CUDA"]
+
+
+@pytest.mark.parametrize("m,k,n", [(1, 8192, 10240), (8, 28672, 8192), (64, 8192, 57344), (17, 1024, 3072)])
+def test_linear_decode_fused_one_launch(m, k, n):
+    """Decode with static scales (and a channel factor c) through fq_linear: one
+    kernel launch, no separate quantization, no memset; outputs bit-exact
+    against the oracle; three calls in a row on one workspace whose bytes past
+    the counter block are garbage, the counters (all words but the grid
+    barrier's generation number, word 1) back at zero after each."""
+    d = synth.decode_static(m, k, n, seed=3)
+    s_k = d["static_scale"]
+    c = synth.generator(m + 5).uniform(0.5, 2.0, k).astype(np.float32)
+    qp = fq.qparams(fq.STATIC)
+    wq, sw = fq.fq_quant_weight(C.dev(d["w"]), fq.qparams(fq.ROW, 1.0), None, C.dev(s_k))
+    X, SK, t = C.dev(d["x"]), C.dev(s_k), fq.Transform(c=C.dev(c))
+    ws = torch.full((fq.fq_linear_workspace_size(m, n, k, fq.STATIC),), 0x5A, dtype=torch.uint8, device="cuda")
+    ws[: fq.SYNC_BYTES].zero_()
+    Y = torch.empty(m, n, dtype=torch.float16, device="cuda")
+    names = _kernel_names(lambda: fq.fq_linear(X, qp, wq, sw, t, static_scale=SK, Y=Y, workspace=ws))
+    assert len(names) == 1 and "gemm_decode_kernel" in names[0], names
+    q_ref, _, _ = O.quant_act(d["x"], O.STATIC, c=c, static_scale=s_k)
+    cols = C.tile_samples(m + k + n, n)
+    qw, sw_ref, _ = O.quant_weight(d["w"][cols], O.ROW, 1.0, qsm_scale=s_k)
+    first = C.host(Y)
+    C.check_gemm_decoupled(first[:, cols], q_ref, None, qw, sw_ref, O.STATIC)
+    for _ in range(2):
+        y = C.host(fq.fq_linear(X, qp, wq, sw, t, static_scale=SK, Y=Y, workspace=ws))
+        assert np.array_equal(y.view(np.uint16), first.view(np.uint16))
+        words = ws[: fq.SYNC_BYTES].view(torch.int32)
+        assert not words[0] and not words[2:].any(), "the counters are not back at zero"
+    xq, _ = fq.fq_quant_act(X, qp, t, SK)
+    y2 = C.host(fq.fq_w4a4_gemm(xq, None, wq, sw, fq.STATIC))
+    assert np.array_equal(y2.view(np.uint16), first.view(np.uint16)), "fused and two-launch paths differ"
+    fq.fq_check_device_error()

@@ -74,7 +74,7 @@ def test_residual_linear_exact(m, k, n):
     qp = fq.qparams(fq.STATIC_RESIDUAL)
     y_lin = C.host(fq.fq_linear(X, qp, wq, sw, static_scale=C.dev(s_k)))
     xq, s_n = fq.fq_quant_act(X, qp, static_scale=C.dev(s_k))
-    ws = torch.empty(max(fq.fq_gemm_workspace_size(m, n, k, fq.ROW), 256), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(max(fq.fq_gemm_workspace_size(m, n, k, fq.ROW), 256), dtype=torch.uint8, device="cuda")
     y = C.host(fq.fq_w4a4_gemm(xq, s_n, wq, sw, fq.ROW, workspace=ws))
     fq.fq_check_device_error()
     assert np.array_equal(y.view(np.uint16), y_lin.view(np.uint16)), "fq_linear differs from quant + GEMM"
