@@ -21,7 +21,10 @@ It restates, step by step and in plain numpy, what the pages define:
   y = acc * s_x * s_w (FlatQuant notes, 核心思想: Y ~ Q(XP) Q(P^-1 W^T));
 * the general quantizer (any b, min-max zero point; FRM-PTQ page) and the
   per-token residual scaling S_n ahead of static quantization (FPTQuant
-  explainer, 伪动态残差缩放).
+  explainer, 伪动态残差缩放);
+* the asymmetric ternary quantizer W^ = alpha T + mu with its iterative
+  closed-form fit, and the product of fp16 activations with such weights
+  (PT2-LLM page, 非对称三值量化器 ATQ).
 
 Precision: the transform is evaluated in float64 and rounded once to float32
 (the "transformed value"); scales, the division and round-half-to-even are
@@ -377,6 +380,108 @@ def linear(x, wq, s_w, gran=ROW, alpha=1.0, p1=None, p2=None, c=None,
     if gran == STATIC:
         return dequant_static(gemm_int(qx, wq), s_w)
     return dequant_group(qx, wq, s_x, s_w)
+
+
+# ------------------------------------------------------------------ ternary weights
+
+TERNARY_BLOCK = 128
+
+
+def ternary_alpha_mu(w, t):
+    """Closed-form (alpha, mu) of one block for a fixed ternary matrix T.
+
+    PT2-LLM page, 非对称三值量化器 ATQ (ITF): with T fixed, the per-row scale
+    alpha* = (m (W o T) 1 - (T 1) o (W 1)) / (m (T o T) 1 - (T 1)^2) (m the
+    block's column count); it is the least-squares alpha when the offset is
+    solved jointly, so the offset is mu* = (W 1 - alpha* T 1) / m.  A row
+    whose denominator is 0 (T constant on the row) gets alpha = 0 and mu = the
+    row mean (then W^ = mu is that row's least-squares fit).
+    w float64 [R, m], t int [R, m] -> (alpha, mu) float64 [R].
+    Parity pinned by: least squares on [T, 1] (numpy lstsq) for random blocks.
+    """
+    w = np.asarray(w, np.float64)
+    t = np.asarray(t, np.float64)
+    m = w.shape[1]
+    num = m * (w * t).sum(1) - t.sum(1) * w.sum(1)
+    den = m * (t * t).sum(1) - t.sum(1) ** 2
+    ok = den != 0
+    alpha = np.where(ok, num / np.where(ok, den, 1.0), 0.0)
+    mu = (w.sum(1) - alpha * t.sum(1)) / m
+    return alpha, mu
+
+
+def ternary_round(w, alpha, mu):
+    """T_ij = argmin over t in {-1, 0, 1} of |Z_ij - t|, Z = (W - mu) / alpha
+    (PT2-LLM page, ITF); ties |Z| = 1/2 go to 0 (round half to even), and a
+    row with alpha = 0 gets T = 0."""
+    w = np.asarray(w, np.float64)
+    a = np.asarray(alpha, np.float64)[:, None]
+    z = np.where(a != 0, (w - np.asarray(mu, np.float64)[:, None]) / np.where(a != 0, a, 1.0), 0.0)
+    return np.clip(np.rint(z), -1, 1).astype(np.int8)
+
+
+def ternary_fit(w, iters: int = 10, block: int = TERNARY_BLOCK):
+    """Asymmetric ternary quantization of weight rows, per block of 128 columns.
+
+    PT2-LLM page, 非对称三值量化器 ATQ, iterative ternary fitting (ITF): mu
+    starts at each row's mean, then `iters` rounds of (T from the current
+    grid, then alpha and mu in closed form for that T).  The page gives no
+    starting alpha; this takes alpha_0 = 2 mean|W - mu_0| (a ternary threshold
+    at mean|W - mu_0|).  Returns (T int8 [N, K], alpha float32 [N, K/block],
+    mu float32 [N, K/block]); alpha and mu are the float64 values rounded to
+    float32, T is the last rounding's.
+    Parity pinned by: the weight error ||W - W^||_F never increasing over the
+    iterations, the closed form against least squares, tests/golden/ternary_worked.txt.
+    """
+    w = np.asarray(w, np.float64)
+    n, k = w.shape
+    nb = k // block
+    t_out = np.zeros((n, k), np.int8)
+    a_out = np.zeros((n, nb), np.float32)
+    m_out = np.zeros((n, nb), np.float32)
+    for g in range(nb):
+        wb = w[:, g * block:(g + 1) * block]
+        mu = wb.mean(1)
+        alpha = 2.0 * np.abs(wb - mu[:, None]).mean(1)
+        t = ternary_round(wb, alpha, mu)
+        for _ in range(iters):
+            alpha, mu = ternary_alpha_mu(wb, t)
+            t = ternary_round(wb, alpha, mu)
+        alpha, mu = ternary_alpha_mu(wb, t)
+        t_out[:, g * block:(g + 1) * block] = t
+        a_out[:, g] = alpha.astype(np.float32)
+        m_out[:, g] = mu.astype(np.float32)
+    return t_out, a_out, m_out
+
+
+def ternary_dequant(t, alpha, mu, block: int = TERNARY_BLOCK) -> np.ndarray:
+    """W^ = alpha T + mu per row and block (PT2-LLM page, ATQ), float64 [N, K]."""
+    t = np.asarray(t, np.float64)
+    a = np.repeat(np.asarray(alpha, np.float64), block, axis=1)
+    m = np.repeat(np.asarray(mu, np.float64), block, axis=1)
+    return a * t + m
+
+
+def ternary_linear(x, t, alpha, mu, block: int = TERNARY_BLOCK) -> np.ndarray:
+    """Y = X W^T with W^ = alpha T + mu and fp16 activations X [M, K], in
+    float64 (the product as defined; weight-only ternarization keeps the
+    activations in fp16).  Returns float64 [M, N].
+    Parity pinned by: pure-Python loops over a tiny case.
+    """
+    return np.asarray(x, np.float64) @ ternary_dequant(t, alpha, mu, block).T
+
+
+def pack_ternary(t) -> np.ndarray:
+    """Ternary codes packed 4 per byte, low bits first: 2 bits per weight,
+    00 = 0, 01 = +1, 11 = -1 (bit 0: nonzero, bit 1: negative).
+    int8 [N, K] -> uint8 [N, K/4].  (T carries log2(3) = 1.58 bits of
+    information per weight; the stored width is 2 bits.)
+    Parity pinned by: hand-packed bytes in tests/golden/ternary_worked.txt."""
+    t = np.asarray(t, np.int64)
+    code = np.where(t == 0, 0, np.where(t > 0, 1, 3))
+    n, k = t.shape
+    c = code.reshape(n, k // 4, 4)
+    return (c[..., 0] | (c[..., 1] << 2) | (c[..., 2] << 4) | (c[..., 3] << 6)).astype(np.uint8)
 
 
 # ------------------------------------------------------------------ sampled rows

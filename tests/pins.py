@@ -454,3 +454,70 @@ def check_residual_exact_sum(o):
 
 
 ALL_CHECKS += [check_residual_golden, check_residual_invariants, check_residual_exact_sum]
+
+
+# ------------------------------------------------------------------ ternary weights (PT2-LLM ATQ)
+
+def check_ternary_golden(o):
+    """Hand-worked ITF rows in tests/golden/ternary_worked.txt (PT2-LLM, ATQ)."""
+    from fractions import Fraction
+    for ln in _lines("ternary_worked.txt"):
+        ws, a_s, m_s, ts, byte = [p.strip() for p in ln.split("|")]
+        w = np.array([float(v) for v in ws.split()], dtype=np.float16)[None, :]
+        t, a, m = o.ternary_fit(w, iters=10, block=w.shape[1])
+        assert np.array_equal(t[0], np.array([int(v) for v in ts.split()], np.int8)), (ln, t)
+        assert a[0, 0] == np.float32(float(Fraction(a_s))), (ln, a)
+        assert m[0, 0] == np.float32(float(Fraction(m_s))), (ln, m)
+        assert int(o.pack_ternary(t)[0, 0]) == int(byte), (ln, o.pack_ternary(t))
+
+
+def check_ternary_closed_form(o):
+    """The closed-form (alpha, mu) for fixed T is the least-squares fit of each
+    row by alpha T + mu (numpy lstsq on [T, 1]), including rows with sum(T) != 0."""
+    g = np.random.Generator(np.random.PCG64(31))
+    w = g.standard_normal((16, 128)) * 0.02 + g.uniform(-0.01, 0.01, (16, 1))
+    t = g.integers(-1, 2, (16, 128))
+    t[0] = 1  # a constant row: alpha = 0, mu = the mean
+    a, m = o.ternary_alpha_mu(w, t)
+    for r in range(1, 16):
+        sol = np.linalg.lstsq(np.stack([t[r].astype(np.float64), np.ones(128)], 1), w[r], rcond=None)[0]
+        assert np.allclose([a[r], m[r]], sol, rtol=1e-10, atol=1e-14), (r, a[r], m[r], sol)
+    assert a[0] == 0 and np.isclose(m[0], w[0].mean())
+
+
+def check_ternary_itf_monotone(o):
+    """Each ITF step solves its sub-problem exactly, so the weight error
+    ||W - W^||_F never increases with the number of iterations; the fit beats
+    the symmetric grid alpha T (mu = 0) on rows with a mean offset."""
+    g = np.random.Generator(np.random.PCG64(32))
+    w = (g.standard_normal((32, 256)) * 0.02 + g.uniform(-0.02, 0.02, (32, 1))).astype(np.float16)
+    w64 = w.astype(np.float64)
+    errs = []
+    for it in range(0, 11):
+        t, a, m = o.ternary_fit(w, iters=it)
+        errs.append(((w64 - o.ternary_dequant(t, a.astype(np.float64), m.astype(np.float64))) ** 2).sum())
+    assert all(errs[i + 1] <= errs[i] * (1 + 1e-9) for i in range(10)), errs
+    t, a, m = o.ternary_fit(w)
+    assert set(np.unique(t)) <= {-1, 0, 1}
+    sym = ((w64 - np.repeat(a.astype(np.float64), 128, 1) * t) ** 2).sum()
+    assert errs[-1] < sym
+
+
+def check_ternary_linear_loops(o):
+    """Y = X (alpha T + mu)^T by plain Python loops on a tiny case (block 4)."""
+    g = np.random.Generator(np.random.PCG64(33))
+    x = g.standard_normal((2, 8)).astype(np.float16)
+    t = g.integers(-1, 2, (3, 8)).astype(np.int8)
+    a = g.uniform(0.01, 0.05, (3, 2)).astype(np.float32)
+    mu = g.uniform(-0.01, 0.01, (3, 2)).astype(np.float32)
+    y = o.ternary_linear(x, t, a, mu, block=4)
+    for i in range(2):
+        for n in range(3):
+            ref = 0.0
+            for k in range(8):
+                ref += float(x[i, k]) * (float(a[n, k // 4]) * int(t[n, k]) + float(mu[n, k // 4]))
+            assert abs(y[i, n] - ref) <= 1e-12 * max(1.0, abs(ref)), (i, n, y[i, n], ref)
+
+
+ALL_CHECKS += [check_ternary_golden, check_ternary_closed_form, check_ternary_itf_monotone,
+               check_ternary_linear_loops]

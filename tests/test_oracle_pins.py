@@ -168,7 +168,56 @@ def _quant_act_residual_times(x, static_scale):
     return quantize(v, np.asarray(static_scale, np.float32)[None, :]), s_n, v  # noqa: F821
 
 
+def _ternary_alpha_mu_no_m(w, t):
+    # the factor m dropped from the numerator of alpha*
+    w = np.asarray(w, np.float64)
+    t = np.asarray(t, np.float64)
+    m = w.shape[1]
+    num = (w * t).sum(1) - t.sum(1) * w.sum(1)
+    den = m * (t * t).sum(1) - t.sum(1) ** 2
+    alpha = np.where(den != 0, num / np.where(den != 0, den, 1.0), 0.0)
+    return alpha, (w.sum(1) - alpha * t.sum(1)) / m
+
+
+def _ternary_alpha_mu_mu_sign(w, t):
+    # mu with the alpha T term added instead of subtracted
+    w = np.asarray(w, np.float64)
+    t = np.asarray(t, np.float64)
+    m = w.shape[1]
+    num = m * (w * t).sum(1) - t.sum(1) * w.sum(1)
+    den = m * (t * t).sum(1) - t.sum(1) ** 2
+    alpha = np.where(den != 0, num / np.where(den != 0, den, 1.0), 0.0)
+    return alpha, (w.sum(1) + alpha * t.sum(1)) / m
+
+
+def _ternary_round_floor(w, alpha, mu):
+    # floor instead of nearest
+    a = np.asarray(alpha, np.float64)[:, None]
+    z = np.where(a != 0, (np.asarray(w, np.float64) - np.asarray(mu, np.float64)[:, None]) / np.where(a != 0, a, 1.0), 0.0)
+    return np.clip(np.floor(z), -1, 1).astype(np.int8)
+
+
+def _ternary_linear_no_mu(x, t, alpha, mu, block=128):
+    # the offset term dropped
+    a = np.repeat(np.asarray(alpha, np.float64), block, axis=1)
+    return np.asarray(x, np.float64) @ (a * np.asarray(t, np.float64)).T
+
+
+def _pack_ternary_swapped(t):
+    # the two code bits swapped (bit 0 negative, bit 1 nonzero)
+    t = np.asarray(t, np.int64)
+    code = np.where(t == 0, 0, np.where(t > 0, 2, 3))
+    n, k = t.shape
+    c = code.reshape(n, k // 4, 4)
+    return (c[..., 0] | (c[..., 1] << 2) | (c[..., 2] << 4) | (c[..., 3] << 6)).astype(np.uint8)
+
+
 MUTANTS = {
+    "ternary_alpha_without_m": dict(ternary_alpha_mu=_ternary_alpha_mu_no_m),
+    "ternary_mu_sign": dict(ternary_alpha_mu=_ternary_alpha_mu_mu_sign),
+    "ternary_round_floor": dict(ternary_round=_ternary_round_floor),
+    "ternary_linear_without_mu": dict(ternary_linear=_ternary_linear_no_mu),
+    "ternary_pack_bits_swapped": dict(pack_ternary=_pack_ternary_swapped),
     "residual_rms_without_mean": dict(residual_rms=_residual_rms_no_mean),
     "residual_rms_without_sqrt": dict(residual_rms=_residual_rms_no_sqrt),
     "residual_multiplied": dict(quant_act_residual=_quant_act_residual_times),
