@@ -43,6 +43,7 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # ends are not in it.
 GEMM_DRAM_BYTES = {"qkv": 16842240, "o": 12640000, "gate_up": 63101696 + 69518336, "down": 44100096 + 29440}
 INT8_OVER_BF16 = 4.5 / 2.25  # nominal dense ratio (B200: 4.5 POPS int8 vs 2.25 PFLOPS bf16)
+ALU_CLOCK_GHZ = 1.965  # clocks.max.sm of this B200 (the ALU roofline of the ternary kernel)
 
 
 def peaks():
@@ -441,14 +442,82 @@ def run_transform_quant(args, dev_index):
     return {
         "metric": METRIC, "workload": "transform_quant", "value": round(gbs, 1), "unit": "GB/s",
         "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
-        "higher_is_better": True, "dtype": "fp16 in, fp32 transform (fp16 hi/lo tensor-core products), int4 out",
+        "higher_is_better": True, "dtype": "fp16 in, exact transform (int8-limb tensor-core products, int32 level sums), int4 out",
         "data": "synthetic",
         "config": {"workload": "transform+quant, X [2048, 4096], 1% outlier channels x30, token 0 x100, "
                                "Kronecker (64, 64), c ~ U[0.5, 2], alpha_a = 0.9, per-token INT4 + fp32 scales",
                    "l2": "256 MiB flush between launches; median of the launches"},
-        "roofline": {"kernel": "quant_act_tc_kernel", "bound": "hbm", "achieved": round(gbs, 1),
+        "roofline": {"kernel": "quant_act_int_kernel", "bound": "hbm", "achieved": round(gbs, 1),
                      "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": round(gbs / pk["hbm_gbs"], 4),
                      "peak_kind": pk_kind, "algorithmic_bytes": int(nbytes), "traffic": None},
+        "clocks": clk,
+    }
+
+
+def run_kv_cache(args, dev_index):
+    """INT4 key cache with FlatQuant's per-head transform: 16384 tokens x 8 heads
+    x 128 (P1 = I_8, P2 = P_h), one fp16 scale per token and head.  Roofline: HBM."""
+    torch, fq, dev, stream, clocks = _suite_common(args, dev_index)
+    d = synth.kv_cache(16384, 8)
+    x = torch.from_numpy(d["x"]).to(dev)
+    p_h = torch.from_numpy(d["p2"]).to(dev)
+    xq, sx = fq.fq_quant_kv(x, p_h)
+    timer = LaunchTimer(dev, stream, clocks)
+    clocks.start()
+    ms = timer.time(lambda: fq.fq_quant_kv(x, p_h, 1.0, xq, sx, stream=stream), args.steps, args.warmup)
+    clk = clocks.stop()
+    m, k = d["m"], d["k"]
+    nbytes = m * k * 2 + m * k // 2 + 2 * m * (k // 128) + 4 * d["n2"] ** 2
+    pk, pk_kind = peaks()
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {
+        "workload": "kv_cache", "value": round(gbs, 1), "unit": "GB/s", "ms_per_step": round(ms, 5),
+        "config": {"workload": "INT4 KV cache (fq_quant_kv), 16384 tokens x 8 heads x 128, per-head P_h, "
+                               "per-(token, head) fp16 scales"},
+        "roofline": {"kernel": "quant_act_int_kernel", "bound": "hbm", "achieved": round(gbs, 1),
+                     "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": round(gbs / pk["hbm_gbs"], 4),
+                     "peak_kind": pk_kind},
+        "clocks": clk,
+    }
+
+
+def run_ternary(args, dev_index):
+    """Ternary-weight decode (PT2-LLM: W^ = alpha T + mu per row and 128-block,
+    fp16 tokens): M in {1, 8} x (K, N) in {(8192, 57344), (28672, 8192)}.
+    Roofline per row: the slower of HBM (2-bit codes + alpha, mu + tokens) and
+    the CUDA-core ALU at one add per weight and token (148 SMs x 128 lanes x
+    the SM clock); the line reports the fraction of that bound."""
+    torch, fq, dev, stream, clocks = _suite_common(args, dev_index)
+    rows, timer = [], LaunchTimer(dev, stream, clocks)
+    pk, pk_kind = peaks()
+    alu_peak = 148 * 128 * ALU_CLOCK_GHZ  # G ops/s
+    clocks.start()
+    for k, n in synth.TERNARY_SHAPES:
+        for m in (1, 8):
+            d = synth.ternary_linear(m, k, n)
+            tq = fq.fq_ternary_pack(torch.from_numpy(d["t"]).to(dev))
+            x = torch.from_numpy(d["x"]).to(dev)
+            al, mu = torch.from_numpy(d["alpha"]).to(dev), torch.from_numpy(d["mu"]).to(dev)
+            y = torch.empty(m, n, dtype=torch.float16, device=dev)
+            ms = timer.time(lambda: fq.fq_ternary_linear(x, tq, al, mu, Y=y, stream=stream), args.steps, args.warmup)
+            nbytes = n * k // 4 + 8 * n * (k // 128) + 2 * m * k + 2 * m * n
+            t_hbm = nbytes / (pk["hbm_gbs"] * 1e9)
+            t_alu = m * n * k / (alu_peak * 1e9)
+            t = ms * 1e-3
+            rows.append({"M": m, "K": k, "N": n, "us": round(ms * 1e3, 2), "gbs": round(nbytes / t / 1e9, 1),
+                         "gops": round(m * n * k / t / 1e9, 1), "bound": "hbm" if t_hbm >= t_alu else "alu",
+                         "frac": round(max(t_hbm, t_alu) / t, 4)})
+            del tq, x, al, mu, y, d
+    clk = clocks.stop()
+    frac = sum(r["frac"] for r in rows) / len(rows)
+    return {
+        "workload": "ternary", "value": round(frac, 4), "unit": "mean fraction of the per-row roofline",
+        "rows": rows,
+        "config": {"workload": "ternary decode, M in {1, 8} x (K, N) in {(8192, 57344), (28672, 8192)}, "
+                               "2-bit codes, per-(row, 128-block) alpha and mu, fp16 tokens"},
+        "roofline": {"kernel": "ternary_linear_kernel", "bound": "hbm / alu per row", "achieved": round(frac, 4),
+                     "peak": 1.0, "unit": "fraction", "frac": round(frac, 4),
+                     "peak_kind": f"{pk_kind} HBM; ALU = 148 x 128 lanes x {ALU_CLOCK_GHZ} GHz"},
         "clocks": clk,
     }
 
@@ -535,13 +604,16 @@ def run_decode(args, dev_index):
                               args.warmup)
             g_ms = timer.time(lambda: fq.fq_w4a4_gemm(xq, None, wq, sw, fq.STATIC, Y=y, workspace=ws, stream=stream),
                               args.steps, args.warmup)
-            # the product call: one launch that quantizes the tokens inside the decode GEMM
+            # the product call (quantization + decode GEMM), and its one-launch form
             l_ms = timer.time(lambda: fq.fq_linear(x, qs, wq, sw, None, static_scale=s_k, Y=y, workspace=lws,
                                                    stream=stream), args.steps, args.warmup)
+            f_ms = timer.time(lambda: fq.fq_linear(x, qs, wq, sw, None, static_scale=s_k, Y=y, workspace=lws,
+                                                   stream=stream, fused=True), args.steps, args.warmup)
             gb = n * k // 2 + 4 * n + m * k // 2 + 2 * m * n
             lb = n * k // 2 + 4 * n + 2 * m * k + 4 * k + 2 * m * n
             rows.append({"M": m, "K": k, "N": n, "linear_us": round(l_ms * 1e3, 2),
-                         "linear_gbs": round(lb / (l_ms * 1e-3) / 1e9, 1), "gemm_us": round(g_ms * 1e3, 2),
+                         "linear_gbs": round(lb / (l_ms * 1e-3) / 1e9, 1), "fused_us": round(f_ms * 1e3, 2),
+                         "gemm_us": round(g_ms * 1e3, 2),
                          "gemm_gbs": round(gb / (g_ms * 1e-3) / 1e9, 1), "quant_us": round(q_ms * 1e3, 2),
                          "bytes": lb})
         del wq, sw, s_k, d0
@@ -558,10 +630,10 @@ def run_decode(args, dev_index):
         "dtype": "int4 (s8 tensor-core MMA, weights on the 128-row side, stream-K int32 partials), fp16 io", "data": "synthetic",
         "config": {"workload": "decode M in {1, 8, 32, 64} x (K, N) in {(8192, 57344), (28672, 8192)}, static "
                                "per-channel activation scales folded into per-channel INT4 weights; fq_linear "
-                               "(tokens quantized inside the decode GEMM launch)",
+                               "(quantization + decode GEMM); fused_us: fq_linear_fused (one launch)",
                    "l2": "256 MiB flush between launches; median of the launches"},
         "rows": rows,
-        "roofline": {"kernel": "gemm_decode_kernel (fused static quantization)", "bound": "hbm",
+        "roofline": {"kernel": "quant_static_kernel + gemm_decode_kernel", "bound": "hbm",
                      "achieved": round(gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
                      "frac": round(gbs / pk["hbm_gbs"], 4), "peak_kind": pk_kind, "traffic": None},
         "clocks": clk,
@@ -593,7 +665,7 @@ def run_configs(args, dev_index):
     import torch
     out = {}
     for name, fn in (("tiny", run_tiny), ("transform_quant", run_transform_quant), ("group", run_group),
-                     ("decode", run_decode)):
+                     ("decode", run_decode), ("kv_cache", run_kv_cache), ("ternary", run_ternary)):
         r = fn(args, dev_index)
         keep = {k: r[k] for k in ("value", "unit", "ms_per_step", "rows", "clocks") if k in r}
         if "roofline" in r:
@@ -752,7 +824,8 @@ def main():
                     help="skip the other workloads (tiny, transform+quant, group, decode) in the default run")
     ap.add_argument("--only", choices=[s[0] for s in SHAPES], default=None,
                     help="run one layer only (for profiling a single launch)")
-    ap.add_argument("--workload", choices=["prefill", "transform_quant", "group", "decode"], default="prefill",
+    ap.add_argument("--workload", choices=["prefill", "transform_quant", "group", "decode", "kv_cache", "ternary"],
+                    default="prefill",
                     help="prefill (default): the decoder-layer prefill step; the others time one kernel family "
                          "on its own workload (1 GPU)")
     ap.add_argument("--shape", default=None,
@@ -764,7 +837,8 @@ def main():
     if args.impl == "reference":
         out = run_reference(args, ws, rank)
     elif args.workload != "prefill":
-        suite = {"transform_quant": run_transform_quant, "group": run_group, "decode": run_decode}[args.workload]
+        suite = {"transform_quant": run_transform_quant, "group": run_group, "decode": run_decode,
+                 "kv_cache": run_kv_cache, "ternary": run_ternary}[args.workload]
         out = suite(args, local) if rank == 0 else None
     else:
         out = run_ours(args, ws, rank, local)

@@ -105,8 +105,10 @@ typedef struct {
  * factors and each row is mapped to c * x followed by P1^T Xbar P2 on its
  * row-major n1 x n2 reshape Xbar.  For weights the caller passes the
  * INVERSES P1^-1, P2^-1 and each weight row w (a column of W^T) is mapped to
- * w / c followed by P1^-1 Wbar (P2^-1)^T.  P1 == NULL means no transform
- * (then P2, n1, n2 are ignored); c == NULL means c = 1. */
+ * w / c followed by P1^-1 Wbar (P2^-1)^T.  P1 == NULL and P2 == NULL: no
+ * transform (n1, n2 ignored); P1 == NULL with P2 given: P1 = I (the n1 rows
+ * of the reshape are transformed on their own, as FlatQuant's per-head P_h
+ * and P_v act on the heads of a token); c == NULL means c = 1. */
 typedef struct {
   int n1, n2;
   const float* P1;
@@ -148,6 +150,21 @@ fq_status fq_quant_weight(const uint16_t* W, int N, int K, const fq_qparams* qp,
 fq_status fq_quant_act(const uint16_t* X, int M, int K, const fq_qparams* qp,
                        const fq_transform* t, const float* static_scale,
                        uint8_t* Xq, void* s_x, void* stream);
+
+/* INT4 key or value cache with FlatQuant's per-head transform (FlatQuant
+ * notes, Transformer 集成: P_h for the key cache, P_v for the value cache,
+ * one head_dim x head_dim matrix applied to every head, not decomposed).
+ * KV fp16 [T, H * 128] (T tokens of H heads of 128, 16-byte aligned);
+ * P_h float32 [128, 128] (device, row-major); alpha the clip ratio in (0, 1].
+ * Each head vector v = x_h P_h is quantized with its own scale
+ * s = fp16((max |v| alpha) / 7): Q uint8 [T, H * 64] packed codes (16-byte
+ * aligned), scales fp16 [T, H] (out).  The same transform, exactness and
+ * codes as fq_quant_act with P1 = I_H, P2 = P_h and FQ_DYNAMIC_GROUP; when
+ * T * H is a multiple of 64, 64 head vectors (of any tokens) share one
+ * kernel item, so small head counts keep the kernel's tiles full.
+ * H in [1, 128].  Enqueues one kernel; allocates nothing. */
+fq_status fq_quant_kv(const uint16_t* KV, int T, int H, const float* P_h, float alpha, uint8_t* Q,
+                      uint16_t* scales, void* stream);
 
 /* fq_quant_act that also writes xhat float32 [M, K], the transformed values
  * that were quantized (for checking the transform on its own). */
@@ -217,11 +234,7 @@ fq_status fq_w4a4_gemm_s32(const uint8_t* Xq, const uint8_t* Wq, int M, int N, i
  * fq_quant_weight with the matching inverse transform (and, for
  * FQ_STATIC_CHANNEL and FQ_STATIC_RESIDUAL, the same static scales folded
  * in; for FQ_ZERO_POINT_MINMAX, the weights' min-max scale block).
- * Decode (M <= 64) with FQ_STATIC_CHANNEL, no Kronecker factors and 16-byte
- * aligned static_scale (and c) runs as ONE cooperative launch: the decode
- * GEMM quantizes the tokens itself (same codes as fq_quant_act) before a
- * grid-wide barrier; where a cooperative launch is not available it falls
- * back to the two launches.  workspace: fq_linear_workspace_size() bytes,
+ * workspace: fq_linear_workspace_size() bytes,
  * 256-byte aligned (the GEMM's scratch with its counter block first, then the
  * packed activations and their scales; pass FQ_DYNAMIC_ROW_ZP there for the
  * min-max quantizer); its first FQ_WORKSPACE_SYNC_BYTES follow the rule of
@@ -230,6 +243,40 @@ fq_status fq_linear(const uint16_t* X, int M, int K, const fq_qparams* act_qp,
                     const fq_transform* t, const float* static_scale,
                     const uint8_t* Wq, const void* s_w, int N, uint16_t* Y,
                     void* workspace, size_t ws_bytes, void* stream);
+
+/* Ternary-weight linear layer (PT2-LLM page, 非对称三值量化器 ATQ):
+ * Y = X W^T with W^ = alpha T + mu per row and block of 128 columns, T in
+ * {-1, 0, +1}, fp16 activations (weight-only ternarization).
+ * X fp16 [M, K] (16-byte aligned); Tq uint8 [N, K/4]: 2 bits per weight,
+ * low bits first, 00 = 0, 01 = +1, 11 = -1 (as fq_ternary_pack writes it;
+ * 16-byte aligned); alpha, mu float32 [N, K/128] row-major; Y fp16 [M, N] (out).
+ * K a multiple of 128 in [128, 65536]; M, N >= 1.
+ * Arithmetic: per token, row and block, s = sum x t and S = sum x in
+ * float32, y = fp16(sum over blocks of alpha s + mu S) accumulated in float32
+ * (the summation order is the kernel's; not bit-reproducible against another
+ * order).  Tokens are processed 8 at a time: M > 8 streams the weights
+ * ceil(M / 8) times.  Enqueues one kernel; allocates nothing. */
+fq_status fq_ternary_linear(const uint16_t* X, int M, int K, const uint8_t* Tq, const float* alpha,
+                            const float* mu, int N, uint16_t* Y, void* stream);
+
+/* Packs int8 T [N, K] (16-byte aligned, K a multiple of 16) into Tq uint8
+ * [N, K/4] (4-byte aligned): 1 -> 01, -1 -> 11, every other value -> 00. */
+fq_status fq_ternary_pack(const int8_t* T, int N, int K, uint8_t* Tq, void* stream);
+
+/* fq_linear as ONE kernel launch, for decode (M <= 64) with FQ_STATIC_CHANNEL,
+ * no Kronecker factors (c allowed) and 16-byte aligned static_scale and c
+ * (MergeQuant's setting): the decode GEMM quantizes the tokens itself, with
+ * the same codes as fq_quant_act, before a grid-wide barrier, so the launch
+ * is cooperative and runs one CTA per SM.  Same arguments, workspace and
+ * results as fq_linear (bit-identical outputs); FQ_ERR_UNSUPPORTED where
+ * the shape or granularity does not qualify or a cooperative launch is not
+ * available.  On B200 the two launches of fq_linear are faster for every
+ * decode shape measured (the single launch keeps half the CTAs resident);
+ * this call is for callers that need one launch per layer. */
+fq_status fq_linear_fused(const uint16_t* X, int M, int K, const fq_qparams* act_qp,
+                          const fq_transform* t, const float* static_scale,
+                          const uint8_t* Wq, const void* s_w, int N, uint16_t* Y,
+                          void* workspace, size_t ws_bytes, void* stream);
 
 /* Scratch sizes in bytes (0 when none is needed).  gran as in the calls. */
 size_t fq_gemm_workspace_size(int M, int N, int K, fq_gran gran);

@@ -11,7 +11,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libfq.so")
-SOURCES = ["abi.cu", "quant.cu", "quant_int.cu", "gemm.cu", "linear.cu"]
+SOURCES = ["abi.cu", "quant.cu", "quant_int.cu", "gemm.cu", "linear.cu", "ternary.cu"]
 HEADERS = ["fq_device.cuh", "fq_host.h", os.path.join("..", "..", "include", "fq.h")]
 
 NVCC_FLAGS = [

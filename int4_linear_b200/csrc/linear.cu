@@ -1,8 +1,8 @@
 // The W4A4 linear layer: online activation quantization into the caller's
 // workspace, then the INT4 x INT4 GEMM, on one stream (FlatQuant notes,
-// 核心思想: Y ~ Q(XP) Q(P^-1 W^T)).  Decode with static per-channel scales
-// and no Kronecker transform (MergeQuant's setting) runs as one launch: the
-// decode GEMM quantizes the tokens itself.
+// 核心思想: Y ~ Q(XP) Q(P^-1 W^T)).  fq_linear_fused runs decode with static
+// per-channel scales and no Kronecker transform (MergeQuant's setting) as one
+// launch: the decode GEMM quantizes the tokens itself.
 #include <algorithm>
 
 #include "fq_host.h"
@@ -48,9 +48,11 @@ size_t fq_linear_workspace_size(int M, int N, int K, fq_gran gran) {
   return fq::linear_workspace_bytes(M, N, K, gran);
 }
 
-fq_status fq_linear(const uint16_t* X, int M, int K, const fq_qparams* act_qp, const fq_transform* t,
-                    const float* static_scale, const uint8_t* Wq, const void* s_w, int N, uint16_t* Y,
-                    void* workspace, size_t ws_bytes, void* stream) {
+namespace {
+// fused: the one-launch decode path (FQ_ERR_UNSUPPORTED where it does not apply)
+fq_status linear_impl(const uint16_t* X, int M, int K, const fq_qparams* act_qp, const fq_transform* t,
+                      const float* static_scale, const uint8_t* Wq, const void* s_w, int N, uint16_t* Y,
+                      void* workspace, size_t ws_bytes, void* stream, bool fused) {
   fq::clear_error();
   if (!act_qp) return fq::fail(FQ_ERR_INVALID, "act_qp is NULL");
   if (M < 1 || K < fq::kGroup || K % fq::kGroup || N < 8 || N % 8)
@@ -68,20 +70,38 @@ fq_status fq_linear(const uint16_t* X, int M, int K, const fq_qparams* act_qp, c
   off += fq::up(size_t(M) * (K / 2));
   void* sx = act_qp->gran == FQ_STATIC_CHANNEL ? nullptr : static_cast<void*>(base + off);
   fq_status st;
-  if (gran == FQ_STATIC_CHANNEL && act_qp->zero_point == 8 && (!t || !t->P1) && fq::aligned(static_scale, 16) &&
-      (!t || !t->c || fq::aligned(t->c, 16))) {
+  if (fused) {
+    if (!(gran == FQ_STATIC_CHANNEL && act_qp->zero_point == 8 && (!t || !t->P1) && fq::aligned(static_scale, 16) &&
+          (!t || !t->c || fq::aligned(t->c, 16))))
+      return fq::fail(FQ_ERR_UNSUPPORTED,
+                      "the one-launch path takes static per-channel scales (16-byte aligned) and no Kronecker factors");
     st = fq::check_act_args(X, M, K, act_qp, t, static_scale, xq, sx);
     if (st != FQ_OK) return st;
     st = fq::decode_linear_fused(X, static_scale, t ? t->c : nullptr, xq, Wq, s_w, M, N, K, Y, gws, gws_bytes,
                                  static_cast<cudaStream_t>(stream));
-    if (st != FQ_ERR_UNSUPPORTED) return st;
-    fq::clear_error();  // not a decode shape: quantize in a launch of its own
+    if (st == FQ_ERR_UNSUPPORTED && !fq_last_error()[0])
+      return fq::fail(FQ_ERR_UNSUPPORTED,
+                      "M = %d is not a decode size (M <= 64), or a cooperative launch is not available", M);
+    return st;
   }
   st = fq_quant_act(X, M, K, act_qp, t, static_scale, xq, sx, stream);
   if (st != FQ_OK) return st;
   // the residual scaling leaves through the per-token epilogue: s_x = S_n
   const fq_gran ggran = gran == FQ_STATIC_RESIDUAL ? FQ_DYNAMIC_ROW : gran;
   return fq_w4a4_gemm(xq, sx, Wq, s_w, M, N, K, ggran, Y, gws, gws_bytes, stream);
+}
+}  // namespace
+
+fq_status fq_linear(const uint16_t* X, int M, int K, const fq_qparams* act_qp, const fq_transform* t,
+                    const float* static_scale, const uint8_t* Wq, const void* s_w, int N, uint16_t* Y,
+                    void* workspace, size_t ws_bytes, void* stream) {
+  return linear_impl(X, M, K, act_qp, t, static_scale, Wq, s_w, N, Y, workspace, ws_bytes, stream, false);
+}
+
+fq_status fq_linear_fused(const uint16_t* X, int M, int K, const fq_qparams* act_qp, const fq_transform* t,
+                          const float* static_scale, const uint8_t* Wq, const void* s_w, int N, uint16_t* Y,
+                          void* workspace, size_t ws_bytes, void* stream) {
+  return linear_impl(X, M, K, act_qp, t, static_scale, Wq, s_w, N, Y, workspace, ws_bytes, stream, true);
 }
 
 }  // extern "C"

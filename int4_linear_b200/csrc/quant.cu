@@ -38,6 +38,7 @@ struct QuantTcParams {
   uint8_t* Q;
   float* s_row;
   __half* s_grp;
+  long long sg_g, sg_m;
   float* xhat;
   unsigned* err;
 };
@@ -78,6 +79,7 @@ struct QuantParams {
 // Xhat[k][l].  Activations: P1^T, so Lc(k, i) = P1[i][k]; weights: P1^-1.
 template <int SIDE>
 __device__ __forceinline__ float left_at(const float* L, int n1, int k, int i) {
+  if (!L) return k == i ? 1.f : 0.f;  // P1 = I
   return SIDE == kAct ? L[i * n1 + k] : L[k * n1 + i];
 }
 // Right factor as used by the row pass: Rr(j, l) multiplies Xbar[i][j] into
@@ -559,9 +561,12 @@ fq_status check_qparams(const fq_qparams* qp, bool act) {
   return FQ_OK;
 }
 
-// dry: validate every argument as for a launch, launch nothing
+// dry: validate every argument as for a launch, launch nothing.  sg_g, sg_m
+// (0: the default group-major [K/128][R]) are element strides of the group
+// scales; only the tensor-core transform kernel takes other strides.
 fq_status quant_common(int side, const uint16_t* X, int R, int K, const fq_qparams* qp, const fq_transform* t,
-                       const float* extra, uint8_t* Q, void* s_out, float* xhat, void* stream, bool dry = false) {
+                       const float* extra, uint8_t* Q, void* s_out, float* xhat, void* stream, bool dry = false,
+                       long long sg_g = 0, long long sg_m = 0) {
   clear_error();
   fq_status st = check_qparams(qp, side == kAct);
   if (st != FQ_OK) return st;
@@ -574,7 +579,7 @@ fq_status quant_common(int side, const uint16_t* X, int R, int K, const fq_qpara
     FQ_CHECK_ARG(extra && aligned(extra, 4), "static scales [K] are required for the static granularities");
   if (qp->gran != FQ_STATIC_CHANNEL)
     FQ_CHECK_ARG(s_out && aligned(s_out, 4), "the scale output must be non-NULL and aligned");
-  if (qp->gran == FQ_STATIC_RESIDUAL && t && (t->P1 || t->c))
+  if (qp->gran == FQ_STATIC_RESIDUAL && t && (t->P1 || t->P2 || t->c))
     return fail(FQ_ERR_UNSUPPORTED, "FQ_STATIC_RESIDUAL takes no transform and no c");
   QuantParams p{};
   p.X = reinterpret_cast<const __half*>(X);
@@ -598,7 +603,7 @@ fq_status quant_common(int side, const uint16_t* X, int R, int K, const fq_qpara
   if (t) {
     p.c = t->c;
     if (t->c) FQ_CHECK_ARG(aligned(t->c, 4), "c must be 4-byte aligned");
-    if (t->P1) {
+    if (t->P1 || t->P2) {
       FQ_CHECK_ARG(t->P2 != nullptr, "P2 is NULL while P1 is given");
       FQ_CHECK_ARG(t->n1 >= 1 && t->n2 >= 1 && t->n1 <= 256 && t->n2 <= 256 && t->n1 * t->n2 == K,
                    "transform tile %d x %d must satisfy n1 * n2 = K = %d with 1 <= n1, n2 <= 256", t->n1, t->n2,
@@ -630,6 +635,8 @@ fq_status quant_common(int side, const uint16_t* X, int R, int K, const fq_qpara
     tp.Q = p.Q;
     tp.s_row = p.s_row;
     tp.s_grp = p.s_grp;
+    tp.sg_g = sg_g ? sg_g : R;
+    tp.sg_m = sg_g ? sg_m : 1;
     tp.xhat = p.xhat;
     tp.err = err;
     return launch_quant_act_tc(tp, s);
@@ -668,6 +675,31 @@ fq_status fq_quant_weight(const uint16_t* W, int N, int K, const fq_qparams* qp,
 fq_status fq_quant_act(const uint16_t* X, int M, int K, const fq_qparams* qp, const fq_transform* t,
                        const float* static_scale, uint8_t* Xq, void* s_x, void* stream) {
   return fq::quant_common(fq::kAct, X, M, K, qp, t, static_scale, Xq, s_x, nullptr, stream);
+}
+
+fq_status fq_quant_kv(const uint16_t* KV, int T, int H, const float* P_h, float alpha, uint8_t* Q, uint16_t* scales,
+                      void* stream) {
+  fq::clear_error();
+  FQ_CHECK_ARG(T >= 1 && H >= 1 && H <= 128, "T = %d must be >= 1 and H = %d in [1, 128]", T, H);
+  FQ_CHECK_ARG(P_h != nullptr, "P_h must be non-NULL");
+  FQ_CHECK_ARG(scales && fq::aligned(scales, 2), "scales must be non-NULL and aligned");
+  fq_qparams qp{};
+  qp.bits = 4;
+  qp.zero_point = 8;
+  qp.gran = FQ_DYNAMIC_GROUP;
+  qp.group_size = fq::kGroup;
+  qp.alpha = alpha;
+  const long long rows = static_cast<long long>(T) * H;  // head-rows of 128
+  if (rows % 64 == 0 && rows / 64 <= 0x7fffffffLL) {
+    // 64 head-rows (of any tokens) per item: P1 = I_64, P2 = P_h; the scale
+    // of head-row r = 64 v + g (item v, group g) goes to r
+    const fq_transform tt{64, 128, nullptr, P_h, nullptr};
+    return fq::quant_common(fq::kAct, KV, int(rows / 64), 64 * 128, &qp, &tt, nullptr, Q, scales, nullptr, stream,
+                            false, 1, 64);
+  }
+  // otherwise one token per item: P1 = I_H, P2 = P_h; head h of token t to t H + h
+  const fq_transform tt{H, 128, nullptr, P_h, nullptr};
+  return fq::quant_common(fq::kAct, KV, T, H * 128, &qp, &tt, nullptr, Q, scales, nullptr, stream, false, 1, H);
 }
 
 fq_status fq_quant_act_debug(const uint16_t* X, int M, int K, const fq_qparams* qp, const fq_transform* t,

@@ -56,6 +56,7 @@ struct QuantTcParams {
   uint8_t* Q;
   float* s_row;
   __half* s_grp;
+  long long sg_g, sg_m;  // element strides of s_grp: group g of token m at g * sg_g + m * sg_m
   float* xhat;
   unsigned* err;
 };
@@ -352,7 +353,12 @@ __global__ void __launch_bounds__(kIntThreads, (N2 == 64 ? 2 : 1)) quant_act_int
     __syncthreads();  // P2 read: the staging bytes take P1
     // P1 stacks: chunk kc (32 columns k), row (3 - b) * 32 + k', byte i = limb b
     // of P1[i][32 kc + k'] (0 past n1); rows 128..159 of a chunk are zero
-    stage(p.P1, n1 * n1, 1);
+    if (p.P1) {
+      stage(p.P1, n1 * n1, 1);
+    } else {  // P1 = I: the rows of the n1 x n2 reshape are transformed on their own
+      for (int e = t; e < n1 * n1; e += kIntThreads) sf[e] = (e / n1 == e % n1) ? 1.f : 0.f;
+      __syncthreads();
+    }
     const int f1 = maxabs(n1 * n1);
     const float s1 = pow2f(-f1);
     for (int e = t; e < NP * (NP / 4); e += kIntThreads) {
@@ -692,7 +698,7 @@ __global__ void __launch_bounds__(kIntThreads, (N2 == 64 ? 2 : 1)) quant_act_int
             sg[tt * 64 + gi] = __half2float(sh);
             const int tkk = tok0 + (N2 == 128 ? g : tt);
             const int kg = N2 == 128 ? kc * 32 + gi : kc * 16 + gi;  // group index within the token
-            if (tkk < M && kg * 128 < n1 * N2) p.s_grp[size_t(kg) * M + tkk] = sh;
+            if (tkk < M && kg * 128 < n1 * N2) p.s_grp[kg * p.sg_g + tkk * p.sg_m] = sh;
           }
           __syncthreads();
         }

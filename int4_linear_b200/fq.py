@@ -48,13 +48,17 @@ class Transform:
     P2: torch.Tensor | None = None
     c: torch.Tensor | None = None
 
+    n1: int = 0  # with P1 None and P2 given: the number of rows of the reshape (P1 = I)
+
     def as_c(self) -> _Transform:
         t = _Transform()
-        if self.P1 is not None:
+        if self.P1 is not None or self.P2 is not None:
             _check(self.P1, torch.float32, "P1")
             _check(self.P2, torch.float32, "P2")
-            t.n1, t.n2 = self.P1.shape[0], self.P2.shape[0]
-            t.P1, t.P2 = self.P1.data_ptr(), self.P2.data_ptr()
+            t.n1 = self.P1.shape[0] if self.P1 is not None else self.n1
+            t.n2 = self.P2.shape[0]
+            t.P1 = self.P1.data_ptr() if self.P1 is not None else None
+            t.P2 = self.P2.data_ptr()
         if self.c is not None:
             _check(self.c, torch.float32, "c")
             t.c = self.c.data_ptr()
@@ -87,6 +91,10 @@ def lib():
         "fq_w4a4_gemm_s32": [vp, vp, i, i, i, vp, vp],
         "fq_w4a4_gemm_noalloc": [vp, vp, vp, vp, i, i, i, i, vp, vp],
         "fq_linear": [vp, i, i, qp, tp, vp, vp, vp, i, vp, vp, sz, vp],
+        "fq_linear_fused": [vp, i, i, qp, tp, vp, vp, vp, i, vp, vp, sz, vp],
+        "fq_ternary_linear": [vp, i, i, vp, vp, vp, i, vp, vp],
+        "fq_quant_kv": [vp, i, i, vp, ctypes.c_float, vp, vp, vp],
+        "fq_ternary_pack": [vp, i, i, vp, vp],
         "fq_check_device_error": [vp],
         "fq_debug_wait_timeout": [ctypes.c_uint, vp],
     }
@@ -262,8 +270,9 @@ def fq_w4a4_gemm_s32(Xq, Wq, acc=None, stream=None):
 
 
 def fq_linear(X, qp: QParams, Wq, s_w, t: Transform | None = None, static_scale=None,
-              Y=None, workspace=None, stream=None):
-    """Y fp16 [M, N] = dequant(Q(X P) Q(P^-1 W^T)), quantization + GEMM on one stream."""
+              Y=None, workspace=None, stream=None, fused=False):
+    """Y fp16 [M, N] = dequant(Q(X P) Q(P^-1 W^T)), quantization + GEMM on one
+    stream (fused=True: fq_linear_fused, one launch at decode sizes)."""
     _check(X, torch.float16, "X")
     _check(Wq, torch.uint8, "Wq")
     _check(static_scale, torch.float32, "static_scale")
@@ -274,10 +283,50 @@ def fq_linear(X, qp: QParams, Wq, s_w, t: Transform | None = None, static_scale=
     gran = ROW_ZP if qp.zero_point == ZERO_POINT_MINMAX else qp.gran
     ws, wsb = _workspace(fq_linear_workspace_size(m, n, k, gran), X.device, workspace)
     tc = t.as_c() if t is not None else None
-    st = lib().fq_linear(X.data_ptr(), m, k, ctypes.byref(qp), ctypes.byref(tc) if tc else None,
+    fn = lib().fq_linear_fused if fused else lib().fq_linear
+    st = fn(X.data_ptr(), m, k, ctypes.byref(qp), ctypes.byref(tc) if tc else None,
                          _p(static_scale), Wq.data_ptr(), _p(s_w), n, Y.data_ptr(), _p(ws), wsb,
                          _s(stream))
     _raise(st)
+    return Y
+
+
+def fq_quant_kv(KV, P_h, alpha: float = 1.0, Q=None, scales=None, stream=None):
+    """INT4 key/value cache: KV fp16 [T, H, 128] (or [T, H * 128]) with the
+    per-head transform P_h [128, 128] -> (Q uint8 [T, H * 64], scales fp16 [T, H])."""
+    _check(KV, torch.float16, "KV")
+    _check(P_h, torch.float32, "P_h")
+    t = KV.shape[0]
+    h = KV[0].numel() // 128
+    Q = torch.empty(t, h * 64, dtype=torch.uint8, device=KV.device) if Q is None else Q
+    scales = torch.empty(t, h, dtype=torch.float16, device=KV.device) if scales is None else scales
+    _raise(lib().fq_quant_kv(KV.data_ptr(), t, h, P_h.data_ptr(), alpha, Q.data_ptr(), scales.data_ptr(),
+                             _s(stream)))
+    return Q, scales
+
+
+def fq_ternary_pack(T, Tq=None, stream=None):
+    """int8 T [N, K] in {-1, 0, 1} -> packed 2-bit codes uint8 [N, K/4]."""
+    _check(T, torch.int8, "T")
+    n, k = T.shape
+    Tq = torch.empty(n, k // 4, dtype=torch.uint8, device=T.device) if Tq is None else Tq
+    _raise(lib().fq_ternary_pack(T.data_ptr(), n, k, Tq.data_ptr(), _s(stream)))
+    return Tq
+
+
+def fq_ternary_linear(X, Tq, alpha, mu, Y=None, stream=None):
+    """Y fp16 [M, N] = X (alpha T + mu)^T for packed ternary codes Tq [N, K/4]
+    and per-(row, 128-block) alpha, mu float32 [N, K/128]."""
+    _check(X, torch.float16, "X")
+    _check(Tq, torch.uint8, "Tq")
+    _check(alpha, torch.float32, "alpha")
+    _check(mu, torch.float32, "mu")
+    m, k = X.shape
+    n = Tq.shape[0]
+    Y = torch.empty(m, n, dtype=torch.float16, device=X.device) if Y is None else Y
+    _check(Y, torch.float16, "Y")
+    _raise(lib().fq_ternary_linear(X.data_ptr(), m, k, Tq.data_ptr(), alpha.data_ptr(), mu.data_ptr(), n,
+                                   Y.data_ptr(), _s(stream)))
     return Y
 
 

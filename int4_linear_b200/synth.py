@@ -220,6 +220,58 @@ def residual_static(m: int, k: int, n: int, seed: int = 0, calib_seed: int = 1,
                 static_scale=s_k, token_scale=r, outlier_cols=cols)
 
 
+def kv_cache(tokens: int, heads: int = 8, head_dim: int = 128, seed: int = 0) -> dict:
+    """Key or value cache entries for INT4 KV quantization with FlatQuant's
+    per-head transform (FlatQuant notes, Transformer 集成: P_h for the keys, P_v
+    for the values, one head_dim x head_dim matrix applied to every head,
+    not decomposed).  As a Kronecker transform of the token's H x D reshape:
+    P1 = I_H, P2 = P_h.
+
+    X fp16 [tokens, heads * head_dim] ~ N(0, 1) with 2 of every head's dims
+    x20 (the same dims in every head: keys carry fixed outlier dims); P_h =
+    random orthogonal x diag(U[0.8, 1.2]).  LLaMA-3-8B-like: 8 KV heads of 128.
+    Draw order: outlier dims (head_dim permutation), X, P_h.
+    """
+    g = generator(seed)
+    dims = g.permutation(head_dim)[:2]
+    cs = np.ones(heads * head_dim)
+    for h_ in range(heads):
+        cs[h_ * head_dim + dims] = 20.0
+    x = _draw(g, (tokens, heads * head_dim), "normal", 1.0, col_scale=cs)
+    p_h, p_h_inv = orthogonal_scaled(g, head_dim)
+    return dict(name=f"kv_cache_{tokens}x{heads}x{head_dim}", x=x, m=tokens, k=heads * head_dim,
+                n1=heads, n2=head_dim, p1=np.eye(heads, dtype=np.float32), p2=p_h, p2_inv=p_h_inv,
+                alpha_a=1.0, outlier_dims=dims)
+
+
+def ternary_linear(m: int, k: int, n: int, seed: int = 0) -> dict:
+    """Decode tokens against ternary weights W^ = alpha T + mu (PT2-LLM page,
+    非对称三值量化器 ATQ), drawn directly (the offline fit needs trained weights).
+
+    X fp16 [m, k] ~ N(0, 1) with 1% outlier channels x30; T int8 [n, k] in
+    {-1, 0, 1} with probabilities (0.275, 0.45, 0.275) (about the share of
+    zeros a ternary fit of Gaussian rows leaves); alpha float32 [n, k/128] ~
+    U[0.01, 0.03]; mu float32 [n, k/128] ~ U[-0.005, 0.005] (the per-row
+    offsets the asymmetric grid exists for).  Draw order: X, T, alpha, mu;
+    the outlier channels come from the stream seed + 1_000_003.
+    """
+    h = generator(seed + 1_000_003)
+    cols = outlier_channels(h, k)
+    cs = np.ones(k)
+    cs[cols] = 30.0
+    g = generator(seed)
+    x = _draw(g, (m, k), "normal", 1.0, col_scale=cs)
+    u = g.uniform(0.0, 1.0, (n, k))
+    t = np.where(u < 0.275, -1, np.where(u < 0.725, 0, 1)).astype(np.int8)
+    alpha = g.uniform(0.01, 0.03, (n, k // GROUP)).astype(np.float32)
+    mu = g.uniform(-0.005, 0.005, (n, k // GROUP)).astype(np.float32)
+    return dict(name=f"ternary_{m}x{k}x{n}", x=x, t=t, alpha=alpha, mu=mu, m=m, k=k, n=n)
+
+
+# Decode shapes of the ternary workload: the LLaMA-3-70B-like gate+up and down.
+TERNARY_SHAPES = [(8192, 57344), (28672, 8192)]
+
+
 # The LLaMA-3-8B-like decoder-layer linears at prefill, M = 2048 tokens:
 # (K, N) for qkv, o, gate+up, down.
 PREFILL_8B_SHAPES = [(4096, 6144), (4096, 4096), (4096, 28672), (14336, 4096)]

@@ -169,3 +169,22 @@ def test_zero_point_gemm_needs_its_workspace(L):
     assert st == fq.FQ_ERR_INVALID and b"workspace" in L.fq_last_error()
     ws = L.fq_linear_workspace_size(8, 256, 256, fq.ROW_ZP)
     assert ws >= 8 * 128 + 3 * 8 * 4 + 8 * 256 * 4
+
+
+def test_ternary_rejects_arguments(L):
+    """Sizes, NULLs and alignment are checked before any launch."""
+    assert L.fq_ternary_linear(A, 1, 100, A, A, A, 8, A, None) == fq.FQ_ERR_INVALID
+    assert L.fq_ternary_linear(A, 0, 128, A, A, A, 8, A, None) == fq.FQ_ERR_INVALID
+    assert L.fq_ternary_linear(A, 1, 128, None, A, A, 8, A, None) == fq.FQ_ERR_INVALID
+    assert L.fq_ternary_linear(A + 8, 1, 128, A, A, A, 8, A, None) == fq.FQ_ERR_INVALID
+    assert b"aligned" in L.fq_last_error()
+    assert L.fq_ternary_pack(A, 4, 24, A, None) == fq.FQ_ERR_INVALID
+    assert L.fq_ternary_pack(A + 4, 4, 32, A, None) == fq.FQ_ERR_INVALID
+
+
+def test_fused_linear_rejects_what_it_does_not_cover(L):
+    """The one-launch decode linear takes static per-channel scales only."""
+    qp = _qp()  # dynamic per-token
+    need = L.fq_linear_workspace_size(8, 256, 256, fq.ROW)
+    st = L.fq_linear_fused(A, 8, 256, ctypes.byref(qp), None, None, A, A, 256, A, A, need, None)
+    assert st == fq.FQ_ERR_UNSUPPORTED and b"static" in L.fq_last_error()

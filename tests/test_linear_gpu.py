@@ -145,8 +145,8 @@ def _kernel_names(fn):
 
 @pytest.mark.parametrize("m,k,n", [(1, 8192, 10240), (8, 28672, 8192), (64, 8192, 57344), (17, 1024, 3072)])
 def test_linear_decode_fused_one_launch(m, k, n):
-    """Decode with static scales (and a channel factor c) through fq_linear: one
-    kernel launch, no separate quantization, no memset; outputs bit-exact
+    """Decode with static scales (and a channel factor c) through fq_linear_fused:
+    one kernel launch, no separate quantization, no memset; outputs bit-exact
     against the oracle; three calls in a row on one workspace whose bytes past
     the counter block are garbage, the counters (all words but the grid
     barrier's generation number, word 1) back at zero after each."""
@@ -159,7 +159,7 @@ def test_linear_decode_fused_one_launch(m, k, n):
     ws = torch.full((fq.fq_linear_workspace_size(m, n, k, fq.STATIC),), 0x5A, dtype=torch.uint8, device="cuda")
     ws[: fq.SYNC_BYTES].zero_()
     Y = torch.empty(m, n, dtype=torch.float16, device="cuda")
-    names = _kernel_names(lambda: fq.fq_linear(X, qp, wq, sw, t, static_scale=SK, Y=Y, workspace=ws))
+    names = _kernel_names(lambda: fq.fq_linear(X, qp, wq, sw, t, static_scale=SK, Y=Y, workspace=ws, fused=True))
     assert len(names) == 1 and "gemm_decode_kernel" in names[0], names
     q_ref, _, _ = O.quant_act(d["x"], O.STATIC, c=c, static_scale=s_k)
     cols = C.tile_samples(m + k + n, n)
@@ -167,11 +167,13 @@ def test_linear_decode_fused_one_launch(m, k, n):
     first = C.host(Y)
     C.check_gemm_decoupled(first[:, cols], q_ref, None, qw, sw_ref, O.STATIC)
     for _ in range(2):
-        y = C.host(fq.fq_linear(X, qp, wq, sw, t, static_scale=SK, Y=Y, workspace=ws))
+        y = C.host(fq.fq_linear(X, qp, wq, sw, t, static_scale=SK, Y=Y, workspace=ws, fused=True))
         assert np.array_equal(y.view(np.uint16), first.view(np.uint16))
         words = ws[: fq.SYNC_BYTES].view(torch.int32)
         assert not words[0] and not words[2:].any(), "the counters are not back at zero"
     xq, _ = fq.fq_quant_act(X, qp, t, SK)
     y2 = C.host(fq.fq_w4a4_gemm(xq, None, wq, sw, fq.STATIC))
     assert np.array_equal(y2.view(np.uint16), first.view(np.uint16)), "fused and two-launch paths differ"
+    y3 = C.host(fq.fq_linear(X, qp, wq, sw, t, static_scale=SK))
+    assert np.array_equal(y3.view(np.uint16), first.view(np.uint16)), "fq_linear differs from fq_linear_fused"
     fq.fq_check_device_error()

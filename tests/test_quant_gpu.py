@@ -115,6 +115,37 @@ def test_quant_act_transform_group():
     _transform_case(d, "group")
 
 
+@pytest.mark.parametrize("tokens,heads", [(64, 8), (1000, 8), (256, 32)])
+def test_quant_kv_cache_per_head(tokens, heads):
+    """INT4 key / value cache: FlatQuant's per-head P_h as the Kronecker
+    transform P1 = I_H, P2 = P_h, one scale per token and head (the 128-group
+    of a 128-wide head); the identity passed as a matrix and as P1 = NULL."""
+    d = synth.kv_cache(tokens, heads)
+    _transform_case(d, "group")
+    x, t = C.dev(d["x"]), fq.Transform(None, C.dev(d["p2"]), n1=heads)
+    q1, s1, v1 = fq.fq_quant_act_debug(x, fq.qparams(fq.GROUP, 1.0), t)
+    q2, s2, v2 = fq.fq_quant_act_debug(x, fq.qparams(fq.GROUP, 1.0), fq.Transform(C.dev(d["p1"]), C.dev(d["p2"])))
+    assert torch.equal(q1, q2) and torch.equal(s1, s2) and torch.equal(v1, v2), "P1 = NULL differs from P1 = I"
+
+
+@pytest.mark.parametrize("tokens,heads", [(64, 8), (1000, 8), (40, 5), (256, 32), (3, 1)])
+def test_fq_quant_kv(tokens, heads):
+    """fq_quant_kv: 64 head vectors per kernel item when tokens * heads is a
+    multiple of 64 (else one token per item); codes and token-major scales
+    against the oracle (the transformed values through the tolerance of
+    reading 12 as everywhere: scales equal or one fp16 step apart at a
+    midpoint, codes equal outside the tie band)."""
+    d = synth.kv_cache(tokens, heads, seed=tokens + heads)
+    q, s = fq.fq_quant_kv(C.dev(d["x"]), C.dev(d["p2"]), 0.95)
+    q_ref, s_ref, v_ref = O.quant_act(d["x"], O.GROUPED, 0.95, d["p1"], d["p2"])
+    sg = C.host(s).astype(np.float32)
+    C.check_scales_group(sg, s_ref, v_ref, 0.95)
+    ex = C.exempt_mask(v_ref, s_ref, sg, O.GROUPED)
+    n_ex, n_diff = C.check_codes(C.unpack(C.host(q)), q_ref, ex)
+    print(f"{d['name']}: boundary-exempt {n_ex}, differing codes {n_diff}")
+    fq.fq_check_device_error()
+
+
 @pytest.mark.parametrize("k", [14336, 28672])
 def test_quant_act_transform_wide(k):
     """(112, 128) keeps the factors in shared memory; (224, 128) reads them through L1."""
