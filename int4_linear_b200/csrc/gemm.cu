@@ -663,7 +663,12 @@ struct PCfg {
   static constexpr int B_WARP0 = 2 + 4 * NA;   // A: warps 2 .. 2 + 4 NA - 1
   static constexpr int EPI_WARP0 = B_WARP0 + NB;
   static constexpr int THREADS = 32 * (EPI_WARP0 + 8);
-  static constexpr int FEED = 4 + 1;           // arrivals per slice and CTA: 4 A-warps, 1 B-warp
+  static constexpr int FEED = 4 + 1;           // CTA 0's arrivals per slice: 4 A-warps, 1 B-warp
+  // CTA 1's feed warps of one slice (the 4 A-warps and the B-warp of turn
+  // g mod NA) meet at named barrier 2 + turn, and one of them publishes the
+  // slice to CTA 0 with a single cluster-scope release (the barrier orders the
+  // group's operand writes before it; release is cumulative)
+  static_assert(NA == NB, "A- and B-warps take the slices in the same turns");
   static_assert(A_COL0 + SU * A_STAGE_COLS <= TMEM_COLS, "tensor memory");
   static_assert(SMEM <= 227 * 1024, "shared memory");
   static_assert(P_STAGE % 1024 == 0 && UNP_STAGE % 1024 == 0 && PA % 1024 == 0, "1024-byte stage alignment");
@@ -711,7 +716,7 @@ __global__ void __launch_bounds__(PCfg<NB>::THREADS, 1)
       mbar_init(&pempty[s], C::FEED);
     }
     for (int s = 0; s < SU; ++s) {
-      mbar_init(&full_u[s], 2 * C::FEED);
+      mbar_init(&full_u[s], C::FEED + 1);
       mbar_init(&empty_u[s], 1);
     }
     mbar_init(acc_full, 1);
@@ -819,37 +824,45 @@ __global__ void __launch_bounds__(PCfg<NB>::THREADS, 1)
     bool ok = true;
     for (uint32_t g = uint32_t(par); g < total; g += C::NA) {
       const int sp = int(g % SP), su = int(g % SU);
-      if (!warp_wait(&pfull[sp], (g / SP) & 1)) {
-        ok = false;
-        break;
-      }
-      const uint8_t* src = smem + C::OFF_P + sp * C::P_STAGE + row * kPK;
+      bool fail = !warp_wait(&pfull[sp], (g / SP) & 1);
       uint4 w[4];
+      if (!fail) {
+        const uint8_t* src = smem + C::OFF_P + sp * C::P_STAGE + row * kPK;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) w[c] = *reinterpret_cast<const uint4*>(src + ((c ^ sw) << 4));
-      if (!warp_wait(&empty_u[su], ((g / SU) & 1) ^ 1)) {
-        ok = false;
-        break;
+        for (int c = 0; c < 4; ++c) w[c] = *reinterpret_cast<const uint4*>(src + ((c ^ sw) << 4));
+        fail = !warp_wait(&empty_u[su], ((g / SU) & 1) ^ 1);
       }
-      tc_fence_after();
-      uint32_t r[32];
+      if (!fail) {
+        tc_fence_after();
+        uint32_t r[32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        unpack8_hi(w[c].x, r[8 * c + 0], r[8 * c + 1]);
-        unpack8_hi(w[c].y, r[8 * c + 2], r[8 * c + 3]);
-        unpack8_hi(w[c].z, r[8 * c + 4], r[8 * c + 5]);
-        unpack8_hi(w[c].w, r[8 * c + 6], r[8 * c + 7]);
+        for (int c = 0; c < 4; ++c) {
+          unpack8_hi(w[c].x, r[8 * c + 0], r[8 * c + 1]);
+          unpack8_hi(w[c].y, r[8 * c + 2], r[8 * c + 3]);
+          unpack8_hi(w[c].z, r[8 * c + 4], r[8 * c + 5]);
+          unpack8_hi(w[c].w, r[8 * c + 6], r[8 * c + 7]);
+        }
+        tmem_st_32x32(ta + uint32_t(su * C::A_STAGE_COLS), r);
+        tmem_wait_st();
+        tc_fence_before();
       }
-      tmem_st_32x32(ta + uint32_t(su * C::A_STAGE_COLS), r);
-      tmem_wait_st();
-      tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&pempty[sp]);
-        if (crank == 0)
+      if (crank == 0) {
+        if (fail) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          mbar_arrive(&pempty[sp]);
           mbar_arrive(&full_u[su]);
-        else
-          mbar_arrive_cluster(&full_u[su], 0);  // cluster-scope release of this warp's operands
+        }
+      } else {
+        // the slice's group meets; its B-warp publishes the slice to CTA 0
+        if (named_barrier_or(2 + par, 160, fail)) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) mbar_arrive(&pempty[sp]);
       }
     }
     if (!ok && lane == 0) record_error(p.err, kErrTimeoutUnpack);
@@ -864,42 +877,54 @@ __global__ void __launch_bounds__(PCfg<NB>::THREADS, 1)
     bool ok = true;
     for (uint32_t g = uint32_t(bw); g < total; g += NB) {
       const int sp = int(g % SP), su = int(g % SU);
-      if (!warp_wait(&pfull[sp], (g / SP) & 1)) {
-        ok = false;
-        break;
+      bool fail = !warp_wait(&pfull[sp], (g / SP) & 1);
+      if (!fail) {
+        const uint8_t* pb = smem + C::OFF_P + sp * C::P_STAGE + C::PA + lane * 16;
+        uint8_t* uk = smem + C::OFF_UNP + su * C::UNP_STAGE;
+        constexpr int kIt = C::BR / 8;  // 8 rows (32 pieces) per step
+#pragma unroll
+        for (int it0 = 0; it0 < kIt; it0 += 4) {
+          uint4 w[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) w[u] = *reinterpret_cast<const uint4*>(pb + (it0 + u) * 512);
+          if (it0 == 0 && !warp_wait(&empty_u[su], ((g / SU) & 1) ^ 1)) {
+            fail = true;
+            break;
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            uint4 o0, o1;
+            unpack8_hi(w[u].x, o0.x, o0.y);
+            unpack8_hi(w[u].y, o0.z, o0.w);
+            unpack8_hi(w[u].z, o1.x, o1.y);
+            unpack8_hi(w[u].w, o1.z, o1.w);
+            *reinterpret_cast<uint4*>(uk + (it0 + u) * 1024 + dst0) = o0;
+            *reinterpret_cast<uint4*>(uk + (it0 + u) * 1024 + dst1) = o1;
+          }
+        }
       }
-      const uint8_t* pb = smem + C::OFF_P + sp * C::P_STAGE + C::PA + lane * 16;
-      uint8_t* uk = smem + C::OFF_UNP + su * C::UNP_STAGE;
-      constexpr int kIt = C::BR / 8;  // 8 rows (32 pieces) per step
-#pragma unroll
-      for (int it0 = 0; it0 < kIt; it0 += 4) {
-        uint4 w[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) w[u] = *reinterpret_cast<const uint4*>(pb + (it0 + u) * 512);
-        if (it0 == 0 && !warp_wait(&empty_u[su], ((g / SU) & 1) ^ 1)) {
+      if (!fail) fence_proxy_async_smem();
+      __syncwarp();
+      if (crank == 0) {
+        if (fail) {
           ok = false;
           break;
         }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          uint4 o0, o1;
-          unpack8_hi(w[u].x, o0.x, o0.y);
-          unpack8_hi(w[u].y, o0.z, o0.w);
-          unpack8_hi(w[u].z, o1.x, o1.y);
-          unpack8_hi(w[u].w, o1.z, o1.w);
-          *reinterpret_cast<uint4*>(uk + (it0 + u) * 1024 + dst0) = o0;
-          *reinterpret_cast<uint4*>(uk + (it0 + u) * 1024 + dst1) = o1;
-        }
-      }
-      if (!ok) break;
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&pempty[sp]);
-        if (crank == 0)
+        if (lane == 0) {
+          mbar_arrive(&pempty[sp]);
           mbar_arrive(&full_u[su]);
-        else
-          mbar_arrive_cluster(&full_u[su], 0);  // cluster-scope release of this warp's operands
+        }
+      } else {
+        // the slice's group (this warp and the 4 A-warps of turn bw) meets;
+        // one cluster-scope release publishes all their operand writes
+        if (named_barrier_or(2 + bw, 160, fail)) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          mbar_arrive(&pempty[sp]);
+          mbar_arrive_cluster(&full_u[su], 0);
+        }
       }
     }
     if (!ok && lane == 0) record_error(p.err, kErrTimeoutUnpack);

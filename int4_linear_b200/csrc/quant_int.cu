@@ -14,13 +14,13 @@
 // sub-row's largest fp16 value, 2^-31 with c; 2^-30 of the largest factor
 // entry; 2^-29 of the intermediate bound), far below float32's.
 //
-// Structure (all shapes n2 in {64, 128}, n1 <= 128; one CTA of 128 threads,
-// thread t = tensor-memory lane t, two CTAs per SM when shared memory allows).
-// An item is G tokens (G = 2 when n1 <= 64, else 1), so that stage A has
-// 128 rows (token s, tile row i):
-//   1. thread (s, i) loads its tile row (n2 fp16 values, times c), picks a
-//      power-of-two scale for it, and writes its XL limbs (XL = 3, 4 with c)
-//      as the K-major A operand rows of stage A;
+// Structure (all shapes n2 in {64, 128}, n1 <= 128; one CTA of 256 threads,
+// two per tile row (tensor-memory lane t and its second half), two CTAs per
+// SM when shared memory allows).  An item is G tokens (G = 2 when n1 <= 64,
+// else 1), so that stage A has 128 rows (token s, tile row i):
+//   1. the threads of row (s, i) load its tile row (n2 fp16 values, times c),
+//      pick a power-of-two scale for it, and write its XL = 4 limbs as the
+//      K-major A operand rows of stage A;
 //   2. stage A: D[(s, i)][(level, l)] = sum_j Xbar_s[i][j] P2[j][l] by
 //      levels: limb products of equal weight 256^L accumulate together.  P2
 //      is held as 4 limbs stacked along N ([p3; p2; p1; p0] per 64-column
@@ -31,11 +31,13 @@
 //      writes V's 4 limbs as the MN-major A operand of stage B (row i of the
 //      operand holds the 128 M positions (s, l));
 //   4. stage B: D[(s, l)][(level, k)] = sum_i V_s[i][l] P1[i][k], P1 as 4
-//      stacked limbs per 64-column chunk of k;
+//      stacked limbs per 32-column chunk of k (five levels, a zero block
+//      padding the stack); P1 = NULL stages the identity;
 //   5. thread = (s, l): levels -> exact 64-bit value -> float32 X̂ (one
 //      rounding), per-token / per-group maxima by warp reductions, scales,
 //      round-half-even codes (reciprocal fast path outside a tie band, IEEE
-//      quotient inside it), a 3-step shuffle transpose into 32-bit stores.
+//      quotient inside it) into a shared-memory code tile that leaves by one
+//      bulk store per item; group scales go out through caller strides.
 #include <cuda_fp16.h>
 
 #include <algorithm>

@@ -48,10 +48,19 @@ __device__ __forceinline__ float ternary_value(uint32_t code) {
   return __int_as_float(int((code & 1u) * 0x3F800000u) | int((code & 2u) << 30));
 }
 
+// The values of two weights from their 4-bit code pair, looked up in a
+// 16-entry float2 table: the 16 entries of 8 bytes fill the 32 banks once,
+// so a warp's lookups never conflict.
+__device__ __forceinline__ float2 ternary_pair(const float2* lut, uint32_t w, int i) {
+  return lut[(w >> (4 * i)) & 15u];
+}
+
 __global__ void __launch_bounds__(kTerThreads) ternary_linear_kernel(const TernaryParams p) {
   extern __shared__ float sS[];  // [kTerMT][K/128] block sums of the token group
+  __shared__ float2 lut[16];     // code pair -> the two weights' values
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int K = p.K, nb = K / kTerBlock, words = K / 16;
+  if (tid < 16) lut[tid] = make_float2(ternary_value(uint32_t(tid)), ternary_value(uint32_t(tid) >> 2));
   pdl_wait();
   for (int m0 = 0; m0 < p.M; m0 += kTerMT) {
     const int mt = min(kTerMT, p.M - m0);
@@ -97,11 +106,11 @@ __global__ void __launch_bounds__(kTerThreads) ternary_linear_kernel(const Terna
         for (int u = 0; u < kTerU; ++u) {
           const int j = j0 + 32 * u;
           if (j >= words) break;
-          float tv[kTerR][16];
+          float2 tv[kTerR][8];
 #pragma unroll
           for (int r = 0; r < kTerR; ++r)
 #pragma unroll
-            for (int i = 0; i < 16; ++i) tv[r][i] = ternary_value(wv[u][r] >> (2 * i));
+            for (int i = 0; i < 8; ++i) tv[r][i] = ternary_pair(lut, wv[u][r], i);
 #pragma unroll
           for (int m = 0; m < kTerMT; ++m) {
             if (m >= mt) break;
@@ -116,8 +125,8 @@ __global__ void __launch_bounds__(kTerThreads) ternary_linear_kernel(const Terna
               const float2 xf = __half22float2(*reinterpret_cast<const __half2*>(&hw[i]));
 #pragma unroll
               for (int r = 0; r < kTerR; ++r) {
-                sr[r] = fmaf(xf.x, tv[r][2 * i], sr[r]);
-                sr[r] = fmaf(xf.y, tv[r][2 * i + 1], sr[r]);
+                sr[r] = fmaf(xf.x, tv[r][i].x, sr[r]);
+                sr[r] = fmaf(xf.y, tv[r][i].y, sr[r]);
               }
             }
 #pragma unroll
