@@ -41,7 +41,7 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # (dram__bytes_read.sum + dram__bytes_write.sum) of this bench command on the
 # current GEMM kernel; the fp16 outputs that still sit in L2 when a launch
 # ends are not in it.
-GEMM_DRAM_BYTES = {"qkv": 16842240, "o": 12640000, "gate_up": 63101696 + 69518336, "down": 44100096 + 29440}
+GEMM_DRAM_BYTES = {"qkv": 16844544 + 768, "o": 12641280, "gate_up": 63201280 + 69606400, "down": 44098816 + 11776}
 INT8_OVER_BF16 = 4.5 / 2.25  # nominal dense ratio (B200: 4.5 POPS int8 vs 2.25 PFLOPS bf16)
 ALU_CLOCK_GHZ = 1.965  # clocks.max.sm of this B200 (the ALU roofline of the ternary kernel)
 

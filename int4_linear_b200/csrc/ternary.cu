@@ -65,20 +65,32 @@ __global__ void __launch_bounds__(kTerThreads) ternary_linear_kernel(const Terna
   for (int m0 = 0; m0 < p.M; m0 += kTerMT) {
     const int mt = min(kTerMT, p.M - m0);
     __syncthreads();  // the previous group's sums are no longer read
-    // block sums: one warp per (token, block), 4 values per lane, coalesced
-    for (int e = warp; e < kTerMT * nb; e += kTerWarps) {
-      const int m = e / nb, g = e - m * nb;
-      float v = 0.f;
-      if (m < mt) {
-        const uint2 raw = __ldg(reinterpret_cast<const uint2*>(p.X + size_t(m0 + m) * K + g * kTerBlock) + lane);
-        const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
-        const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
-        v = (a.x + a.y) + (b.x + b.y);
+    // block sums: one warp per (token, block), 4 values per lane, coalesced,
+    // four sums per warp in flight; the slots of absent tokens are zero
+    for (int e0 = warp; e0 < mt * nb; e0 += 4 * kTerWarps) {
+      float v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int e = e0 + u * kTerWarps;
+        v[u] = 0.f;
+        if (e < mt * nb) {
+          const int m = e / nb, g = e - m * nb;
+          const uint2 raw =
+              __ldg(reinterpret_cast<const uint2*>(p.X + size_t(m0 + m) * K + g * kTerBlock) + lane);
+          const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
+          const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
+          v[u] = (a.x + a.y) + (b.x + b.y);
+        }
       }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      if (lane == 0) sS[e] = v;
+      for (int u = 0; u < 4; ++u) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v[u] += __shfl_xor_sync(0xffffffffu, v[u], o);
+        const int e = e0 + u * kTerWarps;
+        if (lane == 0 && e < mt * nb) sS[e] = v[u];
+      }
     }
+    for (int e = mt * nb + tid; e < kTerMT * nb; e += kTerThreads) sS[e] = 0.f;
     __syncthreads();
     // kTerR rows per warp share every token load; kTerU code words per lane
     // are loaded ahead of their use
@@ -88,20 +100,28 @@ __global__ void __launch_bounds__(kTerThreads) ternary_linear_kernel(const Terna
       for (int r = 0; r < kTerR; ++r)
 #pragma unroll
         for (int m = 0; m < kTerMT; ++m) acc[r][m] = 0.f;
-      for (int j0 = lane; j0 < words; j0 += 32 * kTerU) {
-        uint32_t wv[kTerU][kTerR];
-        float av[kTerU][kTerR];
+      // code words (and alphas) of the next kTerU words per lane are loaded
+      // while the current ones are used
+      uint32_t wv[kTerU][kTerR];
+      float av[kTerU][kTerR];
+      auto load_words = [&](int jb, uint32_t (&w)[kTerU][kTerR], float (&a)[kTerU][kTerR]) {
 #pragma unroll
         for (int u = 0; u < kTerU; ++u) {
-          const int j = j0 + 32 * u;
+          const int j = jb + 32 * u;
 #pragma unroll
           for (int r = 0; r < kTerR; ++r) {
             const int n = n0 + r;
             const bool live = j < words && n < p.N;
-            wv[u][r] = live ? __ldg(p.T + size_t(n) * words + j) : 0u;
-            av[u][r] = live ? __ldg(p.alpha + size_t(n) * nb + (j >> 3)) : 0.f;
+            w[u][r] = live ? __ldg(p.T + size_t(n) * words + j) : 0u;
+            a[u][r] = live ? __ldg(p.alpha + size_t(n) * nb + (j >> 3)) : 0.f;
           }
         }
+      };
+      load_words(lane, wv, av);
+      for (int j0 = lane; j0 < words; j0 += 32 * kTerU) {
+        uint32_t wn[kTerU][kTerR];
+        float an[kTerU][kTerR];
+        load_words(j0 + 32 * kTerU, wn, an);
 #pragma unroll
         for (int u = 0; u < kTerU; ++u) {
           const int j = j0 + 32 * u;
@@ -133,6 +153,13 @@ __global__ void __launch_bounds__(kTerThreads) ternary_linear_kernel(const Terna
             for (int r = 0; r < kTerR; ++r) acc[r][m] = fmaf(av[u][r], sr[r], acc[r][m]);
           }
         }
+#pragma unroll
+        for (int u = 0; u < kTerU; ++u)
+#pragma unroll
+          for (int r = 0; r < kTerR; ++r) {
+            wv[u][r] = wn[u][r];
+            av[u][r] = an[u][r];
+          }
       }
 #pragma unroll
       for (int r = 0; r < kTerR; ++r) {
