@@ -1069,7 +1069,9 @@ __global__ void __launch_bounds__(PCfg<NB>::THREADS, 1)
 // as two CTAs do.
 template <int BN, bool ONE = false>
 struct DecCfg {
-  static constexpr int SP = ONE ? (BN == 64 ? 12 : 16) : (BN == 64 ? 6 : 8);  // packed stages (weights + tokens)
+  // packed stages (weights + tokens); deeper rings (9-11 stages) measured
+  // slower at two CTAs per SM
+  static constexpr int SP = ONE ? (BN == 64 ? 12 : 16) : (BN == 64 ? 6 : 8);
   static constexpr int UG = ONE ? 2 : 1;          // unpacking groups
   static constexpr int ACC = BN < 32 ? 32 : BN;   // columns of one accumulator
   // MMA-issuing threads (warp 1, then warps I_WARP0...): a tcgen05.mma of
