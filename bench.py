@@ -332,7 +332,7 @@ def run_ours(args, ws, rank, local):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "int4 (s8 tensor-core MMA, s32 accumulate), fp32 transform/scales, fp16 io",
+        "dtype": "int4 (s8 tensor-core MMA, s32 accumulate), exact transform (int8-limb MMA, int32 level sums), fp32 scales, fp16 io",
         "data": "synthetic (seeded Gaussian activations with outlier channels, Gaussian weights; stands in for LLaMA activations/weights)",
         "config": {
             "workload": WORKLOAD,

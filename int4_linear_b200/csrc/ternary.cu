@@ -137,20 +137,18 @@ __global__ void __launch_bounds__(kTerThreads) ternary_linear_kernel(const Terna
             const uint4* xp = reinterpret_cast<const uint4*>(p.X + size_t(m0 + m) * K + 16 * j);
             const uint4 r0 = __ldg(xp), r1 = __ldg(xp + 1);
             const uint32_t hw[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
-            float sr[kTerR];
+            // even and odd weights in the two lanes of packed float32 FMAs
+            float2 sr[kTerR];
 #pragma unroll
-            for (int r = 0; r < kTerR; ++r) sr[r] = 0.f;
+            for (int r = 0; r < kTerR; ++r) sr[r] = make_float2(0.f, 0.f);
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
               const float2 xf = __half22float2(*reinterpret_cast<const __half2*>(&hw[i]));
 #pragma unroll
-              for (int r = 0; r < kTerR; ++r) {
-                sr[r] = fmaf(xf.x, tv[r][i].x, sr[r]);
-                sr[r] = fmaf(xf.y, tv[r][i].y, sr[r]);
-              }
+              for (int r = 0; r < kTerR; ++r) sr[r] = ffma2(xf, tv[r][i], sr[r]);
             }
 #pragma unroll
-            for (int r = 0; r < kTerR; ++r) acc[r][m] = fmaf(av[u][r], sr[r], acc[r][m]);
+            for (int r = 0; r < kTerR; ++r) acc[r][m] = fmaf(av[u][r], sr[r].x + sr[r].y, acc[r][m]);
           }
         }
 #pragma unroll
