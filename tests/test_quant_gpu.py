@@ -132,9 +132,9 @@ def test_quant_kv_cache_per_head(tokens, heads):
 def test_fq_quant_kv(tokens, heads):
     """fq_quant_kv: 64 head vectors per kernel item when tokens * heads is a
     multiple of 64 (else one token per item); codes and token-major scales
-    against the oracle (the transformed values through the tolerance of
-    reading 12 as everywhere: scales equal or one fp16 step apart at a
-    midpoint, codes equal outside the tie band)."""
+    against the oracle (the transformed-value tolerance of gpu_checks:
+    scales equal or one fp16 step apart at a midpoint, codes equal outside
+    the tie band)."""
     d = synth.kv_cache(tokens, heads, seed=tokens + heads)
     q, s = fq.fq_quant_kv(C.dev(d["x"]), C.dev(d["p2"]), 0.95)
     q_ref, s_ref, v_ref = O.quant_act(d["x"], O.GROUPED, 0.95, d["p1"], d["p2"])
@@ -143,6 +143,21 @@ def test_fq_quant_kv(tokens, heads):
     ex = C.exempt_mask(v_ref, s_ref, sg, O.GROUPED)
     n_ex, n_diff = C.check_codes(C.unpack(C.host(q)), q_ref, ex)
     print(f"{d['name']}: boundary-exempt {n_ex}, differing codes {n_diff}")
+    fq.fq_check_device_error()
+
+
+def test_fq_quant_kv_bench_size():
+    """The benchmark's KV workload (16384 tokens x 8 heads) in its launch
+    configuration, on sampled tokens covering every 128-token stretch."""
+    d = synth.kv_cache(16384, 8)
+    q, s = fq.fq_quant_kv(C.dev(d["x"]), C.dev(d["p2"]))
+    rows = C.tile_samples(17, 16384)
+    q_ref, s_ref, v_ref = O.quant_act(d["x"][rows], O.GROUPED, 1.0, d["p1"], d["p2"])
+    sg = C.host(s)[rows].astype(np.float32)
+    C.check_scales_group(sg, s_ref, v_ref, 1.0)
+    ex = C.exempt_mask(v_ref, s_ref, sg, O.GROUPED)
+    n_ex, n_diff = C.check_codes(C.unpack(C.host(q)[rows]), q_ref, ex)
+    print(f"{d['name']}: {len(rows)} tokens, boundary-exempt {n_ex}, differing codes {n_diff}")
     fq.fq_check_device_error()
 
 
