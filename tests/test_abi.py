@@ -188,3 +188,27 @@ def test_fused_linear_rejects_what_it_does_not_cover(L):
     need = L.fq_linear_workspace_size(8, 256, 256, fq.ROW)
     st = L.fq_linear_fused(A, 8, 256, ctypes.byref(qp), None, None, A, A, 256, A, A, need, None)
     assert st == fq.FQ_ERR_UNSUPPORTED and b"static" in L.fq_last_error()
+
+
+def test_quant_kv_rejects_arguments(L):
+    """fq_quant_kv: T >= 1, 1 <= H <= 128, P_h and the scale output non-NULL, the
+    same alignment rules as fq_quant_act (checked before any launch)."""
+    assert L.fq_quant_kv(A, 0, 8, A, 1.0, A, A, None) == fq.FQ_ERR_INVALID
+    assert L.fq_quant_kv(A, 4, 129, A, 1.0, A, A, None) == fq.FQ_ERR_INVALID
+    assert L.fq_quant_kv(A, 4, 8, None, 1.0, A, A, None) == fq.FQ_ERR_INVALID
+    assert L.fq_quant_kv(A, 4, 8, A, 1.0, A, None, None) == fq.FQ_ERR_INVALID
+    assert L.fq_quant_kv(A + 8, 8, 8, A, 1.0, A, A, None) == fq.FQ_ERR_INVALID  # X not 16-byte aligned
+    assert L.fq_quant_kv(A, 8, 8, A, 0.0, A, A, None) == fq.FQ_ERR_INVALID      # alpha out of (0, 1]
+
+
+@pytest.mark.parametrize("m,n,k", [(1, 8192, 28672), (8, 57344, 8192), (64, 4096, 4096), (2048, 28672, 4096),
+                                   (4096, 10240, 8192)])
+def test_linear_workspace_holds_its_parts(L, m, n, k):
+    """fq_linear's workspace: the GEMM's part (at least the 16 KB counter block,
+    first), then the packed activations and their scales, each 256-byte aligned."""
+    up = lambda v: (v + 255) // 256 * 256
+    for gran, scale_bytes in ((fq.ROW, 4 * m), (fq.STATIC, 0), (fq.GROUP, 2 * m * (k // 128)),
+                              (fq.STATIC_RESIDUAL, 4 * m), (fq.ROW_ZP, 12 * m)):
+        gemm = max(fq.SYNC_BYTES, L.fq_gemm_workspace_size(m, n, k, gran))
+        need = up(gemm) + up(m * k // 2) + up(scale_bytes)
+        assert L.fq_linear_workspace_size(m, n, k, gran) == need, (gran, m, n, k)
