@@ -515,7 +515,7 @@ def run_ternary(args, dev_index):
         "rows": rows,
         "config": {"workload": "ternary decode, M in {1, 8} x (K, N) in {(8192, 57344), (28672, 8192)}, "
                                "2-bit codes, per-(row, 128-block) alpha and mu, fp16 tokens"},
-        "roofline": {"kernel": "ternary_linear_kernel", "bound": "hbm / alu per row", "achieved": round(frac, 4),
+        "roofline": {"kernel": "ternary_lut_kernel", "bound": "hbm / alu per row", "achieved": round(frac, 4),
                      "peak": 1.0, "unit": "fraction", "frac": round(frac, 4),
                      "peak_kind": f"{pk_kind} HBM; ALU = 148 x 128 lanes x {ALU_CLOCK_GHZ} GHz"},
         "clocks": clk,

@@ -254,8 +254,12 @@ fq_status fq_linear(const uint16_t* X, int M, int K, const fq_qparams* act_qp,
  * Arithmetic: per token, row and block, s = sum x t and S = sum x in
  * float32, y = fp16(sum over blocks of alpha s + mu S) accumulated in float32
  * (the summation order is the kernel's; not bit-reproducible against another
- * order).  Tokens are processed 8 at a time: M > 8 streams the weights
- * ceil(M / 8) times.  Enqueues one kernel; allocates nothing. */
+ * order, but the same on every run).  For M <= 16 and K <= 32768 the partial
+ * products of weight pairs come from per-token tables of the 16 possible pair
+ * sums (each the float32 rounding of the exact sum), one launch of clusters
+ * of ceil(K / 4096) CTAs reads the weights from HBM once; otherwise tokens
+ * are processed 8 at a time and M > 8 streams the weights ceil(M / 8) times.
+ * Enqueues one kernel; allocates nothing. */
 fq_status fq_ternary_linear(const uint16_t* X, int M, int K, const uint8_t* Tq, const float* alpha,
                             const float* mu, int N, uint16_t* Y, void* stream);
 

@@ -20,6 +20,7 @@
 #include <cuda_fp16.h>
 
 #include <algorithm>
+#include <atomic>
 
 #include "fq_device.cuh"
 #include "fq_host.h"
@@ -197,7 +198,222 @@ __global__ void __launch_bounds__(256) ternary_pack_kernel(const int8_t* __restr
   }
 }
 
+// ------------------------------------------------------------------ pair-sum tables (M <= 16, K <= 32768)
+//
+// The partial product of two adjacent weights with one token takes one of
+// nine values, 0, +-a, +-b, +-a +-b (a, b the two fp16 values).  Per token,
+// the CTA writes all 16 code-pair entries of every weight pair of its K
+// slice into shared memory; the product of a weight row is then one table
+// read and half an addition per weight, with no per-weight decoding.
+//
+// A cluster of c CTAs splits K into c slices of at most 4096 columns (256
+// code words) and walks one range of weight rows; each CTA writes its
+// slice's partial sum of every row and token to its shared memory, and after
+// a cluster barrier CTA r sums rows r, r + c, ... over the c slices in rank
+// order through distributed shared memory (a fixed order: the result does not
+// depend on scheduling).
+//
+// Table layout (128 KB, per 4-byte entry): lane l of a warp reads the 16
+// code words 4 l + 128 u + v (v < 4, u < 2) of its row; the pair in the low
+// nibble of byte j of word v (pair 2 j) is looked up in region L at
+// code * 256 + (q / 2) * 4096 + (q % 2) * 128 + 4 l, the pair in the high
+// nibble (pair 2 j + 1) in region H at 65536 + code * 4096 + q * 128 + 4 l,
+// q = (4 j + v) * 2 + u.  Once byte j is shifted to bits 8-15 of a
+// register, (reg & 0xF00) | 4 l and (reg & 0xF000) | 4 l are the byte
+// offsets of both entries up to a constant, and every address of a warp's
+// lookup falls in bank l: no conflicts.
+constexpr int kLutThreads = 512;
+constexpr int kLutWarps = kLutThreads / 32;
+constexpr int kLutSliceWords = 256;      // code words of a CTA's K slice
+constexpr int kLutRegion = 65536;        // bytes per table region (L, H)
+constexpr int kLutPartials = 8192;       // floats of per-chunk partial sums
+constexpr int kLutMaxM = 16;             // tokens per launch on this path
+constexpr int kLutMaxCluster = 8;
+constexpr size_t kLutSmem = 2 * size_t(kLutRegion) + kLutPartials * sizeof(float) + 32 * sizeof(float);
+
+// Entries of the 16 codes of one weight pair: bits 0-1 the first weight's
+// code, bits 2-3 the second's (01 = +1, 11 = -1, 00 and 10 = 0); every entry
+// is the float32 rounding of the exact pair sum.
+__device__ __forceinline__ void pair_entries(float a, float b, float (&e)[16]) {
+  const float s = a + b, d = a - b;
+  const float t[4] = {0.f, a, 0.f, -a};
+#pragma unroll
+  for (int ca = 0; ca < 4; ++ca) {
+    e[ca] = t[ca];
+    e[ca + 8] = t[ca];
+  }
+  e[4] = b, e[5] = s, e[6] = b, e[7] = -d;
+  e[12] = -b, e[13] = d, e[14] = -b, e[15] = -s;
+}
+
+// Sum over the 16 weights pairs of code words w4 (a lane's quad u) of the
+// table entries: 32 lookups.
+template <int U>
+__device__ __forceinline__ float quad_sum(const uint8_t* tab, uint4 w4, uint32_t lb) {
+  const uint32_t wv[4] = {w4.x, w4.y, w4.z, w4.w};
+  float2 s = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int v = 0; v < 4; ++v) {
+    const uint32_t src[4] = {wv[v] << 8, wv[v], wv[v] >> 8, wv[v] >> 16};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int q = (4 * j + v) * 2 + U;
+      const float lo =
+          *reinterpret_cast<const float*>(tab + ((src[j] & 0xF00u) | lb) + (q >> 1) * 4096 + (q & 1) * 128);
+      const float hi = *reinterpret_cast<const float*>(tab + kLutRegion + ((src[j] & 0xF000u) | lb) + q * 128);
+      s = fadd2(s, make_float2(lo, hi));
+    }
+  }
+  return s.x + s.y;
+}
+
+struct LutRow {
+  uint4 w[2];    // the lane's two quads of code words
+  float al[2];   // their blocks' alpha
+  float mu;      // mu of the slice's block `lane`
+};
+
+__global__ void __launch_bounds__(kLutThreads, 1)
+    ternary_lut_kernel(const TernaryParams p, const int slice_words, const int rows_per_cluster, const int chunk_rows) {
+  extern __shared__ __align__(16) uint8_t lsm[];
+  float* part = reinterpret_cast<float*>(lsm + 2 * kLutRegion);  // [M][chunk_rows] partial sums
+  float* sS = part + kLutPartials;                                // [32] block sums of the token
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t c = cluster_size(), rank = cluster_rank();
+  const int cl = blockIdx.x / c;
+  const int words = p.K / 16, nb = p.K / kTerBlock;
+  const int w0 = int(rank) * slice_words;
+  const int ws = max(0, min(words, w0 + slice_words) - w0);  // this CTA's code words
+  const int gb0 = w0 / 8, nbs = ws / 8;                       // its first block, block count (<= 32)
+  const int r_begin = cl * rows_per_cluster, r_end = min(p.N, r_begin + rows_per_cluster);
+  const uint32_t lb = uint32_t(lane) * 4;
+  const bool has0 = 4 * lane < ws, has1 = 4 * lane + 128 < ws;
+  const uint4* tq = reinterpret_cast<const uint4*>(p.T);
+  const size_t row_quads = size_t(words) / 4;
+  pdl_wait();
+  for (int cr0 = r_begin; cr0 < r_end; cr0 += chunk_rows) {
+    const int rc = min(chunk_rows, r_end - cr0);
+    for (int m = 0; m < p.M; ++m) {
+      __syncthreads();  // the previous token's table is no longer read
+      const __half* xm = p.X + size_t(m) * p.K + size_t(w0) * 16;
+      for (int e = tid; e < 2048; e += kLutThreads) {
+        const int region = e >> 10, q = (e >> 5) & 31, ln = e & 31;
+        const int j = q >> 3, v = (q >> 1) & 3, u = q & 1;
+        const int word = 4 * ln + 128 * u + v;
+        float a = 0.f, b = 0.f;
+        if (word < ws) {
+          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(xm + 16 * word + 2 * (2 * j + region)));
+          a = f.x, b = f.y;
+        }
+        float ent[16];
+        pair_entries(a, b, ent);
+        uint8_t* dst = region == 0 ? lsm + (q >> 1) * 4096 + (q & 1) * 128 + 4 * ln
+                                   : lsm + kLutRegion + q * 128 + 4 * ln;
+        const int stride = region == 0 ? 256 : 4096;
+#pragma unroll
+        for (int code = 0; code < 16; ++code) *reinterpret_cast<float*>(dst + code * stride) = ent[code];
+      }
+      // the token's block sums over the slice (for the mu term)
+      for (int g = warp; g < nbs; g += kLutWarps) {
+        const uint2 raw = *reinterpret_cast<const uint2*>(xm + g * kTerBlock + 4 * lane);
+        const float2 fa = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
+        const float2 fb = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
+        float v = (fa.x + fa.y) + (fb.x + fb.y);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane == 0) sS[g] = v;
+      }
+      __syncthreads();
+      const float s_lane = lane < nbs ? sS[lane] : 0.f;
+      float* pm = part + m * chunk_rows;
+      auto load_row = [&](int rr, LutRow& r) {
+        r.w[0] = r.w[1] = make_uint4(0u, 0u, 0u, 0u);
+        r.al[0] = r.al[1] = r.mu = 0.f;
+        if (rr < rc) {
+          const int n = cr0 + rr;
+          const uint4* row = tq + size_t(n) * row_quads + w0 / 4;
+          const float* arow = p.alpha + size_t(n) * nb + gb0;
+          if (has0) r.w[0] = __ldg(row + lane), r.al[0] = __ldg(arow + lane / 2);
+          if (has1) r.w[1] = __ldg(row + lane + 32), r.al[1] = __ldg(arow + lane / 2 + 16);
+          if (lane < nbs) r.mu = __ldg(p.mu + size_t(n) * nb + gb0 + lane);
+        }
+      };
+      auto row_value = [&](const LutRow& r) {
+        float acc = 0.f;
+        if (has0) acc = fmaf(r.al[0], quad_sum<0>(lsm, r.w[0], lb), acc);
+        if (has1) acc = fmaf(r.al[1], quad_sum<1>(lsm, r.w[1], lb), acc);
+        acc = fmaf(r.mu, s_lane, acc);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        return acc;
+      };
+      // two rows per warp in flight: a row's loads are issued one row
+      // computation ahead of their use
+      LutRow ra, rb;
+      load_row(warp, ra);
+      load_row(warp + kLutWarps, rb);
+      for (int rr = warp; rr < rc; rr += 2 * kLutWarps) {
+        const float ya = row_value(ra);
+        load_row(rr + 2 * kLutWarps, ra);
+        if (lane == 0) pm[rr] = ya;
+        if (rr + kLutWarps < rc) {
+          const float yb = row_value(rb);
+          if (lane == 0) pm[rr + kLutWarps] = yb;
+        }
+        load_row(rr + 3 * kLutWarps, rb);
+      }
+    }
+    cluster_sync();  // every CTA's partial sums of the chunk are written
+    const int nr = rc > int(rank) ? (rc - int(rank) + int(c) - 1) / int(c) : 0;
+    for (int e = tid; e < p.M * nr; e += kLutThreads) {
+      const int m = e / nr, rr = int(rank) + int(c) * (e - m * nr);
+      float y = 0.f;
+      for (uint32_t r = 0; r < c; ++r) y += ld_cluster_f32(part + m * chunk_rows + rr, r);
+      p.Y[size_t(m) * p.N + cr0 + rr] = __float2half_rn(y);
+    }
+    cluster_sync();  // the peers have read this CTA's partial sums
+  }
+  pdl_launch_dependents();
+}
+
 }  // namespace
+
+// Clusters of c CTAs of ternary_lut_kernel that fit on the device at once
+// (0 if none or the query fails); cached per c.
+static int lut_clusters(int c) {
+  static std::atomic<int> cache[kLutMaxCluster + 1];
+  static std::atomic<bool> attr_set{false};
+  const int hit = cache[c].load(std::memory_order_relaxed);
+  if (hit != 0) return hit > 0 ? hit : 0;
+  if (!attr_set.load(std::memory_order_relaxed)) {
+    if (cudaFuncSetAttribute(ternary_lut_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kLutSmem)) !=
+        cudaSuccess) {
+      cudaGetLastError();
+      cache[c].store(-1);
+      return 0;
+    }
+    attr_set.store(true);
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(c * sm_count());
+  cfg.blockDim = dim3(kLutThreads);
+  cfg.dynamicSmemBytes = kLutSmem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = unsigned(c);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, ternary_lut_kernel, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    n = 0;
+  }
+  cache[c].store(n > 0 ? n : -1);
+  return n > 0 ? n : 0;
+}
+
 }  // namespace fq
 
 extern "C" {
@@ -221,6 +437,30 @@ fq_status fq_ternary_linear(const uint16_t* X, int M, int K, const uint8_t* Tq, 
   p.M = M;
   p.N = N;
   p.K = K;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // pair-sum tables: one cluster of c CTAs per row range, c K slices of at
+  // most 4096 columns (the table of a slice fills 128 KB)
+  const int words = K / 16;
+  const int c = (words + fq::kLutSliceWords - 1) / fq::kLutSliceWords;
+  if (M <= fq::kLutMaxM && c <= fq::kLutMaxCluster) {
+    const int ncl_max = fq::lut_clusters(c);
+    if (ncl_max > 0) {
+      const int slice_words = ((words + c - 1) / c + 7) / 8 * 8;
+      const int rows_per_cluster = (N + ncl_max - 1) / ncl_max;
+      const int ncl = (N + rows_per_cluster - 1) / rows_per_cluster;
+      // one token: the whole range at once; several: 256-row chunks, whose
+      // code words stay in L2 between the tokens' passes
+      const int chunk_rows = M == 1 ? fq::kLutPartials : std::min(256, fq::kLutPartials / M);
+      const cudaError_t e = fq::launch_pdl_cluster(fq::ternary_lut_kernel, dim3(ncl * c), dim3(fq::kLutThreads),
+                                                   fq::kLutSmem, st, unsigned(c), p, slice_words, rows_per_cluster,
+                                                   chunk_rows);
+      if (e != cudaSuccess) {
+        cudaGetLastError();
+        return fq::fail(FQ_ERR_CUDA, "ternary_lut_kernel: %s", cudaGetErrorString(e));
+      }
+      return fq::check_launch("ternary_lut_kernel");
+    }
+  }
   const size_t smem = size_t(fq::kTerMT) * (K / fq::kTerBlock) * sizeof(float);
   auto kern = fq::ternary_linear_kernel;
   if (smem > 48 * 1024 && cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
@@ -228,8 +468,7 @@ fq_status fq_ternary_linear(const uint16_t* X, int M, int K, const uint8_t* Tq, 
     return fq::fail(FQ_ERR_CUDA, "cannot reserve %zu bytes of shared memory", smem);
   const int rows_per_cta = fq::kTerWarps * fq::kTerR;
   const int grid = std::max(1, std::min((N + rows_per_cta - 1) / rows_per_cta, 4 * fq::sm_count()));
-  const cudaError_t e = fq::launch_pdl(kern, dim3(grid), dim3(fq::kTerThreads), smem,
-                                       static_cast<cudaStream_t>(stream), p);
+  const cudaError_t e = fq::launch_pdl(kern, dim3(grid), dim3(fq::kTerThreads), smem, st, p);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return fq::fail(FQ_ERR_CUDA, "ternary_linear_kernel: %s", cudaGetErrorString(e));

@@ -5,11 +5,14 @@ against the oracle's pack_ternary and ternary_linear.
 Packing is integer work and is compared bit-exactly.  The product is float32
 arithmetic in the kernel's own order against the float64 definition, so
 each output must lie within 1 fp16 ulp of the exact value plus a float32
-accumulation bound derived from the summation: no partial sum passes through
-more than 16 (a 16-weight word) + K/512 (a lane's words) + 5 (the warp
-reduction) + 8 + K/4096 (the block sums of the offset term) roundings, each
-at most 2^-24 of B = sum_k |x_k| (|alpha t_k| + |mu|); the test allows
-(K/16 + 160) 2^-24 B.
+accumulation bound derived from the summation, each rounding at most 2^-24
+of B = sum_k |x_k| (|alpha t_k| + |mu|).  Per-token tables of pair sums
+(M <= 16, K <= 32768): a partial sum passes through 1 (the table entry) + 16
+(a lane's 32 lookups in two float32 lanes) + 3 (alpha) + 8 (the offset term's
+block sum) + 5 (the warp) + 8 (the cluster's slices) roundings.  Direct
+kernel: 16 (a 16-weight word) + K/512 (a lane's words) + 5 (the warp
+reduction) + 8 + K/4096 (the block sums of the offset term).  The test
+allows (K/16 + 160) 2^-24 B.
 """
 import numpy as np
 import pytest
@@ -70,6 +73,39 @@ def test_ternary_linear_decode_full(m, k, n):
     cols = C.tile_samples(m + k + n, n)
     worst = _check_close(y[:, cols], d["x"], d["t"], d["alpha"], d["mu"], cols=cols)
     print(f"{d['name']}: {len(cols)} columns, worst err / bound {worst:.3f}")
+    fq.fq_check_device_error()
+
+
+@pytest.mark.parametrize("m,k,n", [
+    (2, 8192, 20000),   # tables, two K slices, several 256-row chunks per cluster
+    (1, 32768, 300),    # tables, the largest cluster (8 slices)
+    (16, 4224, 130),    # tables, the most tokens; a 33-block K in two ragged slices
+    (1, 12288, 5),      # tables, three slices, fewer rows than clusters
+    (17, 1024, 77),     # direct kernel: more tokens than the tables take
+    (1, 32896, 50),     # direct kernel: K beyond 8 slices of 4096
+])
+def test_ternary_linear_paths(m, k, n):
+    """Both kernels and the edges between them; every output checked below
+    10000 rows, above that columns hitting every 128-row stretch."""
+    d = synth.ternary_linear(m, k, n, seed=m + k + n)
+    tq = fq.fq_ternary_pack(C.dev(d["t"]))
+    y = C.host(fq.fq_ternary_linear(C.dev(d["x"]), tq, C.dev(d["alpha"]), C.dev(d["mu"])))
+    if n < 10000:
+        _check_close(y, d["x"], d["t"], d["alpha"], d["mu"])
+    else:
+        cols = C.tile_samples(m + k + n, n)
+        _check_close(y[:, cols], d["x"], d["t"], d["alpha"], d["mu"], cols=cols)
+    fq.fq_check_device_error()
+
+
+def test_ternary_linear_repeatable():
+    """The summation order is fixed: two launches give the same bits."""
+    d = synth.ternary_linear(8, 8192, 4096, seed=11)
+    tq = fq.fq_ternary_pack(C.dev(d["t"]))
+    args = (C.dev(d["x"]), tq, C.dev(d["alpha"]), C.dev(d["mu"]))
+    y1 = C.host(fq.fq_ternary_linear(*args))
+    y2 = C.host(fq.fq_ternary_linear(*args))
+    assert np.array_equal(y1.view(np.uint16), y2.view(np.uint16))
     fq.fq_check_device_error()
 
 
