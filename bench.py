@@ -380,6 +380,11 @@ def run_ours(args, ws, rank, local):
 # CUDA-event pair with an L2 flush (a 256 MiB write) between launches, outside
 # the timed pair, because these inputs alone may fit in the 126 MB L2.
 
+TIMED_MIN_S = 0.25         # shortest timed region of a workload line
+TIMED_MAX_LAUNCHES = 5000  # most launches a workload line times
+TIMED_PROBE = 5            # launches that estimate the time per launch
+
+
 class LaunchTimer:
     def __init__(self, dev, stream, clocks):
         import torch
@@ -390,11 +395,21 @@ class LaunchTimer:
         self.flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
     def time(self, fn, steps, warmup):
+        """Median launch time over at least `steps` launches, and over enough
+        launches that the timed region lasts TIMED_MIN_S (the clock sampler's
+        period is 50 ms), at most TIMED_MAX_LAUNCHES."""
         torch = self.torch
         for _ in range(warmup):
             fn()
         torch.cuda.synchronize()
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        t0 = time.perf_counter()
+        for _ in range(TIMED_PROBE):
+            self.flush_buf.fill_(1)
+            fn()
+        torch.cuda.synchronize()
+        per = max((time.perf_counter() - t0) / TIMED_PROBE, 1e-6)
+        n = max(steps, min(TIMED_MAX_LAUNCHES, int(TIMED_MIN_S / per) + 1))
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
         self.clocks.active = True
         for a, b in evs:
             self.flush_buf.fill_(1)
