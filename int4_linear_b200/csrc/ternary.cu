@@ -5,18 +5,22 @@
 // Per output (m, n): y = sum_g (alpha[n][g] s[m][n][g] + mu[n][g] S[m][g])
 // with s = sum_{k in g} x[m][k] t[n][k] and S = sum_{k in g} x[m][k], all in
 // float32.  A ternary weight needs no multiplication, but at fp16
-// activations it still costs a CUDA-core instruction or two: the code is
-// turned into +-1.0 / 0 and accumulated with an FMA per token.  The tensor
+// activations it still costs CUDA-core work per weight and token; the tensor
 // core does not help at decode sizes (an MMA of N <= 16 tokens holds its
-// issuer far longer than its arithmetic takes), so this kernel is bound by
-// ALU issue, not by the 2 bits per weight it streams.
+// issuer far longer than its arithmetic takes).  Two kernels:
 //
-// Mapping: one warp per two weight rows at a time (grid-stride over rows);
-// lane l reads the 32-bit code words l, l + 32, ... of both rows (16 weights
-// each, consecutive lanes on consecutive words, four words per lane in
-// flight) and the matching 16 fp16 values of each token once for both rows;
-// the 8 words of a 128-block share its alpha.  The block sums S of the CTA's
-// token group sit in shared memory, one warp per (token, block).
+// ternary_lut_kernel (M <= 16, K <= 32768): per-token tables of the 16
+// possible sums of two adjacent weights' products, one table read and half
+// an addition per weight; K split over a cluster of CTAs (layout and
+// reduction described above the kernel).
+//
+// ternary_linear_kernel (the rest): one warp per two weight rows at a time
+// (grid-stride over rows); lane l reads the 32-bit code words l, l + 32, ...
+// of both rows (16 weights each, consecutive lanes on consecutive words,
+// four words per lane in flight) and the matching 16 fp16 values of each
+// token once for both rows; the 8 words of a 128-block share its alpha.  The
+// block sums S of the CTA's token group sit in shared memory, one warp per
+// (token, block).
 #include <cuda_fp16.h>
 
 #include <algorithm>
@@ -246,7 +250,7 @@ __device__ __forceinline__ void pair_entries(float a, float b, float (&e)[16]) {
   e[12] = -b, e[13] = d, e[14] = -b, e[15] = -s;
 }
 
-// Sum over the 16 weights pairs of code words w4 (a lane's quad u) of the
+// Sum over the 32 weight pairs of a lane's quad U (code words w4) of their
 // table entries: 32 lookups.
 template <int U>
 __device__ __forceinline__ float quad_sum(const uint8_t* tab, uint4 w4, uint32_t lb) {
