@@ -134,9 +134,16 @@ class ClockSampler:
         except Exception:
             self.proc.kill()
         self.t.join(timeout=2)
+        return self.summary(self.lines)
+
+    @staticmethod
+    def summary(lines):
+        """Median SM clock, the max clock and the throttle reasons seen Active
+        in `nvidia-smi --query-gpu=FIELDS --format=csv,noheader,nounits` rows
+        (None without a parsable row)."""
         sm, smax, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        for ln in lines:
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 8:
                 continue
